@@ -1,0 +1,194 @@
+"""CPU oracle for the sparse Mixture-of-Experts layer forward pass.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by ``bench.py``'s CPU-baseline leg. The product path (the CUDA library and
+its Python binding) never imports it, and it imports nothing from the product.
+
+The arithmetic lives in ``moe_oracle.cpp`` (plain C++, fp64 except for the fp32
+router whose summation order is stated there). This module only builds that
+file and marshals numpy / torch CPU arrays into it.
+
+Every function cites its passage in ``moe_oracle.cpp``. All oracle functions
+here are pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``
+(brute-force sorts, closed forms, invariants, and library routines); none is
+parity-unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.cpp")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+CXXFLAGS = ["-O2", "-std=c++17", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-mfma",
+            "-shared", "-fPIC"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``moe_oracle.cpp`` into ``libmoe_oracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["g++", *CXXFLAGS, _SRC, "-o", tmp], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I = ctypes.c_int64
+            lib.oracle_router_logits.argtypes = [P, P, P, I, I, I, P]
+            lib.oracle_topk.argtypes = [P, I, I, I, P, P, P]
+            lib.oracle_permute.argtypes = [P, I, I, I, P, P, P, P]
+            lib.oracle_expert_ffn.argtypes = [P, I, P, P, I, I, P, P]
+            lib.oracle_combine.argtypes = [P, P, P, I, I, I, P]
+            lib.oracle_forward_tokens.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, P, P]
+            for fn in ("oracle_router_logits", "oracle_topk", "oracle_permute", "oracle_expert_ffn",
+                       "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version"):
+                getattr(lib, fn).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+# ---------------------------------------------------------------- marshalling
+
+def _bf16_bits(a) -> np.ndarray:
+    """A bf16 torch tensor (CPU) or a uint16 numpy array -> contiguous uint16 bits."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            assert a.dtype == torch.bfloat16, a.dtype
+            return np.ascontiguousarray(a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.asarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return np.ascontiguousarray(a)
+
+
+def _f32(a) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return np.ascontiguousarray(a.detach().cpu().to(torch.float32).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _check(st: int, what: str):
+    if st == 1:
+        raise ValueError(f"{what}: bad argument")
+    if st == 2:
+        raise FloatingPointError(f"{what}: non-finite input (outside the oracle's contract)")
+    if st != 0:
+        raise RuntimeError(f"{what}: status {st}")
+
+
+# ------------------------------------------------------------------ the steps
+
+def router_logits(x, W_router, bias=None) -> np.ndarray:
+    """Step 1 of moe_oracle.cpp: fp32 logits [T, E] in the stated chunked order."""
+    xb = _bf16_bits(x)
+    Wr = _f32(W_router)
+    T, d = xb.shape
+    d2, E = Wr.shape
+    assert d == d2
+    b = _f32(bias) if bias is not None else None
+    out = np.empty((T, E), dtype=np.float32)
+    _check(_load().oracle_router_logits(_ptr(xb), _ptr(Wr), _ptr(b), T, d, E, _ptr(out)), "router_logits")
+    return out
+
+
+def topk(logits: np.ndarray, k: int, want_probs: bool = False):
+    """Steps 2-3: (idx [T,k] int32, w [T,k] fp64[, probs [T,E] fp64])."""
+    lg = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    probs = np.empty((T, E), dtype=np.float64) if want_probs else None
+    _check(_load().oracle_topk(_ptr(lg), T, E, k, _ptr(idx), _ptr(w), _ptr(probs)), "topk")
+    return (idx, w, probs) if want_probs else (idx, w)
+
+
+def permute(idx: np.ndarray, E: int):
+    """Step 4: (counts [E], offsets [E+1], perm_token [T*k], inv_perm [T,k]) int32."""
+    ix = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = ix.shape
+    counts = np.empty(E, dtype=np.int32)
+    offsets = np.empty(E + 1, dtype=np.int32)
+    perm_token = np.empty(T * k, dtype=np.int32)
+    inv_perm = np.empty((T, k), dtype=np.int32)
+    _check(_load().oracle_permute(_ptr(ix), T, E, k, _ptr(counts), _ptr(offsets), _ptr(perm_token),
+                                  _ptr(inv_perm)), "permute")
+    return counts, offsets, perm_token, inv_perm
+
+
+def expert_ffn(x_rows, W_gate_up_e, W_down_e, want_h: bool = False):
+    """Step 5 for one expert: y [n, d] fp64 (and h [n, f] fp64)."""
+    xr = _bf16_bits(x_rows)
+    Wg = _bf16_bits(W_gate_up_e)
+    Wd = _bf16_bits(W_down_e)
+    n, d = xr.shape
+    d2, f2 = Wg.shape
+    f, d3 = Wd.shape
+    assert d == d2 == d3 and f2 == 2 * f
+    y = np.empty((n, d), dtype=np.float64)
+    h = np.empty((n, f), dtype=np.float64) if want_h else None
+    _check(_load().oracle_expert_ffn(_ptr(xr), n, _ptr(Wg), _ptr(Wd), d, f, _ptr(y), _ptr(h)), "expert_ffn")
+    return (y, h) if want_h else y
+
+
+def combine(y_rows: np.ndarray, inv_perm: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Step 6: out [T, d] fp64."""
+    y = np.ascontiguousarray(y_rows, dtype=np.float64)
+    ip = np.ascontiguousarray(inv_perm, dtype=np.int32)
+    ww = np.ascontiguousarray(w, dtype=np.float64)
+    T, k = ip.shape
+    d = y.shape[1]
+    out = np.empty((T, d), dtype=np.float64)
+    _check(_load().oracle_combine(_ptr(y), _ptr(ip), _ptr(ww), T, d, k, _ptr(out)), "combine")
+    return out
+
+
+def forward(x, W_router, bias, W_gate_up, W_down, k: int, tokens=None):
+    """The whole layer (steps 1-6) for all tokens or the listed ones.
+
+    Returns (out [n, d] fp64, idx [n, k] int32, w [n, k] fp64).
+    """
+    xb = _bf16_bits(x)
+    Wr = _f32(W_router)
+    b = _f32(bias) if bias is not None else None
+    Wg = _bf16_bits(W_gate_up)
+    Wd = _bf16_bits(W_down)
+    T, d = xb.shape
+    E = Wr.shape[1]
+    f = Wd.shape[1]
+    assert Wg.shape == (E, d, 2 * f) and Wd.shape == (E, f, d)
+    tok = None if tokens is None else np.ascontiguousarray(np.asarray(tokens, dtype=np.int64))
+    n = T if tok is None else tok.shape[0]
+    out = np.empty((n, d), dtype=np.float64)
+    idx = np.empty((n, k), dtype=np.int32)
+    w = np.empty((n, k), dtype=np.float64)
+    _check(_load().oracle_forward_tokens(_ptr(xb), _ptr(Wr), _ptr(b), _ptr(Wg), _ptr(Wd), T, d, E, k, f,
+                                         _ptr(tok), n, _ptr(out), _ptr(idx), _ptr(w)), "forward")
+    return out, idx, w

@@ -1,0 +1,287 @@
+// Plain CPU oracle for the forward pass of one sparse Mixture-of-Experts layer.
+//
+// TEST INFRASTRUCTURE ONLY. The tests, the package's smoke() and the bench's
+// CPU-baseline leg call this library to check and to time the CUDA path; the
+// product path never loads it. It shares no source, header, table or helper
+// with the CUDA library: every step below is written out from its definition.
+//
+// What it computes, step by step (page titles abbreviated as
+//   [P2] "Kimi K3: The Open Model That Just Cornered the AI Frontier",
+//   [P3] "Kimi K3: Open Frontier Intelligence"):
+//
+//  1. Router logits l[t,e] = sum_i x[t,i] * W_router[i,e] (+ b[e]).
+//     [P2] section "Mixture-of-Experts with Dynamic Load Balancing", gating
+//     code: one linear gate projection from d_model to n_experts.
+//     The pages fix no precision for it; reading taken: fp32, with x widened
+//     from bf16 exactly, in a stated order (oracle_router_logits below), so
+//     that routing decisions are reproducible bit for bit.
+//  2. probs = softmax over ALL experts ([P2] gating code: softmax is taken
+//     over the last axis before top-k). Computed here in fp64.
+//  3. top-k: the k largest, returned with their (unnormalised) softmax values
+//     ([P2] gating code returns the top-k values and indices as they are).
+//     Selection compares the fp32 logits (softmax is monotone, so this is the
+//     same set as ranking the probabilities in exact arithmetic); equal
+//     logits go to the lower expert index; slots are in descending order.
+//  4. dispatch: a stable counting sort of the (token, slot) pairs by expert
+//     ([P3] section "Operational Execution Flow": tokens are dispatched to
+//     their active routed experts).
+//  5. per-expert SwiGLU FFN in fp64: g = x W_gu[:, 0:f], u = x W_gu[:, f:2f],
+//     h = SiLU(g) * u with SiLU(a) = a / (1 + exp(-a)), y = h W_down.
+//  6. combine: out[t] = sum_j p[t,j] * y[t,j] in fp64 ([P3] "Operational
+//     Execution Flow": the routed output is the probability-weighted sum of
+//     the selected experts' outputs).
+//
+// Build: g++ -O2 -std=c++17 -fopenmp -ffp-contract=off -mfma -shared -fPIC.
+// -ffp-contract=off keeps the compiler from fusing any multiply-add the code
+// does not spell as std::fma; -mfma makes std::fma a single instruction.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+inline float bf16_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof(f));
+  return f;
+}
+
+inline double bf16_to_double(uint16_t b) { return static_cast<double>(bf16_to_float(b)); }
+
+constexpr int64_t kChunk = 128;  // router summation chunk (step 1)
+
+}  // namespace
+
+extern "C" {
+
+// Status codes: 0 ok, 1 bad argument, 2 non-finite input.
+
+int oracle_version(void) { return 1; }
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+// Step 1. logits[t*E + e] in fp32.
+// Order: i runs over consecutive chunks of 128 indices. Inside chunk c the
+// partial p_c starts at +0 and takes p_c = fma(x_i, W[i,e], p_c) for i
+// ascending. Then l = p_0, l = l + p_1, ..., l = l + p_{C-1} (ascending c),
+// then l = l + b_e when a bias is given. Every operation is one correctly
+// rounded fp32 fma or add.
+int oracle_router_logits(const uint16_t* x, const float* Wr, const float* bias,
+                         int64_t T, int64_t d, int64_t E, float* logits) {
+  if (!x || !Wr || !logits || T < 0 || d <= 0 || E <= 0) return 1;
+  const int64_t C = (d + kChunk - 1) / kChunk;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t t = 0; t < T; ++t) {
+    std::vector<float> l(E), p(E);
+    std::vector<float> xf(d);
+    for (int64_t i = 0; i < d; ++i) {
+      xf[i] = bf16_to_float(x[t * d + i]);
+      if (!std::isfinite(xf[i])) bad |= 1;
+    }
+    for (int64_t c = 0; c < C; ++c) {
+      std::fill(p.begin(), p.end(), 0.0f);
+      const int64_t i0 = c * kChunk, i1 = std::min(d, i0 + kChunk);
+      for (int64_t i = i0; i < i1; ++i) {
+        const float xi = xf[i];
+        const float* w = Wr + i * E;
+        for (int64_t e = 0; e < E; ++e) p[e] = std::fma(xi, w[e], p[e]);
+      }
+      if (c == 0) {
+        for (int64_t e = 0; e < E; ++e) l[e] = p[e];
+      } else {
+        for (int64_t e = 0; e < E; ++e) l[e] = l[e] + p[e];
+      }
+    }
+    if (bias)
+      for (int64_t e = 0; e < E; ++e) l[e] = l[e] + bias[e];
+    for (int64_t e = 0; e < E; ++e) logits[t * E + e] = l[e];
+  }
+  return bad ? 2 : 0;
+}
+
+// Steps 2 and 3. For each token: probabilities over all E experts in fp64,
+// then the k experts with the largest logits (ties: lower index first), in
+// descending order, with their unnormalised probabilities.
+// probs (optional, may be NULL) receives all E probabilities.
+int oracle_topk(const float* logits, int64_t T, int64_t E, int64_t k,
+                int32_t* idx, double* w, double* probs) {
+  if (!logits || !idx || !w || T < 0 || E <= 0 || k <= 0 || k > E) return 1;
+  int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * E;
+    double m = -INFINITY;
+    for (int64_t e = 0; e < E; ++e) {
+      if (!std::isfinite(l[e])) bad |= 1;
+      m = std::max(m, static_cast<double>(l[e]));
+    }
+    double s = 0.0;
+    for (int64_t e = 0; e < E; ++e) s += std::exp(static_cast<double>(l[e]) - m);
+    std::vector<int32_t> order(E);
+    for (int64_t e = 0; e < E; ++e) order[e] = static_cast<int32_t>(e);
+    // stable: among equal logits the original (ascending) index order stays
+    std::stable_sort(order.begin(), order.end(),
+                     [l](int32_t a, int32_t b) { return l[a] > l[b]; });
+    for (int64_t j = 0; j < k; ++j) {
+      const int32_t e = order[j];
+      idx[t * k + j] = e;
+      w[t * k + j] = std::exp(static_cast<double>(l[e]) - m) / s;
+    }
+    if (probs)
+      for (int64_t e = 0; e < E; ++e) probs[t * E + e] = std::exp(static_cast<double>(l[e]) - m) / s;
+  }
+  return bad ? 2 : 0;
+}
+
+// Step 4. Stable counting sort of the T*k (token, slot) pairs by expert.
+// counts[e]; offsets[0..E] (exclusive scan, offsets[E] = T*k); perm_token[r]
+// is the token of permuted row r; inv_perm[t*k + j] is the row of (t, j).
+// Inside one expert the rows follow ascending token order.
+int oracle_permute(const int32_t* idx, int64_t T, int64_t E, int64_t k,
+                   int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm) {
+  if (!idx || !counts || !offsets || !perm_token || !inv_perm || T < 0 || E <= 0 || k <= 0) return 1;
+  for (int64_t e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t q = 0; q < T * k; ++q) {
+    const int32_t e = idx[q];
+    if (e < 0 || e >= E) return 1;
+    counts[e] += 1;
+  }
+  offsets[0] = 0;
+  for (int64_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  std::vector<int32_t> cursor(offsets, offsets + E);
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t j = 0; j < k; ++j) {
+      const int32_t e = idx[t * k + j];
+      const int32_t r = cursor[e]++;
+      perm_token[r] = static_cast<int32_t>(t);
+      inv_perm[t * k + j] = r;
+    }
+  }
+  return 0;
+}
+
+// Step 5 for one expert: n input rows x_rows[n, d] (bf16) through that
+// expert's W_gu[d, 2f] and W_down[f, d] (bf16), output y[n, d] in fp64.
+// h (optional, may be NULL) receives SiLU(g)*u as [n, f] fp64.
+int oracle_expert_ffn(const uint16_t* x_rows, int64_t n, const uint16_t* Wgu, const uint16_t* Wd,
+                      int64_t d, int64_t f, double* y, double* h_out) {
+  if ((!x_rows && n > 0) || !Wgu || !Wd || !y || n < 0 || d <= 0 || f <= 0) return 1;
+  const int64_t f2 = 2 * f;
+  const int64_t R = 16;  // rows per block (only to reuse a widened weight row)
+  const int64_t nblk = (n + R - 1) / R;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t b = 0; b < nblk; ++b) {
+    const int64_t r0 = b * R, r1 = std::min(n, r0 + R), nr = r1 - r0;
+    std::vector<double> gu(nr * f2, 0.0), hrow(nr * f), yy(nr * d, 0.0), wrow(std::max(f2, d));
+    for (int64_t i = 0; i < d; ++i) {
+      for (int64_t j = 0; j < f2; ++j) wrow[j] = bf16_to_double(Wgu[i * f2 + j]);
+      for (int64_t r = 0; r < nr; ++r) {
+        const double xi = bf16_to_double(x_rows[(r0 + r) * d + i]);
+        double* acc = &gu[r * f2];
+        for (int64_t j = 0; j < f2; ++j) acc[j] += xi * wrow[j];
+      }
+    }
+    for (int64_t r = 0; r < nr; ++r)
+      for (int64_t j = 0; j < f; ++j) {
+        const double g = gu[r * f2 + j], u = gu[r * f2 + f + j];
+        const double silu = g / (1.0 + std::exp(-g));
+        hrow[r * f + j] = silu * u;
+      }
+    for (int64_t j = 0; j < f; ++j) {
+      for (int64_t c = 0; c < d; ++c) wrow[c] = bf16_to_double(Wd[j * d + c]);
+      for (int64_t r = 0; r < nr; ++r) {
+        const double hj = hrow[r * f + j];
+        double* acc = &yy[r * d];
+        for (int64_t c = 0; c < d; ++c) acc[c] += hj * wrow[c];
+      }
+    }
+    for (int64_t r = 0; r < nr; ++r) {
+      for (int64_t c = 0; c < d; ++c) y[(r0 + r) * d + c] = yy[r * d + c];
+      if (h_out)
+        for (int64_t j = 0; j < f; ++j) h_out[(r0 + r) * f + j] = hrow[r * f + j];
+    }
+  }
+  return 0;
+}
+
+// Step 6. out[t, c] = sum_j w[t, j] * y_rows[inv_perm[t, j], c] (fp64, j ascending).
+int oracle_combine(const double* y_rows, const int32_t* inv_perm, const double* w,
+                   int64_t T, int64_t d, int64_t k, double* out) {
+  if (!y_rows || !inv_perm || !w || !out || T < 0 || d <= 0 || k <= 0) return 1;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t c = 0; c < d; ++c) out[t * d + c] = 0.0;
+    for (int64_t j = 0; j < k; ++j) {
+      const double* yr = y_rows + static_cast<int64_t>(inv_perm[t * k + j]) * d;
+      const double wj = w[t * k + j];
+      for (int64_t c = 0; c < d; ++c) out[t * d + c] += wj * yr[c];
+    }
+  }
+  return 0;
+}
+
+// The whole layer for the tokens listed in `tokens` (n_tok of them; all T
+// when tokens == NULL): steps 1-3 for those tokens, then step 5 per selected
+// (token, expert) pair and step 6. Expert weights are read where they lie
+// (bf16, [E, d, 2f] and [E, f, d]) and widened row by row. out is [n_tok, d]
+// fp64; idx_out [n_tok, k] and w_out [n_tok, k] may be NULL.
+int oracle_forward_tokens(const uint16_t* x, const float* Wr, const float* bias,
+                          const uint16_t* Wgu, const uint16_t* Wd,
+                          int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                          const int64_t* tokens, int64_t n_tok,
+                          double* out, int32_t* idx_out, double* w_out) {
+  if (!x || !Wr || !Wgu || !Wd || !out || T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || f <= 0)
+    return 1;
+  if (!tokens) n_tok = T;
+  std::vector<uint16_t> xs(n_tok * d);
+  for (int64_t q = 0; q < n_tok; ++q) {
+    const int64_t t = tokens ? tokens[q] : q;
+    if (t < 0 || t >= T) return 1;
+    std::memcpy(&xs[q * d], x + t * d, sizeof(uint16_t) * d);
+  }
+  std::vector<float> logits(n_tok * E);
+  int st = oracle_router_logits(xs.data(), Wr, bias, n_tok, d, E, logits.data());
+  if (st) return st;
+  std::vector<int32_t> idx(n_tok * k);
+  std::vector<double> w(n_tok * k);
+  st = oracle_topk(logits.data(), n_tok, E, k, idx.data(), w.data(), nullptr);
+  if (st) return st;
+  // group the selected pairs by expert so each expert's weights are widened once
+  std::vector<int32_t> counts(E), offsets(E + 1), perm_tok(n_tok * k), inv(n_tok * k);
+  st = oracle_permute(idx.data(), n_tok, E, k, counts.data(), offsets.data(), perm_tok.data(), inv.data());
+  if (st) return st;
+  std::vector<double> y(n_tok * k * d);
+  const int64_t f2 = 2 * f;
+  for (int64_t e = 0; e < E; ++e) {
+    const int64_t n = counts[e];
+    if (n == 0) continue;
+    std::vector<uint16_t> rows(n * d);
+    for (int64_t r = 0; r < n; ++r)
+      std::memcpy(&rows[r * d], &xs[static_cast<int64_t>(perm_tok[offsets[e] + r]) * d], sizeof(uint16_t) * d);
+    st = oracle_expert_ffn(rows.data(), n, Wgu + e * d * f2, Wd + e * f * d, d, f,
+                           &y[static_cast<int64_t>(offsets[e]) * d], nullptr);
+    if (st) return st;
+  }
+  st = oracle_combine(y.data(), inv.data(), w.data(), n_tok, d, k, out);
+  if (st) return st;
+  if (idx_out) std::memcpy(idx_out, idx.data(), sizeof(int32_t) * n_tok * k);
+  if (w_out) std::memcpy(w_out, w.data(), sizeof(double) * n_tok * k);
+  return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,146 @@
+"""Seeded synthetic workloads for the sparse Mixture-of-Experts layer forward pass.
+
+This module is shared by the CUDA path's tests and bench and by the CPU oracle's
+tests. It only draws random numbers and fixes shapes: it holds none of the
+layer's arithmetic (no router, softmax, top-k, permutation, FFN or combine).
+
+Shapes follow the model-card figures quoted on the pages:
+  * "Kimi K3: What Open-Source Frontier Models Reveal About RL Scaling for
+    Reasoning", section "The Architecture: MoE, Latent Attention, and Massive
+    Context": 384 experts, 8 selected per token;
+  * "Kimi K3: The Open Model That Just Cornered the AI Frontier", section
+    "Mixture-of-Experts with Dynamic Load Balancing": 256 experts, top-4;
+  * "Kimi K3: Open Frontier Intelligence", section "Operational Execution
+    Flow": 896 routed experts, 16 active per token; hidden size 7168.
+
+Distributions (one reading, stated once here):
+  x         ~ N(0, 1), rounded to bf16 (round-to-nearest-even)
+  W_router  ~ N(0, 0.02^2), fp32 (0.02 is the standard deviation)
+  W_gate_up ~ N(0, 1/d), rounded to bf16, layout [E, d, 2f]
+              (columns 0..f-1 feed the gate, f..2f-1 the up projection)
+  W_down    ~ N(0, 1/f), rounded to bf16, layout [E, f, d]
+  bias      (skewed workload only) b_e = 1.5 * ln(1 / rank_e), rank_e = e + 1
+
+Each tensor draws from its own stream of one seed: x 0, W_router 1,
+W_gate_up 2, W_down 3.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class MoEShape:
+    """Sizes of one MoE layer invocation.
+
+    T tokens, d model width, E experts, k experts per token, f expert hidden
+    width. ``bias`` names the router bias recipe (None or "zipf").
+    """
+
+    name: str
+    T: int
+    d: int
+    E: int
+    k: int
+    f: int
+    bias: Optional[str] = None
+    note: str = field(default="", compare=False)
+
+    def with_T(self, T: int, name: Optional[str] = None) -> "MoEShape":
+        return MoEShape(name or f"{self.name}_T{T}", T, self.d, self.E, self.k, self.f, self.bias, self.note)
+
+    def flops(self) -> float:
+        """Algorithmic FLOPs: router 2*T*d*E plus experts 6*T*k*d*f."""
+        return 2.0 * self.T * self.d * self.E + 6.0 * self.T * self.k * self.d * self.f
+
+    def as_dict(self) -> dict:
+        return {"workload": self.name, "T": self.T, "d": self.d, "E": self.E, "k": self.k, "f": self.f,
+                "router_bias": self.bias or "none"}
+
+
+#: The workloads. "tiny" is small enough for the oracle in seconds; the rest
+#: carry the model-card shapes.
+WORKLOADS = {
+    "tiny": MoEShape("tiny", 64, 128, 8, 2, 256, note="oracle-sized"),
+    "prefill": MoEShape("prefill", 4096, 7168, 384, 8, 2048, note="384 experts top-8"),
+    "decode": MoEShape("decode", 128, 7168, 256, 4, 2048, note="256 experts top-4"),
+    "skewed": MoEShape("skewed", 8192, 7168, 896, 16, 512, bias="zipf", note="896 experts top-16, Zipf-like bias"),
+}
+SWEEP_T = (1, 8, 32, 128, 512)
+for _T in SWEEP_T:
+    WORKLOADS[f"sweep_T{_T}"] = MoEShape(f"sweep_T{_T}", _T, 7168, 896, 16, 512, note="decode sweep")
+
+STREAM_X, STREAM_WR, STREAM_WGU, STREAM_WD = 0, 1, 2, 3
+
+
+def _gen(seed: int, stream: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 1_000_003 + int(stream))
+    return g
+
+
+def zipf_bias(E: int) -> torch.Tensor:
+    """Per-expert router bias b_e = 1.5 * ln(1 / (e + 1)), fp32 (Zipf-like load)."""
+    e = torch.arange(E, dtype=torch.float64)
+    return (1.5 * torch.log(1.0 / (e + 1.0))).to(torch.float32)
+
+
+@dataclass
+class MoEInputs:
+    """One seeded draw of every operand of the layer, on one device."""
+
+    shape: MoEShape
+    x: torch.Tensor                 # [T, d] bf16
+    W_router: torch.Tensor          # [d, E] fp32
+    bias: Optional[torch.Tensor]    # [E] fp32 or None
+    W_gate_up: torch.Tensor         # [E, d, 2f] bf16
+    W_down: torch.Tensor            # [E, f, d] bf16
+
+
+def make_x(shape: MoEShape, seed: int = 0, device="cpu") -> torch.Tensor:
+    g = _gen(seed, STREAM_X, device)
+    return torch.randn(shape.T, shape.d, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_router(shape: MoEShape, seed: int = 0, device="cpu") -> torch.Tensor:
+    g = _gen(seed, STREAM_WR, device)
+    return torch.randn(shape.d, shape.E, generator=g, device=device, dtype=torch.float32) * 0.02
+
+
+def _randn_bf16(shape_t, std: float, g, device, chunk_rows: int = 64) -> torch.Tensor:
+    """N(0, std^2) drawn in fp32 and rounded to bf16, one slab of the leading
+    dimension at a time so a 20+ GB weight never needs an fp32 copy."""
+    out = torch.empty(shape_t, dtype=torch.bfloat16, device=device)
+    lead = shape_t[0]
+    for s in range(0, lead, chunk_rows):
+        e = min(lead, s + chunk_rows)
+        tmp = torch.randn((e - s,) + tuple(shape_t[1:]), generator=g, device=device, dtype=torch.float32)
+        tmp.mul_(std)
+        out[s:e].copy_(tmp)
+        del tmp
+    return out
+
+
+def make_experts(shape: MoEShape, seed: int = 0, device="cpu"):
+    g2 = _gen(seed, STREAM_WGU, device)
+    W_gate_up = _randn_bf16((shape.E, shape.d, 2 * shape.f), 1.0 / math.sqrt(shape.d), g2, device)
+    g3 = _gen(seed, STREAM_WD, device)
+    W_down = _randn_bf16((shape.E, shape.f, shape.d), 1.0 / math.sqrt(shape.f), g3, device)
+    return W_gate_up, W_down
+
+
+def make_inputs(shape: MoEShape, seed: int = 0, device="cpu") -> MoEInputs:
+    """Draw x, W_router, bias, W_gate_up, W_down for ``shape`` on ``device``."""
+    x = make_x(shape, seed, device)
+    W_router = make_router(shape, seed, device)
+    bias = zipf_bias(shape.E).to(device) if shape.bias == "zipf" else None
+    W_gate_up, W_down = make_experts(shape, seed, device)
+    return MoEInputs(shape, x, W_router, bias, W_gate_up, W_down)
+
+
+def custom_shape(T: int, d: int, E: int, k: int, f: int, bias: Optional[str] = None, name: str = "custom") -> MoEShape:
+    return MoEShape(name, T, d, E, k, f, bias)

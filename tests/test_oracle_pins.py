@@ -1,0 +1,323 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks one oracle step against something fixed independently:
+hand-derived IEEE-754 values, closed forms, brute force on tiny inputs,
+invariants the definition implies, or a library routine (numpy / scipy) that
+computes the same well-defined quantity by other code. A plausible slip in the
+oracle -- a dropped term, a swapped gate/up half, a wrong index, an unstable
+sort, renormalised weights -- fails at least one of them
+(``test_oracle_mutations.py`` plants such slips and checks that).
+
+Passages: the gating code on "Kimi K3: The Open Model That Just Cornered the AI
+Frontier" (section "Mixture-of-Experts with Dynamic Load Balancing") and the
+routed-expert sum on "Kimi K3: Open Frontier Intelligence" (section
+"Operational Execution Flow").
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_mixture_experts_route_b200 import inputs as moe_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+U32 = 2.0 ** -24  # unit roundoff of binary32
+
+
+def _bf16(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _np_bf16_to_f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _silu(a):
+    return a / (1.0 + np.exp(-a))
+
+
+def _dense_swiglu(x64, Wgu64, Wd64):
+    f = Wd64.shape[0]
+    g = x64 @ Wgu64[:, :f]
+    u = x64 @ Wgu64[:, f:]
+    return (_silu(g) * u) @ Wd64
+
+
+# ------------------------------------------------------------- router order
+
+def _router_case(case):
+    d, E = case["d"], case["E"]
+    if case["x"] == "all 1.0":
+        x = np.ones((1, d), dtype=np.float32)
+    else:
+        x = np.asarray(case["x"], dtype=np.float32).reshape(1, d)
+    if isinstance(case["W"], str):
+        W = np.ones((d, E), dtype=np.float32)
+        W[0, 0] = 2.0 ** 24
+    else:
+        W = np.asarray(case["W"], dtype=np.float32).reshape(d, E)
+    b = None if case["bias"] is None else np.asarray([case["bias"]] * E, dtype=np.float32)
+    return x, W, b
+
+
+def test_router_order_golden():
+    data = json.load(open(os.path.join(GOLDEN, "router_order.json")))
+    for case in data["cases"]:
+        x, W, b = _router_case(case)
+        got = oracle.router_logits(_bf16(x), W, b)
+        assert got.shape == (1, case["E"])
+        assert float(got[0, 0]) == case["expected"], (case["name"], float(got[0, 0]))
+        for other in case["other_orders"].values():
+            assert other != case["expected"]
+
+
+def test_router_within_fp32_error_bound_of_exact_dot():
+    """|l - l_exact| <= gamma_n * sum|x_i W_ie| (+ u*|b|) with n = 128 + chunks + 1.
+
+    l_exact is the fp64 dot product from numpy; the bound is the textbook
+    forward error of a recursive fp32 sum of fma terms (Higham, Accuracy and
+    Stability of Numerical Algorithms, ch. 3).
+    """
+    rng = np.random.default_rng(7)
+    for (T, d, E, use_bias) in [(5, 384, 33, False), (3, 7168, 64, True), (4, 200, 9, True)]:
+        x = _bf16(rng.standard_normal((T, d)))
+        W = (rng.standard_normal((d, E)) * 0.02).astype(np.float32)
+        b = (rng.standard_normal(E) * 2).astype(np.float32) if use_bias else None
+        got = oracle.router_logits(x, W, b).astype(np.float64)
+        x64 = x.to(torch.float64).numpy()
+        exact = x64 @ W.astype(np.float64)
+        absd = np.abs(x64) @ np.abs(W.astype(np.float64))
+        n = 128 + math.ceil(d / 128) + 1
+        gamma = n * U32 / (1 - n * U32)
+        bound = gamma * absd
+        if b is not None:
+            exact = exact + b
+            bound = bound + gamma * np.abs(b) + U32 * np.abs(exact)
+        assert np.all(np.abs(got - exact) <= bound), np.max(np.abs(got - exact) / bound)
+        # and it is not the fp64 value rounded once (the order matters somewhere)
+        assert got.dtype == np.float64
+
+
+def test_router_rows_independent_and_bias_shift():
+    rng = np.random.default_rng(3)
+    x = _bf16(rng.standard_normal((6, 256)))
+    W = (rng.standard_normal((256, 10)) * 0.02).astype(np.float32)
+    full = oracle.router_logits(x, W)
+    for t in range(6):
+        assert np.array_equal(oracle.router_logits(x[t:t + 1], W)[0], full[t])
+    # a bias of exactly 0 changes nothing (x + 0 == x)
+    assert np.array_equal(oracle.router_logits(x, W, np.zeros(10, np.float32)), full)
+
+
+# ------------------------------------------------------------ softmax/top-k
+
+def test_topk_golden_closed_forms():
+    data = json.load(open(os.path.join(GOLDEN, "gate_topk.json")))
+    for case in data["cases"]:
+        if "logits" in case:
+            lg = np.asarray(case["logits"], dtype=np.float32)[None]
+        else:
+            lg = np.log(np.asarray(case["logits_ln_of"], dtype=np.float64)).astype(np.float32)[None]
+        idx, w = oracle.topk(lg, case["k"])
+        assert idx[0].tolist() == case["idx"], case["name"]
+        np.testing.assert_allclose(w[0], case["w"], rtol=1e-6, err_msg=case["name"])
+
+
+def test_topk_vs_brute_force_sort_and_library_softmax():
+    from scipy.special import softmax
+    rng = np.random.default_rng(11)
+    for (T, E, k) in [(50, 8, 2), (20, 384, 8), (10, 896, 16), (7, 5, 5)]:
+        lg = (rng.standard_normal((T, E)) * 1.7).astype(np.float32)
+        # plant exact ties
+        lg[:, E // 2] = lg[:, 0]
+        lg[0, :] = 0.25
+        idx, w, probs = oracle.topk(lg, k, want_probs=True)
+        ref_p = softmax(lg.astype(np.float64), axis=1)
+        np.testing.assert_allclose(probs, ref_p, rtol=1e-13, atol=0)
+        order = np.argsort(-lg.astype(np.float64), axis=1, kind="stable")[:, :k]
+        assert np.array_equal(idx, order)
+        np.testing.assert_allclose(w, np.take_along_axis(ref_p, order, 1), rtol=1e-13)
+        np.testing.assert_allclose(probs.sum(1), 1.0, atol=1e-12)
+        assert np.all(np.diff(w, axis=1) <= 0)
+        # weights are NOT renormalised: their sum is below 1 whenever k < E
+        if k < E:
+            assert np.all(w.sum(1) < 1.0)
+
+
+# ------------------------------------------------------------------ permute
+
+def test_permute_invariants_and_stable_sort():
+    rng = np.random.default_rng(5)
+    for (T, E, k) in [(64, 8, 2), (300, 37, 5), (1, 16, 16), (129, 896, 16)]:
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+        counts, offsets, perm_token, inv_perm = oracle.permute(idx, E)
+        assert counts.sum() == T * k
+        assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
+        assert offsets[0] == 0 and offsets[-1] == T * k
+        assert np.array_equal(np.diff(offsets), counts)
+        # library stable sort of the flattened (t, j) pairs by expert
+        order = np.argsort(idx.ravel(), kind="stable")
+        assert np.array_equal(perm_token, order // k)
+        inv_ref = np.empty(T * k, dtype=np.int64)
+        inv_ref[order] = np.arange(T * k)
+        assert np.array_equal(inv_perm.ravel(), inv_ref)
+        # bijection and inverse
+        assert np.array_equal(np.sort(inv_perm.ravel()), np.arange(T * k))
+        assert np.array_equal(perm_token[inv_perm], np.repeat(np.arange(T), k).reshape(T, k))
+        for e in range(E):
+            seg = perm_token[offsets[e]:offsets[e + 1]]
+            assert np.all(np.diff(seg) > 0)
+
+
+def test_permute_then_combine_of_x_is_weight_sum_times_x():
+    rng = np.random.default_rng(9)
+    T, d, E, k = 40, 64, 6, 3
+    x = _bf16(rng.standard_normal((T, d)))
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    w = rng.random((T, k))
+    counts, offsets, perm_token, inv_perm = oracle.permute(idx, E)
+    x64 = x.to(torch.float64).numpy()
+    x_perm = x64[perm_token]
+    out = oracle.combine(x_perm, inv_perm, w)
+    np.testing.assert_allclose(out, w.sum(1)[:, None] * x64, rtol=1e-14, atol=1e-300)
+
+
+# --------------------------------------------------------------- expert FFN
+
+def test_expert_ffn_vs_numpy_matmul():
+    rng = np.random.default_rng(13)
+    for (n, d, f) in [(1, 64, 64), (37, 128, 256), (5, 256, 96)]:
+        x = _bf16(rng.standard_normal((n, d)))
+        Wgu = _bf16(rng.standard_normal((d, 2 * f)) / math.sqrt(d))
+        Wd = _bf16(rng.standard_normal((f, d)) / math.sqrt(f))
+        y, h = oracle.expert_ffn(x, Wgu, Wd, want_h=True)
+        x64, Wg64, Wd64 = (_np_bf16_to_f64(t) for t in (x, Wgu, Wd))
+        g = x64 @ Wg64[:, :f]
+        u = x64 @ Wg64[:, f:]
+        np.testing.assert_allclose(h, _silu(g) * u, rtol=1e-11, atol=1e-13)
+        np.testing.assert_allclose(y, _dense_swiglu(x64, Wg64, Wd64), rtol=1e-10, atol=1e-12)
+
+
+def test_silu_closed_forms():
+    # SiLU(0) = 0, SiLU(a) - SiLU(-a) = a, SiLU(ln 3) = 0.75 ln 3
+    d, f = 4, 4
+    Wgu = np.zeros((d, 2 * f), dtype=np.float32)
+    Wd = np.eye(f, d, dtype=np.float32)
+    Wgu[0, :f] = [0.0, 1.0, -1.0, 2.0]   # gate columns
+    Wgu[1, f:] = 1.0                     # up columns = x[1]
+    x = np.array([[1.0, 1.0, 0.0, 0.0]], dtype=np.float32)
+    y = oracle.expert_ffn(_bf16(x), _bf16(Wgu), _bf16(Wd))
+    s = lambda a: a / (1 + math.exp(-a))
+    np.testing.assert_allclose(y[0], [0.0, s(1.0), s(-1.0), s(2.0)], rtol=1e-15)
+    assert abs((y[0, 1] - y[0, 2]) - 1.0) < 1e-15
+    # gate and up halves are not interchangeable: zero up half -> zero output
+    Wgu2 = Wgu.copy()
+    Wgu2[1, f:] = 0.0
+    assert np.all(oracle.expert_ffn(_bf16(x), _bf16(Wgu2), _bf16(Wd)) == 0.0)
+
+
+# ------------------------------------------------------------- whole layer
+
+def _tiny_layer(E=8, k=2, T=64, d=128, f=256, seed=0, bias=None):
+    shape = moe_inputs.custom_shape(T, d, E, k, f, bias=bias)
+    return moe_inputs.make_inputs(shape, seed=seed)
+
+
+def test_forward_E1_k1_is_dense_swiglu():
+    inp = _tiny_layer(E=1, k=1, T=33, d=128, f=64)
+    out, idx, w = oracle.forward(inp.x, inp.W_router, None, inp.W_gate_up, inp.W_down, 1)
+    assert np.all(idx == 0) and np.all(w == 1.0)
+    ref = _dense_swiglu(_np_bf16_to_f64(inp.x), _np_bf16_to_f64(inp.W_gate_up[0]), _np_bf16_to_f64(inp.W_down[0]))
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_forward_identical_experts_is_prob_sum_times_ffn():
+    inp = _tiny_layer(E=6, k=3, T=25, d=128, f=64)
+    Wgu = inp.W_gate_up[:1].expand(6, -1, -1).contiguous()
+    Wd = inp.W_down[:1].expand(6, -1, -1).contiguous()
+    out, idx, w = oracle.forward(inp.x, inp.W_router, None, Wgu, Wd, 3)
+    ffn = _dense_swiglu(_np_bf16_to_f64(inp.x), _np_bf16_to_f64(Wgu[0]), _np_bf16_to_f64(Wd[0]))
+    np.testing.assert_allclose(out, w.sum(1)[:, None] * ffn, rtol=1e-10, atol=1e-12)
+
+
+def test_forward_zero_token_and_hot_expert_and_duplicate_column():
+    inp = _tiny_layer(E=8, k=2, T=16, d=128, f=64)
+    x = inp.x.clone()
+    x[5] = 0
+    out, idx, w = oracle.forward(x, inp.W_router, None, inp.W_gate_up, inp.W_down, 2)
+    assert idx[5].tolist() == [0, 1]
+    np.testing.assert_allclose(w[5], [1 / 8, 1 / 8], rtol=1e-15)
+    assert np.all(out[5] == 0.0)
+    # +100 bias on expert 3: every token puts expert 3 in slot 0
+    b = np.zeros(8, np.float32)
+    b[3] = 100.0
+    _, idx, w = oracle.forward(inp.x, inp.W_router, b, inp.W_gate_up, inp.W_down, 2)
+    assert np.all(idx[:, 0] == 3)
+    counts, *_ = oracle.permute(idx, 8)
+    assert counts[3] == 16
+    # duplicated router column: equal logits, the lower index ranks first
+    Wr = inp.W_router.clone()
+    Wr[:, 6] = Wr[:, 1]
+    lg = oracle.router_logits(inp.x, Wr)
+    assert np.array_equal(lg[:, 6], lg[:, 1])
+    idx, _ = oracle.topk(lg, 3)
+    for row in idx.tolist():
+        if 6 in row:
+            assert 1 in row and row.index(1) < row.index(6)
+
+
+def test_tiny_workload_vs_numpy_cross_implementation():
+    """Whole tiny layer (T=64, d=128, E=8, k=2, f=256, seed 0) against an
+    independent numpy fp64 implementation with its own fp64 routing."""
+    inp = moe_inputs.make_inputs(moe_inputs.WORKLOADS["tiny"], seed=0)
+    k = 2
+    out, idx, w = oracle.forward(inp.x, inp.W_router, None, inp.W_gate_up, inp.W_down, k)
+    x64 = _np_bf16_to_f64(inp.x)
+    lg = x64 @ inp.W_router.numpy().astype(np.float64)
+    # the fp64 and fp32 routings agree wherever the k-th / (k+1)-th gap is
+    # larger than the fp32 error bound; check that holds for this draw
+    srt = np.sort(lg, axis=1)[:, ::-1]
+    gap = srt[:, k - 1] - srt[:, k]
+    assert np.all(gap > 1e-4)
+    order = np.argsort(-lg, axis=1, kind="stable")[:, :k]
+    assert np.array_equal(order, idx)
+    p = np.exp(lg - lg.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    wref = np.take_along_axis(p, order, 1)
+    np.testing.assert_allclose(w, wref, rtol=1e-5)
+    ref = np.zeros_like(x64)
+    for t in range(x64.shape[0]):
+        for j in range(k):
+            e = order[t, j]
+            ref[t] += wref[t, j] * _dense_swiglu(x64[t:t + 1], _np_bf16_to_f64(inp.W_gate_up[e]),
+                                                  _np_bf16_to_f64(inp.W_down[e]))[0]
+    np.testing.assert_allclose(out, ref, rtol=2e-5, atol=1e-7)
+
+
+def test_forward_token_subset_matches_full():
+    inp = moe_inputs.make_inputs(moe_inputs.WORKLOADS["tiny"], seed=0)
+    full, idx, w = oracle.forward(inp.x, inp.W_router, None, inp.W_gate_up, inp.W_down, 2)
+    sel = [0, 7, 63, 7]
+    sub, sidx, sw = oracle.forward(inp.x, inp.W_router, None, inp.W_gate_up, inp.W_down, 2, tokens=sel)
+    assert np.array_equal(sidx, idx[sel])
+    np.testing.assert_allclose(sub, full[sel], rtol=1e-13, atol=1e-15)
+
+
+def test_skewed_bias_recipe():
+    b = moe_inputs.zipf_bias(896).numpy()
+    assert b[0] == 0.0
+    np.testing.assert_allclose(b[9], -1.5 * math.log(10.0), rtol=1e-6)
+    assert np.all(np.diff(b) < 0)
+
+
+def test_oracle_rejects_bad_arguments():
+    with pytest.raises(ValueError):
+        oracle.topk(np.zeros((2, 4), np.float32), 5)
+    with pytest.raises(ValueError):
+        oracle.permute(np.array([[0, 9]], dtype=np.int32), 4)
+    with pytest.raises(FloatingPointError):
+        oracle.topk(np.array([[0.0, np.nan]], dtype=np.float32), 1)
