@@ -1,0 +1,394 @@
+"""Benchmark of the MoE layer forward pass (route -> dispatch -> SwiGLU experts ->
+combine) on B200, printing one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+A step is one moe_forward over one batch of T synthetic tokens with the
+workload's weights resident in HBM. Timing: W untimed warm-up steps, then K
+steps, each between CUDA events on the launching stream, with an L2 flush
+(a write larger than L2) between steps outside the events; barrier and
+synchronize on both sides; the max over ranks. Under torchrun every rank is an
+independent replica with its own tokens (weak scaling, no data-path
+collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_route_b200 import inputs as moe_inputs  # noqa: E402
+
+METRIC = "moe_layer_tokens_per_s"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+KERNELS_PER_STEP = 10  # router 2, dispatch 4, schedule 1, grouped GEMMs 2, combine 1
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- algorithmic
+
+def algorithmic(shape: moe_inputs.MoEShape, counts: np.ndarray):
+    """F_alg and B_alg of one layer pass, plus the dominant kernel's bytes.
+
+    F_alg = 2*T*d*E (router) + 6*T*k*d*f (experts)
+    B_alg = 4*d*E (W_router) + 2*T*d*2 (x in, out) + n_touched*6*d*f (expert
+            weights of experts with at least one row) + 4*E (bias, if any)
+    gate/up GEMM kernel (the dominant one): its compulsory bytes per launch =
+            n_touched*4*d*f (gate and up weights) + T*k*d*2 (rows in)
+            + T*k*f*2 (h out)
+    """
+    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    n_touched = int((counts > 0).sum())
+    F = 2.0 * T * d * E + 6.0 * T * k * d * f
+    B = 4.0 * d * E + 4.0 * T * d + n_touched * 6.0 * d * f + (4.0 * E if shape.bias else 0.0)
+    gu_bytes = n_touched * 4.0 * d * f + 2.0 * T * k * d + 2.0 * T * k * f
+    gu_flops = 4.0 * T * k * d * f
+    return {"F": F, "B": B, "n_touched": n_touched, "gu_bytes": gu_bytes, "gu_flops": gu_flops}
+
+
+def kernel_source_digest() -> str:
+    p = os.path.join(ROOT, "sparse_mixture_experts_route_b200", "csrc", "expert_gemm.cuh")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """dram read+write bytes per launch of the gate/up GEMM from a committed ncu
+    summary, only if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "gemm_gate_up_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except ValueError:
+        return None
+    ent = d.get(workload)
+    if not ent or ent.get("kernel_sha") != kernel_source_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ CPU baseline
+
+def cpu_baseline(inp, shape, budget_s: float = 20.0, seed: int = 1):
+    """The oracle, as it stands, on a bounded sample of the workload, on this
+    host's cores. Per-token cost = router+top-k+combine per token + k expert
+    rows; each part is timed on its own sample and scaled to tokens/s."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    n_route = min(T, 256)
+    toks = np.sort(rng.choice(T, size=n_route, replace=False))
+    xs = inp.x[torch.as_tensor(toks, device=inp.x.device)].cpu()
+    Wr = inp.W_router.cpu()
+    b = inp.bias.cpu() if inp.bias is not None else None
+    t0 = time.perf_counter()
+    lg = oracle.router_logits(xs, Wr, b)
+    idx, w = oracle.topk(lg, k)
+    t_route = (time.perf_counter() - t0) / n_route
+    # expert rows: rows of a few experts chosen by the sample, until the budget
+    rows_done, t_ffn = 0, 0.0
+    experts = list(dict.fromkeys(idx.ravel().tolist()))
+    deadline = time.perf_counter() + budget_s
+    for e in experts:
+        sel = np.argwhere(idx == e)[:, 0]
+        Wg = inp.W_gate_up[e].cpu()
+        Wd = inp.W_down[e].cpu()
+        t1 = time.perf_counter()
+        y = oracle.expert_ffn(xs[torch.as_tensor(sel)], Wg, Wd)
+        t_ffn += time.perf_counter() - t1
+        rows_done += len(sel)
+        if time.perf_counter() > deadline or rows_done >= n_route * k:
+            break
+    t_row = t_ffn / max(rows_done, 1)
+    yy = np.zeros((n_route * k, d))
+    t2 = time.perf_counter()
+    oracle.combine(yy, np.arange(n_route * k, dtype=np.int32).reshape(n_route, k), w)
+    t_comb = (time.perf_counter() - t2) / n_route
+    per_token = t_route + k * t_row + t_comb
+    return {"value": 1.0 / per_token, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"router+top-k+combine on {n_route} sampled tokens, SwiGLU on {rows_done} routed rows "
+                      f"of {shape.name}; tokens/s = 1/(t_route+k*t_row+t_combine)",
+            "seconds": t_route * n_route + t_ffn + t_comb * n_route}
+
+
+# ------------------------------------------------------------------ arms
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    from sparse_mixture_experts_route_b200 import _lib
+    world, rank, local = dist_setup()
+    shape = moe_inputs.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+
+    log(f"[rank {rank}] generating {shape.name} on {dev}")
+    inp = moe_inputs.make_inputs(shape, seed=0, device=dev)
+    if rank != 0:  # each replica routes its own tokens
+        inp.x = moe_inputs.make_x(shape, seed=1000 + rank, device=dev)
+    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    ws = torch.empty(_lib.moe_forward_workspace_size(T, d, E, k, f), dtype=torch.uint8, device=dev)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # routing statistics of this batch (for the algorithmic byte counts)
+    idx, _ = _lib.moe_route(inp.x, inp.W_router, inp.bias, k)
+    offs, _, _, _ = _lib.moe_permute(None, idx, E, with_rows=False)
+    counts = np.diff(offs.cpu().numpy())
+    alg = algorithmic(shape, counts)
+
+    nst = len(_lib.TIMED_STAGES)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        _lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+    assert _lib.get_device_error() == 0, "device error during warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + 2 * nst)] for _ in range(args.steps)]
+    for row in evs:
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.fill_(float(s))                     # L2 flush, outside the step's events
+        evs[s][0].record(stream)
+        _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[s][2:], out, ws)
+        evs[s][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
+    stage_ms = {name: [evs[s][2 + 2 * i].elapsed_time(evs[s][3 + 2 * i]) for s in range(args.steps)]
+                for i, name in enumerate(_lib.TIMED_STAGES)}
+    total_ms = max_over_ranks(sum(step_ms), world)
+    assert _lib.get_device_error() == 0, "device error during timing"
+
+    # end to end through the public call: x from pinned host memory, result back to the host
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        _lib.moe_forward(x_dev, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = []
+    for s in range(args.steps):
+        flush.fill_(float(s))
+        e0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        _lib.moe_forward(x_dev, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    barrier(world)
+    e2e_total = max_over_ranks(sum(e2e_ms), world)
+
+    if rank != 0:
+        return None
+    n = world
+    sec = total_ms / 1e3
+    value = n * T * args.steps / sec
+    ms_per_step = total_ms / args.steps
+    t_step = ms_per_step / 1e3
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    gu_ms = statistics.mean(stage_ms["gemm_gate_up"])
+    gu_achieved = alg["gu_bytes"] / (gu_ms / 1e3) / 1e9
+    traffic = profiled_traffic(shape.name)
+    layer_roof_s = max(alg["F"] / (tc * 1e12), alg["B"] / (hbm * 1e9))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {**shape.as_dict(), "seed": 0, "parallelism": f"replicas{n}",
+                   "l2": "flushed between steps (2x L2 write outside the step events)",
+                   "weights_gb": round(E * 6.0 * d * f / 1e9, 3)},
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
+                     "achieved": gu_achieved, "peak": hbm, "unit": "GB/s", "frac": gu_achieved / hbm,
+                     "traffic": traffic, "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+                     "alg_bytes_per_launch": alg["gu_bytes"], "ms_per_launch": gu_ms},
+        "layer": {"tflops": alg["F"] / t_step / 1e12, "hbm_gbs": alg["B"] / t_step / 1e9,
+                  "F_alg": alg["F"], "B_alg": alg["B"], "n_touched": alg["n_touched"],
+                  "roofline_frac": layer_roof_s / t_step,
+                  "binding_roof": "hbm" if alg["B"] / hbm / 1e9 >= alg["F"] / tc / 1e12 else "tensor",
+                  "tensor_frac_of_peak": alg["F"] / t_step / 1e12 / tc,
+                  "stage_ms": {kname: statistics.mean(v) for kname, v in stage_ms.items()}},
+        "e2e": {"value": n * T * args.steps / (e2e_total / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        log("[rank 0] timing the CPU oracle on a bounded sample")
+        line["cpu_baseline"] = cpu_baseline(inp, shape, budget_s=args.cpu_budget)
+    return line
+
+
+def run_reference(args):
+    """The oracle on the host cores, each step a bounded sample of the workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    shape = moe_inputs.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = moe_inputs.make_inputs(shape, seed=0, device=dev)
+    budget = max(2.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(inp, shape, budget_s=budget)
+    vals = [cpu_baseline(inp, shape, budget_s=budget) for _ in range(args.steps)]
+    tps = [v["value"] for v in vals]
+    value = statistics.mean(tps)
+    cb = dict(vals[-1])
+    cb["value"] = value
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * shape.T / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**shape.as_dict(), "seed": 0, "parallelism": "host cores"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=sorted(moe_inputs.WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and args.impl == "ours":
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of one sparse
+ * Mixture-of-Experts layer:
+ *
+ *   router logits -> softmax over all experts -> top-k -> dispatch (permute)
+ *   -> per-expert SwiGLU feed-forward -> gate-weighted combine (unpermute).
+ *
+ * Passages (page title, then section):
+ *   [P2] "Kimi K3: The Open Model That Just Cornered the AI Frontier",
+ *        section "Mixture-of-Experts with Dynamic Load Balancing", gating code:
+ *        logits from one gate projection, softmax over the expert axis, top-k
+ *        of the probabilities, values and indices returned as they are.
+ *   [P3] "Kimi K3: Open Frontier Intelligence", section "Operational Execution
+ *        Flow": tokens are dispatched to their active routed experts and the
+ *        routed output is the probability-weighted sum of the selected experts'
+ *        outputs; the experts use a GLU feed-forward whose SwiGLU regime the
+ *        page names.
+ *   Model-card shapes: 384 experts top-8 ("Kimi K3: What Open-Source Frontier
+ *   Models Reveal About RL Scaling for Reasoning", section "The Architecture:
+ *   MoE, Latent Attention, and Massive Context"), 256 top-4 ([P2]), 896
+ *   top-16 and d_model 7168 ([P3]).
+ *
+ * Conventions for every entry point
+ *   - Every pointer is a DEVICE pointer owned by the caller, unless stated.
+ *     The library never allocates, frees or synchronises; every call only
+ *     enqueues kernels on `stream` and returns.
+ *   - All tensors are dense, row-major, with no padding between rows.
+ *     bf16 tensors are passed as `const moe_bf16_t*` (the 16-bit patterns).
+ *     x, W_gate_up, W_down, x_perm, h, y_perm and out must be 16-byte aligned.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns a status other than MOE_OK and launches nothing.
+ *   - MOE_ERR_CUDA means a launch failed (cudaGetLastError after the launches).
+ *   - Kernels that wait on hardware barriers wait for a bounded time; if a
+ *     wait runs out they record a code in a per-device error word and return
+ *     early (outputs are then undefined). moe_get_device_error() reads it.
+ *   - Sizes: T >= 1 tokens, d model width, E experts, 1 <= k <= min(E, 16)
+ *     selected experts per token, f expert hidden width. d and f must be
+ *     multiples of 64; E <= 1024; T * k < 2^31; d, f <= 32768.
+ */
+#ifndef MOE_B200_MOE_H_
+#define MOE_B200_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h> /* cudaStream_t */
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t; /* bfloat16 bit pattern */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, size out of range, misalignment */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but beyond this build's limits (k > 16, E > 1024, ...) */
+  MOE_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE = 5       /* a kernel recorded an error (see moe_get_device_error) */
+} moe_status_t;
+
+/* Human-readable name of a status. Never NULL. */
+const char* moe_status_string(moe_status_t status);
+
+/* Maximum k and E supported by the register top-k. */
+#define MOE_MAX_TOPK 16
+#define MOE_MAX_EXPERTS 1024
+
+/* ---------------------------------------------------------------- router --
+ * moe_route: steps 1-3 of the pass ([P2] gating code).
+ *   logits[t, e] = sum_i x[t, i] * W_router[i, e]  (+ router_bias[e])
+ *     computed in fp32 (x widened exactly from bf16) in a fixed order: fma
+ *     inside consecutive chunks of 128 input indices, chunk partials added in
+ *     ascending chunk order, bias added last. The order makes the routing
+ *     reproducible bit for bit.
+ *   probs[t, :] = softmax(logits[t, :]) over all E experts (fp32).
+ *   topk_idx[t, 0..k-1]: the experts with the k largest logits, descending;
+ *     equal logits go to the lower expert index.
+ *   topk_w[t, j] = probs[t, topk_idx[t, j]], NOT renormalised.
+ * Inputs:  x [T, d] bf16; W_router [d, E] fp32; router_bias [E] fp32 or NULL.
+ * Outputs: topk_idx [T, k] int32; topk_w [T, k] fp32.
+ * Scratch: workspace of at least moe_route_workspace_size(T, d, E) bytes,
+ *   256-byte aligned (holds fp32 logits or per-chunk partial sums).
+ */
+size_t moe_route_workspace_size(int T, int d, int E);
+moe_status_t moe_route(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                       int T, int d, int E, int k,
+                       int32_t* topk_idx, float* topk_w,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------- permute --
+ * moe_permute: step 4, dispatch ([P3] tokens are dispatched to their routed
+ * experts). A stable counting sort of the T*k (token, slot) pairs by expert:
+ *   expert_offsets[e] = number of pairs routed to experts < e  ([E+1] int32,
+ *     expert_offsets[E] = T*k);
+ *   rows expert_offsets[e] .. expert_offsets[e+1]-1 hold the tokens routed to
+ *     expert e in ascending token order: perm_token[row] = token ([T*k] int32);
+ *   inv_perm[t*k + j] = row of the pair (t, j)  ([T, k] int32);
+ *   x_perm[row, :] = x[perm_token[row], :]  ([T*k, d] bf16; may be NULL to
+ *     skip the row copy).
+ * Inputs: x [T, d] bf16 (may be NULL when x_perm is NULL); topk_idx [T, k].
+ * Scratch: moe_permute_workspace_size(T, E, k) bytes, 256-byte aligned.
+ */
+size_t moe_permute_workspace_size(int T, int E, int k);
+moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx,
+                         int T, int d, int E, int k,
+                         int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm,
+                         moe_bf16_t* x_perm,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------ expert FFN --
+ * moe_expert_ffn: step 5, every expert's SwiGLU feed-forward on its rows.
+ * For expert e and each row r in expert_offsets[e] .. expert_offsets[e+1]-1:
+ *   g = x_perm[r, :] @ W_gate_up[e][:, 0:f]      (gate half)
+ *   u = x_perm[r, :] @ W_gate_up[e][:, f:2f]     (up half)
+ *   h[r, :] = SiLU(g) * u, SiLU(a) = a / (1 + exp(-a))   -> bf16 [Tk, f]
+ *   y_perm[r, :] = h[r, :] @ W_down[e]                    -> bf16 [Tk, d]
+ * bf16 operands on the tcgen05 tensor cores, fp32 accumulation, fp32
+ * epilogue, round-to-nearest-even to bf16.
+ * Inputs: x_perm [Tk, d] bf16; expert_offsets [E+1] int32 (device; read on the
+ *   device, no host sync); W_gate_up [E, d, 2f] bf16; W_down [E, f, d] bf16.
+ * Outputs: h [Tk, f] bf16 (also the operand of the second GEMM); y_perm [Tk, d].
+ * Scratch: moe_expert_ffn_workspace_size(Tk, E) bytes, 256-byte aligned.
+ */
+size_t moe_expert_ffn_workspace_size(int Tk, int E);
+moe_status_t moe_expert_ffn(const moe_bf16_t* x_perm, const int32_t* expert_offsets,
+                            const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down,
+                            int Tk, int d, int E, int f,
+                            moe_bf16_t* h, moe_bf16_t* y_perm,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------- unpermute --
+ * moe_unpermute: step 6, the gate-weighted combine ([P3] the routed output is
+ * the probability-weighted sum of the selected experts' outputs):
+ *   out[t, :] = sum_{j=0..k-1} topk_w[t, j] * y_perm[inv_perm[t*k + j], :]
+ * accumulated in fp32 in ascending j, stored bf16 [T, d].
+ * Needs no scratch.
+ */
+moe_status_t moe_unpermute(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w,
+                           int T, int d, int k, moe_bf16_t* out, cudaStream_t stream);
+
+/* --------------------------------------------------------------- forward --
+ * moe_forward: the whole pass (route, permute, expert FFN, unpermute) on one
+ * stream, with no host synchronisation. All intermediates are carved from
+ * `workspace` (at least moe_forward_workspace_size(T, d, E, k, f) bytes,
+ * 256-byte aligned). out [T, d] bf16.
+ */
+size_t moe_forward_workspace_size(int T, int d, int E, int k, int f);
+moe_status_t moe_forward(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                         const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down,
+                         int T, int d, int E, int k, int f,
+                         moe_bf16_t* out,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* moe_forward_timed: moe_forward that also records CUDA events around its
+ * kernel groups on `stream`, for live per-kernel timing. `events` holds
+ * 2 * MOE_TIMED_STAGES caller-created events (cudaEventCreate); stage i is
+ * bracketed by events[2*i] and events[2*i+1]:
+ *   0 router (logits + softmax/top-k)   1 dispatch (histogram, scan, scatter,
+ *   row copy, GEMM tile schedule)       2 gate/up grouped GEMM (one kernel)
+ *   3 down grouped GEMM (one kernel)    4 combine (one kernel)
+ * Same arguments, results and errors as moe_forward otherwise; events == NULL
+ * is MOE_ERR_INVALID_ARG.
+ */
+#define MOE_TIMED_STAGES 5
+moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                               const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down,
+                               int T, int d, int E, int k, int f,
+                               moe_bf16_t* out,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                               cudaEvent_t* events);
+
+/* ------------------------------------------------------------ diagnostics --
+ * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
+ * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise
+ * one of MOE_DEVERR_*. This call synchronises the device (it is a debug aid,
+ * not part of the hot path). Returns MOE_ERR_CUDA if the read fails,
+ * MOE_ERR_DEVICE if *code != 0, MOE_OK otherwise.
+ */
+#define MOE_DEVERR_NONE 0u
+#define MOE_DEVERR_WAIT_TIMEOUT_PRODUCER 1u /* TMA producer gave up waiting for a free stage */
+#define MOE_DEVERR_WAIT_TIMEOUT_MMA 2u      /* MMA issuer gave up waiting for operands/accumulator */
+#define MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE 3u /* epilogue gave up waiting for an accumulator */
+#define MOE_DEVERR_SELFTEST_TIMEOUT 4u      /* moe_selftest_wait_timeout fired as intended */
+#define MOE_DEVERR_BAD_ROUTE 5u             /* an expert index outside [0, E) reached the dispatch */
+moe_status_t moe_get_device_error(uint32_t* code, int clear);
+
+/* moe_selftest_wait_timeout: launches one tiny kernel that waits, with a
+ * limit of `timeout_us` microseconds (1..1000000), on a shared-memory barrier
+ * that nothing ever signals, then records MOE_DEVERR_SELFTEST_TIMEOUT and
+ * returns. It checks that bounded waits end and report an error instead of
+ * hanging; it faults nothing. Asynchronous on `stream`.
+ */
+moe_status_t moe_selftest_wait_timeout(int timeout_us, cudaStream_t stream);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H_ */

@@ -1,0 +1,235 @@
+"""ctypes binding of ``libmoe.so`` (the C ABI in include/moe.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, their ``data_ptr()`` and torch's current CUDA stream are passed to
+the C entry point of the same name, and a non-OK status raises ``MoEError``.
+Every step of the layer runs in the library's kernels. Importing this module
+loads the library and raises if it is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run python -m sparse_mixture_experts_route_b200.build")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+Z = ctypes.c_size_t
+
+EXPORTS = {
+    "moe_status_string": ([I], ctypes.c_char_p),
+    "moe_version": ([], I),
+    "moe_route_workspace_size": ([I, I, I], Z),
+    "moe_route": ([P, P, P, I, I, I, I, P, P, P, Z, P], I),
+    "moe_permute_workspace_size": ([I, I, I], Z),
+    "moe_permute": ([P, P, I, I, I, I, P, P, P, P, P, Z, P], I),
+    "moe_expert_ffn_workspace_size": ([I, I], Z),
+    "moe_expert_ffn": ([P, P, P, P, I, I, I, I, P, P, P, Z, P], I),
+    "moe_unpermute": ([P, P, P, I, I, I, P, P], I),
+    "moe_forward_workspace_size": ([I, I, I, I, I], Z),
+    "moe_forward": ([P, P, P, P, P, I, I, I, I, I, P, P, Z, P], I),
+    "moe_get_device_error": ([ctypes.POINTER(ctypes.c_uint32), I], I),
+    "moe_selftest_wait_timeout": ([I, P], I),
+}
+for _name, (_args, _res) in EXPORTS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
+DEVERR_SELFTEST_TIMEOUT = 4
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = _lib.moe_status_string(status).decode()
+        super().__init__(f"{where}: {name}")
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoEError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def version() -> int:
+    return int(_lib.moe_version())
+
+
+def route_workspace_size(T: int, d: int, E: int) -> int:
+    return int(_lib.moe_route_workspace_size(T, d, E))
+
+
+def permute_workspace_size(T: int, E: int, k: int) -> int:
+    return int(_lib.moe_permute_workspace_size(T, E, k))
+
+
+def expert_ffn_workspace_size(Tk: int, E: int) -> int:
+    return int(_lib.moe_expert_ffn_workspace_size(Tk, E))
+
+
+def moe_forward_workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
+    return int(_lib.moe_forward_workspace_size(T, d, E, k, f))
+
+
+def moe_route(x, W_router, router_bias, k: int, workspace=None, stream=None):
+    """Steps 1-3. Returns (topk_idx [T,k] int32, topk_w [T,k] fp32)."""
+    T, d = x.shape
+    E = W_router.shape[1]
+    _need(x, "x", torch.bfloat16, (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    ws = workspace if workspace is not None else _workspace(route_workspace_size(T, d, E), x.device)
+    _check(_lib.moe_route(_ptr(x), _ptr(W_router), _ptr(router_bias), T, d, E, k, _ptr(idx), _ptr(w),
+                          _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
+    return idx, w
+
+
+def moe_permute(x, topk_idx, E: int, with_rows: bool = True, workspace=None, stream=None):
+    """Step 4. Returns (offsets [E+1], perm_token [T*k], inv_perm [T,k], x_perm [T*k,d] or None)."""
+    T, k = topk_idx.shape
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    d = x.shape[1] if x is not None else 64
+    if x is not None:
+        _need(x, "x", torch.bfloat16, (T, d))
+    dev = topk_idx.device
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv_perm = torch.empty(T, k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device=dev) if (with_rows and x is not None) else None
+    ws = workspace if workspace is not None else _workspace(permute_workspace_size(T, E, k), dev)
+    _check(_lib.moe_permute(_ptr(x), _ptr(topk_idx), T, d, E, k, _ptr(offsets), _ptr(perm_token), _ptr(inv_perm),
+                            _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+    return offsets, perm_token, inv_perm, x_perm
+
+
+def moe_expert_ffn(x_perm, expert_offsets, W_gate_up, W_down, workspace=None, stream=None):
+    """Step 5. Returns (h [Tk,f] bf16, y_perm [Tk,d] bf16)."""
+    Tk, d = x_perm.shape
+    E, d2, f2 = W_gate_up.shape
+    f = f2 // 2
+    _need(x_perm, "x_perm", torch.bfloat16, (Tk, d))
+    _need(expert_offsets, "expert_offsets", torch.int32, (E + 1,))
+    _need(W_gate_up, "W_gate_up", torch.bfloat16, (E, d, 2 * f))
+    _need(W_down, "W_down", torch.bfloat16, (E, f, d))
+    h = torch.empty(Tk, f, dtype=torch.bfloat16, device=x_perm.device)
+    y = torch.empty(Tk, d, dtype=torch.bfloat16, device=x_perm.device)
+    ws = workspace if workspace is not None else _workspace(expert_ffn_workspace_size(Tk, E), x_perm.device)
+    _check(_lib.moe_expert_ffn(_ptr(x_perm), _ptr(expert_offsets), _ptr(W_gate_up), _ptr(W_down), Tk, d, E, f,
+                               _ptr(h), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn")
+    return h, y
+
+
+def moe_unpermute(y_perm, inv_perm, topk_w, stream=None, out=None):
+    """Step 6. Returns out [T,d] bf16."""
+    T, k = inv_perm.shape
+    d = y_perm.shape[1]
+    _need(y_perm, "y_perm", torch.bfloat16, (T * k, d))
+    _need(inv_perm, "inv_perm", torch.int32, (T, k))
+    _need(topk_w, "topk_w", torch.float32, (T, k))
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=y_perm.device)
+    _need(out, "out", torch.bfloat16, (T, d))
+    _check(_lib.moe_unpermute(_ptr(y_perm), _ptr(inv_perm), _ptr(topk_w), T, d, k, _ptr(out), _stream(stream)),
+           "moe_unpermute")
+    return out
+
+
+def moe_forward(x, W_router, router_bias, W_gate_up, W_down, k: int, out=None, workspace=None, stream=None):
+    """The whole layer. Returns out [T,d] bf16."""
+    T, d = x.shape
+    E = W_router.shape[1]
+    f = W_down.shape[1]
+    _need(x, "x", torch.bfloat16, (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    _need(W_gate_up, "W_gate_up", torch.bfloat16, (E, d, 2 * f))
+    _need(W_down, "W_down", torch.bfloat16, (E, f, d))
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", torch.bfloat16, (T, d))
+    ws = workspace if workspace is not None else _workspace(moe_forward_workspace_size(T, d, E, k, f), x.device)
+    _check(_lib.moe_forward(_ptr(x), _ptr(W_router), _ptr(router_bias), _ptr(W_gate_up), _ptr(W_down),
+                            T, d, E, k, f, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_forward")
+    return out
+
+
+def get_device_error(clear: bool = True) -> int:
+    """Read (and clear) the current device's error word; synchronises the device."""
+    code = ctypes.c_uint32(0)
+    st = _lib.moe_get_device_error(ctypes.byref(code), 1 if clear else 0)
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoEError(st, "moe_get_device_error")
+    return int(code.value)
+
+
+def selftest_wait_timeout(timeout_us: int, stream=None):
+    _check(_lib.moe_selftest_wait_timeout(int(timeout_us), _stream(stream)), "moe_selftest_wait_timeout")
+
+
+# raw C entry points, for callers that hold device pointers themselves
+raw = _lib
+
+_lib.moe_forward_timed.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P, P]
+_lib.moe_forward_timed.restype = I
+TIMED_STAGES = ("router", "dispatch", "gemm_gate_up", "gemm_down", "combine")
+
+
+def moe_forward_timed(x, W_router, router_bias, W_gate_up, W_down, k: int, events, out, workspace, stream=None):
+    """moe_forward that records ``events`` (2 * len(TIMED_STAGES) torch.cuda.Event
+    with enable_timing=True) around its kernel groups on the launching stream."""
+    T, d = x.shape
+    E = W_router.shape[1]
+    f = W_down.shape[1]
+    assert len(events) == 2 * len(TIMED_STAGES)
+    for ev in events:
+        if ev.cuda_event == 0:  # torch creates the CUDA event on its first record
+            ev.record(torch.cuda.current_stream() if stream is None else stream)
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(ev.cuda_event) for ev in events])
+    _check(_lib.moe_forward_timed(_ptr(x), _ptr(W_router), _ptr(router_bias), _ptr(W_gate_up), _ptr(W_down),
+                                  T, d, E, k, f, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream), arr),
+           "moe_forward_timed")
+    return out

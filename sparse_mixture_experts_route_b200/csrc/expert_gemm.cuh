@@ -1,0 +1,369 @@
+// Grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM, fed by TMA).
+//
+// Computes every expert's SwiGLU feed-forward on its dispatched rows (the
+// routed experts E_i of "Kimi K3: Open Frontier Intelligence", section
+// "Operational Execution Flow"; the page names SwiGLU as the regime its GLU
+// keeps). Two launches of one kernel template:
+//   mode 0 (gate/up):  H[r, j] = SiLU(X[r] . Wgu[e][:, j]) * (X[r] . Wgu[e][:, f + j])
+//   mode 1 (down):     Y[r, c] = H[r] . Wd[e][:, c]
+// for every row r of expert e (rows offsets[e] .. offsets[e+1]-1).
+//
+// Orientation ("swap AB"): the weights are the UMMA A operand (M = 128 output
+// features per tile) and the tokens are the B operand (N = up to 128 rows of
+// one expert), so an expert with 1..128 rows still issues full-height MMAs and
+// each weight byte is read once per token block. D = W^T X^T lands in TMEM with
+// one feature per lane and one token per column.
+//   A: weight tile [64 K rows x 128 features], N-contiguous in memory
+//      -> MN-major operand, two 64-feature boxes, 128-byte swizzle.
+//   B: token rows [128 rows x 64 K], K-contiguous -> K-major, 128-byte swizzle.
+// For mode 0 each tile carries two accumulators side by side in TMEM (gate
+// features j0..j0+127 and the matching up features), so one thread holds g and
+// u for the same (feature, token) and the SiLU-gate is fused in the epilogue.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer (one lane): smem ring of kStages stages;
+//   warp 1      TMEM allocator and MMA issuer (one lane);
+//   warps 2..5  epilogue: tcgen05.ld -> fp32 math -> bf16 stores.
+// Tiles are (expert, feature block, token block), enumerated from the device
+// copy of the expert offsets, so there is no host synchronisation; consecutive
+// tiles share a weight tile when an expert has several token blocks.
+// Every barrier wait is bounded; on a timeout the kernel records an error code,
+// drains what it issued and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kGemmBK = 64;     // K per stage: one 128-byte swizzle row of bf16
+constexpr int kGemmBMF = 128;   // output features per tile (UMMA M)
+constexpr int kGemmBNT = 128;   // token rows per tile (largest UMMA N used)
+constexpr int kGemmThreads = 192;
+
+template <int kMode>
+struct GemmCfg {
+  static constexpr int kNumA = (kMode == 0) ? 2 : 1;          // A operands per stage (gate, up)
+  static constexpr int kABytes = kGemmBK * kGemmBMF * 2;       // 16 KB per A operand
+  static constexpr int kAHalf = kABytes / 2;                   // one 64-feature box (8 KB)
+  static constexpr int kBBytes = kGemmBNT * kGemmBK * 2;       // 16 KB
+  static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
+  static constexpr int kStages = (kMode == 0) ? 4 : 6;
+  static constexpr int kAccCols = kNumA * kGemmBNT;            // TMEM columns per accumulator
+  static constexpr int kTmemCols = 2 * kAccCols;               // double buffered (512 / 256)
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+  static_assert(kTmemCols <= 512, "TMEM has 512 columns");
+};
+
+struct GemmParams {
+  const int32_t* expert_offsets;  // [E + 1] rows per expert (device)
+  const int32_t* tile_prefix;     // [E + 1] token blocks before expert e (device)
+  int E;
+  int K;            // reduction length (d for mode 0, f for mode 1)
+  int n_feat;       // output features (f for mode 0, d for mode 1)
+  int n_feat_tiles; // ceil(n_feat / 128)
+  int up_offset;    // column of the first up feature in W_gate_up (f); unused in mode 1
+  uint16_t* out;    // [Tk, n_feat] bf16
+};
+
+struct TileInfo {
+  int e, nb, row0, nrows;
+};
+
+__device__ __forceinline__ bool decode_tile(const GemmParams& p, int tile, TileInfo& ti) {
+  const int NB = p.n_feat_tiles;
+  const int blocks_total = __ldg(p.tile_prefix + p.E);
+  if (tile >= blocks_total * NB) return false;
+  // owner: the largest e with tile_prefix[e] * NB <= tile
+  int lo = 0, hi = p.E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.tile_prefix + mid) * NB <= tile)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int e = lo;
+  const int tb_count = __ldg(p.tile_prefix + e + 1) - __ldg(p.tile_prefix + e);
+  const int local = tile - __ldg(p.tile_prefix + e) * NB;
+  const int tb = local % tb_count;
+  ti.e = e;
+  ti.nb = local / tb_count;
+  ti.row0 = __ldg(p.expert_offsets + e) + tb * kGemmBNT;
+  ti.nrows = min(kGemmBNT, __ldg(p.expert_offsets + e + 1) - ti.row0);
+  return true;
+}
+
+__device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)); }
+
+template <int kMode>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmParams p) {
+  using Cfg = GemmCfg<kMode>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
+  uint64_t* empty_bar = full_bar + S;
+  uint64_t* acc_full_bar = empty_bar + S;   // [2]
+  uint64_t* acc_empty_bar = acc_full_bar + 2;  // [2]
+  uint64_t* drain_bar = acc_empty_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int KB = p.K / kGemmBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full_bar[b], 1);
+      mbar_init(&acc_empty_bar[b], 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();  // weights: streamed once
+      const uint64_t pol_x = l2_policy_evict_last();   // activations: re-read per feature block
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      TileInfo ti;
+      for (int tile = blockIdx.x; ok && decode_tile(p, tile, ti); tile += gridDim.x) {
+        const int feat0 = ti.nb * kGemmBMF;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
+            record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * Cfg::kStageBytes;
+          mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
+          const int k0 = kb * kGemmBK;
+          tma_load_3d(st, &tmA, &full_bar[s], feat0, k0, ti.e, pol_w);
+          tma_load_3d(st + Cfg::kAHalf, &tmA, &full_bar[s], feat0 + 64, k0, ti.e, pol_w);
+          if (kMode == 0) {
+            tma_load_3d(st + Cfg::kABytes, &tmA, &full_bar[s], p.up_offset + feat0, k0, ti.e, pol_w);
+            tma_load_3d(st + Cfg::kABytes + Cfg::kAHalf, &tmA, &full_bar[s], p.up_offset + feat0 + 64, k0, ti.e,
+                        pol_w);
+          }
+          tma_load_2d(st + Cfg::kNumA * Cfg::kABytes, &tmB, &full_bar[s], k0, ti.row0, pol_x);
+          ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: wait (bounded) for the loads still in flight into the ring
+        for (int i = 0; i < S && i < issued; ++i) {
+          s = (s == 0) ? S - 1 : s - 1;
+          if (s == S - 1) ph ^= 1u;
+          mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      bool any = false;
+      TileInfo ti;
+      for (int tile = blockIdx.x; ok && decode_tile(p, tile, ti); tile += gridDim.x) {
+        const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
+        const uint32_t idesc = umma_idesc_bf16_f32(128u, n_mma, 1u, 0u);
+        if (!mbar_wait_bounded(&acc_empty_bar[acc], acc_ph ^ 1u, kWaitLimitNs, abort_flag)) {
+          record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * Cfg::kAccCols);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
+            record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(smem + s * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + Cfg::kNumA * Cfg::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+            const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            const uint64_t adesc = umma_smem_desc_sw128(a_addr + kk * 2048, Cfg::kAHalf, 1024);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, accum);
+            if (kMode == 0) {
+              const uint64_t adesc_u = umma_smem_desc_sw128(a_addr + Cfg::kABytes + kk * 2048, Cfg::kAHalf, 1024);
+              tc_mma_bf16(d_tmem + kGemmBNT, adesc_u, bdesc, idesc, accum);
+            }
+          }
+          tc_commit(&empty_bar[s]);  // stage s is free once these MMAs have read it
+          any = true;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full_bar[acc]);  // accumulator complete
+        if (++acc == 2) {
+          acc = 0;
+          acc_ph ^= 1u;
+        }
+      }
+      if (any) {
+        // make sure no MMA is still running before TMEM is released
+        tc_commit(drain_bar);
+        mbar_wait_bounded(drain_bar, 0u, kWaitLimitNs, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    TileInfo ti;
+    for (int tile = blockIdx.x; decode_tile(p, tile, ti); tile += gridDim.x) {
+      if (!mbar_wait_bounded(&acc_full_bar[acc], acc_ph, kWaitLimitNs, abort_flag)) {
+        record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after_sync();
+      const int feat = ti.nb * kGemmBMF + q * 32 + lane;
+      const bool feat_ok = feat < p.n_feat;
+      const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * Cfg::kAccCols);
+      for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+        uint32_t g[32];
+        tmem_ld_32x32b_x32(taddr + c0, g);
+        if (kMode == 0) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(taddr + kGemmBNT + c0, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (feat_ok && c0 + i < ti.nrows) {
+              const float h = silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+              const __nv_bfloat16 hb = __float2bfloat16_rn(h);
+              p.out[static_cast<int64_t>(ti.row0 + c0 + i) * p.n_feat + feat] =
+                  *reinterpret_cast<const uint16_t*>(&hb);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (feat_ok && c0 + i < ti.nrows) {
+              const __nv_bfloat16 yb = __float2bfloat16_rn(__uint_as_float(g[i]));
+              p.out[static_cast<int64_t>(ti.row0 + c0 + i) * p.n_feat + feat] =
+                  *reinterpret_cast<const uint16_t*>(&yb);
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty_bar[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_ph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// Token blocks per expert: tile_prefix[e] = sum_{e' < e} ceil(count_e' / 128).
+__global__ void __launch_bounds__(1024)
+    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ tile_prefix) {
+  __shared__ int32_t warp_sums[32];
+  const int e = threadIdx.x;
+  const int32_t cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
+  const int32_t nb = (cnt + kGemmBNT - 1) / kGemmBNT;
+  const int lane = e & 31, w = e >> 5;
+  int32_t incl = nb;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int32_t ws = warp_sums[lane];
+    int32_t wincl = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, wincl, o);
+      if (lane >= o) wincl += y;
+    }
+    warp_sums[lane] = wincl - ws;
+  }
+  __syncthreads();
+  const int32_t excl = warp_sums[w] + incl - nb;
+  if (e < E) {
+    tile_prefix[e] = excl;
+    if (e == E - 1) tile_prefix[E] = excl + nb;
+  }
+}
+
+// A wait that nothing will ever satisfy, bounded by `limit_ns`: checks that
+// bounded waits end and report instead of hanging.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!mbar_wait_bounded(&bar, 0u, limit_ns, nullptr)) record_device_error(4u /* MOE_DEVERR_SELFTEST_TIMEOUT */);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,465 @@
+// C ABI of the MoE layer forward pass (declarations and contracts in
+// include/moe.h). Host code only validates arguments, carves workspaces,
+// encodes TMA descriptors and enqueues kernels; every step of the pass runs in
+// the kernels included below. No call allocates, frees or synchronises
+// (except moe_get_device_error, a documented debug read).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "moe.h"
+
+#include "common.cuh"
+#include "expert_gemm.cuh"
+#include "permute.cuh"
+#include "ptx.cuh"
+#include "router.cuh"
+
+namespace {
+
+using namespace moe;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device one-time set-up: SM count and the dynamic shared-memory limits of
+// the GEMM kernels. Returns MOE_ERR_CUDA if the device cannot be queried.
+moe_status_t device_setup(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& di = g_devices[dev];
+  if (!di.ready) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<0>::kSmemBytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<1>::kSmemBytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return MOE_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    di.num_sms = sms;
+    di.ready = true;
+  }
+  *num_sms = di.num_sms;
+  return MOE_OK;
+}
+
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// ------------------------------------------------------------------ router
+
+enum RouterVariant { kRouterFullBig = 0, kRouterSplitBig = 1, kRouterSplitSmall = 2 };
+
+struct RoutePlan {
+  RouterVariant variant;
+  int nchunks;
+  size_t ws_bytes;
+};
+
+RoutePlan route_plan(int T, int d, int E) {
+  RoutePlan p;
+  p.nchunks = ceil_div(d, kRouterChunk);
+  const int64_t big_tiles = ceil_div64(T, 128) * ceil_div64(E, 64);
+  if (p.nchunks > 1 && T <= 32)
+    p.variant = kRouterSplitSmall;
+  else if (p.nchunks > 1 && big_tiles < 296)
+    p.variant = kRouterSplitBig;
+  else
+    p.variant = kRouterFullBig;
+  const int64_t planes = (p.variant == kRouterFullBig) ? 1 : p.nchunks;
+  p.ws_bytes = align256(static_cast<size_t>(planes) * T * E * sizeof(float));
+  return p;
+}
+
+bool shape_ok(int T, int d, int E, int k) {
+  return T >= 1 && d >= 64 && d % 64 == 0 && d <= 32768 && E >= 1 && k >= 1 && k <= E &&
+         static_cast<int64_t>(T) * k < (int64_t(1) << 31);
+}
+
+moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const float* bias, int T, int d, int E, int k,
+                          int32_t* idx, float* w, void* ws, cudaStream_t stream) {
+  const RoutePlan plan = route_plan(T, d, E);
+  float* lg = static_cast<float*>(ws);
+  switch (plan.variant) {
+    case kRouterFullBig: {
+      dim3 grid(ceil_div(E, 64), ceil_div(T, 128), 1);
+      router_logits_kernel<128, 64, 8, 4, false><<<grid, 256, 0, stream>>>(x, W_router, bias, T, d, E, lg);
+      break;
+    }
+    case kRouterSplitBig: {
+      dim3 grid(ceil_div(E, 64), ceil_div(T, 128), plan.nchunks);
+      router_logits_kernel<128, 64, 8, 4, true><<<grid, 256, 0, stream>>>(x, W_router, nullptr, T, d, E, lg);
+      break;
+    }
+    case kRouterSplitSmall: {
+      dim3 grid(ceil_div(E, 64), ceil_div(T, 32), plan.nchunks);
+      router_logits_kernel<32, 64, 2, 4, true><<<grid, 256, 0, stream>>>(x, W_router, nullptr, T, d, E, lg);
+      break;
+    }
+  }
+  const int nsplit = (plan.variant == kRouterFullBig) ? 1 : plan.nchunks;
+  const int blocks = ceil_div(T, 8);
+  if (E <= 256)
+    router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, nsplit, bias, T, E, k, idx, w);
+  else
+    router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, nsplit, bias, T, E, k, idx, w);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- permute
+
+size_t permute_ws(int T, int E, int k) {
+  const int64_t nblk = ceil_div64(static_cast<int64_t>(T) * k, kPairsPerBlock);
+  return align256(static_cast<size_t>(nblk) * E * sizeof(int32_t));
+}
+
+moe_status_t launch_permute(const moe_bf16_t* x, const int32_t* idx, int T, int d, int E, int k, int32_t* offsets,
+                            int32_t* perm_token, int32_t* inv_perm, moe_bf16_t* x_perm, void* ws,
+                            cudaStream_t stream) {
+  const int64_t n_pairs = static_cast<int64_t>(T) * k;
+  const int nblk = static_cast<int>(ceil_div64(n_pairs, kPairsPerBlock));
+  int32_t* block_hist = static_cast<int32_t*>(ws);
+  const size_t sm = static_cast<size_t>(E) * sizeof(int32_t);
+  permute_hist_kernel<<<nblk, 256, sm, stream>>>(idx, n_pairs, E, block_hist);
+  permute_scan_kernel<<<1, 1024, 0, stream>>>(block_hist, nblk, E, offsets);
+  permute_scatter_kernel<<<nblk, 32, sm, stream>>>(idx, n_pairs, E, k, block_hist, perm_token, inv_perm);
+  if (x_perm != nullptr) {
+    const int rows_per_block = 8;
+    const int64_t blocks = ceil_div64(n_pairs, rows_per_block);
+    permute_copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(x), perm_token, n_pairs, d / 8, reinterpret_cast<uint4*>(x_perm));
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// -------------------------------------------------------------- expert FFN
+
+size_t ffn_ws(int E) { return align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
+
+bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+                const cuuint32_t* box) {
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                              const_cast<void*>(base), dims, strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Weights W[E][K][N] (N contiguous): boxes of 64 features x 64 K rows of one expert.
+bool weight_map(CUtensorMap* map, const moe_bf16_t* W, int E, int K, int N) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(N) * 2, static_cast<cuuint64_t>(N) * K * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  return encode_map(map, W, 3, dims, strides, box);
+}
+
+// Activations A[rows][K] (K contiguous): boxes of 64 K x 128 rows.
+bool act_map(CUtensorMap* map, const moe_bf16_t* A, int rows, int K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kGemmBNT)};
+  return encode_map(map, A, 2, dims, strides, box);
+}
+
+struct FfnPlan {
+  CUtensorMap mA0, mB0, mA1, mB1;
+  GemmParams p0, p1;
+  int grid0, grid1;
+};
+
+moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
+                      int Tk, int d, int E, int f, moe_bf16_t* h, moe_bf16_t* y_perm, void* ws, int num_sms,
+                      FfnPlan* fp) {
+  if (!weight_map(&fp->mA0, Wgu, E, d, 2 * f) || !act_map(&fp->mB0, x_perm, Tk, d) ||
+      !weight_map(&fp->mA1, Wd, E, f, d) || !act_map(&fp->mB1, h, Tk, f))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t blocks_ub = ceil_div64(Tk, kGemmBNT) + (E < Tk ? E : Tk);
+  GemmParams& p0 = fp->p0;
+  p0.expert_offsets = offsets;
+  p0.tile_prefix = static_cast<int32_t*>(ws);
+  p0.E = E;
+  p0.K = d;
+  p0.n_feat = f;
+  p0.n_feat_tiles = ceil_div(f, kGemmBMF);
+  p0.up_offset = f;
+  p0.out = h;
+  const int64_t tiles0 = blocks_ub * p0.n_feat_tiles;
+  fp->grid0 = static_cast<int>(tiles0 < num_sms ? tiles0 : num_sms);
+  GemmParams& p1 = fp->p1;
+  p1 = p0;
+  p1.K = f;
+  p1.n_feat = d;
+  p1.n_feat_tiles = ceil_div(d, kGemmBMF);
+  p1.up_offset = 0;
+  p1.out = y_perm;
+  const int64_t tiles1 = blocks_ub * p1.n_feat_tiles;
+  fp->grid1 = static_cast<int>(tiles1 < num_sms ? tiles1 : num_sms);
+  return MOE_OK;
+}
+
+void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
+  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, const_cast<int32_t*>(fp.p0.tile_prefix));
+}
+void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
+  grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.p0);
+}
+void launch_gemm_down(const FfnPlan& fp, cudaStream_t stream) {
+  grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.p1);
+}
+
+moe_status_t launch_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
+                        int Tk, int d, int E, int f, moe_bf16_t* h, moe_bf16_t* y_perm, void* ws, int num_sms,
+                        cudaStream_t stream) {
+  FfnPlan fp;
+  const moe_status_t st = plan_ffn(x_perm, offsets, Wgu, Wd, Tk, d, E, f, h, y_perm, ws, num_sms, &fp);
+  if (st != MOE_OK) return st;
+  launch_schedule(fp, stream);
+  launch_gemm_gate_up(fp, stream);
+  launch_gemm_down(fp, stream);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- unpermute
+
+moe_status_t launch_unpermute(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* w, int T, int d, int k,
+                              moe_bf16_t* out, cudaStream_t stream) {
+  unpermute_kernel<<<T, 128, 0, stream>>>(reinterpret_cast<const uint4*>(y_perm), inv_perm, w, k, d / 8,
+                                          reinterpret_cast<uint4*>(out));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- forward
+
+struct ForwardLayout {
+  size_t route, idx, w, offsets, perm_token, inv_perm, x_perm, h, y_perm, perm_ws, ffn_ws, total;
+};
+
+ForwardLayout forward_layout(int T, int d, int E, int k, int f) {
+  ForwardLayout L;
+  const size_t Tk = static_cast<size_t>(T) * k;
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t here = at;
+    at += align256(bytes);
+    return here;
+  };
+  L.route = take(route_plan(T, d, E).ws_bytes);
+  L.idx = take(Tk * sizeof(int32_t));
+  L.w = take(Tk * sizeof(float));
+  L.offsets = take((static_cast<size_t>(E) + 1) * sizeof(int32_t));
+  L.perm_token = take(Tk * sizeof(int32_t));
+  L.inv_perm = take(Tk * sizeof(int32_t));
+  L.x_perm = take(Tk * d * 2);
+  L.h = take(Tk * f * 2);
+  L.y_perm = take(Tk * d * 2);
+  L.perm_ws = take(permute_ws(T, E, k));
+  L.ffn_ws = take(ffn_ws(E));
+  L.total = at;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int moe_version(void) { return 100; }
+
+size_t moe_route_workspace_size(int T, int d, int E) {
+  if (T < 1 || d < 1 || E < 1) return 0;
+  return route_plan(T, d, E).ws_bytes;
+}
+
+moe_status_t moe_route(const moe_bf16_t* x, const float* W_router, const float* router_bias, int T, int d, int E,
+                       int k, int32_t* topk_idx, float* topk_w, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  if (!x || !W_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, d, E, k) || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!workspace || !aligned256(workspace) || workspace_bytes < route_plan(T, d, E).ws_bytes) return MOE_ERR_WORKSPACE;
+  return launch_route(x, W_router, router_bias, T, d, E, k, topk_idx, topk_w, workspace, stream);
+}
+
+size_t moe_permute_workspace_size(int T, int E, int k) {
+  if (T < 1 || E < 1 || k < 1) return 0;
+  return permute_ws(T, E, k);
+}
+
+moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                         int32_t* expert_offsets, int32_t* perm_token, int32_t* inv_perm, moe_bf16_t* x_perm,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!topk_idx || !expert_offsets || !perm_token || !inv_perm) return MOE_ERR_INVALID_ARG;
+  if (x_perm != nullptr && (x == nullptr || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, d, E, k)) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!workspace || !aligned256(workspace) || workspace_bytes < permute_ws(T, E, k)) return MOE_ERR_WORKSPACE;
+  return launch_permute(x, topk_idx, T, d, E, k, expert_offsets, perm_token, inv_perm, x_perm, workspace, stream);
+}
+
+size_t moe_expert_ffn_workspace_size(int Tk, int E) {
+  if (Tk < 0 || E < 1) return 0;
+  return ffn_ws(E);
+}
+
+moe_status_t moe_expert_ffn(const moe_bf16_t* x_perm, const int32_t* expert_offsets, const moe_bf16_t* W_gate_up,
+                            const moe_bf16_t* W_down, int Tk, int d, int E, int f, moe_bf16_t* h, moe_bf16_t* y_perm,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!x_perm || !expert_offsets || !W_gate_up || !W_down || !h || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (Tk < 1 || d < 64 || d % 64 || f < 64 || f % 64 || d > 32768 || f > 32768 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(W_gate_up) || !aligned16(W_down) || !aligned16(h) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!workspace || !aligned256(workspace) || workspace_bytes < ffn_ws(E)) return MOE_ERR_WORKSPACE;
+  int sms = 0;
+  const moe_status_t st = device_setup(&sms);
+  if (st != MOE_OK) return st;
+  return launch_ffn(x_perm, expert_offsets, W_gate_up, W_down, Tk, d, E, f, h, y_perm, workspace, sms, stream);
+}
+
+moe_status_t moe_unpermute(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w, int T, int d, int k,
+                           moe_bf16_t* out, cudaStream_t stream) {
+  if (!y_perm || !inv_perm || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || d < 64 || d % 64 || d > 32768 || k < 1 || !aligned16(y_perm) || !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  return launch_unpermute(y_perm, inv_perm, topk_w, T, d, k, out, stream);
+}
+
+size_t moe_forward_workspace_size(int T, int d, int E, int k, int f) {
+  if (T < 1 || d < 1 || E < 1 || k < 1 || f < 1) return 0;
+  return forward_layout(T, d, E, k, f).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                          const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, int T, int d, int E, int k, int f,
+                          moe_bf16_t* out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                          cudaEvent_t* ev) {
+  if (!x || !W_router || !W_gate_up || !W_down || !out) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, d, E, k) || f < 64 || f % 64 || f > 32768) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W_gate_up) || !aligned16(W_down) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  const ForwardLayout L = forward_layout(T, d, E, k, f);
+  if (!workspace || !aligned256(workspace) || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  int sms = 0;
+  moe_status_t st = device_setup(&sms);
+  if (st != MOE_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_token = reinterpret_cast<int32_t*>(ws + L.perm_token);
+  int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  moe_bf16_t* x_perm = reinterpret_cast<moe_bf16_t*>(ws + L.x_perm);
+  moe_bf16_t* h = reinterpret_cast<moe_bf16_t*>(ws + L.h);
+  moe_bf16_t* y_perm = reinterpret_cast<moe_bf16_t*>(ws + L.y_perm);
+  const int Tk = T * k;
+  FfnPlan fp;
+  st = plan_ffn(x_perm, offsets, W_gate_up, W_down, Tk, d, E, f, h, y_perm, ws + L.ffn_ws, sms, &fp);
+  if (st != MOE_OK) return st;
+  auto mark = [&](int i) {
+    if (ev) cudaEventRecord(ev[i], stream);
+  };
+  mark(0);
+  st = launch_route(x, W_router, router_bias, T, d, E, k, idx, w, ws + L.route, stream);
+  if (st != MOE_OK) return st;
+  mark(1);
+  mark(2);
+  st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, x_perm, ws + L.perm_ws, stream);
+  if (st != MOE_OK) return st;
+  launch_schedule(fp, stream);
+  mark(3);
+  mark(4);
+  launch_gemm_gate_up(fp, stream);
+  mark(5);
+  mark(6);
+  launch_gemm_down(fp, stream);
+  mark(7);
+  mark(8);
+  st = launch_unpermute(y_perm, inv_perm, w, T, d, k, out, stream);
+  mark(9);
+  if (st != MOE_OK) return st;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_forward(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                         const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, int T, int d, int E, int k, int f,
+                         moe_bf16_t* out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return forward_impl(x, W_router, router_bias, W_gate_up, W_down, T, d, E, k, f, out, workspace, workspace_bytes,
+                      stream, nullptr);
+}
+
+moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                               const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, int T, int d, int E, int k,
+                               int f, moe_bf16_t* out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                               cudaEvent_t* events) {
+  if (!events) return MOE_ERR_INVALID_ARG;
+  return forward_impl(x, W_router, router_bias, W_gate_up, W_down, T, d, E, k, f, out, workspace, workspace_bytes,
+                      stream, events);
+}
+
+moe_status_t moe_get_device_error(uint32_t* code, int clear) {
+  if (!code) return MOE_ERR_INVALID_ARG;
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, moe::g_device_error, sizeof(v)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (clear && v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(moe::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  *code = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+moe_status_t moe_selftest_wait_timeout(int timeout_us, cudaStream_t stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return MOE_ERR_INVALID_ARG;
+  moe::selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"

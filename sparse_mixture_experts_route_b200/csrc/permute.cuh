@@ -1,0 +1,174 @@
+// Dispatch (permute) and combine (unpermute).
+//
+// Dispatch follows "Kimi K3: Open Frontier Intelligence", section
+// "Operational Execution Flow": each token is sent to its active routed
+// experts. Layout built here: a stable counting sort of the T*k (token, slot)
+// pairs by expert, so expert e owns rows offsets[e] .. offsets[e+1]-1 in
+// ascending token order. Three passes, no atomics that decide an order:
+//   hist    per block of kPairsPerBlock consecutive pairs: a per-expert count;
+//   scan    per expert: total, exclusive scan over experts (offsets), and each
+//           block's first row for each expert;
+//   scatter per block, one warp walking its pairs in order 32 at a time; the
+//           rank among equal experts inside a group of 32 comes from
+//           __match_any_sync, so the result is the sequential counting sort.
+// The combine (same page and section: the routed output is the
+// probability-weighted sum of the selected experts' outputs) accumulates the k
+// rows of a token in fp32 in ascending slot order.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPairsPerBlock = 512;
+
+__global__ void __launch_bounds__(256)
+    permute_hist_kernel(const int32_t* __restrict__ topk_idx, int64_t n_pairs, int E, int32_t* __restrict__ block_hist) {
+  extern __shared__ int32_t cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int64_t q0 = static_cast<int64_t>(blockIdx.x) * kPairsPerBlock;
+  const int64_t q1 = min(n_pairs, q0 + kPairsPerBlock);
+  for (int64_t q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
+    const int e = topk_idx[q];
+    if (e >= 0 && e < E)
+      atomicAdd(&cnt[e], 1);
+    else
+      record_device_error(5u /* MOE_DEVERR_BAD_ROUTE */);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) block_hist[static_cast<int64_t>(blockIdx.x) * E + e] = cnt[e];
+}
+
+// One block of 1024 threads; thread e owns expert e (E <= 1024).
+// In: block_hist[nblk][E] counts. Out: offsets[0..E]; block_hist rewritten in
+// place with each block's first row per expert.
+__global__ void __launch_bounds__(1024)
+    permute_scan_kernel(int32_t* __restrict__ block_hist, int nblk, int E, int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_sums[32];
+  const int e = threadIdx.x;
+  int32_t total = 0;
+  if (e < E)
+    for (int b = 0; b < nblk; ++b) total += block_hist[static_cast<int64_t>(b) * E + e];
+  // exclusive scan of `total` over the block
+  const int lane = e & 31, w = e >> 5;
+  int32_t incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int32_t ws = warp_sums[lane];
+    int32_t wincl = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, wincl, o);
+      if (lane >= o) wincl += y;
+    }
+    warp_sums[lane] = wincl - ws;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int32_t excl = warp_sums[w] + incl - total;
+  if (e < E) {
+    offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + total;
+    int32_t run = excl;
+    for (int b = 0; b < nblk; ++b) {
+      const int64_t at = static_cast<int64_t>(b) * E + e;
+      const int32_t c = block_hist[at];
+      block_hist[at] = run;
+      run += c;
+    }
+  }
+}
+
+// One warp per block of kPairsPerBlock pairs.
+__global__ void __launch_bounds__(32)
+    permute_scatter_kernel(const int32_t* __restrict__ topk_idx, int64_t n_pairs, int E, int k,
+                           const int32_t* __restrict__ block_base, int32_t* __restrict__ perm_token,
+                           int32_t* __restrict__ inv_perm) {
+  extern __shared__ int32_t base[];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) base[e] = block_base[static_cast<int64_t>(blockIdx.x) * E + e];
+  __syncwarp();
+  const int64_t q0 = static_cast<int64_t>(blockIdx.x) * kPairsPerBlock;
+  const int64_t q1 = min(n_pairs, q0 + kPairsPerBlock);
+  for (int64_t g = q0; g < q1; g += 32) {
+    const int64_t q = g + lane;
+    const bool valid = q < q1;
+    int e = valid ? topk_idx[q] : -1;
+    if (valid && (e < 0 || e >= E)) e = -2;  // reported by the hist pass; never written
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int32_t row = 0;
+    if (e >= 0) row = base[e] + rank;
+    __syncwarp();
+    if (e >= 0 && rank == 0) base[e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      perm_token[row] = static_cast<int32_t>(q / k);
+      inv_perm[q] = row;
+    }
+  }
+}
+
+// x_perm[row, :] = x[perm_token[row], :], 16-byte vectors, one warp per row.
+__global__ void __launch_bounds__(256)
+    permute_copy_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_token, int64_t n_rows,
+                             int vec_per_row, uint4* __restrict__ x_perm) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= n_rows) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t src = static_cast<int64_t>(perm_token[row]) * vec_per_row;
+  const int64_t dst = row * vec_per_row;
+  for (int v = lane; v < vec_per_row; v += 32) x_perm[dst + v] = __ldg(x + src + v);
+}
+
+// out[t, :] = sum_j w[t, j] * y_perm[inv_perm[t, j], :]; fp32, ascending j.
+// One block per token, 8 bf16 per thread per step.
+__global__ void __launch_bounds__(128)
+    unpermute_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ inv_perm,
+                     const float* __restrict__ topk_w, int k, int vec_per_row, uint4* __restrict__ out) {
+  const int64_t t = blockIdx.x;
+  int32_t rows[16];
+  float ws[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < k) {
+      rows[j] = inv_perm[t * k + j];
+      ws[j] = topk_w[t * k + j];
+    }
+  }
+  for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < k) {
+        const uint4 y = __ldg(y_perm + static_cast<int64_t>(rows[j]) * vec_per_row + v);
+        const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] = __fmaf_rn(ws[j], __uint_as_float(yw[q] << 16), acc[2 * q]);
+          acc[2 * q + 1] = __fmaf_rn(ws[j], __uint_as_float(yw[q] & 0xFFFF0000u), acc[2 * q + 1]);
+        }
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+      o[q] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    out[t * vec_per_row + v] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace moe

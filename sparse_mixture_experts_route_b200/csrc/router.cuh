@@ -1,0 +1,236 @@
+// Router: logits, softmax over all experts, top-k.
+//
+// Follows the gating code on "Kimi K3: The Open Model That Just Cornered the
+// AI Frontier" (section "Mixture-of-Experts with Dynamic Load Balancing"): one
+// gate projection from d_model to n_experts, softmax over the expert axis,
+// top-k of the probabilities, values returned without renormalisation.
+//
+// Numerics (the pages fix none): fp32 with x widened exactly from bf16.
+// Summation order, fixed so routing is reproducible bit for bit:
+//   p_c = fma chain over the 128 consecutive input indices of chunk c (from +0),
+//   l   = ((p_0 + p_1) + p_2) + ... + p_{C-1},   then l = l + b_e.
+// Selection compares these fp32 logits (softmax is monotone, so the chosen set
+// equals top-k of the probabilities); equal logits go to the lower index.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kRouterChunk = 128;  // input indices per ordered partial sum
+constexpr int kRouterBK = 32;      // input indices staged in shared memory per step
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Logits of a [BM tokens x BN experts] tile.
+//   SPLIT = false: the CTA walks every chunk in order and writes final logits
+//                  (+ bias) to out[t * E + e].
+//   SPLIT = true : the CTA handles chunk blockIdx.z only and writes its partial
+//                  p_c to out[(c * T + t) * E + e]; router_topk_kernel adds the
+//                  partials in ascending c. Both modes give identical bits.
+// Requires d % 32 == 0. Threads: (BM / TM) * (BN / TN).
+template <int BM, int BN, int TM, int TN, bool SPLIT>
+__global__ void __launch_bounds__((BM / TM) * (BN / TN))
+    router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
+                         const float* __restrict__ bias, int T, int d, int E, float* __restrict__ out) {
+  constexpr int NT = (BM / TM) * (BN / TN);
+  constexpr int TX = BN / TN;
+  static_assert(TM % 2 == 0 && TN == 4, "micro-tile layout");
+  __shared__ __align__(16) float xs[2][kRouterBK][BM];
+  __shared__ __align__(16) float ws[2][kRouterBK][BN];
+
+  const int tid = threadIdx.x;
+  const int tx = tid % TX, ty = tid / TX;
+  const int e0 = blockIdx.x * BN, t0 = blockIdx.y * BM;
+  const int nchunks = (d + kRouterChunk - 1) / kRouterChunk;
+  const int c_begin = SPLIT ? blockIdx.z : 0;
+  const int c_end = SPLIT ? blockIdx.z + 1 : nchunks;
+  const int k_begin = c_begin * kRouterChunk;
+  const int k_end = min(d, c_end * kRouterChunk);
+  const int nsteps = (k_end - k_begin) / kRouterBK;
+
+  // staging registers for the next step
+  constexpr int XV = (BM * kRouterBK / 8 + NT - 1) / NT;  // uint4 (8 bf16) loads of x per thread
+  constexpr int WV = (BN * kRouterBK + NT - 1) / NT;      // scalar loads of W per thread
+  uint4 xr[XV];
+  float wr[WV];
+
+  auto load_step = [&](int k0) {
+#pragma unroll
+    for (int v = 0; v < XV; ++v) {
+      const int m = tid + v * NT;  // m in [0, BM*BK/8)
+      const int r = m / (kRouterBK / 8), cg = m % (kRouterBK / 8);
+      const int t = t0 + r;
+      if (m < BM * kRouterBK / 8 && t < T)
+        xr[v] = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d + k0 + cg * 8);
+      else
+        xr[v] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int v = 0; v < WV; ++v) {
+      const int m = tid + v * NT;
+      const int kk = m / BN, col = m % BN;
+      const int e = e0 + col;
+      wr[v] = (m < BN * kRouterBK && e < E) ? __ldg(W + static_cast<int64_t>(k0 + kk) * E + e) : 0.0f;
+    }
+  };
+  auto store_step = [&](int buf) {
+#pragma unroll
+    for (int v = 0; v < XV; ++v) {
+      const int m = tid + v * NT;
+      if (m < BM * kRouterBK / 8) {
+        const int r = m / (kRouterBK / 8), cg = m % (kRouterBK / 8);
+        const uint32_t w4[4] = {xr[v].x, xr[v].y, xr[v].z, xr[v].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          xs[buf][cg * 8 + 2 * q][r] = __uint_as_float(w4[q] << 16);
+          xs[buf][cg * 8 + 2 * q + 1][r] = __uint_as_float(w4[q] & 0xFFFF0000u);
+        }
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < WV; ++v) {
+      const int m = tid + v * NT;
+      if (m < BN * kRouterBK) ws[buf][m / BN][m % BN] = wr[v];
+    }
+  };
+
+  float acc[TM][TN], lsum[TM][TN];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f, lsum[i][j] = 0.0f;
+
+  if (nsteps > 0) {
+    load_step(k_begin);
+    store_step(0);
+  }
+  __syncthreads();
+  for (int s = 0; s < nsteps; ++s) {
+    const int buf = s & 1;
+    const int k0 = k_begin + s * kRouterBK;
+    if (s + 1 < nsteps) load_step(k0 + kRouterBK);
+#pragma unroll
+    for (int kk = 0; kk < kRouterBK; ++kk) {
+      float a[TM], b[TN];
+#pragma unroll
+      for (int i = 0; i < TM; i += 2) {
+        const float2 v = *reinterpret_cast<const float2*>(&xs[buf][kk][ty * TM + i]);
+        a[i] = v.x;
+        a[i + 1] = v.y;
+      }
+      const float4 bv = *reinterpret_cast<const float4*>(&ws[buf][kk][tx * TN]);
+      b[0] = bv.x, b[1] = bv.y, b[2] = bv.z, b[3] = bv.w;
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = __fmaf_rn(a[i], b[j], acc[i][j]);
+    }
+    // end of a 128-index chunk (or of the input): fold the chunk partial in order
+    const int k_next = k0 + kRouterBK;
+    if (!SPLIT && (k_next % kRouterChunk == 0 || k_next == k_end)) {
+      const bool first = (k_next <= kRouterChunk);
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) {
+          lsum[i][j] = first ? acc[i][j] : __fadd_rn(lsum[i][j], acc[i][j]);
+          acc[i][j] = 0.0f;
+        }
+    }
+    if (s + 1 < nsteps) store_step(buf ^ 1);
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int t = t0 + ty * TM + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < TN; ++j) {
+      const int e = e0 + tx * TN + j;
+      if (e >= E) continue;
+      if (SPLIT) {
+        out[(static_cast<int64_t>(blockIdx.z) * T + t) * E + e] = acc[i][j];
+      } else {
+        float l = lsum[i][j];
+        if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e));
+        out[static_cast<int64_t>(t) * E + e] = l;
+      }
+    }
+  }
+}
+
+// One warp per token: (optionally) add the per-chunk partials in ascending
+// chunk order and the bias, softmax over all E experts in fp32, then k rounds
+// of warp arg-max (ties -> lower index). MAXV >= ceil(E / 32).
+template <int MAXV>
+__global__ void __launch_bounds__(256)
+    router_topk_kernel(const float* __restrict__ lg, int nsplit, const float* __restrict__ bias, int T, int E,
+                       int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const int t = warp;
+  float v[MAXV];
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int e = i * 32 + lane;
+    float l = -INFINITY;
+    if (e < E) {
+      if (nsplit == 1) {
+        l = lg[static_cast<int64_t>(t) * E + e];
+      } else {
+        l = lg[static_cast<int64_t>(t) * E + e];
+        for (int c = 1; c < nsplit; ++c) l = __fadd_rn(l, lg[(static_cast<int64_t>(c) * T + t) * E + e]);
+        if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e));
+      }
+      m = fmaxf(m, l);
+    }
+    v[i] = l;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i)
+    if (i * 32 + lane < E) s += expf(v[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+
+  uint32_t taken = 0u;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == 0) {
+      topk_idx[static_cast<int64_t>(t) * k + j] = bi;
+      topk_w[static_cast<int64_t>(t) * k + j] = expf(bv - m) / s;
+    }
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,137 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point that
+include/moe.h declares, sizes its workspaces consistently, and rejects bad
+arguments on the host with the documented status before launching anything.
+No test here launches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_mixture_experts_route_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_unpermute", "moe_forward",
+                     "moe_forward_workspace_size", "moe_status_string", "moe_get_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from sparse_mixture_experts_route_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (moe_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_library_is_sm100a_only_and_static_runtime(lib):
+    from sparse_mixture_experts_route_b200 import build
+    deps = subprocess.run(["ldd", build.LIB], capture_output=True, text=True).stdout
+    assert "libcudart" not in deps  # runtime linked statically
+    assert "libtorch" not in deps
+    fl = build.flags()
+    assert "arch=compute_100a,code=sm_100a" in fl
+
+
+def _setup(lib):
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_status_string.argtypes = [I]
+    for n in ("moe_route_workspace_size", "moe_permute_workspace_size", "moe_expert_ffn_workspace_size",
+              "moe_forward_workspace_size"):
+        getattr(lib, n).restype = Z
+    lib.moe_route_workspace_size.argtypes = [I, I, I]
+    lib.moe_permute_workspace_size.argtypes = [I, I, I]
+    lib.moe_expert_ffn_workspace_size.argtypes = [I, I]
+    lib.moe_forward_workspace_size.argtypes = [I, I, I, I, I]
+    lib.moe_route.argtypes = [P, P, P, I, I, I, I, P, P, P, Z, P]
+    lib.moe_permute.argtypes = [P, P, I, I, I, I, P, P, P, P, P, Z, P]
+    lib.moe_expert_ffn.argtypes = [P, P, P, P, I, I, I, I, P, P, P, Z, P]
+    lib.moe_unpermute.argtypes = [P, P, P, I, I, I, P, P]
+    lib.moe_forward.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P]
+    lib.moe_selftest_wait_timeout.argtypes = [I, P]
+    return lib
+
+
+def test_status_strings(lib):
+    lib = _setup(lib)
+    names = [lib.moe_status_string(i).decode() for i in range(6)]
+    assert names == ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_WORKSPACE", "MOE_ERR_CUDA",
+                     "MOE_ERR_DEVICE"]
+    assert lib.moe_status_string(99).decode() == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    lib = _setup(lib)
+    for (T, d, E, k, f) in [(64, 128, 8, 2, 256), (4096, 7168, 384, 8, 2048), (128, 7168, 256, 4, 2048),
+                            (8192, 7168, 896, 16, 512), (1, 7168, 896, 16, 512)]:
+        fw = lib.moe_forward_workspace_size(T, d, E, k, f)
+        rw = lib.moe_route_workspace_size(T, d, E)
+        pw = lib.moe_permute_workspace_size(T, E, k)
+        ew = lib.moe_expert_ffn_workspace_size(T * k, E)
+        Tk = T * k
+        inter = Tk * 4 * 4 + (E + 1) * 4 + Tk * d * 2 * 2 + Tk * f * 2
+        assert fw >= rw + pw + ew + inter
+        assert fw % 256 == 0 and rw % 256 == 0 and pw % 256 == 0 and ew % 256 == 0
+        assert rw >= T * E * 4
+        assert fw < rw + pw + ew + inter + 12 * 256
+    assert lib.moe_forward_workspace_size(0, 128, 8, 2, 256) == 0
+
+
+FAKE = 0x10000  # a 256-byte aligned non-null address; never dereferenced on these paths
+
+
+def test_route_argument_checks(lib):
+    lib = _setup(lib)
+    p = ctypes.c_void_p(FAKE)
+    ws = lib.moe_route_workspace_size(64, 128, 8)
+    assert lib.moe_route(None, p, None, 64, 128, 8, 2, p, p, p, ws, None) == 1
+    assert lib.moe_route(p, p, None, 0, 128, 8, 2, p, p, p, ws, None) == 1          # T = 0
+    assert lib.moe_route(p, p, None, 64, 100, 8, 2, p, p, p, ws, None) == 1         # d % 64
+    assert lib.moe_route(p, p, None, 64, 128, 8, 9, p, p, p, ws, None) == 1         # k > E
+    assert lib.moe_route(p, p, None, 64, 128, 32, 17, p, p, p, 1 << 30, None) == 2  # k > 16
+    assert lib.moe_route(p, p, None, 64, 128, 2048, 2, p, p, p, 1 << 30, None) == 2  # E > 1024
+    assert lib.moe_route(p, p, None, 64, 128, 8, 2, p, p, p, ws - 1, None) == 3     # workspace too small
+    assert lib.moe_route(p, p, None, 64, 128, 8, 2, p, p, None, ws, None) == 3      # no workspace
+    assert lib.moe_route(p, p, None, 64, 128, 8, 2, p, p, ctypes.c_void_p(FAKE + 16), ws, None) == 3
+    assert lib.moe_route(ctypes.c_void_p(FAKE + 2), p, None, 64, 128, 8, 2, p, p, p, ws, None) == 1  # x align
+
+
+def test_other_argument_checks(lib):
+    lib = _setup(lib)
+    p = ctypes.c_void_p(FAKE)
+    pw = lib.moe_permute_workspace_size(64, 8, 2)
+    assert lib.moe_permute(p, None, 64, 128, 8, 2, p, p, p, p, p, pw, None) == 1
+    assert lib.moe_permute(None, p, 64, 128, 8, 2, p, p, p, p, p, pw, None) == 1      # rows need x
+    assert lib.moe_permute(p, p, 64, 128, 8, 2, p, p, p, p, p, pw - 256, None) == 3
+    ew = lib.moe_expert_ffn_workspace_size(128, 8)
+    assert lib.moe_expert_ffn(p, p, p, p, 128, 128, 8, 100, p, p, p, ew, None) == 1    # f % 64
+    assert lib.moe_expert_ffn(p, p, p, p, 128, 128, 2000, 256, p, p, p, 1 << 20, None) == 2
+    assert lib.moe_expert_ffn(p, p, p, p, 128, 128, 8, 256, p, p, p, 0, None) == 3
+    assert lib.moe_unpermute(p, p, p, 64, 128, 17, p, None) == 2
+    assert lib.moe_unpermute(p, p, p, 64, 120, 2, p, None) == 1
+    fw = lib.moe_forward_workspace_size(64, 128, 8, 2, 256)
+    assert lib.moe_forward(p, p, None, p, p, 64, 128, 8, 2, 256, None, p, fw, None) == 1
+    assert lib.moe_forward(p, p, None, p, p, 64, 128, 8, 2, 250, p, p, fw, None) == 1
+    assert lib.moe_forward(p, p, None, p, p, 64, 128, 8, 2, 256, p, p, fw - 256, None) == 3
+    assert lib.moe_selftest_wait_timeout(0, None) == 1
+    assert lib.moe_selftest_wait_timeout(2_000_000, None) == 1

@@ -1,0 +1,226 @@
+"""GPU parity of every C-ABI step against the CPU oracle, on seeded inputs at
+sizes the oracle finishes in seconds that still span several tiles and ragged
+tails (partial router chunks, partial feature tiles, multi-block experts,
+empty experts). Routing indices, counts, offsets and permutations are compared
+bit for bit; floating-point outputs use the layer tolerance in parity.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_mixture_experts_route_b200 import inputs as moe_inputs
+import moe_parity as parity
+
+pytestmark = pytest.mark.gpu
+
+U32 = 2.0 ** -24
+
+
+@pytest.fixture(scope="module")
+def lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from sparse_mixture_experts_route_b200 import _lib
+    _lib.get_device_error(clear=True)
+    return _lib
+
+
+def _inputs(T, d, E, k, f, seed=0, bias=None):
+    shape = moe_inputs.custom_shape(T, d, E, k, f, bias=bias)
+    return moe_inputs.make_inputs(shape, seed=seed, device="cpu")
+
+
+def _cuda(inp):
+    return type(inp)(inp.shape, inp.x.cuda(), inp.W_router.cuda(),
+                     inp.bias.cuda() if inp.bias is not None else None,
+                     inp.W_gate_up.cuda(), inp.W_down.cuda())
+
+
+SHAPES = [
+    # (T, d, E, k, f)
+    (64, 128, 8, 2, 256),      # the tiny workload
+    (333, 320, 20, 3, 192),    # ragged: last router chunk of 64, half feature tiles, 999 rows
+    (1, 256, 16, 4, 128),      # a single token
+    (2560, 256, 1024, 16, 64), # router without split (many tiles), 1024 experts
+    (50, 128, 8, 8, 128),      # k = E
+    (200, 192, 5, 1, 64),      # k = 1, E not a multiple of 4
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_route_bit_exact(lib, shape):
+    T, d, E, k, f = shape
+    inp = _inputs(T, d, E, k, f)
+    g = _cuda(inp)
+    idx, w = lib.moe_route(g.x, g.W_router, None, k)
+    torch.cuda.synchronize()
+    _, ridx, rw = parity.oracle_route(inp, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=1e-5, atol=1e-7)
+    assert lib.get_device_error() == 0
+
+
+def test_route_bias_ties_zero_rows(lib):
+    T, d, E, k, f = 96, 384, 12, 3, 64
+    inp = _inputs(T, d, E, k, f)
+    Wr = inp.W_router.clone()
+    Wr[:, 7] = Wr[:, 2]            # exact ties between experts 2 and 7
+    x = inp.x.clone()
+    x[10] = 0                      # all-zero token: logits all 0 (+bias)
+    x[11] = 0
+    bias = torch.zeros(E, dtype=torch.float32)
+    bias[5] = 0.25
+    for b in (None, bias):
+        idx, w = lib.moe_route(x.cuda(), Wr.cuda(), b.cuda() if b is not None else None, k)
+        lg = oracle.router_logits(x, Wr, b)
+        ridx, rw = oracle.topk(lg, k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-5, atol=1e-7)
+    # the zero tokens with a bias on expert 5 pick 5 then 0, 1
+    assert idx[10].tolist() == [5, 0, 1]
+
+
+def test_route_zipf_bias_and_hot_expert(lib):
+    T, d, E, k, f = 257, 256, 64, 4, 64
+    inp = _inputs(T, d, E, k, f, bias="zipf")
+    g = _cuda(inp)
+    idx, w = lib.moe_route(g.x, g.W_router, g.bias, k)
+    _, ridx, rw = parity.oracle_route(inp, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-5, atol=1e-7)
+    hot = torch.zeros(E, dtype=torch.float32)
+    hot[3] = 100.0
+    idx, _ = lib.moe_route(g.x, g.W_router, hot.cuda(), k)
+    assert torch.all(idx[:, 0] == 3)
+
+
+@pytest.mark.parametrize("shape", [(64, 128, 8, 2, 256), (333, 320, 20, 3, 192), (2000, 128, 896, 16, 64),
+                                   (1, 128, 4, 4, 64)], ids=lambda s: "x".join(map(str, s)))
+def test_permute_bit_exact(lib, shape):
+    T, d, E, k, f = shape
+    inp = _inputs(T, d, E, k, f)
+    _, ridx, _ = parity.oracle_route(inp, k)
+    counts, offsets, perm_token, inv_perm = oracle.permute(ridx, E)
+    x = inp.x.cuda()
+    g_off, g_perm, g_inv, g_xp = lib.moe_permute(x, torch.from_numpy(ridx).cuda(), E)
+    torch.cuda.synchronize()
+    assert np.array_equal(g_off.cpu().numpy(), offsets)
+    assert np.array_equal(g_perm.cpu().numpy(), perm_token)
+    assert np.array_equal(g_inv.cpu().numpy(), inv_perm)
+    assert torch.equal(g_xp.cpu(), inp.x[torch.from_numpy(perm_token).long()])
+    assert lib.get_device_error() == 0
+
+
+def test_permute_all_tokens_one_expert(lib):
+    T, E, k = 700, 16, 1
+    idx = torch.full((T, k), 9, dtype=torch.int32)
+    x = torch.randn(T, 64).to(torch.bfloat16)
+    off, perm, inv, xp = lib.moe_permute(x.cuda(), idx.cuda(), E)
+    exp = [0] * 10 + [T] * 7
+    assert off.cpu().tolist() == exp
+    assert perm.cpu().tolist() == list(range(T))
+    assert torch.equal(xp.cpu(), x)
+
+
+def _ffn_check(lib, inp, k):
+    E, f = inp.W_down.shape[0], inp.W_down.shape[1]
+    _, ridx, rw = parity.oracle_route(inp, k)
+    counts, offsets, perm_token, inv_perm = oracle.permute(ridx, E)
+    x_perm = inp.x[torch.from_numpy(perm_token).long()]
+    h, y = lib.moe_expert_ffn(x_perm.cuda(), torch.from_numpy(offsets).cuda(), inp.W_gate_up.cuda(),
+                              inp.W_down.cuda())
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    ref_h = np.zeros((len(perm_token), f))
+    ref_y = np.zeros((len(perm_token), inp.x.shape[1]))
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if a == b:
+            continue
+        ye, he = oracle.expert_ffn(x_perm[a:b], inp.W_gate_up[e], inp.W_down[e], want_h=True)
+        ref_h[a:b] = he
+        ref_y[a:b] = ye
+    parity.assert_layer_close(h, ref_h, "h")
+    parity.assert_layer_close(y, ref_y, "y_perm")
+    # per-expert as well, so one wrong expert cannot hide in the average
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b > a:
+            parity.assert_layer_close(y[a:b], ref_y[a:b], f"expert {e}")
+    return h, y
+
+
+@pytest.mark.parametrize("shape", [(64, 128, 8, 2, 256), (333, 320, 20, 3, 192), (1, 256, 16, 4, 128),
+                                   (400, 128, 6, 2, 384)], ids=lambda s: "x".join(map(str, s)))
+def test_expert_ffn(lib, shape):
+    T, d, E, k, f = shape
+    _ffn_check(lib, _inputs(T, d, E, k, f), k)
+
+
+def test_expert_ffn_hot_expert_multi_block(lib):
+    # every token in expert 3 -> 300 rows = token blocks of 128, 128, 44; other experts empty
+    T, d, E, k, f = 300, 128, 8, 1, 128
+    inp = _inputs(T, d, E, k, f)
+    inp.W_router.zero_()
+    inp.W_router[:, 3] = 0.0
+    b = torch.zeros(E)
+    b[3] = 100.0
+    inp = type(inp)(inp.shape, inp.x, inp.W_router, b, inp.W_gate_up, inp.W_down)
+    _ffn_check(lib, inp, k)
+
+
+def test_unpermute(lib):
+    T, d, k = 77, 192, 3
+    rows = T * k
+    y = (torch.randn(rows, d) * 3).to(torch.bfloat16)
+    inv = torch.randperm(rows).to(torch.int32).reshape(T, k)
+    w = torch.rand(T, k, dtype=torch.float32)
+    out = lib.moe_unpermute(y.cuda(), inv.cuda(), w.cuda())
+    ref = oracle.combine(parity.to_np64(y), inv.numpy(), w.numpy().astype(np.float64))
+    absref = oracle.combine(np.abs(parity.to_np64(y)), inv.numpy(), np.abs(w.numpy().astype(np.float64)))
+    # fp32 fma chain of k terms, then one bf16 rounding
+    gam = k * U32 / (1 - k * U32)
+    bound = 2.0 ** -8 * np.abs(ref) + gam * absref * (1 + 2.0 ** -8) + 1e-30
+    assert np.all(np.abs(parity.to_np64(out) - ref) <= bound)
+
+
+@pytest.mark.parametrize("shape", SHAPES + [(300, 128, 8, 2, 128)], ids=lambda s: "x".join(map(str, s)))
+def test_forward(lib, shape):
+    T, d, E, k, f = shape
+    inp = _inputs(T, d, E, k, f)
+    g = _cuda(inp)
+    out = lib.moe_forward(g.x, g.W_router, None, g.W_gate_up, g.W_down, k)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    ref, ridx, rw = oracle.forward(inp.x, inp.W_router, None, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(out, ref, "forward")
+    # the same call twice gives identical bits (no order decided by atomics)
+    out2 = lib.moe_forward(g.x, g.W_router, None, g.W_gate_up, g.W_down, k)
+    assert torch.equal(out, out2)
+
+
+def test_forward_zipf_bias(lib):
+    T, d, E, k, f = 256, 256, 64, 8, 128
+    inp = _inputs(T, d, E, k, f, bias="zipf")
+    g = _cuda(inp)
+    out = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k)
+    ref, _, _ = oracle.forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(out, ref, "forward zipf")
+
+
+def test_bounded_wait_reports_instead_of_hanging(lib):
+    assert lib.get_device_error(clear=True) == 0
+    lib.selftest_wait_timeout(2000)  # 2 ms on a barrier nothing signals
+    assert lib.get_device_error(clear=True) == lib.DEVERR_SELFTEST_TIMEOUT
+    assert lib.get_device_error(clear=True) == 0
+    # the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
+
+
+def test_python_binding_rejects_bad_tensors(lib):
+    x = torch.zeros(4, 128, dtype=torch.float32, device="cuda")
+    with pytest.raises(TypeError):
+        lib.moe_route(x, torch.zeros(128, 8, device="cuda"), None, 2)
+    xb = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lib.MoEError):
+        lib.moe_route(xb, torch.zeros(128, 8, device="cuda"), None, 9)
