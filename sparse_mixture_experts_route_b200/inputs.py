@@ -70,6 +70,9 @@ WORKLOADS = {
     "decode": MoEShape("decode", 128, 7168, 256, 4, 2048, note="256 experts top-4"),
     "skewed": MoEShape("skewed", 8192, 7168, 896, 16, 512, bias="zipf", note="896 experts top-16, Zipf-like bias"),
 }
+#: Prefill-shaped but with 32 experts (2.8 GB of weights, still > L2): the
+#: size used for full ncu captures of the kernels.
+WORKLOADS["prefill_small"] = MoEShape("prefill_small", 1024, 7168, 32, 8, 2048, note="profiling size")
 SWEEP_T = (1, 8, 32, 128, 512)
 for _T in SWEEP_T:
     WORKLOADS[f"sweep_T{_T}"] = MoEShape(f"sweep_T{_T}", _T, 7168, 896, 16, 512, note="decode sweep")
