@@ -171,6 +171,33 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const
                                void* workspace, size_t workspace_bytes, cudaStream_t stream,
                                cudaEvent_t* events);
 
+/* ---------------------------------------------------- allocation-free router --
+ * moe_route_noalloc: moe_route for callers that cannot allocate device memory
+ * -- for example code running inside a host framework that owns every device
+ * allocation, or a serving loop that must not call into an allocator between
+ * steps. The pages have no counterpart to this entry point; it exists only for
+ * such callers. The caller still passes the inputs and outputs; the scratch
+ * that moe_route takes as `workspace` is instead a fixed array inside the
+ * library, MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4 MiB) per device, held by every
+ * GPU that loads the library until the process exits.
+ * Same arguments (minus the workspace), results and errors as moe_route, plus:
+ *   - sizes whose scratch, moe_route_workspace_size(T, d, E), exceeds
+ *     MOE_ROUTE_NOALLOC_SCRATCH_BYTES return MOE_ERR_UNSUPPORTED and launch
+ *     nothing (for d = 7168, E = 896 that is T > 20);
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on that device;
+ *   - every call on a device shares the one array: calls that overlap on the
+ *     GPU (different streams, no ordering between them) race and give
+ *     undefined results. Nothing needs clearing between calls, because each
+ *     call writes every scratch element it reads before reading it.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status_t moe_route_noalloc(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                               int T, int d, int E, int k,
+                               int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
 /* ------------------------------------------------------------ diagnostics --
  * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
  * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise

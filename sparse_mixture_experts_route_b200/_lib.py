@@ -233,3 +233,24 @@ def moe_forward_timed(x, W_router, router_bias, W_gate_up, W_down, k: int, event
                                   T, d, E, k, f, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream), arr),
            "moe_forward_timed")
     return out
+
+_lib.moe_route_noalloc.argtypes = [P, P, P, I, I, I, I, P, P, P]
+_lib.moe_route_noalloc.restype = I
+ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_route_noalloc(x, W_router, router_bias, k: int, topk_idx, topk_w, stream=None):
+    """Steps 1-3 with the library's fixed device scratch instead of a workspace,
+    for callers that cannot allocate device memory. Writes into the given
+    topk_idx [T,k] int32 and topk_w [T,k] fp32; allocates nothing."""
+    T, d = x.shape
+    E = W_router.shape[1]
+    _need(x, "x", torch.bfloat16, (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    _need(topk_w, "topk_w", torch.float32, (T, k))
+    _check(_lib.moe_route_noalloc(_ptr(x), _ptr(W_router), _ptr(router_bias), T, d, E, k, _ptr(topk_idx),
+                                  _ptr(topk_w), _stream(stream)), "moe_route_noalloc")
+    return topk_idx, topk_w

@@ -443,6 +443,51 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const
                       stream, events);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------ allocation-free router scratch
+//
+// The scratch of moe_route_noalloc: one fixed array per device, so callers
+// that cannot allocate device memory can still route. Host code must not use
+// the symbol itself as a pointer (on the host it names a stand-in, not device
+// memory); noalloc_route_scratch() looks up the device address once per
+// device, with that device current, and the kernels get that address.
+static __device__ __align__(256) unsigned char g_route_noalloc_scratch[MOE_ROUTE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+void* g_route_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_route_noalloc_mutex;
+
+moe_status_t noalloc_route_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_route_noalloc_mutex);
+  if (g_route_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_route_noalloc_ptr[dev] = p;
+  }
+  *out = g_route_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_noalloc(const moe_bf16_t* x, const float* W_router, const float* router_bias, int T, int d,
+                               int E, int k, int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+  if (!x || !W_router || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, d, E, k) || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (route_plan(T, d, E).ws_bytes > MOE_ROUTE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const moe_status_t st = noalloc_route_scratch(&scratch);
+  if (st != MOE_OK) return st;
+  return launch_route(x, W_router, router_bias, T, d, E, k, topk_idx, topk_w, scratch, stream);
+}
+
 moe_status_t moe_get_device_error(uint32_t* code, int clear) {
   if (!code) return MOE_ERR_INVALID_ARG;
   unsigned int v = 0;
