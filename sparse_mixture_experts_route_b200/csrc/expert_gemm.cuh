@@ -72,7 +72,7 @@ struct GemmParams {
 };
 
 struct TileInfo {
-  int e, nb, row0, nrows;
+  int e, nb, row0, nrows, nblocks;  // nblocks: token blocks of expert e
 };
 
 __device__ __forceinline__ bool decode_tile(const GemmParams& p, int tile, TileInfo& ti) {
@@ -93,6 +93,7 @@ __device__ __forceinline__ bool decode_tile(const GemmParams& p, int tile, TileI
   const int local = tile - __ldg(p.tile_prefix + e) * NB;
   const int tb = local % tb_count;
   ti.e = e;
+  ti.nblocks = tb_count;
   ti.nb = local / tb_count;
   ti.row0 = __ldg(p.expert_offsets + e) + tb * kGemmBNT;
   ti.nrows = min(kGemmBNT, __ldg(p.expert_offsets + e + 1) - ti.row0);
@@ -151,7 +152,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();  // weights: streamed once
+      // weights of an expert with one token block are read once: evict first;
+      // with several blocks the neighbouring tiles re-read them: normal priority
+      const uint64_t pol_w_once = l2_policy_evict_first();
+      const uint64_t pol_w_shared = l2_policy_evict_normal();
       const uint64_t pol_x = l2_policy_evict_last();   // activations: re-read per feature block
       int s = 0;
       uint32_t ph = 0;
@@ -160,6 +164,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       TileInfo ti;
       for (int tile = blockIdx.x; ok && decode_tile(p, tile, ti); tile += gridDim.x) {
         const int feat0 = ti.nb * kGemmBMF;
+        const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);

@@ -17,6 +17,7 @@
 #include "permute.cuh"
 #include "ptx.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 
 namespace {
 
@@ -53,6 +54,9 @@ moe_status_t device_setup(int* num_sms) {
     if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<1>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(router_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rt_smem_bytes(128)) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -74,19 +78,60 @@ inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) &
 
 // ------------------------------------------------------------------ router
 
-enum RouterVariant { kRouterFullBig = 0, kRouterSplitBig = 1, kRouterSplitSmall = 2 };
+enum RouterVariant {
+  kRouterFullBig = 0,
+  kRouterSplitBig = 1,
+  kRouterSplitSmall = 2,
+  kRouterSplitTiny = 3,
+  kRouterTensorCore = 4
+};
+
+// Tokens from which the tensor-core screen + exact re-check router is used.
+constexpr int kRouterTcMinTokens = 256;
 
 struct RoutePlan {
   RouterVariant variant;
   int nchunks;
   size_t ws_bytes;
+  // tensor-core variant: expert tile width and workspace offsets
+  int ne = 0, nparts = 0;
+  size_t off_A = 0, off_wt32 = 0, off_hi = 0, off_lo = 0, off_part = 0, off_wnorm = 0, off_xnorm = 0;
 };
 
 RoutePlan route_plan(int T, int d, int E) {
   RoutePlan p;
   p.nchunks = ceil_div(d, kRouterChunk);
   const int64_t big_tiles = ceil_div64(T, 128) * ceil_div64(E, 64);
-  if (p.nchunks > 1 && T <= 32)
+  if (T >= kRouterTcMinTokens && d % 64 == 0 && d <= 8192 && E >= 16) {
+    p.variant = kRouterTensorCore;
+    const int64_t ttiles = ceil_div64(T, kRtM);
+    p.ne = 32;
+    for (int ne : {128, 64}) {
+      if (ttiles * ceil_div64(E, ne) >= 148) {
+        p.ne = ne;
+        break;
+      }
+    }
+    p.nparts = ceil_div(d, 256);
+    size_t at = 0;
+    auto take = [&](size_t bytes) {
+      const size_t here = at;
+      at += align256(bytes);
+      return here;
+    };
+    p.off_A = take(static_cast<size_t>(T) * E * 4);
+    p.off_wt32 = take(static_cast<size_t>(E) * 128 * ceil_div(d, 128) * 4);
+    p.off_hi = take(static_cast<size_t>(E) * d * 2);
+    p.off_lo = take(static_cast<size_t>(E) * d * 2);
+    p.off_part = take(static_cast<size_t>(p.nparts) * E * 8);
+    p.off_wnorm = take(static_cast<size_t>(E + 1) * 4);
+    p.off_xnorm = take(static_cast<size_t>(T) * 4);
+    p.ws_bytes = at;
+    return p;
+  }
+  if (p.nchunks > 1 && T <= 8)
+    p.variant = kRouterSplitTiny;
+  else if (p.nchunks > 1 && T <= 32)
     p.variant = kRouterSplitSmall;
   else if (p.nchunks > 1 && big_tiles < 296)
     p.variant = kRouterSplitBig;
@@ -102,14 +147,58 @@ bool shape_ok(int T, int d, int E, int k) {
          static_cast<int64_t>(T) * k < (int64_t(1) << 31);
 }
 
+bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+                const cuuint32_t* box);
+
+moe_status_t launch_route_tc(const RoutePlan& plan, const moe_bf16_t* x, const float* W_router, const float* bias,
+                             int T, int d, int E, int k, int32_t* idx, float* w, void* ws, cudaStream_t stream) {
+  int sms = 0;
+  const moe_status_t st = device_setup(&sms);
+  if (st != MOE_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* A = reinterpret_cast<float*>(base + plan.off_A);
+  float* wt32 = reinterpret_cast<float*>(base + plan.off_wt32);
+  uint16_t* hi = reinterpret_cast<uint16_t*>(base + plan.off_hi);
+  uint16_t* lo = reinterpret_cast<uint16_t*>(base + plan.off_lo);
+  double* part = reinterpret_cast<double*>(base + plan.off_part);
+  float* wnorm = reinterpret_cast<float*>(base + plan.off_wnorm);
+  float* xnorm = reinterpret_cast<float*>(base + plan.off_xnorm);
+  CUtensorMap mX, mHi, mLo;
+  {
+    const cuuint64_t dx[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
+    const cuuint64_t sx[1] = {static_cast<cuuint64_t>(d) * 2};
+    const cuuint32_t bx[2] = {64, static_cast<cuuint32_t>(kRtM)};
+    const cuuint64_t dw[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E)};
+    const cuuint32_t bw[2] = {64, static_cast<cuuint32_t>(plan.ne)};
+    if (!encode_map(&mX, x, 2, dx, sx, bx) || !encode_map(&mHi, hi, 2, dw, sx, bw) || !encode_map(&mLo, lo, 2, dw, sx, bw))
+      return MOE_ERR_INVALID_ARG;
+  }
+  router_prep_kernel<<<dim3(ceil_div(E, 32), plan.nparts), dim3(32, 8), 0, stream>>>(W_router, d, E, hi, lo, part);
+  router_interleave_kernel<<<dim3(ceil_div(E, 32), 32), dim3(32, 8), 0, stream>>>(W_router, d, E, ceil_div(d, 128),
+                                                                                   wt32);
+  router_wnorm_kernel<<<1, 1024, 0, stream>>>(part, plan.nparts, E, wnorm);
+  router_xnorm_kernel<<<ceil_div(T * 32, 256), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), T, d / 8, xnorm);
+  router_screen_kernel<<<dim3(ceil_div(E, plan.ne), ceil_div(T, kRtM)), kRtThreads, rt_smem_bytes(plan.ne), stream>>>(
+      mX, mHi, mLo, bias, T, d, E, plan.ne, A);
+  const size_t xs_bytes = static_cast<size_t>(ceil_div(d, 128)) * 128 * sizeof(float);
+  if (E <= 256)
+    router_recheck_kernel<8><<<T, 128, xs_bytes, stream>>>(A, x, wt32, bias, xnorm, wnorm, T, d, E, k, idx, w);
+  else
+    router_recheck_kernel<32><<<T, 128, xs_bytes, stream>>>(A, x, wt32, bias, xnorm, wnorm, T, d, E, k, idx, w);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const float* bias, int T, int d, int E, int k,
                           int32_t* idx, float* w, void* ws, cudaStream_t stream) {
   const RoutePlan plan = route_plan(T, d, E);
+  if (plan.variant == kRouterTensorCore) return launch_route_tc(plan, x, W_router, bias, T, d, E, k, idx, w, ws, stream);
   float* lg = static_cast<float*>(ws);
   switch (plan.variant) {
+    case kRouterTensorCore:
+      break;
     case kRouterFullBig: {
-      dim3 grid(ceil_div(E, 64), ceil_div(T, 128), 1);
-      router_logits_kernel<128, 64, 8, 4, false><<<grid, 256, 0, stream>>>(x, W_router, bias, T, d, E, lg);
+      dim3 grid(ceil_div(E, 64), ceil_div(T, 64), 1);
+      router_logits_kernel<64, 64, 4, 4, false><<<grid, 256, 0, stream>>>(x, W_router, bias, T, d, E, lg);
       break;
     }
     case kRouterSplitBig: {
@@ -122,13 +211,22 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
       router_logits_kernel<32, 64, 2, 4, true><<<grid, 256, 0, stream>>>(x, W_router, nullptr, T, d, E, lg);
       break;
     }
+    case kRouterSplitTiny: {
+      dim3 grid(ceil_div(E, 128), 1, plan.nchunks);
+      router_logits_kernel<8, 128, 2, 4, true><<<grid, 128, 0, stream>>>(x, W_router, nullptr, T, d, E, lg);
+      break;
+    }
   }
-  const int nsplit = (plan.variant == kRouterFullBig) ? 1 : plan.nchunks;
+  if (plan.variant != kRouterFullBig) {
+    const int64_t n = static_cast<int64_t>(T) * E;
+    router_reduce_partials_kernel<<<static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, stream>>>(
+        lg, plan.nchunks, bias, T, E);
+  }
   const int blocks = ceil_div(T, 8);
   if (E <= 256)
-    router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, nsplit, bias, T, E, k, idx, w);
+    router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, 1, nullptr, T, E, k, idx, w);
   else
-    router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, nsplit, bias, T, E, k, idx, w);
+    router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, 1, nullptr, T, E, k, idx, w);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -248,10 +346,27 @@ moe_status_t launch_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const 
 
 // --------------------------------------------------------------- unpermute
 
+template <int K>
+void launch_unpermute_k(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* w, int T, int d,
+                        moe_bf16_t* out, cudaStream_t stream) {
+  const int vpr = d / 8;
+  const int64_t n = static_cast<int64_t>(T) * vpr;
+  unpermute_kernel<K><<<static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(y_perm), inv_perm, w, T, vpr, reinterpret_cast<uint4*>(out));
+}
+
 moe_status_t launch_unpermute(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* w, int T, int d, int k,
                               moe_bf16_t* out, cudaStream_t stream) {
-  unpermute_kernel<<<T, 128, 0, stream>>>(reinterpret_cast<const uint4*>(y_perm), inv_perm, w, k, d / 8,
-                                          reinterpret_cast<uint4*>(out));
+  switch (k) {
+#define MOE_UNPERMUTE_CASE(K) \
+  case K: launch_unpermute_k<K>(y_perm, inv_perm, w, T, d, out, stream); break;
+    MOE_UNPERMUTE_CASE(1) MOE_UNPERMUTE_CASE(2) MOE_UNPERMUTE_CASE(3) MOE_UNPERMUTE_CASE(4)
+    MOE_UNPERMUTE_CASE(5) MOE_UNPERMUTE_CASE(6) MOE_UNPERMUTE_CASE(7) MOE_UNPERMUTE_CASE(8)
+    MOE_UNPERMUTE_CASE(9) MOE_UNPERMUTE_CASE(10) MOE_UNPERMUTE_CASE(11) MOE_UNPERMUTE_CASE(12)
+    MOE_UNPERMUTE_CASE(13) MOE_UNPERMUTE_CASE(14) MOE_UNPERMUTE_CASE(15) MOE_UNPERMUTE_CASE(16)
+#undef MOE_UNPERMUTE_CASE
+    default: return MOE_ERR_UNSUPPORTED;
+  }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -130,45 +130,45 @@ __global__ void __launch_bounds__(256)
   for (int v = lane; v < vec_per_row; v += 32) x_perm[dst + v] = __ldg(x + src + v);
 }
 
-// out[t, :] = sum_j w[t, j] * y_perm[inv_perm[t, j], :]; fp32, ascending j.
-// One block per token, 8 bf16 per thread per step.
-__global__ void __launch_bounds__(128)
+// out[t, :] = sum_j w[t, j] * y_perm[inv_perm[t, j], :]; fp32 fma in ascending
+// j, one rounding to bf16. One thread per 16-byte vector (8 values) of one
+// token, with K (the number of slots) fixed at compile time so all K row loads
+// are in flight together.
+template <int K>
+__global__ void __launch_bounds__(256)
     unpermute_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ inv_perm,
-                     const float* __restrict__ topk_w, int k, int vec_per_row, uint4* __restrict__ out) {
-  const int64_t t = blockIdx.x;
-  int32_t rows[16];
-  float ws[16];
+                     const float* __restrict__ topk_w, int64_t T, int vec_per_row, uint4* __restrict__ out) {
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t t = g / vec_per_row;
+  const int v = static_cast<int>(g - t * vec_per_row);
+  if (t >= T) return;
+  uint4 y[K];
+  float ws[K];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    if (j < k) {
-      rows[j] = inv_perm[t * k + j];
-      ws[j] = topk_w[t * k + j];
-    }
+  for (int j = 0; j < K; ++j) {
+    const int32_t row = __ldg(inv_perm + t * K + j);
+    ws[j] = __ldg(topk_w + t * K + j);
+    y[j] = __ldg(y_perm + static_cast<int64_t>(row) * vec_per_row + v);
   }
-  for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) {
-    float acc[8];
+  float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j < k) {
-        const uint4 y = __ldg(y_perm + static_cast<int64_t>(rows[j]) * vec_per_row + v);
-        const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[2 * q] = __fmaf_rn(ws[j], __uint_as_float(yw[q] << 16), acc[2 * q]);
-          acc[2 * q + 1] = __fmaf_rn(ws[j], __uint_as_float(yw[q] & 0xFFFF0000u), acc[2 * q + 1]);
-        }
-      }
-    }
-    uint32_t o[4];
+  for (int j = 0; j < K; ++j) {
+    const uint32_t yw[4] = {y[j].x, y[j].y, y[j].z, y[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
-      o[q] = *reinterpret_cast<const uint32_t*>(&p);
+      acc[2 * q] = __fmaf_rn(ws[j], __uint_as_float(yw[q] << 16), acc[2 * q]);
+      acc[2 * q + 1] = __fmaf_rn(ws[j], __uint_as_float(yw[q] & 0xFFFF0000u), acc[2 * q + 1]);
     }
-    out[t * vec_per_row + v] = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    o[q] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  out[t * vec_per_row + v] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace moe

@@ -31,16 +31,17 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 //   SPLIT = false: the CTA walks every chunk in order and writes final logits
 //                  (+ bias) to out[t * E + e].
 //   SPLIT = true : the CTA handles chunk blockIdx.z only and writes its partial
-//                  p_c to out[(c * T + t) * E + e]; router_topk_kernel adds the
-//                  partials in ascending c. Both modes give identical bits.
+//                  p_c to out[(c * T + t) * E + e]; router_reduce_partials_kernel
+//                  adds the partials in ascending c. Both modes give identical bits.
 // Requires d % 32 == 0. Threads: (BM / TM) * (BN / TN).
 template <int BM, int BN, int TM, int TN, bool SPLIT>
-__global__ void __launch_bounds__((BM / TM) * (BN / TN))
+__global__ void __launch_bounds__((BM / TM) * (BN / TN), 2)
     router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W,
                          const float* __restrict__ bias, int T, int d, int E, float* __restrict__ out) {
   constexpr int NT = (BM / TM) * (BN / TN);
   constexpr int TX = BN / TN;
   static_assert(TM % 2 == 0 && TN == 4, "micro-tile layout");
+  static_assert(NT >= 64 && NT <= 256, "block size");
   __shared__ __align__(16) float xs[2][kRouterBK][BM];
   __shared__ __align__(16) float ws[2][kRouterBK][BN];
 
@@ -164,6 +165,28 @@ __global__ void __launch_bounds__((BM / TM) * (BN / TN))
       }
     }
   }
+}
+
+// Split mode, second half: thread per (t, e) adds the C per-chunk partials in
+// ascending chunk order, then the bias, writing the final logit over plane 0.
+// Each thread reads only its own column of partials, so the in-place write is safe.
+__global__ void __launch_bounds__(256)
+    router_reduce_partials_kernel(float* __restrict__ lg, int nsplit, const float* __restrict__ bias, int T, int E) {
+  const int64_t n = static_cast<int64_t>(T) * E;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float l = lg[i];
+  int c = 1;
+  for (; c + 8 <= nsplit; c += 8) {
+    float p[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) p[u] = lg[static_cast<int64_t>(c + u) * n + i];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) l = __fadd_rn(l, p[u]);
+  }
+  for (; c < nsplit; ++c) l = __fadd_rn(l, lg[static_cast<int64_t>(c) * n + i]);
+  if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + static_cast<int>(i % E)));
+  lg[i] = l;
 }
 
 // One warp per token: (optionally) add the per-chunk partials in ascending

@@ -15,6 +15,15 @@ import oracle
 MAX_ABS_FRAC = 1e-2
 MEAN_REL = 5e-3
 
+# Router weights (probabilities of the selected experts). Routing indices are
+# bit-exact; the weights are fp32 softmax values whose denominator, on the
+# many-token router, sums screened logits for the non-candidate experts. The
+# tensor-core fp32 accumulation behind those logits errs by up to ~1.5e-4 at
+# d = 7168, so a relative tolerance of 5e-4 (3x margin) is used; it is 10x
+# below the layer's mean-relative output tolerance, which the weights only scale.
+W_RTOL = 5e-4
+W_ATOL = 1e-7
+
 
 def to_np64(t) -> np.ndarray:
     if isinstance(t, torch.Tensor):

@@ -39,7 +39,7 @@ def test_full_size_workload(lib, name, n_sample):
     assert lib.get_device_error() == 0
     _, ridx, rw = parity.oracle_route(inp, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
     counts, roffs, rperm, rinv = oracle.permute(ridx, E)
     assert counts.sum() == T * k
     assert np.array_equal(offs.cpu().numpy(), roffs)

@@ -55,7 +55,7 @@ def test_route_bit_exact(lib, shape):
     torch.cuda.synchronize()
     _, ridx, rw = parity.oracle_route(inp, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
     assert lib.get_device_error() == 0
 
 
@@ -74,7 +74,7 @@ def test_route_bias_ties_zero_rows(lib):
         lg = oracle.router_logits(x, Wr, b)
         ridx, rw = oracle.topk(lg, k)
         assert np.array_equal(idx.cpu().numpy(), ridx)
-        np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-5, atol=1e-7)
+        np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
     # the zero tokens with a bias on expert 5 pick 5 then 0, 1
     assert idx[10].tolist() == [5, 0, 1]
 
@@ -86,7 +86,7 @@ def test_route_zipf_bias_and_hot_expert(lib):
     idx, w = lib.moe_route(g.x, g.W_router, g.bias, k)
     _, ridx, rw = parity.oracle_route(inp, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
     hot = torch.zeros(E, dtype=torch.float32)
     hot[3] = 100.0
     idx, _ = lib.moe_route(g.x, g.W_router, hot.cuda(), k)
@@ -224,3 +224,25 @@ def test_python_binding_rejects_bad_tensors(lib):
     xb = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lib.MoEError):
         lib.moe_route(xb, torch.zeros(128, 8, device="cuda"), None, 9)
+
+
+@pytest.mark.parametrize("E,k,bias_on", [(64, 8, False), (896, 16, True)])
+def test_route_tensor_core_screen_ties_and_fallback(lib, E, k, bias_on):
+    """Many tokens (the tensor-core screen + exact re-check router): exact ties
+    from duplicated router columns, all-zero tokens (every logit equal, so the
+    candidate window overflows and every expert is recomputed), and a bias."""
+    T, d = 300, 512
+    inp = _inputs(T, d, E, k, 64, bias="zipf" if bias_on else None)
+    Wr = inp.W_router.clone()
+    Wr[:, E - 1] = Wr[:, 1]
+    Wr[:, E // 2] = Wr[:, 0]
+    x = inp.x.clone()
+    x[7] = 0
+    x[299] = 0
+    idx, w = lib.moe_route(x.cuda(), Wr.cuda(), inp.bias.cuda() if inp.bias is not None else None, k)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    lg = oracle.router_logits(x, Wr, inp.bias)
+    ridx, rw = oracle.topk(lg, k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
