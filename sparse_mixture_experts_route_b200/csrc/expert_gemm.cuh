@@ -9,16 +9,24 @@
 // for every row r of expert e (rows offsets[e] .. offsets[e+1]-1).
 //
 // Orientation ("swap AB"): the weights are the UMMA A operand (M = 128 output
-// features per tile) and the tokens are the B operand (N = up to 128 rows of
-// one expert), so an expert with 1..128 rows still issues full-height MMAs and
-// each weight byte is read once per token block. D = W^T X^T lands in TMEM with
-// one feature per lane and one token per column.
+// features per MMA) and the tokens are the B operand (N = the rows of one
+// token block of one expert), so an expert with 1..16 rows still issues
+// full-height MMAs and each weight byte is read once per token block. D = W^T X^T
+// lands in TMEM with one feature per lane and one token per column.
 //   A: weight tile [64 K rows x 128 features], N-contiguous in memory
 //      -> MN-major operand, two 64-feature boxes, 128-byte swizzle.
-//   B: token rows [128 rows x 64 K], K-contiguous -> K-major, 128-byte swizzle.
-// For mode 0 each tile carries two accumulators side by side in TMEM (gate
-// features j0..j0+127 and the matching up features), so one thread holds g and
-// u for the same (feature, token) and the SiLU-gate is fused in the epilogue.
+//   B: token rows [N rows x 64 K], K-contiguous -> K-major, 128-byte swizzle.
+// Every tile carries two A operands and two accumulators side by side in TMEM:
+//   mode 0: gate features j0..j0+127 and the matching up features, so one
+//           thread holds g and u of the same (feature, token): the SiLU-gate is
+//           fused in the epilogue. Token blocks are 256 rows: a block with more
+//           than 128 rows issues N = 256 MMAs and uses all 512 TMEM columns,
+//           which halves the weight traffic of heavily loaded experts.
+//   mode 1: output features n0..n0+127 and n0+128..n0+255 (256 per tile), so
+//           each row of H is read once per 256 output features. Token blocks are
+//           128 rows.
+// TMEM holds two 256-column slots: a tile with N <= 128 uses one slot (the
+// epilogue of one tile overlaps the MMAs of the next), a tile with N > 128 both.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one lane): smem ring of kStages stages;
@@ -40,42 +48,47 @@
 
 namespace moe {
 
-constexpr int kGemmBK = 64;     // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGemmBMF = 128;   // output features per tile (UMMA M)
-constexpr int kGemmBNT = 128;   // token rows per tile (largest UMMA N used)
+constexpr int kGemmBK = 64;         // K per stage: one 128-byte swizzle row of bf16
+constexpr int kGemmBMF = 128;       // output features per A operand (UMMA M)
 constexpr int kGemmThreads = 192;
+constexpr int kGemmBoxRows = 128;   // rows of the large B box
+constexpr int kGemmSmallBox = 32;   // rows of the small B box (tiles of <= 32 rows)
+constexpr int kTmemSlotCols = 256;
+
+__host__ __device__ constexpr int gemm_block_rows(int mode) { return mode == 0 ? 256 : 128; }
 
 template <int kMode>
 struct GemmCfg {
-  static constexpr int kNumA = (kMode == 0) ? 2 : 1;          // A operands per stage (gate, up)
-  static constexpr int kABytes = kGemmBK * kGemmBMF * 2;       // 16 KB per A operand
-  static constexpr int kAHalf = kABytes / 2;                   // one 64-feature box (8 KB)
-  static constexpr int kBBytes = kGemmBNT * kGemmBK * 2;       // 16 KB
-  static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
-  static constexpr int kStages = (kMode == 0) ? 4 : 6;
-  static constexpr int kAccCols = kNumA * kGemmBNT;            // TMEM columns per accumulator
-  static constexpr int kTmemCols = 2 * kAccCols;               // double buffered (512 / 256)
+  static constexpr int kABytes = kGemmBK * kGemmBMF * 2;         // 16 KB per A operand
+  static constexpr int kAHalf = kABytes / 2;                     // one 64-feature box (8 KB)
+  static constexpr int kBRows = gemm_block_rows(kMode);          // 256 / 128
+  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB / 16 KB
+  static constexpr int kStageBytes = 2 * kABytes + kBBytes;      // 64 KB / 48 KB
+  static constexpr int kStages = (kMode == 0) ? 3 : 4;
+  static constexpr int kTmemCols = 2 * kTmemSlotCols;            // 512
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
-  static_assert(kTmemCols <= 512, "TMEM has 512 columns");
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct GemmParams {
   const int32_t* expert_offsets;  // [E + 1] rows per expert (device)
   const int32_t* tile_prefix;     // [E + 1] token blocks before expert e (device)
   int E;
-  int K;            // reduction length (d for mode 0, f for mode 1)
-  int n_feat;       // output features (f for mode 0, d for mode 1)
-  int n_feat_tiles; // ceil(n_feat / 128)
-  int up_offset;    // column of the first up feature in W_gate_up (f); unused in mode 1
-  uint16_t* out;    // [Tk, n_feat] bf16
+  int K;             // reduction length (d for mode 0, f for mode 1)
+  int n_feat;        // output features (f for mode 0, d for mode 1)
+  int n_feat_tiles;  // mode 0: ceil(f / 128); mode 1: ceil(d / 256)
+  int a1_offset;     // column of the second A operand: f + j0 (mode 0) or n0 + 128 (mode 1), minus j0 / n0
+  uint16_t* out;     // [Tk, n_feat] bf16
 };
 
 struct TileInfo {
   int e, nb, row0, nrows, nblocks;  // nblocks: token blocks of expert e
 };
 
+template <int kMode>
 __device__ __forceinline__ bool decode_tile(const GemmParams& p, int tile, TileInfo& ti) {
+  constexpr int BR = gemm_block_rows(kMode);
   const int NB = p.n_feat_tiles;
   const int blocks_total = __ldg(p.tile_prefix + p.E);
   if (tile >= blocks_total * NB) return false;
@@ -95,24 +108,47 @@ __device__ __forceinline__ bool decode_tile(const GemmParams& p, int tile, TileI
   ti.e = e;
   ti.nblocks = tb_count;
   ti.nb = local / tb_count;
-  ti.row0 = __ldg(p.expert_offsets + e) + tb * kGemmBNT;
-  ti.nrows = min(kGemmBNT, __ldg(p.expert_offsets + e + 1) - ti.row0);
+  ti.row0 = __ldg(p.expert_offsets + e) + tb * BR;
+  ti.nrows = min(BR, __ldg(p.expert_offsets + e + 1) - ti.row0);
   return true;
+}
+
+// TMEM slot use of one tile: a tile with more than 128 rows takes both slots.
+struct SlotPlan {
+  int first, count;
+};
+__device__ __forceinline__ SlotPlan slot_plan(int nrows, int& next_slot) {
+  SlotPlan sp;
+  if (nrows > 128) {
+    sp.first = 0;
+    sp.count = 2;
+    next_slot = 0;
+  } else {
+    sp.first = next_slot;
+    sp.count = 1;
+    next_slot ^= 1;
+  }
+  return sp;
 }
 
 __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)); }
 
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<const uint16_t*>(&b);
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmBs, const GemmParams p) {
   using Cfg = GemmCfg<kMode>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
   uint64_t* empty_bar = full_bar + S;
-  uint64_t* acc_full_bar = empty_bar + S;   // [2]
+  uint64_t* acc_full_bar = empty_bar + S;      // [2] one per TMEM slot
   uint64_t* acc_empty_bar = acc_full_bar + 2;  // [2]
   uint64_t* drain_bar = acc_empty_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -139,6 +175,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBs);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -156,15 +193,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // with several blocks the neighbouring tiles re-read them: normal priority
       const uint64_t pol_w_once = l2_policy_evict_first();
       const uint64_t pol_w_shared = l2_policy_evict_normal();
-      const uint64_t pol_x = l2_policy_evict_last();   // activations: re-read per feature block
+      const uint64_t pol_x = l2_policy_evict_last();  // activations: re-read per feature block
       int s = 0;
       uint32_t ph = 0;
       int issued = 0;
       bool ok = true;
       TileInfo ti;
-      for (int tile = blockIdx.x; ok && decode_tile(p, tile, ti); tile += gridDim.x) {
-        const int feat0 = ti.nb * kGemmBMF;
+      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, tile, ti); tile += gridDim.x) {
+        const int f0 = ti.nb * (kMode == 0 ? kGemmBMF : 2 * kGemmBMF);
+        const int f1 = f0 + p.a1_offset;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
+        const bool small_box = ti.nrows <= kGemmSmallBox;
+        const int nbox = small_box ? 1 : (ti.nrows + kGemmBoxRows - 1) / kGemmBoxRows;
+        const uint32_t b_bytes = small_box ? kGemmSmallBox * kGemmBK * 2 : nbox * kGemmBoxRows * kGemmBK * 2;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
@@ -173,16 +214,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           uint8_t* st = smem + s * Cfg::kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[s], Cfg::kStageBytes);
+          mbar_arrive_expect_tx(&full_bar[s], 2 * Cfg::kABytes + b_bytes);
           const int k0 = kb * kGemmBK;
-          tma_load_3d(st, &tmA, &full_bar[s], feat0, k0, ti.e, pol_w);
-          tma_load_3d(st + Cfg::kAHalf, &tmA, &full_bar[s], feat0 + 64, k0, ti.e, pol_w);
-          if (kMode == 0) {
-            tma_load_3d(st + Cfg::kABytes, &tmA, &full_bar[s], p.up_offset + feat0, k0, ti.e, pol_w);
-            tma_load_3d(st + Cfg::kABytes + Cfg::kAHalf, &tmA, &full_bar[s], p.up_offset + feat0 + 64, k0, ti.e,
-                        pol_w);
+          tma_load_3d(st, &tmA, &full_bar[s], f0, k0, ti.e, pol_w);
+          tma_load_3d(st + Cfg::kAHalf, &tmA, &full_bar[s], f0 + 64, k0, ti.e, pol_w);
+          tma_load_3d(st + Cfg::kABytes, &tmA, &full_bar[s], f1, k0, ti.e, pol_w);
+          tma_load_3d(st + Cfg::kABytes + Cfg::kAHalf, &tmA, &full_bar[s], f1 + 64, k0, ti.e, pol_w);
+          uint8_t* bdst = st + 2 * Cfg::kABytes;
+          if (small_box) {
+            tma_load_2d(bdst, &tmBs, &full_bar[s], k0, ti.row0, pol_x);
+          } else {
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(bdst + b * kGemmBoxRows * kGemmBK * 2, &tmB, &full_bar[s], k0, ti.row0 + b * kGemmBoxRows,
+                          pol_x);
           }
-          tma_load_2d(st + Cfg::kNumA * Cfg::kABytes, &tmB, &full_bar[s], k0, ti.row0, pol_x);
           ++issued;
           if (++s == S) {
             s = 0;
@@ -204,21 +249,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      int acc = 0;
-      uint32_t acc_ph = 0;
+      uint32_t uses[2] = {0u, 0u};  // completed uses of each TMEM slot
+      int next_slot = 0;
       bool ok = true;
       bool any = false;
       TileInfo ti;
-      for (int tile = blockIdx.x; ok && decode_tile(p, tile, ti); tile += gridDim.x) {
+      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, tile, ti); tile += gridDim.x) {
         const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
         const uint32_t idesc = umma_idesc_bf16_f32(128u, n_mma, 1u, 0u);
-        if (!mbar_wait_bounded(&acc_empty_bar[acc], acc_ph ^ 1u, kWaitLimitNs, abort_flag)) {
-          record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
-          *abort_flag = 1;
-          break;
+        const SlotPlan sp = slot_plan(ti.nrows, next_slot);
+        for (int j = 0; j < sp.count && ok; ++j) {
+          const int sl = sp.first + j;
+          if (!mbar_wait_bounded(&acc_empty_bar[sl], (uses[sl] & 1u) ^ 1u, kWaitLimitNs, abort_flag)) {
+            record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+            *abort_flag = 1;
+            ok = false;
+          }
         }
+        if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * Cfg::kAccCols);
+        // accumulator 0 at the slot start; accumulator 1 after N columns (128 or 256)
+        const uint32_t d0 = tmem_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
+        const uint32_t d1 = d0 + (sp.count == 2 ? 256u : 128u);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
             record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
@@ -228,17 +280,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           tc_fence_after_sync();
           const uint32_t a_addr = smem_u32(smem + s * Cfg::kStageBytes);
-          const uint32_t b_addr = a_addr + Cfg::kNumA * Cfg::kABytes;
+          const uint32_t b_addr = a_addr + 2 * Cfg::kABytes;
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 16; ++kk) {
             const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-            const uint64_t adesc = umma_smem_desc_sw128(a_addr + kk * 2048, Cfg::kAHalf, 1024);
+            const uint64_t adesc0 = umma_smem_desc_sw128(a_addr + kk * 2048, Cfg::kAHalf, 1024);
+            const uint64_t adesc1 = umma_smem_desc_sw128(a_addr + Cfg::kABytes + kk * 2048, Cfg::kAHalf, 1024);
             const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, accum);
-            if (kMode == 0) {
-              const uint64_t adesc_u = umma_smem_desc_sw128(a_addr + Cfg::kABytes + kk * 2048, Cfg::kAHalf, 1024);
-              tc_mma_bf16(d_tmem + kGemmBNT, adesc_u, bdesc, idesc, accum);
-            }
+            tc_mma_bf16(d0, adesc0, bdesc, idesc, accum);
+            tc_mma_bf16(d1, adesc1, bdesc, idesc, accum);
           }
           tc_commit(&empty_bar[s]);  // stage s is free once these MMAs have read it
           any = true;
@@ -248,10 +298,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit(&acc_full_bar[acc]);  // accumulator complete
-        if (++acc == 2) {
-          acc = 0;
-          acc_ph ^= 1u;
+        for (int j = 0; j < sp.count; ++j) {
+          tc_commit(&acc_full_bar[sp.first + j]);  // accumulators complete
+          ++uses[sp.first + j];
         }
       }
       if (any) {
@@ -264,53 +313,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int acc = 0;
-    uint32_t acc_ph = 0;
+    uint32_t uses[2] = {0u, 0u};
+    int next_slot = 0;
+    bool ok = true;
     TileInfo ti;
-    for (int tile = blockIdx.x; decode_tile(p, tile, ti); tile += gridDim.x) {
-      if (!mbar_wait_bounded(&acc_full_bar[acc], acc_ph, kWaitLimitNs, abort_flag)) {
-        record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
-        *abort_flag = 1;
-        break;
+    for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, tile, ti); tile += gridDim.x) {
+      const SlotPlan sp = slot_plan(ti.nrows, next_slot);
+      for (int j = 0; j < sp.count && ok; ++j) {
+        const int sl = sp.first + j;
+        if (!mbar_wait_bounded(&acc_full_bar[sl], uses[sl] & 1u, kWaitLimitNs, abort_flag)) {
+          record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
+          *abort_flag = 1;
+          ok = false;
+        }
       }
+      if (!ok) break;
       tc_fence_after_sync();
-      const int feat = ti.nb * kGemmBMF + q * 32 + lane;
-      const bool feat_ok = feat < p.n_feat;
-      const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(acc * Cfg::kAccCols);
+      const uint32_t t0 = tmem_base + lane_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
+      const uint32_t t1 = t0 + (sp.count == 2 ? 256u : 128u);
+      const int fa = ti.nb * (kMode == 0 ? kGemmBMF : 2 * kGemmBMF) + q * 32 + lane;
+      const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
+      const bool fa_ok = fa < p.n_feat;
+      const bool fb_ok = (kMode == 1) && fb < p.n_feat;
       for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
-        uint32_t g[32];
-        tmem_ld_32x32b_x32(taddr + c0, g);
+        uint32_t g[32], u[32];
+        tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
+        tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
+        tmem_ld_wait();
+        uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + c0) * p.n_feat;
+        const int nv = min(32, ti.nrows - c0);
         if (kMode == 0) {
-          uint32_t u[32];
-          tmem_ld_32x32b_x32(taddr + kGemmBNT + c0, u);
-          tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (feat_ok && c0 + i < ti.nrows) {
-              const float h = silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-              const __nv_bfloat16 hb = __float2bfloat16_rn(h);
-              p.out[static_cast<int64_t>(ti.row0 + c0 + i) * p.n_feat + feat] =
-                  *reinterpret_cast<const uint16_t*>(&hb);
-            }
+            if (fa_ok && i < nv)
+              orow[static_cast<int64_t>(i) * p.n_feat + fa] =
+                  bf16_bits(silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]));
           }
         } else {
-          tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (feat_ok && c0 + i < ti.nrows) {
-              const __nv_bfloat16 yb = __float2bfloat16_rn(__uint_as_float(g[i]));
-              p.out[static_cast<int64_t>(ti.row0 + c0 + i) * p.n_feat + feat] =
-                  *reinterpret_cast<const uint16_t*>(&yb);
+            if (i < nv) {
+              if (fa_ok) orow[static_cast<int64_t>(i) * p.n_feat + fa] = bf16_bits(__uint_as_float(g[i]));
+              if (fb_ok) orow[static_cast<int64_t>(i) * p.n_feat + fb] = bf16_bits(__uint_as_float(u[i]));
             }
           }
         }
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty_bar[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_ph ^= 1u;
+      for (int j = 0; j < sp.count; ++j) {
+        if (lane == 0) mbar_arrive(&acc_empty_bar[sp.first + j]);
+        ++uses[sp.first + j];
       }
     }
   }
@@ -323,37 +376,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// Token blocks per expert: tile_prefix[e] = sum_{e' < e} ceil(count_e' / 128).
+// Token blocks per expert for both GEMMs:
+//   prefix0[e] = sum_{e' < e} ceil(count_e' / 256)  (gate/up, 256-row blocks)
+//   prefix1[e] = sum_{e' < e} ceil(count_e' / 128)  (down, 128-row blocks)
 __global__ void __launch_bounds__(1024)
-    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ tile_prefix) {
-  __shared__ int32_t warp_sums[32];
+    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ prefix0,
+                         int32_t* __restrict__ prefix1) {
+  __shared__ int32_t warp_sums[2][32];
   const int e = threadIdx.x;
   const int32_t cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
-  const int32_t nb = (cnt + kGemmBNT - 1) / kGemmBNT;
+  const int32_t nb[2] = {(cnt + gemm_block_rows(0) - 1) / gemm_block_rows(0),
+                         (cnt + gemm_block_rows(1) - 1) / gemm_block_rows(1)};
   const int lane = e & 31, w = e >> 5;
-  int32_t incl = nb;
+  int32_t incl[2];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+  for (int m = 0; m < 2; ++m) {
+    incl[m] = nb[m];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl[m], o);
+      if (lane >= o) incl[m] += y;
+    }
+    if (lane == 31) warp_sums[m][w] = incl[m];
   }
-  if (lane == 31) warp_sums[w] = incl;
   __syncthreads();
-  if (w == 0) {
-    const int32_t ws = warp_sums[lane];
+  if (w < 2) {
+    const int m = w;
+    const int32_t ws = warp_sums[m][lane];
     int32_t wincl = ws;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int32_t y = __shfl_up_sync(0xffffffffu, wincl, o);
       if (lane >= o) wincl += y;
     }
-    warp_sums[lane] = wincl - ws;
+    warp_sums[m][lane] = wincl - ws;
   }
   __syncthreads();
-  const int32_t excl = warp_sums[w] + incl - nb;
   if (e < E) {
-    tile_prefix[e] = excl;
-    if (e == E - 1) tile_prefix[E] = excl + nb;
+    int32_t* outs[2] = {prefix0, prefix1};
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int32_t excl = warp_sums[m][w] + incl[m] - nb[m];
+      outs[m][e] = excl;
+      if (e == E - 1) outs[m][E] = excl + nb[m];
+    }
   }
 }
 

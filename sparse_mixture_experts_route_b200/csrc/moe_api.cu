@@ -54,7 +54,7 @@ moe_status_t device_setup(int* num_sms) {
     if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<1>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
-    if (cudaFuncSetAttribute(router_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rt_smem_bytes(128)) !=
+    if (cudaFuncSetAttribute(router_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScrSmemBytes) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
     if (g_encode == nullptr) {
@@ -93,9 +93,10 @@ struct RoutePlan {
   RouterVariant variant;
   int nchunks;
   size_t ws_bytes;
-  // tensor-core variant: expert tile width and workspace offsets
-  int ne = 0, nparts = 0;
-  size_t off_A = 0, off_wt32 = 0, off_hi = 0, off_lo = 0, off_part = 0, off_wnorm = 0, off_xnorm = 0;
+  // tensor-core variant: K split of the screen and workspace offsets
+  int nsplit = 1, kb_per_split = 0, nparts = 0;
+  size_t off_A = 0, off_wt32 = 0, off_hi = 0, off_lo = 0, off_part = 0, off_wnorm = 0, off_xnorm = 0, off_xc = 0,
+         off_ovf = 0;
 };
 
 RoutePlan route_plan(int T, int d, int E) {
@@ -104,14 +105,15 @@ RoutePlan route_plan(int T, int d, int E) {
   const int64_t big_tiles = ceil_div64(T, 128) * ceil_div64(E, 64);
   if (T >= kRouterTcMinTokens && d % 64 == 0 && d <= 8192 && E >= 16) {
     p.variant = kRouterTensorCore;
-    const int64_t ttiles = ceil_div64(T, kRtM);
-    p.ne = 32;
-    for (int ne : {128, 64}) {
-      if (ttiles * ceil_div64(E, ne) >= 148) {
-        p.ne = ne;
-        break;
-      }
-    }
+    // split K so the screen has about two CTAs per SM of a 148-SM part; every
+    // split keeps at least 8 K blocks
+    const int KB = d / kRtBK;
+    const int64_t tiles = ceil_div64(T, kScrT) * ceil_div64(E, kScrE);
+    int ns = static_cast<int>(ceil_div64(296, tiles));
+    ns = ns < 1 ? 1 : ns;
+    ns = ns > KB / 8 ? (KB / 8 > 0 ? KB / 8 : 1) : ns;
+    p.kb_per_split = ceil_div(KB, ns);
+    p.nsplit = ceil_div(KB, p.kb_per_split);  // every split non-empty
     p.nparts = ceil_div(d, 256);
     size_t at = 0;
     auto take = [&](size_t bytes) {
@@ -119,13 +121,14 @@ RoutePlan route_plan(int T, int d, int E) {
       at += align256(bytes);
       return here;
     };
-    p.off_A = take(static_cast<size_t>(T) * E * 4);
-    p.off_wt32 = take(static_cast<size_t>(E) * 128 * ceil_div(d, 128) * 4);
+    p.off_A = take(static_cast<size_t>(p.nsplit) * T * E * 4);
+    p.off_wt32 = take(static_cast<size_t>(E) * 128 * 64 * 4);
     p.off_hi = take(static_cast<size_t>(E) * d * 2);
     p.off_lo = take(static_cast<size_t>(E) * d * 2);
     p.off_part = take(static_cast<size_t>(p.nparts) * E * 8);
     p.off_wnorm = take(static_cast<size_t>(E + 1) * 4);
     p.off_xnorm = take(static_cast<size_t>(T) * 4);
+    p.off_ovf = take(static_cast<size_t>(T + 1) * 4);
     p.ws_bytes = at;
     return p;
   }
@@ -163,28 +166,39 @@ moe_status_t launch_route_tc(const RoutePlan& plan, const moe_bf16_t* x, const f
   double* part = reinterpret_cast<double*>(base + plan.off_part);
   float* wnorm = reinterpret_cast<float*>(base + plan.off_wnorm);
   float* xnorm = reinterpret_cast<float*>(base + plan.off_xnorm);
+  int32_t* ovf = reinterpret_cast<int32_t*>(base + plan.off_ovf);
+  const int C = ceil_div(d, 128);
   CUtensorMap mX, mHi, mLo;
   {
     const cuuint64_t dx[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T)};
     const cuuint64_t sx[1] = {static_cast<cuuint64_t>(d) * 2};
-    const cuuint32_t bx[2] = {64, static_cast<cuuint32_t>(kRtM)};
+    const cuuint32_t bx[2] = {64, 128};
     const cuuint64_t dw[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(E)};
-    const cuuint32_t bw[2] = {64, static_cast<cuuint32_t>(plan.ne)};
-    if (!encode_map(&mX, x, 2, dx, sx, bx) || !encode_map(&mHi, hi, 2, dw, sx, bw) || !encode_map(&mLo, lo, 2, dw, sx, bw))
+    if (!encode_map(&mX, x, 2, dx, sx, bx) || !encode_map(&mHi, hi, 2, dw, sx, bx) || !encode_map(&mLo, lo, 2, dw, sx, bx))
       return MOE_ERR_INVALID_ARG;
   }
   router_prep_kernel<<<dim3(ceil_div(E, 32), plan.nparts), dim3(32, 8), 0, stream>>>(W_router, d, E, hi, lo, part);
-  router_interleave_kernel<<<dim3(ceil_div(E, 32), 32), dim3(32, 8), 0, stream>>>(W_router, d, E, ceil_div(d, 128),
-                                                                                   wt32);
+  router_interleave_kernel<<<dim3(ceil_div(E, 32), 32), dim3(32, 8), 0, stream>>>(W_router, d, E, C, wt32);
   router_wnorm_kernel<<<1, 1024, 0, stream>>>(part, plan.nparts, E, wnorm);
-  router_xnorm_kernel<<<ceil_div(T * 32, 256), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), T, d / 8, xnorm);
-  router_screen_kernel<<<dim3(ceil_div(E, plan.ne), ceil_div(T, kRtM)), kRtThreads, rt_smem_bytes(plan.ne), stream>>>(
-      mX, mHi, mLo, bias, T, d, E, plan.ne, A);
-  const size_t xs_bytes = static_cast<size_t>(ceil_div(d, 128)) * 128 * sizeof(float);
-  if (E <= 256)
-    router_recheck_kernel<8><<<T, 128, xs_bytes, stream>>>(A, x, wt32, bias, xnorm, wnorm, T, d, E, k, idx, w);
-  else
-    router_recheck_kernel<32><<<T, 128, xs_bytes, stream>>>(A, x, wt32, bias, xnorm, wnorm, T, d, E, k, idx, w);
+  router_xnorm_kernel<<<ceil_div(T * 32, 256), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), T, d / 8, xnorm,
+                                                                 ovf);
+  router_screen_kernel<<<dim3(ceil_div(T, kScrT), ceil_div(E, kScrE), plan.nsplit), kRtThreads, kScrSmemBytes,
+                         stream>>>(mX, mHi, mLo, T, d, E, plan.kb_per_split, A);
+  // add the K-split planes in order and the bias: A = plane 0
+  router_reduce_partials_kernel<<<static_cast<unsigned>(ceil_div64(static_cast<int64_t>(T) * E, 256)), 256, 0,
+                                  stream>>>(A, plan.nsplit, bias, T, E);
+  const bool full = (d % 128) == 0;
+  const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+#define MOE_RECHECK(MAXV, FULL)                                                                                   \
+  router_recheck_kernel<MAXV, FULL><<<T, kRcWarps * 32, 0, stream>>>(A, xb, wt32, bias, xnorm, wnorm, T, d, E, k, idx, \
+                                                                     w, ovf)
+  if (E <= 256) {
+    if (full) MOE_RECHECK(8, true); else MOE_RECHECK(8, false);
+  } else {
+    if (full) MOE_RECHECK(32, true); else MOE_RECHECK(32, false);
+  }
+#undef MOE_RECHECK
+  router_fallback_kernel<<<T, 128, 0, stream>>>(ovf, xb, wt32, bias, d, E, k, idx, w);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -224,9 +238,9 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
   }
   const int blocks = ceil_div(T, 8);
   if (E <= 256)
-    router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, 1, nullptr, T, E, k, idx, w);
+    router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
   else
-    router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, 1, nullptr, T, E, k, idx, w);
+    router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -258,7 +272,7 @@ moe_status_t launch_permute(const moe_bf16_t* x, const int32_t* idx, int T, int 
 
 // -------------------------------------------------------------- expert FFN
 
-size_t ffn_ws(int E) { return align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
+size_t ffn_ws(int E) { return 2 * align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
 
 bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
                 const cuuint32_t* box) {
@@ -278,16 +292,16 @@ bool weight_map(CUtensorMap* map, const moe_bf16_t* W, int E, int K, int N) {
   return encode_map(map, W, 3, dims, strides, box);
 }
 
-// Activations A[rows][K] (K contiguous): boxes of 64 K x 128 rows.
-bool act_map(CUtensorMap* map, const moe_bf16_t* A, int rows, int K) {
+// Activations A[rows][K] (K contiguous): boxes of 64 K x `box_rows` rows.
+bool act_map(CUtensorMap* map, const moe_bf16_t* A, int rows, int K, int box_rows) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kGemmBNT)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   return encode_map(map, A, 2, dims, strides, box);
 }
 
 struct FfnPlan {
-  CUtensorMap mA0, mB0, mA1, mB1;
+  CUtensorMap mA0, mB0, mBs0, mA1, mB1, mBs1;
   GemmParams p0, p1;
   int grid0, grid1;
 };
@@ -295,41 +309,46 @@ struct FfnPlan {
 moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
                       int Tk, int d, int E, int f, moe_bf16_t* h, moe_bf16_t* y_perm, void* ws, int num_sms,
                       FfnPlan* fp) {
-  if (!weight_map(&fp->mA0, Wgu, E, d, 2 * f) || !act_map(&fp->mB0, x_perm, Tk, d) ||
-      !weight_map(&fp->mA1, Wd, E, f, d) || !act_map(&fp->mB1, h, Tk, f))
+  if (!weight_map(&fp->mA0, Wgu, E, d, 2 * f) || !act_map(&fp->mB0, x_perm, Tk, d, kGemmBoxRows) ||
+      !act_map(&fp->mBs0, x_perm, Tk, d, kGemmSmallBox) || !weight_map(&fp->mA1, Wd, E, f, d) ||
+      !act_map(&fp->mB1, h, Tk, f, kGemmBoxRows) || !act_map(&fp->mBs1, h, Tk, f, kGemmSmallBox))
     return MOE_ERR_INVALID_ARG;
-  const int64_t blocks_ub = ceil_div64(Tk, kGemmBNT) + (E < Tk ? E : Tk);
+  int32_t* prefix0 = static_cast<int32_t*>(ws);
+  int32_t* prefix1 = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ffn_ws(E) / 2);
+  const int64_t min_e_tk = E < Tk ? E : Tk;
   GemmParams& p0 = fp->p0;
   p0.expert_offsets = offsets;
-  p0.tile_prefix = static_cast<int32_t*>(ws);
+  p0.tile_prefix = prefix0;
   p0.E = E;
   p0.K = d;
   p0.n_feat = f;
   p0.n_feat_tiles = ceil_div(f, kGemmBMF);
-  p0.up_offset = f;
+  p0.a1_offset = f;
   p0.out = h;
-  const int64_t tiles0 = blocks_ub * p0.n_feat_tiles;
+  const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(0)) + min_e_tk) * p0.n_feat_tiles;
   fp->grid0 = static_cast<int>(tiles0 < num_sms ? tiles0 : num_sms);
   GemmParams& p1 = fp->p1;
   p1 = p0;
+  p1.tile_prefix = prefix1;
   p1.K = f;
   p1.n_feat = d;
-  p1.n_feat_tiles = ceil_div(d, kGemmBMF);
-  p1.up_offset = 0;
+  p1.n_feat_tiles = ceil_div(d, 2 * kGemmBMF);
+  p1.a1_offset = kGemmBMF;
   p1.out = y_perm;
-  const int64_t tiles1 = blocks_ub * p1.n_feat_tiles;
+  const int64_t tiles1 = (ceil_div64(Tk, gemm_block_rows(1)) + min_e_tk) * p1.n_feat_tiles;
   fp->grid1 = static_cast<int>(tiles1 < num_sms ? tiles1 : num_sms);
   return MOE_OK;
 }
 
 void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
-  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, const_cast<int32_t*>(fp.p0.tile_prefix));
+  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, const_cast<int32_t*>(fp.p0.tile_prefix),
+                                               const_cast<int32_t*>(fp.p1.tile_prefix));
 }
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
-  grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.p0);
+  grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
 }
 void launch_gemm_down(const FfnPlan& fp, cudaStream_t stream) {
-  grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.p1);
+  grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
 }
 
 moe_status_t launch_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,

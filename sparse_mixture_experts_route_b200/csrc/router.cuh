@@ -189,35 +189,25 @@ __global__ void __launch_bounds__(256)
   lg[i] = l;
 }
 
-// One warp per token: (optionally) add the per-chunk partials in ascending
-// chunk order and the bias, softmax over all E experts in fp32, then k rounds
+// One warp per token: softmax over all E final logits in fp32, then k rounds
 // of warp arg-max (ties -> lower index). MAXV >= ceil(E / 32).
 template <int MAXV>
 __global__ void __launch_bounds__(256)
-    router_topk_kernel(const float* __restrict__ lg, int nsplit, const float* __restrict__ bias, int T, int E,
-                       int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    router_topk_kernel(const float* __restrict__ lg, int T, int E, int k, int32_t* __restrict__ topk_idx,
+                       float* __restrict__ topk_w) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
   const int t = warp;
   float v[MAXV];
-  float m = -INFINITY;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int e = i * 32 + lane;
-    float l = -INFINITY;
-    if (e < E) {
-      if (nsplit == 1) {
-        l = lg[static_cast<int64_t>(t) * E + e];
-      } else {
-        l = lg[static_cast<int64_t>(t) * E + e];
-        for (int c = 1; c < nsplit; ++c) l = __fadd_rn(l, lg[(static_cast<int64_t>(c) * T + t) * E + e]);
-        if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e));
-      }
-      m = fmaxf(m, l);
-    }
-    v[i] = l;
+    v[i] = (e < E) ? __ldcs(lg + static_cast<int64_t>(t) * E + e) : -INFINITY;
   }
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) m = fmaxf(m, v[i]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float s = 0.0f;

@@ -5,12 +5,14 @@
 // Load Balancing": softmax over all experts, top-k, unnormalised values) and the
 // same bits, in less time when T * E is large:
 //
-//  1. prep: W_router [d, E] fp32 -> a chunk-interleaved exact copy Wc [E][128][C]
-//     fp32 (Wc[e][j][c] = W[128 c + j][e]) and Wt_hi / Wt_lo [E, d] bf16 with Wt_hi = bf16(W), Wt_lo = bf16(W - Wt_hi),
+//  1. prep: W_router [d, E] fp32 -> a chunk-interleaved exact copy Wc
+//     [E][128][32][2] fp32 (offset j of chunks l and l + 32 side by side) and
+//     Wt_hi / Wt_lo [E, d] bf16 with Wt_hi = bf16(W), Wt_lo = bf16(W - Wt_hi),
 //     so |W - Wt_hi - Wt_lo| <= 2^-17 |W|; an upper bound of each column norm
 //     ||W_e||_2 and of each token norm ||x_t||_2.
 //  2. screen: A[t, e] = x_t . Wt_hi[e] + x_t . Wt_lo[e] (+ b_e) on tcgen05
-//     (bf16 x bf16 products are exact in fp32; fp32 accumulation in TMEM).
+//     (bf16 x bf16 products are exact in fp32; fp32 accumulation in TMEM), with
+//     the K range split over CTAs and the partials added in a fixed order.
 //  3. re-check, per token: tau = k-th largest A; every expert with
 //     A_e >= tau - 2 eps_t is a candidate, where eps_t bounds |A - L| for the
 //     exact-order fp32 logit L (below); each candidate's L is recomputed in the
@@ -40,15 +42,10 @@
 
 namespace moe {
 
-constexpr int kRtM = 128;          // tokens per tile (UMMA M)
 constexpr int kRtBK = 64;          // K per stage
-constexpr int kRtStages = 4;
 constexpr int kRtThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kMaxCand = 32;       // candidate window capacity per token
 constexpr float kRtEpsRel = 1.0f / 2048.0f;
-
-__host__ __device__ constexpr int rt_stage_bytes(int ne) { return kRtM * kRtBK * 2 + 2 * ne * kRtBK * 2; }
-__host__ __device__ constexpr int rt_smem_bytes(int ne) { return kRtStages * rt_stage_bytes(ne) + 256 + 1024; }
 
 // ---------------------------------------------------------------- 1. prep
 
@@ -97,26 +94,26 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// W [d, E] -> Wc [E][128][C] fp32 with Wc[e][j][c] = W[c * 128 + j][e] (0 past
-// d): for one expert and one offset j inside a chunk, the C chunks are adjacent,
-// so a warp whose lanes each run one chunk's fma chain reads 32 consecutive
-// floats per step. Block (32, 8) handles 32 experts x 4 offsets j x all chunks.
+// W [d, E] -> Wc [E][128][32][2] fp32: Wc[e][j][l][h] = W[128 c + j][e] for
+// chunk c = 32 h + l (0 past d). For one expert and one offset j inside a
+// chunk, lane l of a warp reads chunks l and l + 32 with one 8-byte load.
+// Block (32, 8) handles 32 experts x 4 offsets j x all chunks (C <= 64).
 __global__ void __launch_bounds__(256)
     router_interleave_kernel(const float* __restrict__ W, int d, int E, int C, float* __restrict__ Wc) {
-  __shared__ float tile[4][64][33];  // [j][c][e]; C <= 64 (d <= 8192)
+  __shared__ float tile[4][64][33];  // [j][c][e]
   const int e0 = blockIdx.x * 32, j0 = blockIdx.y * 4;
   const int tx = threadIdx.x, ty = threadIdx.y;
-  for (int rc = ty; rc < 4 * C; rc += 8) {
-    const int j = rc / C, c = rc - j * C;
+  for (int rc = ty; rc < 4 * 64; rc += 8) {
+    const int j = rc / 64, c = rc - j * 64;
     const int i = c * 128 + j0 + j, e = e0 + tx;
-    tile[j][c][tx] = (i < d && e < E) ? __ldg(W + static_cast<int64_t>(i) * E + e) : 0.0f;
+    tile[j][c][tx] = (c < C && i < d && e < E) ? __ldg(W + static_cast<int64_t>(i) * E + e) : 0.0f;
   }
   __syncthreads();
   for (int r = ty; r < 32 * 4; r += 8) {
     const int el = r / 4, j = r % 4, e = e0 + el;
     if (e >= E) continue;
-    float* dst = Wc + (static_cast<int64_t>(e) * 128 + j0 + j) * C;
-    for (int c = tx; c < C; c += 32) dst[c] = tile[j][c][el];
+    float2* dst = reinterpret_cast<float2*>(Wc + (static_cast<int64_t>(e) * 128 + j0 + j) * 64);
+    dst[tx] = make_float2(tile[j][tx][el], tile[j][tx + 32][el]);
   }
 }
 
@@ -147,8 +144,11 @@ __global__ void __launch_bounds__(1024)
 
 // xnorm[t] >= ||x_t||_2: warp per token, fp32 sum of squares scaled up by
 // (1 + 2^-10), which exceeds the relative error of the fp32 sum for d <= 32768.
+// Also resets the re-check's overflow counter.
 __global__ void __launch_bounds__(256)
-    router_xnorm_kernel(const uint4* __restrict__ x, int T, int vec_per_row, float* __restrict__ xnorm) {
+    router_xnorm_kernel(const uint4* __restrict__ x, int T, int vec_per_row, float* __restrict__ xnorm,
+                        int32_t* __restrict__ overflow) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) overflow[0] = 0;  // the re-check appends to it
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -170,27 +170,36 @@ __global__ void __launch_bounds__(256)
 
 // -------------------------------------------------------------- 2. screen
 
-// A[t, e] = x_t . (Wt_hi[e] + Wt_lo[e]) (+ b_e), fp32, for one tile of 128
-// tokens x NE experts per CTA. Both operands K-major with 128-byte swizzle.
+// Apart[s][t][e] = sum over the s-th K range of x_t . (Wt_hi[e] + Wt_lo[e]),
+// fp32, for one tile of 128 experts (UMMA M, A operand) x 256 tokens (N, B
+// operand) per CTA; the K ranges are summed in order by the re-check. Both
+// operands K-major with 128-byte swizzle; two MMAs (hi, lo) per K step into one
+// accumulator of 256 TMEM columns.
+constexpr int kScrE = 128;           // experts per tile
+constexpr int kScrT = 256;           // tokens per tile
+constexpr int kScrStages = 3;
+constexpr int kScrStageBytes = 2 * kScrE * kRtBK * 2 + kScrT * kRtBK * 2;  // 64 KB
+constexpr int kScrSmemBytes = kScrStages * kScrStageBytes + 256 + 1024;
+
 __global__ void __launch_bounds__(kRtThreads, 1)
     router_screen_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmHi,
-                         const __grid_constant__ CUtensorMap tmLo, const float* __restrict__ bias, int T, int d,
-                         int E, int ne, float* __restrict__ A) {
+                         const __grid_constant__ CUtensorMap tmLo, int T, int d, int E, int kb_per_split,
+                         float* __restrict__ Apart) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int stage_bytes = rt_stage_bytes(ne);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kRtStages * stage_bytes);
-  uint64_t* empty_bar = full_bar + kRtStages;
-  uint64_t* acc_bar = empty_bar + kRtStages;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + kScrStages * kScrStageBytes);
+  uint64_t* empty_bar = full_bar + kScrStages;
+  uint64_t* acc_bar = empty_bar + kScrStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.y * kRtM, e0 = blockIdx.x * ne;
+  const int t0 = blockIdx.x * kScrT, e0 = blockIdx.y * kScrE, split = blockIdx.z;
   const int KB = d / kRtBK;
-  const uint32_t tmem_cols = static_cast<uint32_t>(ne < 32 ? 32 : ne);
+  const int kb0 = split * kb_per_split, kb1 = min(KB, kb0 + kb_per_split);
+  constexpr uint32_t kCols = 256;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRtStages; ++s) {
+    for (int s = 0; s < kScrStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -200,7 +209,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     fence_proxy_async_shared();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_alloc(tmem_slot, kCols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -218,39 +227,41 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       uint32_t ph = 0;
       int issued = 0;
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
           record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
           *abort_flag = 1;
           ok = false;
           break;
         }
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&full_bar[s], static_cast<uint32_t>(stage_bytes));
-        tma_load_2d(st, &tmX, &full_bar[s], kb * kRtBK, t0, pol);
-        tma_load_2d(st + kRtM * kRtBK * 2, &tmHi, &full_bar[s], kb * kRtBK, e0, pol);
-        tma_load_2d(st + kRtM * kRtBK * 2 + ne * kRtBK * 2, &tmLo, &full_bar[s], kb * kRtBK, e0, pol);
+        uint8_t* st = smem + s * kScrStageBytes;
+        mbar_arrive_expect_tx(&full_bar[s], static_cast<uint32_t>(kScrStageBytes));
+        const int k0 = kb * kRtBK;
+        tma_load_2d(st, &tmHi, &full_bar[s], k0, e0, pol);
+        tma_load_2d(st + kScrE * kRtBK * 2, &tmLo, &full_bar[s], k0, e0, pol);
+        tma_load_2d(st + 2 * kScrE * kRtBK * 2, &tmX, &full_bar[s], k0, t0, pol);
+        tma_load_2d(st + 2 * kScrE * kRtBK * 2 + 128 * kRtBK * 2, &tmX, &full_bar[s], k0, t0 + 128, pol);
         ++issued;
-        if (++s == kRtStages) {
+        if (++s == kScrStages) {
           s = 0;
           ph ^= 1u;
         }
       }
       if (!ok) {
-        for (int i = 0; i < kRtStages && i < issued; ++i) {
-          s = (s == 0) ? kRtStages - 1 : s - 1;
-          if (s == kRtStages - 1) ph ^= 1u;
+        for (int i = 0; i < kScrStages && i < issued; ++i) {
+          s = (s == 0) ? kScrStages - 1 : s - 1;
+          if (s == kScrStages - 1) ph ^= 1u;
           mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, nullptr);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(128u, static_cast<uint32_t>(ne), 0u, 0u);
+      const uint32_t idesc = umma_idesc_bf16_f32(128u, 256u, 0u, 0u);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
           record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
           *abort_flag = 1;
@@ -258,48 +269,42 @@ __global__ void __launch_bounds__(kRtThreads, 1)
           break;
         }
         tc_fence_after_sync();
-        const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
-        const uint32_t hi_addr = a_addr + kRtM * kRtBK * 2;
-        const uint32_t lo_addr = hi_addr + ne * kRtBK * 2;
+        const uint32_t hi_addr = smem_u32(smem + s * kScrStageBytes);
+        const uint32_t lo_addr = hi_addr + kScrE * kRtBK * 2;
+        const uint32_t x_addr = lo_addr + kScrE * kRtBK * 2;
 #pragma unroll
         for (int kk = 0; kk < kRtBK / 16; ++kk) {
-          const uint64_t adesc = umma_smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+          const uint64_t xdesc = umma_smem_desc_sw128(x_addr + kk * 32, 16, 1024);
           const uint64_t hdesc = umma_smem_desc_sw128(hi_addr + kk * 32, 16, 1024);
           const uint64_t ldesc = umma_smem_desc_sw128(lo_addr + kk * 32, 16, 1024);
-          tc_mma_bf16(tmem_base, adesc, hdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_bf16(tmem_base, adesc, ldesc, idesc, 1u);
+          tc_mma_bf16(tmem_base, hdesc, xdesc, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16(tmem_base, ldesc, xdesc, idesc, 1u);
         }
         tc_commit(&empty_bar[s]);
-        if (++s == kRtStages) {
+        if (++s == kScrStages) {
           s = 0;
           ph ^= 1u;
         }
       }
-      tc_commit(acc_bar);  // also drains: completes when every MMA above has
+      tc_commit(acc_bar);  // completes when every MMA above has
       if (!ok) mbar_wait_bounded(acc_bar, 0u, kWaitLimitNs, nullptr);
     }
   } else {
     const int q = warp & 3;
-    const int r = q * 32 + lane;
-    const int t = t0 + r;
+    const int e = e0 + q * 32 + lane;  // this thread's TMEM lane = expert
     if (mbar_wait_bounded(acc_bar, 0u, kWaitLimitNs, abort_flag)) {
       tc_fence_after_sync();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 0; c0 < ne; c0 += 32) {
+      float* plane = Apart + static_cast<int64_t>(split) * T * E;
+      const int nt = min(kScrT, T - t0);
+      for (int c0 = 0; c0 < nt; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c0), v);
         tmem_ld_wait();
-        if (t < T) {
-          float* row = A + static_cast<int64_t>(t) * E;
+        if (e < E) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = e0 + c0 + i;
-            if (e < E) {
-              float a = __uint_as_float(v[i]);
-              if (bias != nullptr) a = __fadd_rn(a, __ldg(bias + e));
-              row[e] = a;
-            }
-          }
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < nt) plane[static_cast<int64_t>(t0 + c0 + i) * E + e] = __uint_as_float(v[i]);
         }
       }
     } else {
@@ -311,88 +316,147 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, tmem_cols);
+    tmem_dealloc(tmem_base, kCols);
   }
 }
 
 // ------------------------------------------------------------ 3. re-check
 
-// One CTA (128 threads) per token.
-//   warp 0: softmax statistics over A and the candidate window;
-//   warps 0-3: exact-order logits of the candidates; lane l runs the fma chains
-//              of chunks l and l + 32 (reading the chunk-interleaved copy Wc
-//              and x staged as xs[j][c], both conflict-free and coalesced);
-//   warp 0: top-k over the candidates by (L desc, index asc); the softmax
-//           denominator uses L for the candidates and A for every other expert.
-template <int MAXV>
-__global__ void __launch_bounds__(128)
+constexpr int kRcWarps = 4;               // warps per CTA; one CTA per token
+constexpr int kRcXsBytes = 128 * 32 * 4;  // x staged as [j][l] bf16 pairs (16 KB)
+
+// Stage x_t as xs[j][l] = (x[128 l + j], x[128 (l + 32) + j]) bf16 pairs (0 past
+// d) with 16-byte loads; `tid` / `nthreads` split the work.
+__device__ __forceinline__ void stage_x_pairs(const uint16_t* __restrict__ xt, int d, int tid, int nthreads,
+                                              uint32_t* xs) {
+  uint16_t* xh = reinterpret_cast<uint16_t*>(xs);
+  const uint4* xv = reinterpret_cast<const uint4*>(xt);
+  for (int v = tid; v < 128 * 64 / 8; v += nthreads) {  // 8 values of one chunk per vector
+    const int i0 = v * 8, c = i0 >> 7, j0 = i0 & 127;
+    uint4 q = make_uint4(0u, 0u, 0u, 0u);
+    if (i0 < d) q = __ldg(xv + v);
+    const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      xh[((j0 + 2 * u) * 32 + (c & 31)) * 2 + (c >> 5)] = static_cast<uint16_t>(w4[u] & 0xFFFFu);
+      xh[((j0 + 2 * u + 1) * 32 + (c & 31)) * 2 + (c >> 5)] = static_cast<uint16_t>(w4[u] >> 16);
+    }
+  }
+}
+
+// Chunk partials of the exact-order logit of one expert: lane l runs the fma
+// chains of chunks l and l + 32 (each from +0, offsets j ascending), reading
+// its two chunks of Wc with one 8-byte load and of xs with one 4-byte load per
+// offset; 16 offsets of loads are issued before their fmas. FULL: d % 128 == 0.
+template <bool FULL>
+__device__ __forceinline__ void exact_chunk_pairs(const uint32_t* __restrict__ xs, const float2* __restrict__ wce,
+                                                  int d, int lane, float& p0, float& p1) {
+  const int n0 = FULL ? 128 : max(0, min(128, d - lane * 128));
+  const int n1 = FULL ? 128 : max(0, min(128, d - (lane + 32) * 128));
+  p0 = 0.0f;
+  p1 = 0.0f;
+  for (int j = 0; j < 128; j += 16) {
+    float2 w[16];
+    uint32_t xv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      w[u] = __ldg(wce + (j + u) * 32 + lane);
+      xv[u] = xs[(j + u) * 32 + lane];
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float xa = __uint_as_float(xv[u] << 16), xb = __uint_as_float(xv[u] & 0xFFFF0000u);
+      if (FULL || j + u < n0) p0 = __fmaf_rn(xa, w[u].x, p0);
+      if (FULL || j + u < n1) p1 = __fmaf_rn(xb, w[u].y, p1);
+    }
+  }
+}
+
+// Ordered sum of C chunk partials (ascending c), read from shared memory in
+// batches of 8.
+__device__ __forceinline__ float ordered_chunk_sum(const float* part, int C) {
+  float l = part[0];
+  for (int c0 = 1; c0 < C; c0 += 8) {
+    float pc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) pc[u] = part[min(c0 + u, 63)];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c0 + u < C) l = __fadd_rn(l, pc[u]);
+  }
+  return l;
+}
+
+// One CTA (4 warps) per token. A[t, :] holds the screened logits with the
+// bias already added (router_reduce_partials_kernel).
+//  1. warp 0: softmax statistics; candidates by descending A (ties -> lower
+//     index) up to the window A >= tau - 2 eps; warps 1-3 meanwhile stage x.
+//     A token whose window holds more than kMaxCand experts is appended to
+//     `overflow` and finished by router_fallback_kernel.
+//  2. all warps: exact-order logits of the candidates (candidate j by warp j % 4).
+//  3. warp 0: top-k over the candidates by (L desc, index asc); the softmax
+//     denominator uses L for the candidates and A for the other experts.
+template <int MAXV, bool FULL>
+__global__ void __launch_bounds__(kRcWarps * 32, 6)
     router_recheck_kernel(const float* __restrict__ A, const uint16_t* __restrict__ x, const float* __restrict__ Wc,
                           const float* __restrict__ bias, const float* __restrict__ xnorm,
                           const float* __restrict__ wnorm, int T, int d, int E, int k, int32_t* __restrict__ topk_idx,
-                          float* __restrict__ topk_w) {
-  constexpr int kChunk = 128;
-  extern __shared__ float xs[];  // [kChunk][C]: xs[j * C + c] = x[c * 128 + j] (0 past d)
-  __shared__ int s_cand[1024];
-  __shared__ float s_L[1024];
-  __shared__ float s_A[1024];
-  __shared__ float s_part[4][64];
+                          float* __restrict__ topk_w, int32_t* __restrict__ overflow) {
+  __shared__ uint32_t xs[kRcXsBytes / 4];
+  __shared__ float s_part[kRcWarps][64];
+  __shared__ int s_e[kMaxCand];
+  __shared__ float s_a[kMaxCand], s_l[kMaxCand];
   __shared__ int s_nc;
   __shared__ float s_m, s_s;
-
-  const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int C = (d + kChunk - 1) / kChunk;
-
-  for (int i = threadIdx.x; i < kChunk * C; i += blockDim.x) {
-    const int c = i / kChunk, j = i - c * kChunk;  // coalesced reads of x along i
-    const float v = (i < d) ? __uint_as_float(static_cast<uint32_t>(x[static_cast<int64_t>(t) * d + i]) << 16) : 0.0f;
-    xs[j * C + c] = v;
-  }
+  const int t = blockIdx.x;
+  const int C = (d + 127) / 128;
 
   if (warp == 0) {
     float v[MAXV];
-    float m = -INFINITY, amax = 0.0f;
+    float m = -INFINITY, amax = 0.0f, bmax = 0.0f;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i) {
       const int e = i * 32 + lane;
-      v[i] = (e < E) ? A[static_cast<int64_t>(t) * E + e] : -INFINITY;
-      if (e < E) {
+      v[i] = (e < E) ? __ldcs(A + static_cast<int64_t>(t) * E + e) : -INFINITY;
+    }
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      if (i * 32 + lane < E) {
         m = fmaxf(m, v[i]);
         amax = fmaxf(amax, fabsf(v[i]));
       }
     }
+    if (bias != nullptr)
+      for (int e = lane; e < E; e += 32) bmax = fmaxf(bmax, fabsf(__ldg(bias + e)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
     }
-    float s = 0.0f;
+    float ssum = 0.0f;
 #pragma unroll
     for (int i = 0; i < MAXV; ++i)
-      if (i * 32 + lane < E) s += expf(v[i] - m);
+      if (i * 32 + lane < E) ssum += expf(v[i] - m);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    float bmax = 0.0f;
-    if (bias != nullptr) {
-      for (int e = lane; e < E; e += 32) bmax = fmaxf(bmax, fabsf(__ldg(bias + e)));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
-    }
-    const float eps = kRtEpsRel * __ldg(xnorm + t) * __ldg(wnorm + E) + (amax + bmax + 1.0f) * (1.0f / 1048576.0f);
+    for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    const float eps =
+        kRtEpsRel * __ldg(xnorm + t) * __ldg(wnorm + E) + (amax + bmax + 1.0f) * (1.0f / 1048576.0f);
 
-    // extract by descending A (ties -> lower index) until past the window
     uint32_t taken = 0u;
     int nc = 0;
     float tau = 0.0f;
-    bool overflow = false;
     const int limit = (E <= kMaxCand) ? E : kMaxCand;
+    bool overflowed = false;
     while (true) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < MAXV; ++i) {
         const int e = i * 32 + lane;
-        if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv)) {
+        const bool cand = e < E && !((taken >> i) & 1u);
+        if (cand && (bi == 0x7fffffff || v[i] > bv)) {
           bv = v[i];
           bi = e;
         }
@@ -409,109 +473,151 @@ __global__ void __launch_bounds__(128)
       if (bi == 0x7fffffff) break;                  // every expert taken
       if (nc == k - 1) tau = bv;
       if (nc >= k && bv < tau - 2.0f * eps) break;  // outside the window
-      if (nc == limit) {
-        overflow = true;
+      if (nc == limit) {                            // window too wide: exact fallback
+        overflowed = true;
         break;
       }
       if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
       if (lane == 0) {
-        s_cand[nc] = bi;
-        s_A[nc] = bv;
+        s_e[nc] = bi;
+        s_a[nc] = bv;
       }
       ++nc;
     }
-    if (overflow) {  // recompute every expert of this token (exact, slow, rare)
-#pragma unroll
-      for (int i = 0; i < MAXV; ++i) {
-        const int e = i * 32 + lane;
-        if (e < E) {
-          s_cand[e] = e;
-          s_A[e] = v[i];
-        }
-      }
-      nc = E;
-    }
     if (lane == 0) {
+      if (overflowed) {
+        const int slot = atomicAdd(overflow, 1);
+        overflow[1 + slot] = t;
+        nc = 0;
+      }
       s_nc = nc;
       s_m = m;
-      s_s = s;
+      s_s = ssum;
     }
+  } else {
+    stage_x_pairs(x + static_cast<int64_t>(t) * d, d, threadIdx.x - 32, (kRcWarps - 1) * 32, xs);
+  }
+  __syncthreads();
+  const int nc = s_nc;
+  if (nc == 0) return;  // overflowed: finished by the fallback kernel
+
+  // 2. exact-order logits; candidates in ascending expert order across warps
+  //    would share L1 lines, but the list is short, so it is taken as extracted
+  for (int j = warp; j < nc; j += kRcWarps) {
+    const int e = s_e[j];
+    float p0, p1;
+    exact_chunk_pairs<FULL>(xs, reinterpret_cast<const float2*>(Wc + static_cast<int64_t>(e) * 128 * 64), d, lane, p0,
+                            p1);
+    s_part[warp][lane] = p0;
+    s_part[warp][lane + 32] = p1;
+    __syncwarp();
+    if (lane == 0) {
+      float l = ordered_chunk_sum(s_part[warp], C);
+      if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e));
+      s_l[j] = l;
+    }
+    __syncwarp();
   }
   __syncthreads();
 
-  const int nc = s_nc;
-  for (int j = warp; j < nc; j += 4) {
-    const int e = s_cand[j];
-    const float* wc = Wc + static_cast<int64_t>(e) * kChunk * C;
-    const int c0 = lane, c1 = lane + 32;
-    const int n0 = min(kChunk, d - c0 * kChunk), n1 = min(kChunk, d - c1 * kChunk);
-    float p0 = 0.0f, p1 = 0.0f;
-    if (c1 < C) {
-#pragma unroll 8
-      for (int i = 0; i < kChunk; ++i) {
-        const float w0 = __ldg(wc + i * C + c0), w1 = __ldg(wc + i * C + c1);
-        if (i < n0) p0 = __fmaf_rn(xs[i * C + c0], w0, p0);
-        if (i < n1) p1 = __fmaf_rn(xs[i * C + c1], w1, p1);
+  // 3. top-k by (L desc, index asc); denominator with exact L for candidates
+  if (warp == 0) {
+    const float m = s_m;
+    const bool mine = lane < nc;
+    const int my_e = mine ? s_e[lane] : 0x7fffffff;
+    const float my_l = mine ? s_l[lane] : -INFINITY;
+    float corr = mine ? (expf(my_l - m) - expf(s_a[lane] - m)) : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, o);
+    const float s = s_s + corr;
+    bool used = !mine;
+    for (int j = 0; j < k; ++j) {
+      float bv = used ? -INFINITY : my_l;
+      int bi = used ? 0x7fffffff : my_e;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+          bv = ov;
+          bi = oi;
+        }
       }
-    } else if (c0 < C) {
-#pragma unroll 8
-      for (int i = 0; i < kChunk; ++i) {
-        const float w0 = __ldg(wc + i * C + c0);
-        if (i < n0) p0 = __fmaf_rn(xs[i * C + c0], w0, p0);
+      if (!used && bi == my_e) used = true;
+      if (lane == 0) {
+        topk_idx[static_cast<int64_t>(t) * k + j] = bi;
+        topk_w[static_cast<int64_t>(t) * k + j] = expf(bv - m) / s;
       }
     }
-    if (c0 < C) s_part[warp][c0] = p0;
-    if (c1 < C) s_part[warp][c1] = p1;
+  }
+}
+
+// Tokens whose candidate window overflowed: every expert's exact-order logit,
+// then the top-k over all of them (exact softmax). One CTA (4 warps) per
+// listed token; the grid is an upper bound and blocks past the count return.
+__global__ void __launch_bounds__(128)
+    router_fallback_kernel(const int32_t* __restrict__ overflow, const uint16_t* __restrict__ x,
+                           const float* __restrict__ Wc, const float* __restrict__ bias, int d, int E, int k,
+                           int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  __shared__ uint32_t xs[128 * 32];
+  __shared__ float s_l[1024];
+  __shared__ float s_part[4][64];
+  if (static_cast<int>(blockIdx.x) >= overflow[0]) return;
+  const int t = overflow[1 + blockIdx.x];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = (d + 127) / 128;
+  stage_x_pairs(x + static_cast<int64_t>(t) * d, d, threadIdx.x, 128, xs);
+  __syncthreads();
+  for (int e = warp; e < E; e += 4) {
+    float p0, p1;
+    exact_chunk_pairs<false>(xs, reinterpret_cast<const float2*>(Wc + static_cast<int64_t>(e) * 128 * 64), d, lane, p0,
+                             p1);
+    s_part[warp][lane] = p0;
+    s_part[warp][lane + 32] = p1;
     __syncwarp();
     if (lane == 0) {
       float l = s_part[warp][0];
       for (int c = 1; c < C; ++c) l = __fadd_rn(l, s_part[warp][c]);
       if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e));
-      s_L[j] = l;
+      s_l[e] = l;
     }
     __syncwarp();
   }
   __syncthreads();
-
-  if (warp == 0) {
-    const float m = s_m;
-    // denominator: exact-order logits for the candidates, screened ones elsewhere
-    float corr = 0.0f;
-    for (int c = lane; c < nc; c += 32) corr += expf(s_L[c] - m) - expf(s_A[c] - m);
+  if (warp != 0) return;
+  float m = -INFINITY;
+  for (int e = lane; e < E; e += 32) m = fmaxf(m, s_l[e]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, o);
-    const float s = s_s + corr;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff, bslot = -1;
-      for (int c = lane; c < nc; c += 32) {
-        const int e = s_cand[c];
-        if (e < 0) continue;
-        const float L = s_L[c];
-        if (bi == 0x7fffffff || L > bv || (L == bv && e < bi)) {
-          bv = L;
-          bi = e;
-          bslot = c;
-        }
-      }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.0f;
+  for (int e = lane; e < E; e += 32) s += expf(s_l[e] - m);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
-        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-          bv = ov;
-          bi = oi;
-          bslot = os;
-        }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int e = lane; e < E; e += 32) {
+      const float l = s_l[e];
+      if (l != -INFINITY && (bi == 0x7fffffff || l > bv)) {  // ascending e per lane: first max wins ties
+        bv = l;
+        bi = e;
       }
-      if (lane == 0) {
-        topk_idx[static_cast<int64_t>(t) * k + j] = bi;
-        topk_w[static_cast<int64_t>(t) * k + j] = expf(bv - m) / s;
-        s_cand[bslot] = -1;  // taken
-      }
-      __syncwarp();
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (lane == 0) {
+      topk_idx[static_cast<int64_t>(t) * k + j] = bi;
+      topk_w[static_cast<int64_t>(t) * k + j] = expf(bv - m) / s;
+      s_l[bi] = -INFINITY;  // taken
+    }
+    __syncwarp();
   }
 }
 
