@@ -222,13 +222,30 @@ def barrier(world):
         dist.barrier()
 
 
+def _collective_device():
+    import torch.distributed as dist
+    return torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+
+
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's time (a timing reduction, not a data-path collective)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_collective_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_x_seed(rank: int) -> int:
+    """Seed of a replica's tokens: rank 0 uses the workload's seed 0, every other
+    rank its own stream, so replicas route different tokens (weak scaling)."""
+    return 0 if rank == 0 else 1000 + rank
+
+
+def aggregate_tokens_per_s(T: int, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * T * steps / (max_total_ms / 1e3)
 
 
 def run_ours(args):
@@ -241,7 +258,7 @@ def run_ours(args):
     log(f"[rank {rank}] generating {shape.name} on {dev}")
     inp = moe_inputs.make_inputs(shape, seed=0, device=dev)
     if rank != 0:  # each replica routes its own tokens
-        inp.x = moe_inputs.make_x(shape, seed=1000 + rank, device=dev)
+        inp.x = moe_inputs.make_x(shape, seed=replica_x_seed(rank), device=dev)
     T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
     ws = torch.empty(_lib.moe_forward_workspace_size(T, d, E, k, f), dtype=torch.uint8, device=dev)
     out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
@@ -317,8 +334,7 @@ def run_ours(args):
     if rank != 0:
         return None
     n = world
-    sec = total_ms / 1e3
-    value = n * T * args.steps / sec
+    value = aggregate_tokens_per_s(T, args.steps, n, total_ms)
     ms_per_step = total_ms / args.steps
     t_step = ms_per_step / 1e3
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -344,7 +360,7 @@ def run_ours(args):
                   "binding_roof": "hbm" if alg["B"] / hbm / 1e9 >= alg["F"] / tc / 1e12 else "tensor",
                   "tensor_frac_of_peak": alg["F"] / t_step / 1e12 / tc,
                   "stage_ms": {kname: statistics.mean(v) for kname, v in stage_ms.items()}},
-        "e2e": {"value": n * T * args.steps / (e2e_total / 1e3), "unit": UNIT,
+        "e2e": {"value": aggregate_tokens_per_s(T, args.steps, n, e2e_total), "unit": UNIT,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
