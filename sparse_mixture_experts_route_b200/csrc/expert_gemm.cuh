@@ -67,7 +67,8 @@ struct GemmCfg {
   static constexpr int kStages = (kMode == 0) ? 3 : 4;
   static constexpr int kTmemCols = 2 * kTmemSlotCols;            // 512
   static constexpr int kBarrierBytes = 256;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+  static constexpr int kTableBytes = 2 * (1024 + 1) * 4 + 8;  // shared copies of tile_prefix and expert_offsets
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + kTableBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
@@ -86,30 +87,32 @@ struct TileInfo {
   int e, nb, row0, nrows, nblocks;  // nblocks: token blocks of expert e
 };
 
+// Tile -> (expert, feature block, token block), from shared-memory copies of
+// the tile prefix (pre[0..E]) and the expert offsets (off[0..E]).
 template <int kMode>
-__device__ __forceinline__ bool decode_tile(const GemmParams& p, int tile, TileInfo& ti) {
+__device__ __forceinline__ bool decode_tile(const GemmParams& p, const int32_t* pre, const int32_t* off, int tile,
+                                            TileInfo& ti) {
   constexpr int BR = gemm_block_rows(kMode);
   const int NB = p.n_feat_tiles;
-  const int blocks_total = __ldg(p.tile_prefix + p.E);
-  if (tile >= blocks_total * NB) return false;
-  // owner: the largest e with tile_prefix[e] * NB <= tile
+  if (tile >= pre[p.E] * NB) return false;
+  // owner: the largest e with pre[e] * NB <= tile
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.tile_prefix + mid) * NB <= tile)
+    if (pre[mid] * NB <= tile)
       lo = mid;
     else
       hi = mid - 1;
   }
   const int e = lo;
-  const int tb_count = __ldg(p.tile_prefix + e + 1) - __ldg(p.tile_prefix + e);
-  const int local = tile - __ldg(p.tile_prefix + e) * NB;
+  const int tb_count = pre[e + 1] - pre[e];
+  const int local = tile - pre[e] * NB;
   const int tb = local % tb_count;
   ti.e = e;
   ti.nblocks = tb_count;
   ti.nb = local / tb_count;
-  ti.row0 = __ldg(p.expert_offsets + e) + tb * BR;
-  ti.nrows = min(BR, __ldg(p.expert_offsets + e + 1) - ti.row0);
+  ti.row0 = off[e] + tb * BR;
+  ti.nrows = min(BR, off[e + 1] - ti.row0);
   return true;
 }
 
@@ -153,10 +156,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain_bar = acc_empty_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_pre = reinterpret_cast<int32_t*>(smem + S * Cfg::kStageBytes + Cfg::kBarrierBytes);
+  int32_t* s_off = s_pre + (p.E + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int KB = p.K / kGemmBK;
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    s_pre[i] = __ldg(p.tile_prefix + i);
+    s_off[i] = __ldg(p.expert_offsets + i);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -199,7 +208,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int issued = 0;
       bool ok = true;
       TileInfo ti;
-      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, tile, ti); tile += gridDim.x) {
+      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
         const int f0 = ti.nb * (kMode == 0 ? kGemmBMF : 2 * kGemmBMF);
         const int f1 = f0 + p.a1_offset;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
@@ -254,7 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool any = false;
       TileInfo ti;
-      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, tile, ti); tile += gridDim.x) {
+      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
         const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
         const uint32_t idesc = umma_idesc_bf16_f32(128u, n_mma, 1u, 0u);
         const SlotPlan sp = slot_plan(ti.nrows, next_slot);
@@ -317,7 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int next_slot = 0;
     bool ok = true;
     TileInfo ti;
-    for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, tile, ti); tile += gridDim.x) {
+    for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
       const SlotPlan sp = slot_plan(ti.nrows, next_slot);
       for (int j = 0; j < sp.count && ok; ++j) {
         const int sl = sp.first + j;

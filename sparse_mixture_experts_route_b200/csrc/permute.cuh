@@ -118,16 +118,25 @@ __global__ void __launch_bounds__(32)
   }
 }
 
-// x_perm[row, :] = x[perm_token[row], :], 16-byte vectors, one warp per row.
+// x_perm[row, :] = x[perm_token[row], :], 16-byte vectors, one warp per row;
+// each lane keeps 4 loads in flight.
 __global__ void __launch_bounds__(256)
     permute_copy_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_token, int64_t n_rows,
                              int vec_per_row, uint4* __restrict__ x_perm) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= n_rows) return;
   const int lane = threadIdx.x & 31;
-  const int64_t src = static_cast<int64_t>(perm_token[row]) * vec_per_row;
-  const int64_t dst = row * vec_per_row;
-  for (int v = lane; v < vec_per_row; v += 32) x_perm[dst + v] = __ldg(x + src + v);
+  const uint4* src = x + static_cast<int64_t>(__ldg(perm_token + row)) * vec_per_row;
+  uint4* dst = x_perm + row * vec_per_row;
+  int v = lane;
+  for (; v + 96 < vec_per_row; v += 128) {
+    const uint4 a = __ldg(src + v), b = __ldg(src + v + 32), c = __ldg(src + v + 64), d = __ldg(src + v + 96);
+    __stcs(dst + v, a);
+    __stcs(dst + v + 32, b);
+    __stcs(dst + v + 64, c);
+    __stcs(dst + v + 96, d);
+  }
+  for (; v < vec_per_row; v += 32) __stcs(dst + v, __ldg(src + v));
 }
 
 // out[t, :] = sum_j w[t, j] * y_perm[inv_perm[t, j], :]; fp32 fma in ascending
