@@ -55,6 +55,10 @@ constexpr int kGemmBoxRows = 128;   // rows of the large B box
 constexpr int kGemmSmallBox = 32;   // rows of the small B box (tiles of <= 32 rows)
 constexpr int kTmemSlotCols = 256;
 
+// Modes: 0 gate/up with 256-row token blocks (3 stages of 64 KB), 2 gate/up
+// with 128-row token blocks (4 stages of 48 KB: more stages in flight when no
+// expert fills a 256-row block), 1 down (128-row blocks, 4 stages of 48 KB).
+__host__ __device__ constexpr bool gemm_is_gate_up(int mode) { return mode != 1; }
 __host__ __device__ constexpr int gemm_block_rows(int mode) { return mode == 0 ? 256 : 128; }
 
 template <int kMode>
@@ -62,7 +66,7 @@ struct GemmCfg {
   static constexpr int kABytes = kGemmBK * kGemmBMF * 2;         // 16 KB per A operand
   static constexpr int kAHalf = kABytes / 2;                     // one 64-feature box (8 KB)
   static constexpr int kBRows = gemm_block_rows(kMode);          // 256 / 128
-  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB / 16 KB
+  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB (mode 0) / 16 KB
   static constexpr int kStageBytes = 2 * kABytes + kBBytes;      // 64 KB / 48 KB
   static constexpr int kStages = (kMode == 0) ? 3 : 4;
   static constexpr int kTmemCols = 2 * kTmemSlotCols;            // 512
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       TileInfo ti;
       for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
-        const int f0 = ti.nb * (kMode == 0 ? kGemmBMF : 2 * kGemmBMF);
+        const int f0 = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF);
         const int f1 = f0 + p.a1_offset;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
         const bool small_box = ti.nrows <= kGemmSmallBox;
@@ -340,7 +344,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after_sync();
       const uint32_t t0 = tmem_base + lane_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
       const uint32_t t1 = t0 + (sp.count == 2 ? 256u : 128u);
-      const int fa = ti.nb * (kMode == 0 ? kGemmBMF : 2 * kGemmBMF) + q * 32 + lane;
+      const int fa = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF) + q * 32 + lane;
       const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
       const bool fa_ok = fa < p.n_feat;
       const bool fb_ok = (kMode == 1) && fb < p.n_feat;
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld_wait();
         uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + c0) * p.n_feat;
         const int nv = min(32, ti.nrows - c0);
-        if (kMode == 0) {
+        if (gemm_is_gate_up(kMode)) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             if (fa_ok && i < nv)
@@ -386,16 +390,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // Token blocks per expert for both GEMMs:
-//   prefix0[e] = sum_{e' < e} ceil(count_e' / 256)  (gate/up, 256-row blocks)
-//   prefix1[e] = sum_{e' < e} ceil(count_e' / 128)  (down, 128-row blocks)
+//   prefix0[e] = sum_{e' < e} ceil(count_e' / rows0)  (gate/up, rows0 = 256 or 128)
+//   prefix1[e] = sum_{e' < e} ceil(count_e' / 128)    (down)
 __global__ void __launch_bounds__(1024)
-    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int32_t* __restrict__ prefix0,
+    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int rows0, int32_t* __restrict__ prefix0,
                          int32_t* __restrict__ prefix1) {
   __shared__ int32_t warp_sums[2][32];
   const int e = threadIdx.x;
   const int32_t cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
-  const int32_t nb[2] = {(cnt + gemm_block_rows(0) - 1) / gemm_block_rows(0),
-                         (cnt + gemm_block_rows(1) - 1) / gemm_block_rows(1)};
+  const int32_t nb[2] = {(cnt + rows0 - 1) / rows0, (cnt + gemm_block_rows(1) - 1) / gemm_block_rows(1)};
   const int lane = e & 31, w = e >> 5;
   int32_t incl[2];
 #pragma unroll

@@ -49,7 +49,9 @@ moe_status_t device_setup(int* num_sms) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<0>::kSmemBytes) != cudaSuccess)
+                             GemmCfg<0>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<2>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<1>::kSmemBytes) != cudaSuccess)
@@ -304,6 +306,7 @@ struct FfnPlan {
   CUtensorMap mA0, mB0, mBs0, mA1, mB1, mBs1;
   GemmParams p0, p1;
   int grid0, grid1;
+  int mode0;  // 0: 256-row gate/up blocks, 2: 128-row gate/up blocks
 };
 
 moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
@@ -325,7 +328,9 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p0.n_feat_tiles = ceil_div(f, kGemmBMF);
   p0.a1_offset = f;
   p0.out = h;
-  const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(0)) + min_e_tk) * p0.n_feat_tiles;
+  // 256-row blocks pay off only when experts average more than 128 rows
+  fp->mode0 = (static_cast<int64_t>(Tk) > static_cast<int64_t>(E) * 128) ? 0 : 2;
+  const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(fp->mode0)) + min_e_tk) * p0.n_feat_tiles;
   fp->grid0 = static_cast<int>(tiles0 < num_sms ? tiles0 : num_sms);
   GemmParams& p1 = fp->p1;
   p1 = p0;
@@ -341,11 +346,15 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
 }
 
 void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
-  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, const_cast<int32_t*>(fp.p0.tile_prefix),
+  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, gemm_block_rows(fp.mode0),
+                                               const_cast<int32_t*>(fp.p0.tile_prefix),
                                                const_cast<int32_t*>(fp.p1.tile_prefix));
 }
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
-  grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
+  if (fp.mode0 == 0)
+    grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
+  else
+    grouped_gemm_kernel<2><<<fp.grid0, kGemmThreads, GemmCfg<2>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
 }
 void launch_gemm_down(const FfnPlan& fp, cudaStream_t stream) {
   grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);

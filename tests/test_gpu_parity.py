@@ -150,7 +150,8 @@ def _ffn_check(lib, inp, k):
 
 
 @pytest.mark.parametrize("shape", [(64, 128, 8, 2, 256), (333, 320, 20, 3, 192), (1, 256, 16, 4, 128),
-                                   (400, 128, 6, 2, 384)], ids=lambda s: "x".join(map(str, s)))
+                                   (400, 128, 6, 2, 384), (600, 128, 4, 2, 256)],
+                         ids=lambda s: "x".join(map(str, s)))
 def test_expert_ffn(lib, shape):
     T, d, E, k, f = shape
     _ffn_check(lib, _inputs(T, d, E, k, f), k)
@@ -183,7 +184,10 @@ def test_unpermute(lib):
     assert np.all(np.abs(parity.to_np64(out) - ref) <= bound)
 
 
-@pytest.mark.parametrize("shape", SHAPES + [(300, 128, 8, 2, 128)], ids=lambda s: "x".join(map(str, s)))
+# (600, 128, 4, 2, 128): about 300 rows per expert, so the gate/up GEMM takes
+# 256-row token blocks (N = 256 MMAs) with partial remainders
+@pytest.mark.parametrize("shape", SHAPES + [(300, 128, 8, 2, 128), (600, 128, 4, 2, 128)],
+                         ids=lambda s: "x".join(map(str, s)))
 def test_forward(lib, shape):
     T, d, E, k, f = shape
     inp = _inputs(T, d, E, k, f)
