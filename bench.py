@@ -362,7 +362,9 @@ def run_ours(args):
         "config": {**shape.as_dict(), "seed": 0, "parallelism": f"replicas{n}",
                    "l2": "flushed between steps (2x L2 write, then 2x L2 read, outside the step events)",
                    "weights_gb": round(E * 6.0 * d * f / 1e9, 3)},
-        "roofline": {"bound": "hbm", "kernel": "grouped_gemm_kernel<0> (gate/up + SwiGLU)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("grouped_gemm_kernel<0>" if T * k > 128 * E else "grouped_gemm_kernel<2>")
+                               + " (gate/up + SwiGLU)",
                      "achieved": gu_achieved, "peak": hbm, "unit": "GB/s", "frac": gu_achieved / hbm,
                      "traffic": traffic, "peak_source": f"{peak_src} hbm_gbs (burst copy)",
                      "alg_bytes_per_launch": alg["gu_bytes"], "ms_per_launch": gu_ms},
