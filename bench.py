@@ -300,6 +300,22 @@ def run_ours(args):
     for row in evs:
         for ev in row:
             ev.record(stream)
+    graph = None
+    if args.graph == "on":
+        # one step captured as a CUDA graph (the library never allocates or
+        # synchronises, so its launches capture as they are)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            _lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+            with torch.cuda.graph(graph, stream=side):
+                _lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            flush_l2(1)
+            graph.replay()
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
@@ -308,13 +324,28 @@ def run_ours(args):
     for s in range(args.steps):
         flush_l2(s)                               # L2 flush, outside the step's events
         evs[s][0].record(stream)
-        _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[s][2:], out, ws)
+        if graph is not None:
+            graph.replay()
+        else:
+            _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[s][2:], out, ws)
         evs[s][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     step_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
-    stage_ms = {name: [evs[s][2 + 2 * i].elapsed_time(evs[s][3 + 2 * i]) for s in range(args.steps)]
+    if graph is not None:
+        # per-kernel-group times (and the roofline kernel's duration) from a few
+        # eager timed steps: events cannot time nodes inside a graph replay
+        n_eager = min(args.steps, 5)
+        _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[0][2:], out, ws)
+        for s in range(n_eager):
+            flush_l2(s)
+            _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[s][2:], out, ws)
+        torch.cuda.synchronize()
+        stage_steps = range(n_eager)
+    else:
+        stage_steps = range(args.steps)
+    stage_ms = {name: [evs[s][2 + 2 * i].elapsed_time(evs[s][3 + 2 * i]) for s in stage_steps]
                 for i, name in enumerate(_lib.TIMED_STAGES)}
     total_ms = max_over_ranks(sum(step_ms), world)
     assert _lib.get_device_error() == 0, "device error during timing"
@@ -360,6 +391,7 @@ def run_ours(args):
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {**shape.as_dict(), "seed": 0, "parallelism": f"replicas{n}",
+                   "launch": "cuda_graph_replay" if graph is not None else "eager",
                    "l2": "flushed between steps (2x L2 write, then 2x L2 read, outside the step events)",
                    "weights_gb": round(E * 6.0 * d * f / 1e9, 3)},
         "roofline": {"bound": "hbm",
@@ -419,6 +451,8 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(moe_inputs.WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", default="on", choices=["on", "off"],
+                    help="time replays of one step captured as a CUDA graph (on) or eager calls (off)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

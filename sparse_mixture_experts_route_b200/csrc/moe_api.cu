@@ -234,15 +234,15 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
     }
   }
   if (plan.variant != kRouterFullBig) {
-    const int64_t n = static_cast<int64_t>(T) * E;
-    router_reduce_partials_kernel<<<static_cast<unsigned>(ceil_div64(n, 256)), 256, 0, stream>>>(
-        lg, plan.nchunks, bias, T, E);
+    // ordered sum of the chunk partials, bias, softmax and top-k: one block per token
+    router_reduce_topk_kernel<<<T, 256, 0, stream>>>(lg, plan.nchunks, bias, T, E, k, idx, w);
+  } else {
+    const int blocks = ceil_div(T, 8);
+    if (E <= 256)
+      router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
+    else
+      router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
   }
-  const int blocks = ceil_div(T, 8);
-  if (E <= 256)
-    router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
-  else
-    router_topk_kernel<32><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -549,9 +549,18 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
   if (st != MOE_OK) return st;
   mark(1);
   mark(2);
-  st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, x_perm, ws + L.perm_ws, stream);
-  if (st != MOE_OK) return st;
-  launch_schedule(fp, stream);
+  if (Tk <= kSmallDispatchPairs) {
+    // one block: counts, offsets, stable scatter and both GEMM tile prefixes; then the row copy
+    dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, gemm_block_rows(fp.mode0), offsets, perm_token,
+                                                  inv_perm, const_cast<int32_t*>(fp.p0.tile_prefix),
+                                                  const_cast<int32_t*>(fp.p1.tile_prefix));
+    permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(x), perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
+  } else {
+    st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, x_perm, ws + L.perm_ws, stream);
+    if (st != MOE_OK) return st;
+    launch_schedule(fp, stream);
+  }
   mark(3);
   mark(4);
   launch_gemm_gate_up(fp, stream);

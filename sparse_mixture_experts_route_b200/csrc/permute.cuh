@@ -181,3 +181,89 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace moe
+
+namespace moe {
+
+constexpr int kSmallDispatchPairs = 2048;  // fused single-block dispatch up to this many (token, slot) pairs
+
+// Dispatch for few pairs in one block of 1024 threads (E <= 1024): per-expert
+// counts, exclusive scan (offsets), the stable counting-sort scatter (one warp
+// walks the pairs in order, 32 at a time, ranks from __match_any_sync), and the
+// token-block prefixes of both grouped GEMMs (blocks of rows0 and of 128 rows),
+// so a decode step needs one launch here instead of four.
+__global__ void __launch_bounds__(1024)
+    dispatch_small_kernel(const int32_t* __restrict__ topk_idx, int n_pairs, int E, int k, int rows0,
+                          int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm,
+                          int32_t* __restrict__ prefix0, int32_t* __restrict__ prefix1) {
+  __shared__ int32_t cnt[1024];
+  __shared__ int32_t base[1024];
+  __shared__ int32_t wsum[3][32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  cnt[tid] = 0;
+  __syncthreads();
+  for (int q = tid; q < n_pairs; q += 1024) {
+    const int e = topk_idx[q];
+    if (e >= 0 && e < E)
+      atomicAdd(&cnt[e], 1);
+    else
+      record_device_error(5u /* MOE_DEVERR_BAD_ROUTE */);
+  }
+  __syncthreads();
+  // exclusive scans over experts: rows, 128-row blocks and rows0-row blocks
+  const int32_t c = (tid < E) ? cnt[tid] : 0;
+  int32_t v[3] = {c, (c + rows0 - 1) / rows0, (c + 127) / 128};
+  int32_t incl[3];
+#pragma unroll
+  for (int m = 0; m < 3; ++m) {
+    incl[m] = v[m];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl[m], o);
+      if (lane >= o) incl[m] += y;
+    }
+    if (lane == 31) wsum[m][w] = incl[m];
+  }
+  __syncthreads();
+  if (w < 3) {
+    const int32_t ws = wsum[w][lane];
+    int32_t wi = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    wsum[w][lane] = wi - ws;
+  }
+  __syncthreads();
+  if (tid < E) {
+    int32_t* outs[3] = {offsets, prefix0, prefix1};
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const int32_t excl = wsum[m][w] + incl[m] - v[m];
+      outs[m][tid] = excl;
+      if (tid == E - 1) outs[m][E] = excl + v[m];
+      if (m == 0) base[tid] = excl;
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    for (int g = 0; g < n_pairs; g += 32) {
+      const int q = g + lane;
+      int e = (q < n_pairs) ? topk_idx[q] : -1;
+      if (q < n_pairs && (e < 0 || e >= E)) e = -2;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      int32_t row = 0;
+      if (e >= 0) row = base[e] + rank;
+      __syncwarp();
+      if (e >= 0 && rank == 0) base[e] += __popc(peers);
+      __syncwarp();
+      if (e >= 0) {
+        perm_token[row] = q / k;
+        inv_perm[q] = row;
+      }
+    }
+  }
+}
+
+}  // namespace moe

@@ -247,3 +247,157 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// Small-T router, second half, one block of 256 threads per token:
+//  1. thread i owns experts i, i + 256, ...: l = plane 0 + plane 1 + ... (in
+//     ascending chunk order) + bias, kept in shared memory;
+//  2. warp w takes the experts e with (e / 32) % 8 == w: softmax partials (its
+//     own max and sum) and its local top-k by (logit desc, index asc);
+//  3. warp 0 merges the 8 local lists (k rounds of warp arg-max) and rescales
+//     the partial sums to the global max, in warp order.
+__global__ void __launch_bounds__(256)
+    router_reduce_topk_kernel(const float* __restrict__ lg, int nsplit, const float* __restrict__ bias, int T, int E,
+                              int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  __shared__ float s_l[1024];
+  __shared__ float s_cv[8][16];
+  __shared__ int s_ci[8][16];
+  __shared__ float s_wm[8], s_ws[8];
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int64_t n = static_cast<int64_t>(T) * E;
+  // 1. ordered sums of the chunk partials
+  float acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + 256 * i;
+    acc[i] = (e < E) ? __ldcs(lg + static_cast<int64_t>(t) * E + e) : 0.0f;
+  }
+  for (int c0 = 1; c0 < nsplit; c0 += 8) {
+    float p[8][4];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = tid + 256 * i;
+        p[u][i] = (c0 + u < nsplit && e < E) ? __ldcs(lg + (c0 + u) * n + static_cast<int64_t>(t) * E + e) : 0.0f;
+      }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (c0 + u < nsplit) acc[i] = __fadd_rn(acc[i], p[u][i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + 256 * i;
+    if (e < E) s_l[e] = (bias != nullptr) ? __fadd_rn(acc[i], __ldg(bias + e)) : acc[i];
+  }
+  __syncthreads();
+
+  // 2. per-warp softmax partials and local top-k over experts e = 256 i + 32 w + lane
+  float v[4];
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 256 * i + 32 * w + lane;
+    v[i] = (e < E) ? s_l[e] : -INFINITY;
+    m = fmaxf(m, v[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (256 * i + 32 * w + lane < E) s += expf(v[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) {
+    s_wm[w] = m;
+    s_ws[w] = s;
+  }
+  uint32_t taken = 0u;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 256 * i + 32 * w + lane;
+      if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi != 0x7fffffff && ((bi & 31) == lane) && (((bi >> 5) & 7) == w)) taken |= 1u << (bi >> 8);
+    if (lane == 0) {
+      s_cv[w][j] = bv;
+      s_ci[w][j] = bi;
+    }
+  }
+  __syncthreads();
+
+  // 3. merge
+  if (w == 0) {
+    float gm = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) gm = fmaxf(gm, s_wm[q]);
+    float gs = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (s_wm[q] != -INFINITY) gs += s_ws[q] * expf(s_wm[q] - gm);
+    // candidates: lane holds entries lane, lane + 32, ... of the 8 x k list
+    float cv[4];
+    int ci[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int slot = lane + 32 * r;
+      const int q = slot / 16, j = slot % 16;
+      const bool ok = q < 8 && j < k;
+      cv[r] = ok ? s_cv[q][j] : -INFINITY;
+      ci[r] = ok ? s_ci[q][j] : 0x7fffffff;
+    }
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff, br = -1;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (ci[r] != 0x7fffffff && (bi == 0x7fffffff || cv[r] > bv || (cv[r] == bv && ci[r] < bi))) {
+          bv = cv[r];
+          bi = ci[r];
+          br = r;
+        }
+      int wb = bi;
+      float wv = bv;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, wb, o);
+        if (oi != 0x7fffffff && (wb == 0x7fffffff || ov > wv || (ov == wv && oi < wb))) {
+          wv = ov;
+          wb = oi;
+        }
+      }
+      if (br >= 0 && bi == wb) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          if (r == br) ci[r] = 0x7fffffff;  // taken
+      }
+      if (lane == 0) {
+        topk_idx[static_cast<int64_t>(t) * k + j] = wb;
+        topk_w[static_cast<int64_t>(t) * k + j] = expf(wv - gm) / gs;
+      }
+    }
+  }
+}
+
+}  // namespace moe
