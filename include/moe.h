@@ -171,6 +171,32 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const
                                void* workspace, size_t workspace_bytes, cudaStream_t stream,
                                cudaEvent_t* events);
 
+/* moe_forward_host: moe_forward with x and out in HOST memory -- the call a
+ * host program makes when its activations live on the CPU side. On `stream`,
+ * in this order: one cudaMemcpyAsync of x_host [T, d] bf16 into a staging
+ * buffer at the start of `workspace`, the whole pass (exactly the kernels of
+ * moe_forward), and one cudaMemcpyAsync of the result into out_host [T, d].
+ * Returns once that work is enqueued; out_host holds the result when `stream`
+ * has run it (synchronise the stream, or an event recorded after the call).
+ * x_host must stay unchanged until then.
+ * x_host and out_host should be page-locked (cudaHostAlloc/cudaHostRegister):
+ * then the copies run asynchronously, and calls on two streams with two
+ * workspaces overlap one call's copies with the other's kernels. Pageable
+ * buffers work too, but the copies then run synchronously with the host.
+ * Weights (and the bias) are device pointers, as in moe_forward.
+ * Workspace: moe_forward_host_workspace_size(T, d, E, k, f) bytes, 256-byte
+ * aligned = two [T, d] bf16 staging buffers (each rounded up to 256 bytes)
+ * followed by moe_forward's workspace.
+ * Errors: as moe_forward; a device (or managed) pointer for x_host or
+ * out_host is MOE_ERR_INVALID_ARG, a failed copy is MOE_ERR_CUDA.
+ */
+size_t moe_forward_host_workspace_size(int T, int d, int E, int k, int f);
+moe_status_t moe_forward_host(const moe_bf16_t* x_host, const float* W_router, const float* router_bias,
+                              const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down,
+                              int T, int d, int E, int k, int f,
+                              moe_bf16_t* out_host,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------- allocation-free router --
  * moe_route_noalloc: moe_route for callers that cannot allocate device memory
  * -- for example code running inside a host framework that owns every device

@@ -86,9 +86,12 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def _workspace(nbytes: int, device) -> torch.Tensor:
+def _workspace(nbytes: int, device, stream=None) -> torch.Tensor:
     # torch's caching allocator returns 512-byte aligned blocks
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    if stream is not None:
+        ws.record_stream(stream)  # not reused before `stream` has finished with it
+    return ws
 
 
 def version() -> int:
@@ -121,7 +124,7 @@ def moe_route(x, W_router, router_bias, k: int, workspace=None, stream=None):
         _need(router_bias, "router_bias", torch.float32, (E,))
     idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
     w = torch.empty(T, k, dtype=torch.float32, device=x.device)
-    ws = workspace if workspace is not None else _workspace(route_workspace_size(T, d, E), x.device)
+    ws = workspace if workspace is not None else _workspace(route_workspace_size(T, d, E), x.device, stream)
     _check(_lib.moe_route(_ptr(x), _ptr(W_router), _ptr(router_bias), T, d, E, k, _ptr(idx), _ptr(w),
                           _ptr(ws), ws.numel(), _stream(stream)), "moe_route")
     return idx, w
@@ -139,7 +142,7 @@ def moe_permute(x, topk_idx, E: int, with_rows: bool = True, workspace=None, str
     perm_token = torch.empty(T * k, dtype=torch.int32, device=dev)
     inv_perm = torch.empty(T, k, dtype=torch.int32, device=dev)
     x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device=dev) if (with_rows and x is not None) else None
-    ws = workspace if workspace is not None else _workspace(permute_workspace_size(T, E, k), dev)
+    ws = workspace if workspace is not None else _workspace(permute_workspace_size(T, E, k), dev, stream)
     _check(_lib.moe_permute(_ptr(x), _ptr(topk_idx), T, d, E, k, _ptr(offsets), _ptr(perm_token), _ptr(inv_perm),
                             _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
     return offsets, perm_token, inv_perm, x_perm
@@ -156,7 +159,7 @@ def moe_expert_ffn(x_perm, expert_offsets, W_gate_up, W_down, workspace=None, st
     _need(W_down, "W_down", torch.bfloat16, (E, f, d))
     h = torch.empty(Tk, f, dtype=torch.bfloat16, device=x_perm.device)
     y = torch.empty(Tk, d, dtype=torch.bfloat16, device=x_perm.device)
-    ws = workspace if workspace is not None else _workspace(expert_ffn_workspace_size(Tk, E), x_perm.device)
+    ws = workspace if workspace is not None else _workspace(expert_ffn_workspace_size(Tk, E), x_perm.device, stream)
     _check(_lib.moe_expert_ffn(_ptr(x_perm), _ptr(expert_offsets), _ptr(W_gate_up), _ptr(W_down), Tk, d, E, f,
                                _ptr(h), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)), "moe_expert_ffn")
     return h, y
@@ -191,10 +194,55 @@ def moe_forward(x, W_router, router_bias, W_gate_up, W_down, k: int, out=None, w
     if out is None:
         out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
     _need(out, "out", torch.bfloat16, (T, d))
-    ws = workspace if workspace is not None else _workspace(moe_forward_workspace_size(T, d, E, k, f), x.device)
+    ws = workspace if workspace is not None else _workspace(moe_forward_workspace_size(T, d, E, k, f), x.device, stream)
     _check(_lib.moe_forward(_ptr(x), _ptr(W_router), _ptr(router_bias), _ptr(W_gate_up), _ptr(W_down),
                             T, d, E, k, f, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)), "moe_forward")
     return out
+
+
+_lib.moe_forward_host_workspace_size.argtypes = [I, I, I, I, I]
+_lib.moe_forward_host_workspace_size.restype = Z
+_lib.moe_forward_host.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P]
+_lib.moe_forward_host.restype = I
+
+
+def moe_forward_host_workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
+    return int(_lib.moe_forward_host_workspace_size(T, d, E, k, f))
+
+
+def _need_host(t: torch.Tensor, name: str, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be in host memory")
+    if t.dtype != torch.bfloat16 or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 tensor of shape {tuple(shape)}")
+
+
+def moe_forward_host(x_host, W_router, router_bias, W_gate_up, W_down, k: int, out_host=None, workspace=None,
+                     stream=None):
+    """The whole layer with x and the result in host memory: the library copies
+    x in, runs the pass and copies the result back, all on ``stream``.
+    out_host holds the result once the stream has run the call (pin both host
+    tensors for asynchronous copies)."""
+    T, d = x_host.shape
+    E = W_router.shape[1]
+    f = W_down.shape[1]
+    _need_host(x_host, "x_host", (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    _need(W_gate_up, "W_gate_up", torch.bfloat16, (E, d, 2 * f))
+    _need(W_down, "W_down", torch.bfloat16, (E, f, d))
+    if out_host is None:
+        out_host = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    _need_host(out_host, "out_host", (T, d))
+    ws = workspace if workspace is not None else _workspace(moe_forward_host_workspace_size(T, d, E, k, f),
+                                                             W_router.device, stream)
+    _check(_lib.moe_forward_host(_ptr(x_host), _ptr(W_router), _ptr(router_bias), _ptr(W_gate_up), _ptr(W_down),
+                                 T, d, E, k, f, _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_forward_host")
+    return out_host
 
 
 def get_device_error(clear: bool = True) -> int:

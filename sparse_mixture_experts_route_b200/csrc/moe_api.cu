@@ -595,6 +595,40 @@ moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const
                       stream, events);
 }
 
+size_t moe_forward_host_workspace_size(int T, int d, int E, int k, int f) {
+  const size_t fw = moe_forward_workspace_size(T, d, E, k, f);
+  if (fw == 0) return 0;
+  return 2 * align256(static_cast<size_t>(T) * d * sizeof(moe_bf16_t)) + fw;
+}
+
+moe_status_t moe_forward_host(const moe_bf16_t* x_host, const float* W_router, const float* router_bias,
+                              const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, int T, int d, int E, int k,
+                              int f, moe_bf16_t* out_host, void* workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+  if (!x_host || !W_router || !W_gate_up || !W_down || !out_host) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, d, E, k) || f < 64 || f % 64 || f > 32768) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  const size_t stage = align256(static_cast<size_t>(T) * d * sizeof(moe_bf16_t));
+  const size_t need = moe_forward_host_workspace_size(T, d, E, k, f);
+  if (!workspace || !aligned256(workspace) || workspace_bytes < need) return MOE_ERR_WORKSPACE;
+  // x and out must be host memory (pageable or page-locked), never device memory
+  for (const void* hp : {static_cast<const void*>(x_host), static_cast<const void*>(out_host)}) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, hp) != cudaSuccess) return MOE_ERR_CUDA;
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return MOE_ERR_INVALID_ARG;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  moe_bf16_t* x_dev = reinterpret_cast<moe_bf16_t*>(ws);
+  moe_bf16_t* out_dev = reinterpret_cast<moe_bf16_t*>(ws + stage);
+  const size_t bytes = static_cast<size_t>(T) * d * sizeof(moe_bf16_t);
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const moe_status_t st = forward_impl(x_dev, W_router, router_bias, W_gate_up, W_down, T, d, E, k, f, out_dev,
+                                       ws + 2 * stage, workspace_bytes - 2 * stage, stream, nullptr);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 }  // extern "C"
 
 // ------------------------------------------------ allocation-free router scratch

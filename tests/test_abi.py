@@ -69,6 +69,9 @@ def _setup(lib):
     lib.moe_unpermute.argtypes = [P, P, P, I, I, I, P, P]
     lib.moe_forward.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P]
     lib.moe_selftest_wait_timeout.argtypes = [I, P]
+    lib.moe_forward_host_workspace_size.restype = Z
+    lib.moe_forward_host_workspace_size.argtypes = [I, I, I, I, I]
+    lib.moe_forward_host.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P]
     return lib
 
 
@@ -135,3 +138,23 @@ def test_other_argument_checks(lib):
     assert lib.moe_forward(p, p, None, p, p, 64, 128, 8, 2, 256, p, p, fw - 256, None) == 3
     assert lib.moe_selftest_wait_timeout(0, None) == 1
     assert lib.moe_selftest_wait_timeout(2_000_000, None) == 1
+
+
+def test_host_buffer_forward_checks(lib):
+    """moe_forward_host: two 256-byte-rounded [T, d] bf16 staging buffers ahead
+    of moe_forward's workspace; bad arguments are refused before any CUDA call."""
+    lib = _setup(lib)
+    for (T, d, E, k, f) in [(64, 128, 8, 2, 256), (4096, 7168, 384, 8, 2048), (3, 64, 8, 2, 64)]:
+        stage = -(-T * d * 2 // 256) * 256
+        assert lib.moe_forward_host_workspace_size(T, d, E, k, f) == 2 * stage + lib.moe_forward_workspace_size(
+            T, d, E, k, f)
+    assert lib.moe_forward_host_workspace_size(0, 128, 8, 2, 256) == 0
+    p = ctypes.c_void_p(FAKE)
+    hw = lib.moe_forward_host_workspace_size(64, 128, 8, 2, 256)
+    assert lib.moe_forward_host(None, p, None, p, p, 64, 128, 8, 2, 256, p, p, hw, None) == 1    # no x
+    assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 2, 256, None, p, hw, None) == 1    # no out
+    assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 2, 250, p, p, hw, None) == 1       # f % 64
+    assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 17, 256, p, p, hw, None) == 1      # k > E
+    assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 32, 17, 256, p, p, 1 << 30, None) == 2  # k > 16
+    assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 2, 256, p, p, hw - 256, None) == 3
+    assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 2, 256, p, ctypes.c_void_p(FAKE + 8), hw, None) == 3

@@ -211,6 +211,34 @@ def test_forward_zipf_bias(lib):
     parity.assert_layer_close(out, ref, "forward zipf")
 
 
+@pytest.mark.parametrize("shape", [(333, 320, 20, 3, 192), (600, 128, 4, 2, 128)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_forward_host_buffers(lib, shape):
+    """moe_forward_host: x and out in pinned host memory, copies inside the
+    call; same bits as moe_forward, and within tolerance of the oracle.
+    Two calls on two streams with their own workspaces give the same result."""
+    T, d, E, k, f = shape
+    inp = _inputs(T, d, E, k, f, bias="zipf")
+    g = _cuda(inp)
+    x_host = g.x.cpu().pin_memory()
+    dev = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k)
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    outs = [lib.moe_forward_host(x_host, g.W_router, g.bias, g.W_gate_up, g.W_down, k, stream=st) for st in streams]
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    for o in outs:
+        assert o.device.type == "cpu" and torch.equal(o, dev.cpu())
+    ref, _, _ = oracle.forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(outs[0], ref, "forward host buffers")
+    # a device pointer where host memory is required is refused
+    with pytest.raises(lib.MoEError):
+        ws = torch.empty(lib.moe_forward_host_workspace_size(T, d, E, k, f), dtype=torch.uint8, device="cuda")
+        st = lib.raw.moe_forward_host(g.x.data_ptr(), g.W_router.data_ptr(), None, g.W_gate_up.data_ptr(),
+                                      g.W_down.data_ptr(), T, d, E, k, f, outs[0].data_ptr(), ws.data_ptr(),
+                                      ws.numel(), None)
+        lib._check(st, "moe_forward_host")
+
+
 def test_bounded_wait_reports_instead_of_hanging(lib):
     assert lib.get_device_error(clear=True) == 0
     lib.selftest_wait_timeout(2000)  # 2 ms on a barrier nothing signals
