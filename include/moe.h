@@ -237,6 +237,7 @@ moe_status_t moe_route_noalloc(const moe_bf16_t* x, const float* W_router, const
 #define MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE 3u /* epilogue gave up waiting for an accumulator */
 #define MOE_DEVERR_SELFTEST_TIMEOUT 4u      /* moe_selftest_wait_timeout fired as intended */
 #define MOE_DEVERR_BAD_ROUTE 5u             /* an expert index outside [0, E) reached the dispatch */
+#define MOE_DEVERR_WAIT_TIMEOUT_ROUTER 6u   /* few-token router gave up waiting for its W tile */
 moe_status_t moe_get_device_error(uint32_t* code, int clear);
 
 /* moe_selftest_wait_timeout: launches one tiny kernel that waits, with a

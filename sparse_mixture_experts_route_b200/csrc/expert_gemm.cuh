@@ -85,10 +85,24 @@ struct GemmParams {
   int n_feat_tiles;  // mode 0: ceil(f / 128); mode 1: ceil(d / 256)
   int a1_offset;     // column of the second A operand: f + j0 (mode 0) or n0 + 128 (mode 1), minus j0 / n0
   uint16_t* out;     // [Tk, n_feat] bf16
+  // K split (mode 2 only; ksplit == 1 elsewhere): output tile t is computed as
+  // ksplit partial products over K blocks [s * kb_per_split, ...), written to
+  // part[t][s] as fp32; for each 32-feature slice, the last of the ksplit
+  // CTAs to finish it (a ticket) adds them in ascending s and applies the
+  // SiLU-gate. tickets[] start at zero and
+  // are put back to zero.
+  int ksplit;
+  int kb_per_split;
+  float* part;            // [tiles][ksplit][2][128 rows][128 features] fp32
+  unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
 };
+
+// fp32 elements of one split partial: gate and up, 128 rows x 128 features
+constexpr int kSplitPartFloats = 2 * 128 * kGemmBMF;
 
 struct TileInfo {
   int e, nb, row0, nrows, nblocks;  // nblocks: token blocks of expert e
+  int bt, ks, kb0, kb1;             // output tile, K split, K-block range [kb0, kb1)
 };
 
 // Tile -> (expert, feature block, token block), from shared-memory copies of
@@ -98,25 +112,32 @@ __device__ __forceinline__ bool decode_tile(const GemmParams& p, const int32_t* 
                                             TileInfo& ti) {
   constexpr int BR = gemm_block_rows(kMode);
   const int NB = p.n_feat_tiles;
-  if (tile >= pre[p.E] * NB) return false;
-  // owner: the largest e with pre[e] * NB <= tile
+  // consecutive tiles are the K splits of one output tile
+  const int bt = tile / p.ksplit;
+  const int ks = tile - bt * p.ksplit;
+  if (bt >= pre[p.E] * NB) return false;
+  // owner: the largest e with pre[e] * NB <= bt
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (pre[mid] * NB <= tile)
+    if (pre[mid] * NB <= bt)
       lo = mid;
     else
       hi = mid - 1;
   }
   const int e = lo;
   const int tb_count = pre[e + 1] - pre[e];
-  const int local = tile - pre[e] * NB;
+  const int local = bt - pre[e] * NB;
   const int tb = local % tb_count;
   ti.e = e;
   ti.nblocks = tb_count;
   ti.nb = local / tb_count;
   ti.row0 = off[e] + tb * BR;
   ti.nrows = min(BR, off[e + 1] - ti.row0);
+  ti.bt = bt;
+  ti.ks = ks;
+  ti.kb0 = ks * p.kb_per_split;
+  ti.kb1 = min(p.K / kGemmBK, ti.kb0 + p.kb_per_split);
   return true;
 }
 
@@ -165,7 +186,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int KB = p.K / kGemmBK;
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
     s_pre[i] = __ldg(p.tile_prefix + i);
     s_off[i] = __ldg(p.expert_offsets + i);
@@ -219,7 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool small_box = ti.nrows <= kGemmSmallBox;
         const int nbox = small_box ? 1 : (ti.nrows + kGemmBoxRows - 1) / kGemmBoxRows;
         const uint32_t b_bytes = small_box ? kGemmSmallBox * kGemmBK * 2 : nbox * kGemmBoxRows * kGemmBK * 2;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
             *abort_flag = 1;
@@ -284,7 +304,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // accumulator 0 at the slot start; accumulator 1 after N columns (128 or 256)
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
         const uint32_t d1 = d0 + (sp.count == 2 ? 256u : 128u);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
             record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
             *abort_flag = 1;
@@ -299,7 +319,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
             const uint64_t adesc0 = umma_smem_desc_sw128(a_addr + kk * 2048, Cfg::kAHalf, 1024);
             const uint64_t adesc1 = umma_smem_desc_sw128(a_addr + Cfg::kABytes + kk * 2048, Cfg::kAHalf, 1024);
-            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
             tc_mma_bf16(d0, adesc0, bdesc, idesc, accum);
             tc_mma_bf16(d1, adesc1, bdesc, idesc, accum);
           }
@@ -348,6 +368,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
       const bool fa_ok = fa < p.n_feat;
       const bool fb_ok = (kMode == 1) && fb < p.n_feat;
+      if (kMode == 2 && p.ksplit > 1) {
+        // K split: this CTA's fp32 partial to part[bt][ks]; the slot is free
+        // as soon as it is read
+        const int fl = q * 32 + lane;
+        float* mine = p.part + (static_cast<int64_t>(ti.bt) * p.ksplit + ti.ks) * kSplitPartFloats;
+        for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
+          tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
+          tmem_ld_wait();
+          const int nv = min(32, ti.nrows - c0);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i < nv) {
+              __stcg(mine + (c0 + i) * kGemmBMF + fl, __uint_as_float(g[i]));
+              __stcg(mine + (128 + c0 + i) * kGemmBMF + fl, __uint_as_float(u[i]));
+            }
+          }
+        }
+        tc_fence_before_sync();
+        __syncwarp();
+        for (int j = 0; j < sp.count; ++j) {
+          if (lane == 0) mbar_arrive(&acc_empty_bar[sp.first + j]);
+          ++uses[sp.first + j];
+        }
+        // ticket per (output tile, warp): the last split to finish these 32
+        // features adds the partials in ascending split order
+        __threadfence();
+        __syncwarp();
+        unsigned int tk = 0u;
+        if (lane == 0) tk = atomicAdd(&p.tickets[ti.bt * 4 + q], 1u);
+        tk = __shfl_sync(0xffffffffu, tk, 0);
+        if (tk == static_cast<unsigned int>(p.ksplit - 1)) {
+          __threadfence();
+          const float* all = p.part + static_cast<int64_t>(ti.bt) * p.ksplit * kSplitPartFloats;
+          for (int i = 0; i < ti.nrows; ++i) {
+            float gs = __ldcg(all + i * kGemmBMF + fl);
+            float us = __ldcg(all + (128 + i) * kGemmBMF + fl);
+            for (int sk = 1; sk < p.ksplit; ++sk) {
+              gs = __fadd_rn(gs, __ldcg(all + sk * kSplitPartFloats + i * kGemmBMF + fl));
+              us = __fadd_rn(us, __ldcg(all + sk * kSplitPartFloats + (128 + i) * kGemmBMF + fl));
+            }
+            if (fa_ok)
+              p.out[static_cast<int64_t>(ti.row0 + i) * p.n_feat + fa] = bf16_bits(silu_f32(gs) * us);
+          }
+          if (lane == 0) p.tickets[ti.bt * 4 + q] = 0u;
+        }
+        continue;
+      }
       for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
         uint32_t g[32], u[32];
         tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);

@@ -17,6 +17,7 @@
 #include "permute.cuh"
 #include "ptx.cuh"
 #include "router.cuh"
+#include "router_stream.cuh"
 #include "router_tc.cuh"
 
 namespace {
@@ -56,6 +57,13 @@ moe_status_t device_setup(int* num_sms) {
     if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<1>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(router_stream_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             router_stream_smem_bytes(1)) != cudaSuccess ||
+        cudaFuncSetAttribute(router_stream_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             router_stream_smem_bytes(4)) != cudaSuccess ||
+        cudaFuncSetAttribute(router_stream_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             router_stream_smem_bytes(16)) != cudaSuccess)
+      return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(router_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScrSmemBytes) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
@@ -85,7 +93,8 @@ enum RouterVariant {
   kRouterSplitBig = 1,
   kRouterSplitSmall = 2,
   kRouterSplitTiny = 3,
-  kRouterTensorCore = 4
+  kRouterTensorCore = 4,
+  kRouterStream = 5
 };
 
 // Tokens from which the tensor-core screen + exact re-check router is used.
@@ -99,6 +108,8 @@ struct RoutePlan {
   int nsplit = 1, kb_per_split = 0, nparts = 0;
   size_t off_A = 0, off_wt32 = 0, off_hi = 0, off_lo = 0, off_part = 0, off_wnorm = 0, off_xnorm = 0, off_xc = 0,
          off_ovf = 0;
+  // few-token variant: chunk partials, final logits, tickets
+  size_t off_logits = 0, off_tickets = 0;
 };
 
 RoutePlan route_plan(int T, int d, int E) {
@@ -131,6 +142,18 @@ RoutePlan route_plan(int T, int d, int E) {
     p.off_wnorm = take(static_cast<size_t>(E + 1) * 4);
     p.off_xnorm = take(static_cast<size_t>(T) * 4);
     p.off_ovf = take(static_cast<size_t>(T + 1) * 4);
+    p.ws_bytes = at;
+    return p;
+  }
+  if (T <= kRsMaxTokens && E % 4 == 0) {
+    // one launch: every chunk of W_router in flight at once, reductions by the last CTAs
+    p.variant = kRouterStream;
+    const int G = ceil_div(E, kRsExperts);
+    size_t at = align256(static_cast<size_t>(p.nchunks) * T * E * sizeof(float));
+    p.off_logits = at;
+    at += align256(static_cast<size_t>(T) * E * sizeof(float));
+    p.off_tickets = at;
+    at += align256(static_cast<size_t>(G + 1) * sizeof(unsigned int));
     p.ws_bytes = at;
     return p;
   }
@@ -209,8 +232,34 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
   const RoutePlan plan = route_plan(T, d, E);
   if (plan.variant == kRouterTensorCore) return launch_route_tc(plan, x, W_router, bias, T, d, E, k, idx, w, ws, stream);
   float* lg = static_cast<float*>(ws);
-  switch (plan.variant) {
+  RouterVariant variant = plan.variant;
+  if (variant == kRouterStream && !aligned16(W_router)) variant = T <= 8 ? kRouterSplitTiny : kRouterSplitSmall;
+  if (variant == kRouterStream) {
+    int sms = 0;
+    const moe_status_t st = device_setup(&sms);
+    if (st != MOE_OK) return st;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* logits = reinterpret_cast<float*>(base + plan.off_logits);
+    unsigned int* tickets = reinterpret_cast<unsigned int*>(base + plan.off_tickets);
+    const int G = ceil_div(E, kRsExperts);
+    if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(G + 1) * sizeof(unsigned int), stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const dim3 grid(G, plan.nchunks);
+    const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+    if (T == 1)
+      router_stream_kernel<1><<<grid, kRsThreads, router_stream_smem_bytes(1), stream>>>(
+          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
+    else if (T <= 4)
+      router_stream_kernel<4><<<grid, kRsThreads, router_stream_smem_bytes(4), stream>>>(
+          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
+    else
+      router_stream_kernel<16><<<grid, kRsThreads, router_stream_smem_bytes(16), stream>>>(
+          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  switch (variant) {
     case kRouterTensorCore:
+    case kRouterStream:
       break;
     case kRouterFullBig: {
       dim3 grid(ceil_div(E, 64), ceil_div(T, 64), 1);
@@ -233,7 +282,7 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
       break;
     }
   }
-  if (plan.variant != kRouterFullBig) {
+  if (variant != kRouterFullBig) {
     // ordered sum of the chunk partials, bias, softmax and top-k: one block per token
     router_reduce_topk_kernel<<<T, 256, 0, stream>>>(lg, plan.nchunks, bias, T, E, k, idx, w);
   } else {
@@ -274,7 +323,27 @@ moe_status_t launch_permute(const moe_bf16_t* x, const int32_t* idx, int T, int 
 
 // -------------------------------------------------------------- expert FFN
 
-size_t ffn_ws(int E) { return 2 * align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
+// K split of the gate/up GEMM when an upper bound on its output tiles is at
+// most half of kSplitTargetCtas (one CTA per SM of a 148-SM part): each tile
+// becomes ksplit CTAs over disjoint K ranges, so a few-token step streams the
+// touched experts' weights with every SM instead of a third of them.
+constexpr int kSplitTargetCtas = 148;
+constexpr int kSplitMaxK = 4;
+
+// Workspace of the expert FFN: the two tile-prefix arrays, then (only when a K
+// split is possible for this Tk and E, i.e. min(E, Tk) <= kSplitTargetCtas / 2)
+// the split partials (at most kSplitTargetCtas tile-splits) and tickets.
+size_t ffn_split_part_bytes() {
+  return align256(static_cast<size_t>(kSplitTargetCtas) * kSplitPartFloats * sizeof(float));
+}
+size_t ffn_split_ticket_bytes() { return align256(static_cast<size_t>(kSplitTargetCtas / 2) * 4 * sizeof(unsigned)); }
+bool ffn_split_possible(int Tk, int E) { return (E < Tk ? E : Tk) <= kSplitTargetCtas / 2; }
+size_t ffn_prefix_bytes(int E) { return align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
+size_t ffn_ws(int Tk, int E) {
+  size_t b = 2 * ffn_prefix_bytes(E);
+  if (ffn_split_possible(Tk, E)) b += ffn_split_part_bytes() + ffn_split_ticket_bytes();
+  return b;
+}
 
 bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
                 const cuuint32_t* box) {
@@ -307,6 +376,7 @@ struct FfnPlan {
   GemmParams p0, p1;
   int grid0, grid1;
   int mode0;  // 0: 256-row gate/up blocks, 2: 128-row gate/up blocks
+  size_t split_ticket_bytes;  // tickets to clear before a K-split gate/up launch (0: no split)
 };
 
 moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
@@ -317,7 +387,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
       !act_map(&fp->mB1, h, Tk, f, kGemmBoxRows) || !act_map(&fp->mBs1, h, Tk, f, kGemmSmallBox))
     return MOE_ERR_INVALID_ARG;
   int32_t* prefix0 = static_cast<int32_t*>(ws);
-  int32_t* prefix1 = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ffn_ws(E) / 2);
+  int32_t* prefix1 = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ffn_prefix_bytes(E));
   const int64_t min_e_tk = E < Tk ? E : Tk;
   GemmParams& p0 = fp->p0;
   p0.expert_offsets = offsets;
@@ -331,9 +401,33 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   // 256-row blocks pay off only when experts average more than 128 rows
   fp->mode0 = (static_cast<int64_t>(Tk) > static_cast<int64_t>(E) * 128) ? 0 : 2;
   const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(fp->mode0)) + min_e_tk) * p0.n_feat_tiles;
-  fp->grid0 = static_cast<int>(tiles0 < num_sms ? tiles0 : num_sms);
+  const int KB0 = d / kGemmBK;
+  int ksplit = 1;
+  if (fp->mode0 == 2 && ffn_split_possible(Tk, E) && 2 * tiles0 <= kSplitTargetCtas) {
+    ksplit = static_cast<int>(kSplitTargetCtas / tiles0);
+    ksplit = ksplit > kSplitMaxK ? kSplitMaxK : ksplit;
+    ksplit = ksplit > KB0 / 8 ? KB0 / 8 : ksplit;
+    if (ksplit < 2) ksplit = 1;
+  }
+  p0.kb_per_split = ceil_div(KB0, ksplit);
+  p0.ksplit = ceil_div(KB0, p0.kb_per_split);  // every split non-empty
+  p0.part = nullptr;
+  p0.tickets = nullptr;
+  fp->split_ticket_bytes = 0;
+  if (p0.ksplit > 1) {
+    uint8_t* base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
+    p0.part = reinterpret_cast<float*>(base);
+    p0.tickets = reinterpret_cast<unsigned int*>(base + ffn_split_part_bytes());
+    fp->split_ticket_bytes = static_cast<size_t>(tiles0) * 4 * sizeof(unsigned);
+  }
+  const int64_t ctas0 = tiles0 * p0.ksplit;
+  fp->grid0 = static_cast<int>(ctas0 < num_sms ? ctas0 : num_sms);
   GemmParams& p1 = fp->p1;
   p1 = p0;
+  p1.ksplit = 1;
+  p1.kb_per_split = f / kGemmBK;
+  p1.part = nullptr;
+  p1.tickets = nullptr;
   p1.tile_prefix = prefix1;
   p1.K = f;
   p1.n_feat = d;
@@ -351,6 +445,7 @@ void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
                                                const_cast<int32_t*>(fp.p1.tile_prefix));
 }
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
+  if (fp.split_ticket_bytes > 0) cudaMemsetAsync(fp.p0.tickets, 0, fp.split_ticket_bytes, stream);
   if (fp.mode0 == 0)
     grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
   else
@@ -423,7 +518,7 @@ ForwardLayout forward_layout(int T, int d, int E, int k, int f) {
   L.h = take(Tk * f * 2);
   L.y_perm = take(Tk * d * 2);
   L.perm_ws = take(permute_ws(T, E, k));
-  L.ffn_ws = take(ffn_ws(E));
+  L.ffn_ws = take(ffn_ws(T * k, E));
   L.total = at;
   return L;
 }
@@ -479,7 +574,7 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
 
 size_t moe_expert_ffn_workspace_size(int Tk, int E) {
   if (Tk < 0 || E < 1) return 0;
-  return ffn_ws(E);
+  return ffn_ws(Tk, E);
 }
 
 moe_status_t moe_expert_ffn(const moe_bf16_t* x_perm, const int32_t* expert_offsets, const moe_bf16_t* W_gate_up,
@@ -490,7 +585,7 @@ moe_status_t moe_expert_ffn(const moe_bf16_t* x_perm, const int32_t* expert_offs
   if (!aligned16(x_perm) || !aligned16(W_gate_up) || !aligned16(W_down) || !aligned16(h) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
   if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
-  if (!workspace || !aligned256(workspace) || workspace_bytes < ffn_ws(E)) return MOE_ERR_WORKSPACE;
+  if (!workspace || !aligned256(workspace) || workspace_bytes < ffn_ws(Tk, E)) return MOE_ERR_WORKSPACE;
   int sms = 0;
   const moe_status_t st = device_setup(&sms);
   if (st != MOE_OK) return st;

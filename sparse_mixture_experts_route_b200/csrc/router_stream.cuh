@@ -1,0 +1,249 @@
+// Few-token router in one launch: logits, softmax over all experts and top-k
+// for T <= 16 tokens, the decode regime where the step reads the whole fp32
+// gate matrix W_router[d, E] for a handful of rows and is bound by that read.
+//
+// Same gate and numerics as router.cuh (one linear map d -> E, softmax over
+// the expert axis, top-k of the probabilities without renormalisation, as in
+// the gating code on "Kimi K3: The Open Model That Just Cornered the AI
+// Frontier", section "Mixture-of-Experts with Dynamic Load Balancing"), and
+// the same fixed fp32 order, so the logits are bit-identical to the other
+// router kernels:
+//   p_c = fma chain over the 128 input indices of chunk c, from +0, ascending;
+//   l   = ((p_0 + p_1) + ...) + p_{C-1}, then + b_e.
+//
+// Layout of the work: CTA (g, c) owns experts [128 g, 128 g + 128) and input
+// chunk c. It pulls its W tile (<= 128 rows of <= 512 bytes) into shared
+// memory with one bulk copy per row, all issued up front on one mbarrier, so
+// the whole matrix is in flight at once across the grid; widens its chunk of
+// x for every token; and writes p_c for every (token, expert) it owns.
+// The last CTA of expert group g to finish (an atomic ticket, after a fence)
+// adds the group's C partials in ascending c (+ bias) into the final logits;
+// the last group to finish then takes softmax and top-k for every token, one
+// warp per token. Which CTA does a reduction depends on timing, but every sum
+// is taken in the fixed order, so the results are deterministic.
+// The tickets must be zero at launch; the last CTAs put them back to zero.
+#pragma once
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kRsExperts = 128;  // experts per CTA
+constexpr int kRsRows = 128;     // input indices per CTA (one chunk)
+constexpr int kRsThreads = 256;
+constexpr int kRsMaxTokens = 16;
+
+__host__ __device__ constexpr int router_stream_smem_bytes(int tmax) {
+  return kRsRows * kRsExperts * 4 + kRsRows * tmax * 4;
+}
+
+// Order-preserving map of a non-NaN float to an unsigned key.
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Softmax over the E final logits of one token and its top-k (equal logits go
+// to the lower index), by one warp. Values are read through L2 (they were
+// written by other CTAs of this launch).
+template <int MAXV>
+__device__ __forceinline__ void warp_softmax_topk(const float* row, int E, int k, int lane, int32_t* out_idx,
+                                                  float* out_w) {
+  float v[MAXV];
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int e = i * 32 + lane;
+    v[i] = (e < E) ? __ldcg(row + e) : -INFINITY;
+  }
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) m = fmaxf(m, v[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i)
+    if (i * 32 + lane < E) s += expf(v[i] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+
+  uint32_t taken = 0u;
+  for (int j = 0; j < k; ++j) {
+    // this lane's best remaining value; its values are in ascending expert
+    // order, so a strict '>' keeps the lowest index among equal values
+    float bv = -INFINITY;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+    const uint32_t key = bi < 0 ? 0u : float_order_key(bv);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+    const uint32_t win = __reduce_min_sync(0xffffffffu, (bi >= 0 && key == kmax) ? static_cast<uint32_t>(bi)
+                                                                                   : 0xffffffffu);
+    const int wi = static_cast<int>(win);
+    if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
+    const float wv = __shfl_sync(0xffffffffu, bv, wi & 31);
+    if (lane == 0) {
+      out_idx[j] = wi;
+      out_w[j] = expf(wv - m) / s;
+    }
+  }
+}
+
+template <int TMAX>
+__global__ void __launch_bounds__(kRsThreads)
+    router_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, const float* __restrict__ bias,
+                         int T, int d, int E, int k, float* __restrict__ part, float* __restrict__ logits,
+                         unsigned int* __restrict__ tickets, int32_t* __restrict__ topk_idx,
+                         float* __restrict__ topk_w) {
+  static_assert(TMAX == 1 || TMAX == 4 || TMAX == 16, "token tile");
+  extern __shared__ __align__(128) uint8_t rs_smem[];
+  float* ws = reinterpret_cast<float*>(rs_smem);  // [kRsRows][kRsExperts]
+  float* xs = ws + kRsRows * kRsExperts;          // [kRsRows][TMAX]
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ unsigned int s_ticket;
+
+  const int g = blockIdx.x, c = blockIdx.y;
+  const int G = gridDim.x, C = gridDim.y;
+  const int e0 = g * kRsExperts;
+  const int ne = min(kRsExperts, E - e0);  // a multiple of 4 (E % 4 == 0)
+  const int r0 = c * kRsRows;
+  const int nr = min(kRsRows, d - r0);     // 128, or 64 for the last chunk when d % 128 == 64
+  const int tid = threadIdx.x;
+
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nr * ne * 4));
+  __syncthreads();
+  {
+    const uint64_t pol = l2_policy_evict_first();  // read once per call
+    for (int r = tid; r < nr; r += kRsThreads)
+      bulk_load(ws + r * kRsExperts, W + static_cast<int64_t>(r0 + r) * E + e0, static_cast<uint32_t>(ne * 4), &bar,
+                pol);
+  }
+  // the chunk of x for every token, widened exactly: xs[i][t]
+  for (int v = tid; v < TMAX * (kRsRows / 8); v += kRsThreads) {
+    const int t = v / (kRsRows / 8), q = v % (kRsRows / 8);
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T && q * 8 < nr) u = *reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d + r0 + q * 8);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      xs[(q * 8 + 2 * h) * TMAX + t] = __uint_as_float(w4[h] << 16);
+      xs[(q * 8 + 2 * h + 1) * TMAX + t] = __uint_as_float(w4[h] & 0xFFFF0000u);
+    }
+  }
+  __syncthreads();
+  if (!mbar_wait_bounded(&bar, 0u, kWaitLimitNs, nullptr)) {
+    record_device_error(6u /* MOE_DEVERR_WAIT_TIMEOUT_ROUTER */);
+    return;
+  }
+
+  // p_c for experts e0 + 2p, e0 + 2p + 1 and tokens q*TS .. q*TS + TS - 1
+  constexpr int NS = TMAX >= 4 ? 4 : 1;
+  constexpr int TS = TMAX / NS;
+  const int p = tid & 63, q = tid >> 6;
+  if (q < NS && 2 * p < ne) {
+    float acc[TS][2];
+#pragma unroll
+    for (int j = 0; j < TS; ++j) acc[j][0] = acc[j][1] = 0.0f;
+#pragma unroll 8
+    for (int i = 0; i < nr; ++i) {
+      const float2 w2 = *reinterpret_cast<const float2*>(ws + i * kRsExperts + 2 * p);
+      float xv[TS];
+      if constexpr (TS >= 4) {
+#pragma unroll
+        for (int j = 0; j < TS; j += 4) {
+          const float4 x4 = *reinterpret_cast<const float4*>(xs + i * TMAX + q * TS + j);
+          xv[j] = x4.x, xv[j + 1] = x4.y, xv[j + 2] = x4.z, xv[j + 3] = x4.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < TS; ++j) xv[j] = xs[i * TMAX + q * TS + j];
+      }
+#pragma unroll
+      for (int j = 0; j < TS; ++j) {
+        acc[j][0] = __fmaf_rn(xv[j], w2.x, acc[j][0]);
+        acc[j][1] = __fmaf_rn(xv[j], w2.y, acc[j][1]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < TS; ++j) {
+      const int t = q * TS + j;
+      if (t < T)
+        *reinterpret_cast<float2*>(part + (static_cast<int64_t>(c) * T + t) * E + e0 + 2 * p) =
+            make_float2(acc[j][0], acc[j][1]);
+    }
+  }
+
+  // the last CTA of this expert group adds the group's partials in chunk order
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_ticket = atomicAdd(&tickets[g], 1u);
+  __syncthreads();
+  if (s_ticket != static_cast<unsigned int>(C - 1)) return;
+  __threadfence();
+  const int npairs = ne / 2;
+  const int64_t plane = static_cast<int64_t>(T) * E;
+  for (int it = tid; it < T * npairs; it += kRsThreads) {
+    const int t = it / npairs, e = e0 + 2 * (it % npairs);
+    const float* src = part + static_cast<int64_t>(t) * E + e;
+    float2 l = __ldcg(reinterpret_cast<const float2*>(src));
+    int cc = 1;
+    for (; cc + 8 <= C; cc += 8) {
+      float2 pv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pv[u] = __ldcg(reinterpret_cast<const float2*>(src + (cc + u) * plane));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        l.x = __fadd_rn(l.x, pv[u].x);
+        l.y = __fadd_rn(l.y, pv[u].y);
+      }
+    }
+    for (; cc < C; ++cc) {
+      const float2 pv = __ldcg(reinterpret_cast<const float2*>(src + cc * plane));
+      l.x = __fadd_rn(l.x, pv.x);
+      l.y = __fadd_rn(l.y, pv.y);
+    }
+    if (bias != nullptr) {
+      l.x = __fadd_rn(l.x, __ldg(bias + e));
+      l.y = __fadd_rn(l.y, __ldg(bias + e + 1));
+    }
+    *reinterpret_cast<float2*>(logits + static_cast<int64_t>(t) * E + e) = l;
+  }
+
+  // the last group to finish takes softmax and top-k for every token
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    tickets[g] = 0u;
+    s_ticket = atomicAdd(&tickets[G], 1u);
+  }
+  __syncthreads();
+  if (s_ticket != static_cast<unsigned int>(G - 1)) return;
+  __threadfence();
+  if (tid == 0) tickets[G] = 0u;
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int t = warp; t < T; t += kRsThreads / 32) {
+    const float* row = logits + static_cast<int64_t>(t) * E;
+    int32_t* oi = topk_idx + static_cast<int64_t>(t) * k;
+    float* ow = topk_w + static_cast<int64_t>(t) * k;
+    if (E <= 256)
+      warp_softmax_topk<8>(row, E, k, lane, oi, ow);
+    else
+      warp_softmax_topk<32>(row, E, k, lane, oi, ow);
+  }
+}
+
+}  // namespace moe

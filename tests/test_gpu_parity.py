@@ -59,6 +59,66 @@ def test_route_bit_exact(lib, shape):
     assert lib.get_device_error() == 0
 
 
+# The few-token router (T <= 16, E % 4 == 0): one launch that streams every
+# chunk of W_router at once and reduces in the last CTAs. Ragged last chunk
+# (d % 128 == 64), partial last expert group (E % 128 != 0), one chunk only,
+# k = E, 1024 experts, the full-width decode shape, and a bias.
+STREAM_SHAPES = [
+    # (T, d, E, k, bias)
+    (1, 7168, 896, 16, None),
+    (1, 7168, 896, 16, "zipf"),
+    (3, 320, 20, 3, None),
+    (4, 256, 200, 8, "zipf"),
+    (5, 128, 1024, 16, None),
+    (16, 448, 132, 4, None),
+    (16, 64, 8, 8, None),
+    (9, 7168, 384, 8, "zipf"),
+    (2, 128, 6, 1, None),     # E % 4 != 0: the split-chunk router instead
+]
+
+
+@pytest.mark.parametrize("shape", STREAM_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_route_few_tokens(lib, shape):
+    T, d, E, k, bias = shape
+    inp = _inputs(T, d, E, k, 64, bias=bias)
+    g = _cuda(inp)
+    for _ in range(2):  # the tickets return to zero: a second call reuses the workspace as is
+        ws = torch.empty(lib.route_workspace_size(T, d, E), dtype=torch.uint8, device="cuda") if _ == 0 else ws
+        idx, w = lib.moe_route(g.x, g.W_router, g.bias, k, workspace=ws)
+        torch.cuda.synchronize()
+        assert lib.get_device_error() == 0
+        _, ridx, rw = parity.oracle_route(inp, k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+
+
+def test_route_few_tokens_ties_and_unaligned_weights(lib):
+    """Exact ties and all-zero tokens on the few-token router; a W_router that is
+    not 16-byte aligned (4-byte offset) takes the split-chunk router, same bits."""
+    T, d, E, k = 6, 384, 12, 3
+    inp = _inputs(T, d, E, k, 64)
+    Wr = inp.W_router.clone()
+    Wr[:, 7] = Wr[:, 2]
+    x = inp.x.clone()
+    x[1] = 0
+    bias = torch.zeros(E, dtype=torch.float32)
+    bias[5] = 0.25
+    lg = oracle.router_logits(x, Wr, bias)
+    ridx, rw = oracle.topk(lg, k)
+    idx, w = lib.moe_route(x.cuda(), Wr.cuda(), bias.cuda(), k)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    assert idx[1].tolist() == [5, 0, 1]
+    store = torch.empty(d * E + 1, dtype=torch.float32, device="cuda")
+    Wr_off = store[1:].view(d, E)
+    Wr_off.copy_(Wr.cuda())
+    assert Wr_off.data_ptr() % 16 != 0
+    idx2, w2 = lib.moe_route(x.cuda(), Wr_off, bias.cuda(), k)
+    assert torch.equal(idx2, idx)
+    np.testing.assert_allclose(w2.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    assert lib.get_device_error() == 0
+
+
 def test_route_bias_ties_zero_rows(lib):
     T, d, E, k, f = 96, 384, 12, 3, 64
     inp = _inputs(T, d, E, k, f)
@@ -155,6 +215,38 @@ def _ffn_check(lib, inp, k):
 def test_expert_ffn(lib, shape):
     T, d, E, k, f = shape
     _ffn_check(lib, _inputs(T, d, E, k, f), k)
+
+
+# Few output tiles: the gate/up GEMM splits K over 2 or 4 CTAs per tile and
+# the last split adds the fp32 partials in order (f = 192: a half-empty
+# feature tile). Two calls give identical bits (the tickets return to zero).
+@pytest.mark.parametrize("shape", [(8, 1024, 8, 2, 128), (4, 2048, 16, 4, 256), (3, 1024, 8, 2, 192)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_expert_ffn_k_split(lib, shape):
+    T, d, E, k, f = shape
+    inp = _inputs(T, d, E, k, f)
+    h, y = _ffn_check(lib, inp, k)
+    _, ridx, _ = parity.oracle_route(inp, k)
+    _, offsets, perm_token, _ = oracle.permute(ridx, E)
+    x_perm = inp.x[torch.from_numpy(perm_token).long()]
+    h2, y2 = lib.moe_expert_ffn(x_perm.cuda(), torch.from_numpy(offsets).cuda(), inp.W_gate_up.cuda(),
+                                inp.W_down.cuda())
+    assert torch.equal(h, h2) and torch.equal(y, y2)
+
+
+def test_forward_one_token_full_width(lib):
+    """T = 1 at d = 7168, E = 896, k = 16, f = 512 (the first decode-sweep point):
+    few-token router, one-block dispatch, K-split gate/up GEMM."""
+    T, d, E, k, f = 1, 7168, 896, 16, 512
+    inp = _inputs(T, d, E, k, f)
+    g = _cuda(inp)
+    out = lib.moe_forward(g.x, g.W_router, None, g.W_gate_up, g.W_down, k)
+    out2 = lib.moe_forward(g.x, g.W_router, None, g.W_gate_up, g.W_down, k)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    assert torch.equal(out, out2)
+    ref, _, _ = oracle.forward(inp.x, inp.W_router, None, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(out, ref, "forward T=1")
 
 
 def test_expert_ffn_hot_expert_multi_block(lib):
