@@ -242,7 +242,8 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
     float* logits = reinterpret_cast<float*>(base + plan.off_logits);
     unsigned int* tickets = reinterpret_cast<unsigned int*>(base + plan.off_tickets);
     const int G = ceil_div(E, kRsExperts);
-    if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(G + 1) * sizeof(unsigned int), stream) != cudaSuccess)
+    if (T == 1 &&
+        cudaMemsetAsync(tickets, 0, static_cast<size_t>(G + 1) * sizeof(unsigned int), stream) != cudaSuccess)
       return MOE_ERR_CUDA;
     const dim3 grid(G, plan.nchunks);
     const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
@@ -255,6 +256,7 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
     else
       router_stream_kernel<16><<<grid, kRsThreads, router_stream_smem_bytes(16), stream>>>(
           xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
+    if (T > 1) router_reduce_topk_kernel<<<T, 256, 0, stream>>>(lg, plan.nchunks, bias, T, E, k, idx, w);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
   switch (variant) {

@@ -23,6 +23,12 @@ namespace moe {
 constexpr int kRouterChunk = 128;  // input indices per ordered partial sum
 constexpr int kRouterBK = 32;      // input indices staged in shared memory per step
 
+// Order-preserving map of a non-NaN float to an unsigned key.
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
@@ -250,22 +256,239 @@ __global__ void __launch_bounds__(256)
 
 namespace moe {
 
+// Softmax statistics of one token's E <= 1024 logits held in shared memory,
+// by a CTA of 256 threads: M = max_e l_e and S = sum_e exp(l_e - M), the sum
+// taken per warp in a fixed shuffle order and then over the warps in order.
+__device__ __forceinline__ void cta_softmax_stats_256(const float* s_l, int E, float* M, float* S) {
+  __shared__ float s_wm[8], s_ws[8];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  float m = -INFINITY;
+  for (int e = tid; e < E; e += 256) m = fmaxf(m, s_l[e]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_wm[w] = m;
+  __syncthreads();
+  float gm = s_wm[0];
+#pragma unroll
+  for (int q = 1; q < 8; ++q) gm = fmaxf(gm, s_wm[q]);
+  float s = 0.0f;
+  for (int e = tid; e < E; e += 256) s += expf(s_l[e] - gm);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) s_ws[w] = s;
+  __syncthreads();
+  float gs = s_ws[0];
+#pragma unroll
+  for (int q = 1; q < 8; ++q) gs += s_ws[q];
+  *M = gm;
+  *S = gs;
+}
+
+// For warp 0: the bin of a 256-bin histogram (hist, bins ascending) that
+// holds the kk-th largest element, and how many elements lie in higher bins.
+__device__ __forceinline__ void warp_find_bin_from_top(const unsigned* hist, unsigned kk, unsigned* bin,
+                                                       unsigned* above) {
+  const int lane = threadIdx.x & 31;
+  unsigned h[8];
+  unsigned tot = 0u;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    h[q] = hist[lane * 8 + q];
+    tot += h[q];
+  }
+  unsigned suf = tot;  // inclusive suffix sum over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  unsigned cum = suf - tot;  // elements in the bins of higher lanes
+#pragma unroll
+  for (int q = 7; q >= 0; --q) {
+    if (cum < kk && cum + h[q] >= kk) {
+      *bin = static_cast<unsigned>(lane * 8 + q);
+      *above = cum;
+    }
+    cum += h[q];
+  }
+}
+
+// Top-k by (logit desc, index asc) of one token's E <= 1024 logits held in
+// shared memory, by a CTA of 256 threads, without sequential arg-max rounds:
+// two 8-bit histogram passes over the top 16 bits of the order keys locate
+// the bin that holds the k-th largest logit; every logit in or above that bin
+// is a candidate, and a candidate's output slot is its exact rank among the
+// candidates by the key (order key of the logit, -0 taken as +0; then the
+// complemented index), a total order. Returns false, writing nothing, when
+// more than 64 logits are candidates (heavy ties); the caller then takes
+// cta_topk_rounds_256.
+__device__ __forceinline__ bool cta_topk_histogram_256(const float* s_l, int E, int k, float M, float S,
+                                                       int32_t* out_idx, float* out_w) {
+  __shared__ unsigned s_hist[256];
+  __shared__ unsigned s_sel[4];
+  __shared__ unsigned s_ncand;
+  __shared__ uint64_t s_ckey[64];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  uint32_t key[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + 256 * i;
+    key[i] = (e < E) ? float_order_key(s_l[e] + 0.0f) : 0u;
+  }
+  // pass 1: the top byte of the key
+  s_hist[tid] = 0u;
+  if (tid == 0) s_ncand = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (tid + 256 * i < E) atomicAdd(&s_hist[key[i] >> 24], 1u);
+  __syncthreads();
+  if (w == 0) warp_find_bin_from_top(s_hist, static_cast<unsigned>(k), &s_sel[0], &s_sel[1]);
+  __syncthreads();
+  const unsigned b1 = s_sel[0], above1 = s_sel[1];
+  // pass 2: the second byte, within that bin
+  s_hist[tid] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (tid + 256 * i < E && (key[i] >> 24) == b1) atomicAdd(&s_hist[(key[i] >> 16) & 255u], 1u);
+  __syncthreads();
+  if (w == 0) warp_find_bin_from_top(s_hist, static_cast<unsigned>(k) - above1, &s_sel[2], &s_sel[3]);
+  __syncthreads();
+  const unsigned thr = (b1 << 8) | s_sel[2];
+  const unsigned ncand = above1 + s_sel[3] + s_hist[s_sel[2]];
+  if (ncand > 64u) return false;  // the same for every thread: all read the same shared values
+  // collect the candidates (slot order does not matter: ranks decide)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + 256 * i;
+    if (e < E && (key[i] >> 16) >= thr) {
+      const unsigned slot = atomicAdd(&s_ncand, 1u);
+      s_ckey[slot] = (static_cast<uint64_t>(key[i]) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(e));
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    for (unsigned r = lane; r < ncand; r += 32) {
+      const uint64_t kk = s_ckey[r];
+      int rank = 0;
+      for (unsigned q = 0; q < ncand; ++q) rank += (s_ckey[q] > kk) ? 1 : 0;
+      if (rank < k) {
+        const int e = static_cast<int>(~static_cast<uint32_t>(kk & 0xffffffffu));
+        out_idx[rank] = e;
+        out_w[rank] = expf(s_l[e] - M) / S;
+      }
+    }
+  }
+  return true;
+}
+
+// Top-k by k rounds of arg-max (the general case, any ties): warp w takes the
+// experts e with (e / 32) % 8 == w and finds its local top-k; warp 0 merges
+// the 8 local lists. Weights exp(l - M) / S.
+__device__ __forceinline__ void cta_topk_rounds_256(const float* s_l, int E, int k, float M, float S,
+                                                    int32_t* out_idx, float* out_w) {
+  __shared__ float s_cv[8][16];
+  __shared__ int s_ci[8][16];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = 256 * i + 32 * w + lane;
+    v[i] = (e < E) ? s_l[e] : -INFINITY;
+  }
+  // k rounds of warp arg-max by (logit desc, index asc): a lane's values are in
+  // ascending expert order, so a strict '>' keeps its lowest index among equal
+  // values; across lanes the largest order key wins, then the lowest index
+  uint32_t taken = 0u;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 256 * i + 32 * w + lane;
+      if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+    const uint32_t key = bi < 0 ? 0u : float_order_key(bv);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+    const uint32_t win =
+        __reduce_min_sync(0xffffffffu, (bi >= 0 && key == kmax) ? static_cast<uint32_t>(bi) : 0xffffffffu);
+    const int wi = static_cast<int>(win);  // 0xffffffff (-1) when this warp has no expert left
+    if (wi >= 0 && (wi & 31) == lane) taken |= 1u << (wi >> 8);
+    const float wv = __shfl_sync(0xffffffffu, bv, wi >= 0 ? (wi & 31) : 0);
+    if (lane == 0) {
+      s_cv[w][j] = wi >= 0 ? wv : -INFINITY;
+      s_ci[w][j] = wi >= 0 ? wi : 0x7fffffff;
+    }
+  }
+  __syncthreads();
+
+  // merge
+  if (w == 0) {
+    // candidates: lane holds entries lane, lane + 32, ... of the 8 x k list
+    float cv[4];
+    int ci[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int slot = lane + 32 * r;
+      const int q = slot / 16, j = slot % 16;
+      const bool ok = q < 8 && j < k;
+      cv[r] = ok ? s_cv[q][j] : -INFINITY;
+      ci[r] = ok ? s_ci[q][j] : 0x7fffffff;
+    }
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff, br = -1;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (ci[r] != 0x7fffffff && (bi == 0x7fffffff || cv[r] > bv || (cv[r] == bv && ci[r] < bi))) {
+          bv = cv[r];
+          bi = ci[r];
+          br = r;
+        }
+      const uint32_t key = br < 0 ? 0u : float_order_key(bv);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+      const uint32_t win =
+          __reduce_min_sync(0xffffffffu, (br >= 0 && key == kmax) ? static_cast<uint32_t>(bi) : 0xffffffffu);
+      const int wb = static_cast<int>(win);
+      const int owner = __reduce_min_sync(0xffffffffu, (br >= 0 && bi == wb) ? static_cast<uint32_t>(lane) : 32u);
+      const float wv = __shfl_sync(0xffffffffu, bv, owner & 31);
+      if (lane == owner) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          if (r == br) ci[r] = 0x7fffffff;  // taken
+      }
+      if (lane == 0) {
+        out_idx[j] = wb;
+        out_w[j] = expf(wv - M) / S;
+      }
+    }
+  }
+}
+
+// Softmax over one token's E <= 1024 final logits, held in shared memory, and
+// their top-k by (logit desc, index asc), by a CTA of 256 threads. Writes
+// out_idx[0..k) and out_w[0..k) = exp(l - M) / S. Every thread of the CTA
+// must call it.
+__device__ __forceinline__ void cta_softmax_topk_256(const float* s_l, int E, int k, int32_t* out_idx, float* out_w) {
+  float M, S;
+  cta_softmax_stats_256(s_l, E, &M, &S);
+  if (!cta_topk_histogram_256(s_l, E, k, M, S, out_idx, out_w)) cta_topk_rounds_256(s_l, E, k, M, S, out_idx, out_w);
+}
+
 // Small-T router, second half, one block of 256 threads per token:
 //  1. thread i owns experts i, i + 256, ...: l = plane 0 + plane 1 + ... (in
 //     ascending chunk order) + bias, kept in shared memory;
-//  2. warp w takes the experts e with (e / 32) % 8 == w: softmax partials (its
-//     own max and sum) and its local top-k by (logit desc, index asc);
-//  3. warp 0 merges the 8 local lists (k rounds of warp arg-max) and rescales
-//     the partial sums to the global max, in warp order.
+//  2. softmax and top-k of those logits (cta_softmax_topk_256).
 __global__ void __launch_bounds__(256)
     router_reduce_topk_kernel(const float* __restrict__ lg, int nsplit, const float* __restrict__ bias, int T, int E,
                               int k, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   __shared__ float s_l[1024];
-  __shared__ float s_cv[8][16];
-  __shared__ int s_ci[8][16];
-  __shared__ float s_wm[8], s_ws[8];
   const int t = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int tid = threadIdx.x;
   const int64_t n = static_cast<int64_t>(T) * E;
   // 1. ordered sums of the chunk partials
   float acc[4];
@@ -296,108 +519,7 @@ __global__ void __launch_bounds__(256)
   }
   __syncthreads();
 
-  // 2. per-warp softmax partials and local top-k over experts e = 256 i + 32 w + lane
-  float v[4];
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int e = 256 * i + 32 * w + lane;
-    v[i] = (e < E) ? s_l[e] : -INFINITY;
-    m = fmaxf(m, v[i]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float s = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (256 * i + 32 * w + lane < E) s += expf(v[i] - m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) {
-    s_wm[w] = m;
-    s_ws[w] = s;
-  }
-  uint32_t taken = 0u;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = 256 * i + 32 * w + lane;
-      if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv)) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi != 0x7fffffff && ((bi & 31) == lane) && (((bi >> 5) & 7) == w)) taken |= 1u << (bi >> 8);
-    if (lane == 0) {
-      s_cv[w][j] = bv;
-      s_ci[w][j] = bi;
-    }
-  }
-  __syncthreads();
-
-  // 3. merge
-  if (w == 0) {
-    float gm = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) gm = fmaxf(gm, s_wm[q]);
-    float gs = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (s_wm[q] != -INFINITY) gs += s_ws[q] * expf(s_wm[q] - gm);
-    // candidates: lane holds entries lane, lane + 32, ... of the 8 x k list
-    float cv[4];
-    int ci[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int slot = lane + 32 * r;
-      const int q = slot / 16, j = slot % 16;
-      const bool ok = q < 8 && j < k;
-      cv[r] = ok ? s_cv[q][j] : -INFINITY;
-      ci[r] = ok ? s_ci[q][j] : 0x7fffffff;
-    }
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff, br = -1;
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-        if (ci[r] != 0x7fffffff && (bi == 0x7fffffff || cv[r] > bv || (cv[r] == bv && ci[r] < bi))) {
-          bv = cv[r];
-          bi = ci[r];
-          br = r;
-        }
-      int wb = bi;
-      float wv = bv;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, wb, o);
-        if (oi != 0x7fffffff && (wb == 0x7fffffff || ov > wv || (ov == wv && oi < wb))) {
-          wv = ov;
-          wb = oi;
-        }
-      }
-      if (br >= 0 && bi == wb) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-          if (r == br) ci[r] = 0x7fffffff;  // taken
-      }
-      if (lane == 0) {
-        topk_idx[static_cast<int64_t>(t) * k + j] = wb;
-        topk_w[static_cast<int64_t>(t) * k + j] = expf(wv - gm) / gs;
-      }
-    }
-  }
+  cta_softmax_topk_256(s_l, E, k, topk_idx + static_cast<int64_t>(t) * k, topk_w + static_cast<int64_t>(t) * k);
 }
 
 }  // namespace moe

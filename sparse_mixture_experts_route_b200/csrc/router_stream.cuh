@@ -1,6 +1,7 @@
-// Few-token router in one launch: logits, softmax over all experts and top-k
-// for T <= 16 tokens, the decode regime where the step reads the whole fp32
-// gate matrix W_router[d, E] for a handful of rows and is bound by that read.
+// Few-token router: logits, softmax over all experts and top-k for T <= 16
+// tokens (one launch for T = 1), the decode regime where the step reads the
+// whole fp32 gate matrix W_router[d, E] for a handful of rows and is bound by
+// that read.
 //
 // Same gate and numerics as router.cuh (one linear map d -> E, softmax over
 // the expert axis, top-k of the probabilities without renormalisation, as in
@@ -16,18 +17,21 @@
 // memory with one bulk copy per row, all issued up front on one mbarrier, so
 // the whole matrix is in flight at once across the grid; widens its chunk of
 // x for every token; and writes p_c for every (token, expert) it owns.
-// The last CTA of expert group g to finish (an atomic ticket, after a fence)
-// adds the group's C partials in ascending c (+ bias) into the final logits;
-// the last group to finish then takes softmax and top-k for every token, one
-// warp per token. Which CTA does a reduction depends on timing, but every sum
-// is taken in the fixed order, so the results are deterministic.
-// The tickets must be zero at launch; the last CTAs put them back to zero.
+// With one token the same launch finishes the job: the last CTA of expert
+// group g to finish (an atomic ticket, after a fence) adds the group's C
+// partials in ascending c (+ bias) into the final logits; the last group to
+// finish then takes softmax and top-k with all 256 threads. Which CTA does a
+// reduction depends on timing, but every sum is taken in the fixed order, so
+// the results are deterministic. The tickets must be zero at launch; the last
+// CTAs put them back to zero. With more tokens the kernel writes the partials
+// only and router_reduce_topk_kernel follows.
 #pragma once
 
 #include <cstdint>
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "router.cuh"
 
 namespace moe {
 
@@ -38,64 +42,6 @@ constexpr int kRsMaxTokens = 16;
 
 __host__ __device__ constexpr int router_stream_smem_bytes(int tmax) {
   return kRsRows * kRsExperts * 4 + kRsRows * tmax * 4;
-}
-
-// Order-preserving map of a non-NaN float to an unsigned key.
-__device__ __forceinline__ uint32_t float_order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Softmax over the E final logits of one token and its top-k (equal logits go
-// to the lower index), by one warp. Values are read through L2 (they were
-// written by other CTAs of this launch).
-template <int MAXV>
-__device__ __forceinline__ void warp_softmax_topk(const float* row, int E, int k, int lane, int32_t* out_idx,
-                                                  float* out_w) {
-  float v[MAXV];
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int e = i * 32 + lane;
-    v[i] = (e < E) ? __ldcg(row + e) : -INFINITY;
-  }
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) m = fmaxf(m, v[i]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float s = 0.0f;
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i)
-    if (i * 32 + lane < E) s += expf(v[i] - m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-
-  uint32_t taken = 0u;
-  for (int j = 0; j < k; ++j) {
-    // this lane's best remaining value; its values are in ascending expert
-    // order, so a strict '>' keeps the lowest index among equal values
-    float bv = -INFINITY;
-    int bi = -1;
-#pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
-        bv = v[i];
-        bi = e;
-      }
-    }
-    const uint32_t key = bi < 0 ? 0u : float_order_key(bv);
-    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-    const uint32_t win = __reduce_min_sync(0xffffffffu, (bi >= 0 && key == kmax) ? static_cast<uint32_t>(bi)
-                                                                                   : 0xffffffffu);
-    const int wi = static_cast<int>(win);
-    if ((wi & 31) == lane) taken |= 1u << (wi >> 5);
-    const float wv = __shfl_sync(0xffffffffu, bv, wi & 31);
-    if (lane == 0) {
-      out_idx[j] = wi;
-      out_w[j] = expf(wv - m) / s;
-    }
-  }
 }
 
 template <int TMAX>
@@ -187,7 +133,13 @@ __global__ void __launch_bounds__(kRsThreads)
     }
   }
 
-  // the last CTA of this expert group adds the group's partials in chunk order
+  // Several tokens: the ordered sums, softmax and top-k run as a second launch
+  // (router_reduce_topk_kernel, one CTA per token), which spreads the T x E x C
+  // partial reads and the T top-k selections over the whole GPU.
+  if constexpr (TMAX > 1) return;
+
+  // One token: the last CTA of this expert group adds the group's partials in
+  // chunk order (all C loads of a pair issued before the adds)
   __threadfence();
   __syncthreads();
   if (tid == 0) s_ticket = atomicAdd(&tickets[g], 1u);
@@ -196,17 +148,17 @@ __global__ void __launch_bounds__(kRsThreads)
   __threadfence();
   const int npairs = ne / 2;
   const int64_t plane = static_cast<int64_t>(T) * E;
-  for (int it = tid; it < T * npairs; it += kRsThreads) {
-    const int t = it / npairs, e = e0 + 2 * (it % npairs);
-    const float* src = part + static_cast<int64_t>(t) * E + e;
+  if (tid < npairs) {
+    const int e = e0 + 2 * tid;
+    const float* src = part + e;  // token 0
     float2 l = __ldcg(reinterpret_cast<const float2*>(src));
     int cc = 1;
-    for (; cc + 8 <= C; cc += 8) {
-      float2 pv[8];
+    for (; cc + 16 <= C; cc += 16) {
+      float2 pv[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) pv[u] = __ldcg(reinterpret_cast<const float2*>(src + (cc + u) * plane));
+      for (int u = 0; u < 16; ++u) pv[u] = __ldcg(reinterpret_cast<const float2*>(src + (cc + u) * plane));
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         l.x = __fadd_rn(l.x, pv[u].x);
         l.y = __fadd_rn(l.y, pv[u].y);
       }
@@ -220,10 +172,11 @@ __global__ void __launch_bounds__(kRsThreads)
       l.x = __fadd_rn(l.x, __ldg(bias + e));
       l.y = __fadd_rn(l.y, __ldg(bias + e + 1));
     }
-    *reinterpret_cast<float2*>(logits + static_cast<int64_t>(t) * E + e) = l;
+    *reinterpret_cast<float2*>(logits + e) = l;
   }
 
-  // the last group to finish takes softmax and top-k for every token
+  // the last group to finish takes softmax and top-k with the whole CTA
+  __shared__ float s_l[1024];
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -234,16 +187,9 @@ __global__ void __launch_bounds__(kRsThreads)
   if (s_ticket != static_cast<unsigned int>(G - 1)) return;
   __threadfence();
   if (tid == 0) tickets[G] = 0u;
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int t = warp; t < T; t += kRsThreads / 32) {
-    const float* row = logits + static_cast<int64_t>(t) * E;
-    int32_t* oi = topk_idx + static_cast<int64_t>(t) * k;
-    float* ow = topk_w + static_cast<int64_t>(t) * k;
-    if (E <= 256)
-      warp_softmax_topk<8>(row, E, k, lane, oi, ow);
-    else
-      warp_softmax_topk<32>(row, E, k, lane, oi, ow);
-  }
+  for (int e = tid; e < E; e += kRsThreads) s_l[e] = __ldcg(logits + e);
+  __syncthreads();
+  cta_softmax_topk_256(s_l, E, k, topk_idx, topk_w);
 }
 
 }  // namespace moe

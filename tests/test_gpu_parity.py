@@ -92,6 +92,21 @@ def test_route_few_tokens(lib, shape):
         np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
 
 
+@pytest.mark.parametrize("T", [1, 6])
+def test_route_all_equal_logits(lib, T):
+    """All-zero tokens: every logit is 0, so all E = 896 experts tie. The
+    histogram top-k sees more than 64 candidates and hands over to the
+    arg-max rounds: experts 0..k-1 in order, each with weight 1/E."""
+    d, E, k = 256, 896, 16
+    x = torch.zeros(T, d, dtype=torch.bfloat16, device="cuda")
+    Wr = torch.randn(d, E, dtype=torch.float32, device="cuda") * 0.02
+    idx, w = lib.moe_route(x, Wr, None, k)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    assert idx.tolist() == [list(range(k))] * T
+    np.testing.assert_allclose(w.cpu().numpy(), np.full((T, k), 1.0 / E), rtol=1e-6)
+
+
 def test_route_few_tokens_ties_and_unaligned_weights(lib):
     """Exact ties and all-zero tokens on the few-token router; a W_router that is
     not 16-byte aligned (4-byte offset) takes the split-chunk router, same bits."""
