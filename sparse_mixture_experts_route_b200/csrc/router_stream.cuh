@@ -139,40 +139,28 @@ __global__ void __launch_bounds__(kRsThreads)
   if constexpr (TMAX > 1) return;
 
   // One token: the last CTA of this expert group adds the group's partials in
-  // chunk order (all C loads of a pair issued before the adds)
+  // chunk order
   __threadfence();
   __syncthreads();
   if (tid == 0) s_ticket = atomicAdd(&tickets[g], 1u);
   __syncthreads();
   if (s_ticket != static_cast<unsigned int>(C - 1)) return;
   __threadfence();
-  const int npairs = ne / 2;
-  const int64_t plane = static_cast<int64_t>(T) * E;
-  if (tid < npairs) {
-    const int e = e0 + 2 * tid;
-    const float* src = part + e;  // token 0
-    float2 l = __ldcg(reinterpret_cast<const float2*>(src));
-    int cc = 1;
-    for (; cc + 16 <= C; cc += 16) {
-      float2 pv[16];
+  if (tid < ne) {
+    // one expert per thread; 28 chunk partials in flight, then the ordered adds
+    const int e = e0 + tid;
+    const float* src = part + e;  // token 0; plane c at src + c * E
+    float l = __ldcg(src);
+    for (int c0 = 1; c0 < C; c0 += 28) {
+      float pv[28];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) pv[u] = __ldcg(reinterpret_cast<const float2*>(src + (cc + u) * plane));
+      for (int u = 0; u < 28; ++u) pv[u] = (c0 + u < C) ? __ldcg(src + static_cast<int64_t>(c0 + u) * E) : 0.0f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        l.x = __fadd_rn(l.x, pv[u].x);
-        l.y = __fadd_rn(l.y, pv[u].y);
-      }
+      for (int u = 0; u < 28; ++u)
+        if (c0 + u < C) l = __fadd_rn(l, pv[u]);
     }
-    for (; cc < C; ++cc) {
-      const float2 pv = __ldcg(reinterpret_cast<const float2*>(src + cc * plane));
-      l.x = __fadd_rn(l.x, pv.x);
-      l.y = __fadd_rn(l.y, pv.y);
-    }
-    if (bias != nullptr) {
-      l.x = __fadd_rn(l.x, __ldg(bias + e));
-      l.y = __fadd_rn(l.y, __ldg(bias + e + 1));
-    }
-    *reinterpret_cast<float2*>(logits + e) = l;
+    if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e));
+    logits[e] = l;
   }
 
   // the last group to finish takes softmax and top-k with the whole CTA
