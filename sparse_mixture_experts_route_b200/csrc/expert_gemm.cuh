@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int fa = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF) + q * 32 + lane;
       const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
       const bool fa_ok = fa < p.n_feat;
-      const bool fb_ok = (kMode == 1) && fb < p.n_feat;
+      const bool fb_ok = !gemm_is_gate_up(kMode) && fb < p.n_feat;
       if (kMode == 2 && p.ksplit > 1) {
         // K split: this CTA's fp32 partial to part[bt][ks]; the slot is free
         // as soon as it is read
@@ -460,14 +460,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // Token blocks per expert for both GEMMs:
 //   prefix0[e] = sum_{e' < e} ceil(count_e' / rows0)  (gate/up, rows0 = 256 or 128)
-//   prefix1[e] = sum_{e' < e} ceil(count_e' / 128)    (down)
+//   prefix1[e] = sum_{e' < e} ceil(count_e' / rows1)  (down, rows1 = 128)
 __global__ void __launch_bounds__(1024)
-    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int rows0, int32_t* __restrict__ prefix0,
-                         int32_t* __restrict__ prefix1) {
+    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int rows0, int rows1, int32_t* __restrict__ prefix0,
+                         int32_t* __restrict__ prefix1, unsigned int* __restrict__ zero_buf, int zero_n) {
   __shared__ int32_t warp_sums[2][32];
   const int e = threadIdx.x;
+  for (int i = e; i < zero_n; i += 1024) zero_buf[i] = 0u;  // K-split tickets of the gate/up GEMM
   const int32_t cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
-  const int32_t nb[2] = {(cnt + rows0 - 1) / rows0, (cnt + gemm_block_rows(1) - 1) / gemm_block_rows(1)};
+  const int32_t nb[2] = {(cnt + rows0 - 1) / rows0, (cnt + rows1 - 1) / rows1};
   const int lane = e & 31, w = e >> 5;
   int32_t incl[2];
 #pragma unroll

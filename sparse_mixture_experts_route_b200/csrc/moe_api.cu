@@ -377,8 +377,9 @@ struct FfnPlan {
   CUtensorMap mA0, mB0, mBs0, mA1, mB1, mBs1;
   GemmParams p0, p1;
   int grid0, grid1;
-  int mode0;  // 0: 256-row gate/up blocks, 2: 128-row gate/up blocks
-  size_t split_ticket_bytes;  // tickets to clear before a K-split gate/up launch (0: no split)
+  int mode0;  // gate/up: 0 256-row blocks, 2 128-row blocks
+  int mode1;  // down: 1 (128-row blocks)
+  int split_ticket_words;  // K-split tickets the schedule kernel clears (0: no split)
 };
 
 moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
@@ -402,6 +403,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p0.out = h;
   // 256-row blocks pay off only when experts average more than 128 rows
   fp->mode0 = (static_cast<int64_t>(Tk) > static_cast<int64_t>(E) * 128) ? 0 : 2;
+  fp->mode1 = 1;
   const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(fp->mode0)) + min_e_tk) * p0.n_feat_tiles;
   const int KB0 = d / kGemmBK;
   int ksplit = 1;
@@ -415,12 +417,12 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p0.ksplit = ceil_div(KB0, p0.kb_per_split);  // every split non-empty
   p0.part = nullptr;
   p0.tickets = nullptr;
-  fp->split_ticket_bytes = 0;
+  fp->split_ticket_words = 0;
   if (p0.ksplit > 1) {
     uint8_t* base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
     p0.part = reinterpret_cast<float*>(base);
     p0.tickets = reinterpret_cast<unsigned int*>(base + ffn_split_part_bytes());
-    fp->split_ticket_bytes = static_cast<size_t>(tiles0) * 4 * sizeof(unsigned);
+    fp->split_ticket_words = static_cast<int>(tiles0) * 4;
   }
   const int64_t ctas0 = tiles0 * p0.ksplit;
   fp->grid0 = static_cast<int>(ctas0 < num_sms ? ctas0 : num_sms);
@@ -436,18 +438,18 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p1.n_feat_tiles = ceil_div(d, 2 * kGemmBMF);
   p1.a1_offset = kGemmBMF;
   p1.out = y_perm;
-  const int64_t tiles1 = (ceil_div64(Tk, gemm_block_rows(1)) + min_e_tk) * p1.n_feat_tiles;
+  const int64_t tiles1 = (ceil_div64(Tk, gemm_block_rows(fp->mode1)) + min_e_tk) * p1.n_feat_tiles;
   fp->grid1 = static_cast<int>(tiles1 < num_sms ? tiles1 : num_sms);
   return MOE_OK;
 }
 
 void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
   gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, gemm_block_rows(fp.mode0),
-                                               const_cast<int32_t*>(fp.p0.tile_prefix),
-                                               const_cast<int32_t*>(fp.p1.tile_prefix));
+                                               gemm_block_rows(fp.mode1), const_cast<int32_t*>(fp.p0.tile_prefix),
+                                               const_cast<int32_t*>(fp.p1.tile_prefix), fp.p0.tickets,
+                                               fp.split_ticket_words);
 }
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
-  if (fp.split_ticket_bytes > 0) cudaMemsetAsync(fp.p0.tickets, 0, fp.split_ticket_bytes, stream);
   if (fp.mode0 == 0)
     grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
   else
@@ -648,9 +650,11 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
   mark(2);
   if (Tk <= kSmallDispatchPairs) {
     // one block: counts, offsets, stable scatter and both GEMM tile prefixes; then the row copy
-    dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, gemm_block_rows(fp.mode0), offsets, perm_token,
-                                                  inv_perm, const_cast<int32_t*>(fp.p0.tile_prefix),
-                                                  const_cast<int32_t*>(fp.p1.tile_prefix));
+    dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, gemm_block_rows(fp.mode0), gemm_block_rows(fp.mode1),
+                                                  offsets, perm_token, inv_perm,
+                                                  const_cast<int32_t*>(fp.p0.tile_prefix),
+                                                  const_cast<int32_t*>(fp.p1.tile_prefix), fp.p0.tickets,
+                                                  fp.split_ticket_words);
     permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
         reinterpret_cast<const uint4*>(x), perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
   } else {

@@ -189,17 +189,21 @@ constexpr int kSmallDispatchPairs = 2048;  // fused single-block dispatch up to 
 // Dispatch for few pairs in one block of 1024 threads (E <= 1024): per-expert
 // counts, exclusive scan (offsets), the stable counting-sort scatter (one warp
 // walks the pairs in order, 32 at a time, ranks from __match_any_sync), and the
-// token-block prefixes of both grouped GEMMs (blocks of rows0 and of 128 rows),
-// so a decode step needs one launch here instead of four.
+// token-block prefixes of both grouped GEMMs (blocks of rows0 and of rows1
+// rows), so a decode step needs one launch here instead of four. It also
+// clears zero_n words at zero_buf (the K-split tickets of the gate/up GEMM
+// that follows; zero_n may be 0).
 __global__ void __launch_bounds__(1024)
-    dispatch_small_kernel(const int32_t* __restrict__ topk_idx, int n_pairs, int E, int k, int rows0,
+    dispatch_small_kernel(const int32_t* __restrict__ topk_idx, int n_pairs, int E, int k, int rows0, int rows1,
                           int32_t* __restrict__ offsets, int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm,
-                          int32_t* __restrict__ prefix0, int32_t* __restrict__ prefix1) {
+                          int32_t* __restrict__ prefix0, int32_t* __restrict__ prefix1, unsigned int* __restrict__ zero_buf,
+                          int zero_n) {
   __shared__ int32_t cnt[1024];
   __shared__ int32_t base[1024];
   __shared__ int32_t wsum[3][32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   cnt[tid] = 0;
+  for (int i = tid; i < zero_n; i += 1024) zero_buf[i] = 0u;
   __syncthreads();
   for (int q = tid; q < n_pairs; q += 1024) {
     const int e = topk_idx[q];
@@ -209,9 +213,9 @@ __global__ void __launch_bounds__(1024)
       record_device_error(5u /* MOE_DEVERR_BAD_ROUTE */);
   }
   __syncthreads();
-  // exclusive scans over experts: rows, 128-row blocks and rows0-row blocks
+  // exclusive scans over experts: rows, rows0-row blocks and rows1-row blocks
   const int32_t c = (tid < E) ? cnt[tid] : 0;
-  int32_t v[3] = {c, (c + rows0 - 1) / rows0, (c + 127) / 128};
+  int32_t v[3] = {c, (c + rows0 - 1) / rows0, (c + rows1 - 1) / rows1};
   int32_t incl[3];
 #pragma unroll
   for (int m = 0; m < 3; ++m) {

@@ -293,7 +293,10 @@ def test_unpermute(lib):
 
 # (600, 128, 4, 2, 128): about 300 rows per expert, so the gate/up GEMM takes
 # 256-row token blocks (N = 256 MMAs) with partial remainders
-@pytest.mark.parametrize("shape", SHAPES + [(300, 128, 8, 2, 128), (600, 128, 4, 2, 128)],
+# (32, 256, 2, 2, 128) and (33, ...): every expert has exactly T rows, one
+# token block each with N = 32 and N = 48 MMAs
+@pytest.mark.parametrize("shape", SHAPES + [(300, 128, 8, 2, 128), (600, 128, 4, 2, 128), (32, 256, 2, 2, 128),
+                                            (33, 256, 2, 2, 128)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_forward(lib, shape):
     T, d, E, k, f = shape
