@@ -314,12 +314,9 @@ moe_status_t launch_permute(const moe_bf16_t* x, const int32_t* idx, int T, int 
   permute_hist_kernel<<<nblk, 256, sm, stream>>>(idx, n_pairs, E, block_hist);
   permute_scan_kernel<<<1, 1024, 0, stream>>>(block_hist, nblk, E, offsets);
   permute_scatter_kernel<<<nblk, 32, sm, stream>>>(idx, n_pairs, E, k, block_hist, perm_token, inv_perm);
-  if (x_perm != nullptr) {
-    const int rows_per_block = 8;
-    const int64_t blocks = ceil_div64(n_pairs, rows_per_block);
-    permute_copy_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), perm_token, n_pairs, d / 8, reinterpret_cast<uint4*>(x_perm));
-  }
+  if (x_perm != nullptr)  // token-major: each row of x is read once and written k times
+    permute_copy_tokens_kernel<<<static_cast<unsigned>(T), 128, 0, stream>>>(
+        reinterpret_cast<const uint4*>(x), inv_perm, k, d / 8, reinterpret_cast<uint4*>(x_perm));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -50,9 +50,17 @@ __global__ void __launch_bounds__(1024)
     permute_scan_kernel(int32_t* __restrict__ block_hist, int nblk, int E, int32_t* __restrict__ offsets) {
   __shared__ int32_t warp_sums[32];
   const int e = threadIdx.x;
+  constexpr int kBatch = 16;  // block counts in flight per thread
   int32_t total = 0;
   if (e < E)
-    for (int b = 0; b < nblk; ++b) total += block_hist[static_cast<int64_t>(b) * E + e];
+    for (int b0 = 0; b0 < nblk; b0 += kBatch) {
+      int32_t c[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        c[u] = (b0 + u < nblk) ? block_hist[static_cast<int64_t>(b0 + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) total += c[u];
+    }
   // exclusive scan of `total` over the block
   const int lane = e & 31, w = e >> 5;
   int32_t incl = total;
@@ -79,11 +87,17 @@ __global__ void __launch_bounds__(1024)
     offsets[e] = excl;
     if (e == E - 1) offsets[E] = excl + total;
     int32_t run = excl;
-    for (int b = 0; b < nblk; ++b) {
-      const int64_t at = static_cast<int64_t>(b) * E + e;
-      const int32_t c = block_hist[at];
-      block_hist[at] = run;
-      run += c;
+    for (int b0 = 0; b0 < nblk; b0 += kBatch) {
+      int32_t c[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        c[u] = (b0 + u < nblk) ? block_hist[static_cast<int64_t>(b0 + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (b0 + u < nblk) {
+          block_hist[static_cast<int64_t>(b0 + u) * E + e] = run;
+          run += c[u];
+        }
     }
   }
 }
@@ -137,6 +151,40 @@ __global__ void __launch_bounds__(256)
     __stcs(dst + v + 96, d);
   }
   for (; v < vec_per_row; v += 32) __stcs(dst + v, __ldg(src + v));
+}
+
+// x_perm[inv_perm[t, j], :] = x[t, :] for every slot j of token t: one CTA of
+// 128 threads per token reads the row once (8 vectors of 16 bytes per thread
+// per pass) and writes its k copies, so x crosses HBM once however many
+// experts a token picks. Same result as the row-by-row gather.
+__global__ void __launch_bounds__(128)
+    permute_copy_tokens_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv_perm, int k,
+                               int vec_per_row, uint4* __restrict__ x_perm) {
+  constexpr int kVec = 8;
+  const int64_t t = blockIdx.x;
+  const int tid = threadIdx.x;
+  int32_t dst_row[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) dst_row[j] = (j < k) ? __ldg(inv_perm + t * k + j) : 0;
+  const uint4* src = x + t * vec_per_row;
+  for (int v0 = 0; v0 < vec_per_row; v0 += 128 * kVec) {
+    uint4 r[kVec];
+#pragma unroll
+    for (int u = 0; u < kVec; ++u) {
+      const int v = v0 + u * 128 + tid;
+      if (v < vec_per_row) r[u] = __ldg(src + v);
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= k) break;
+      uint4* dst = x_perm + static_cast<int64_t>(dst_row[j]) * vec_per_row;
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int v = v0 + u * 128 + tid;
+        if (v < vec_per_row) __stcs(dst + v, r[u]);
+      }
+    }
+  }
 }
 
 // out[t, :] = sum_j w[t, j] * y_perm[inv_perm[t, j], :]; fp32 fma in ascending
