@@ -87,11 +87,15 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
 
 
 def _workspace(nbytes: int, device, stream=None) -> torch.Tensor:
-    # torch's caching allocator returns 512-byte aligned blocks
-    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
-    if stream is not None:
-        ws.record_stream(stream)  # not reused before `stream` has finished with it
-    return ws
+    """Scratch for one call, allocated on the stream the call runs on: torch's
+    caching allocator hands a freed block only to later allocations on the same
+    stream, which run after this call's work, so a workspace freed when the
+    binding returns is never reused by work that overlaps the call. (Blocks
+    are 512-byte aligned.)"""
+    if stream is None:
+        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def version() -> int:

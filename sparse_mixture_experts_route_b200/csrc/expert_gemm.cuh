@@ -85,59 +85,93 @@ struct GemmParams {
   int n_feat_tiles;  // mode 0: ceil(f / 128); mode 1: ceil(d / 256)
   int a1_offset;     // column of the second A operand: f + j0 (mode 0) or n0 + 128 (mode 1), minus j0 / n0
   uint16_t* out;     // [Tk, n_feat] bf16
-  // K split (mode 2 only; ksplit == 1 elsewhere): output tile t is computed as
-  // ksplit partial products over K blocks [s * kb_per_split, ...), written to
-  // part[t][s] as fp32; for each 32-feature slice, the last of the ksplit
-  // CTAs to finish it (a ticket) adds them in ascending s and applies the
-  // SiLU-gate. tickets[] start at zero and
-  // are put back to zero.
-  int ksplit;
-  int kb_per_split;
-  float* part;            // [tiles][ksplit][2][128 rows][128 features] fp32
+  // Stream-K (stream_k != 0; modes 1 and 2): the units (output tile t, K block
+  // kb), t-major, are split evenly over the CTAs, CTA c taking units
+  // [c * per, (c + 1) * per) with per = ceil(units / gridDim.x), so every SM
+  // streams the same number of weight blocks however few tiles there are. A
+  // CTA's share is a run of work items, each one tile's K-block range; an item
+  // that covers a tile's whole K range is finished as usual, a partial item
+  // writes its fp32 accumulators to part[slot] (slot 2c for the CTA's first
+  // item, 2c + 1 for its last), and for each 32-feature slice the last of the
+  // tile's contributors to finish (a ticket) adds the partials in ascending
+  // CTA order, which is ascending K, and finishes the tile. tickets[] start at
+  // zero and are put back to zero.
+  int stream_k;
+  float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
   unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
 };
 
-// fp32 elements of one split partial: gate and up, 128 rows x 128 features
+// fp32 elements of one partial: two accumulators, 128 rows x 128 features
 constexpr int kSplitPartFloats = 2 * 128 * kGemmBMF;
 
 struct TileInfo {
   int e, nb, row0, nrows, nblocks;  // nblocks: token blocks of expert e
-  int bt, ks, kb0, kb1;             // output tile, K split, K-block range [kb0, kb1)
+  int t, kb0, kb1;                  // tile index, K-block range [kb0, kb1) of this item
+  bool partial;                     // the item covers only part of the tile's K range
+  int slot;                         // partial slot of this CTA's item
 };
 
-// Tile -> (expert, feature block, token block), from shared-memory copies of
+// Tile t -> (expert, feature block, token block), from shared-memory copies of
 // the tile prefix (pre[0..E]) and the expert offsets (off[0..E]).
 template <int kMode>
-__device__ __forceinline__ bool decode_tile(const GemmParams& p, const int32_t* pre, const int32_t* off, int tile,
+__device__ __forceinline__ void decode_tile(const GemmParams& p, const int32_t* pre, const int32_t* off, int t,
                                             TileInfo& ti) {
   constexpr int BR = gemm_block_rows(kMode);
   const int NB = p.n_feat_tiles;
-  // consecutive tiles are the K splits of one output tile
-  const int bt = tile / p.ksplit;
-  const int ks = tile - bt * p.ksplit;
-  if (bt >= pre[p.E] * NB) return false;
-  // owner: the largest e with pre[e] * NB <= bt
+  // owner: the largest e with pre[e] * NB <= t
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (pre[mid] * NB <= bt)
+    if (pre[mid] * NB <= t)
       lo = mid;
     else
       hi = mid - 1;
   }
   const int e = lo;
   const int tb_count = pre[e + 1] - pre[e];
-  const int local = bt - pre[e] * NB;
+  const int local = t - pre[e] * NB;
   const int tb = local % tb_count;
   ti.e = e;
   ti.nblocks = tb_count;
   ti.nb = local / tb_count;
   ti.row0 = off[e] + tb * BR;
   ti.nrows = min(BR, off[e + 1] - ti.row0);
-  ti.bt = bt;
-  ti.ks = ks;
-  ti.kb0 = ks * p.kb_per_split;
-  ti.kb1 = min(p.K / kGemmBK, ti.kb0 + p.kb_per_split);
+  ti.t = t;
+}
+
+// Units of stream-K work per CTA (see GemmParams).
+__device__ __forceinline__ int stream_k_per(int ntiles, int KB) {
+  return (ntiles * KB + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+}
+
+// The it-th work item of this CTA: tiles blockIdx.x, blockIdx.x + gridDim.x,
+// ... with their whole K range, or, with stream-K, the tiles its unit range
+// touches with the K blocks inside that range.
+template <int kMode>
+__device__ __forceinline__ bool work_item(const GemmParams& p, const int32_t* pre, const int32_t* off, int it,
+                                          TileInfo& ti) {
+  const int KB = p.K / kGemmBK;
+  const int ntiles = pre[p.E] * p.n_feat_tiles;
+  if (!p.stream_k) {
+    const int t = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+    if (t >= ntiles) return false;
+    decode_tile<kMode>(p, pre, off, t, ti);
+    ti.kb0 = 0;
+    ti.kb1 = KB;
+    ti.partial = false;
+    ti.slot = -1;
+    return true;
+  }
+  const int per = stream_k_per(ntiles, KB);
+  const int u0 = static_cast<int>(blockIdx.x) * per;
+  const int u1 = min(ntiles * KB, u0 + per);
+  const int t = u0 / KB + it;
+  if (u0 >= u1 || t * KB >= u1) return false;
+  decode_tile<kMode>(p, pre, off, t, ti);
+  ti.kb0 = max(u0, t * KB) - t * KB;
+  ti.kb1 = min(u1, (t + 1) * KB) - t * KB;
+  ti.partial = ti.kb0 > 0 || ti.kb1 < KB;
+  ti.slot = 2 * static_cast<int>(blockIdx.x) + (it == 0 ? 0 : 1);
   return true;
 }
 
@@ -232,7 +266,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int issued = 0;
       bool ok = true;
       TileInfo ti;
-      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
+      for (int it = 0; ok && work_item<kMode>(p, s_pre, s_off, it, ti); ++it) {
         const int f0 = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF);
         const int f1 = f0 + p.a1_offset;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
@@ -287,7 +321,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       bool any = false;
       TileInfo ti;
-      for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
+      for (int it = 0; ok && work_item<kMode>(p, s_pre, s_off, it, ti); ++it) {
         const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
         const uint32_t idesc = umma_idesc_bf16_f32(128u, n_mma, 1u, 0u);
         const SlotPlan sp = slot_plan(ti.nrows, next_slot);
@@ -350,7 +384,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int next_slot = 0;
     bool ok = true;
     TileInfo ti;
-    for (int tile = blockIdx.x; ok && decode_tile<kMode>(p, s_pre, s_off, tile, ti); tile += gridDim.x) {
+    for (int it = 0; ok && work_item<kMode>(p, s_pre, s_off, it, ti); ++it) {
       const SlotPlan sp = slot_plan(ti.nrows, next_slot);
       for (int j = 0; j < sp.count && ok; ++j) {
         const int sl = sp.first + j;
@@ -368,11 +402,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
       const bool fa_ok = fa < p.n_feat;
       const bool fb_ok = !gemm_is_gate_up(kMode) && fb < p.n_feat;
-      if (kMode == 2 && p.ksplit > 1) {
-        // K split: this CTA's fp32 partial to part[bt][ks]; the slot is free
-        // as soon as it is read
+      if (kMode != 0 && ti.partial) {
+        // stream-K partial item: fp32 accumulators to part[slot]; the TMEM
+        // slot is free as soon as it is read
         const int fl = q * 32 + lane;
-        float* mine = p.part + (static_cast<int64_t>(ti.bt) * p.ksplit + ti.ks) * kSplitPartFloats;
+        float* mine = p.part + static_cast<int64_t>(ti.slot) * kSplitPartFloats;
         for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
           uint32_t g[32], u[32];
           tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
@@ -393,27 +427,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) mbar_arrive(&acc_empty_bar[sp.first + j]);
           ++uses[sp.first + j];
         }
-        // ticket per (output tile, warp): the last split to finish these 32
-        // features adds the partials in ascending split order
+        // the tile's contributors are CTAs c_first..c_last; per (tile, warp),
+        // the last one to finish adds their partials in CTA order (K order)
+        const int KB = p.K / kGemmBK;
+        const int per = stream_k_per(s_pre[p.E] * p.n_feat_tiles, KB);
+        const int c_first = (ti.t * KB) / per, c_last = ((ti.t + 1) * KB - 1) / per;
         __threadfence();
         __syncwarp();
         unsigned int tk = 0u;
-        if (lane == 0) tk = atomicAdd(&p.tickets[ti.bt * 4 + q], 1u);
+        if (lane == 0) tk = atomicAdd(&p.tickets[ti.t * 4 + q], 1u);
         tk = __shfl_sync(0xffffffffu, tk, 0);
-        if (tk == static_cast<unsigned int>(p.ksplit - 1)) {
+        if (tk == static_cast<unsigned int>(c_last - c_first)) {
           __threadfence();
-          const float* all = p.part + static_cast<int64_t>(ti.bt) * p.ksplit * kSplitPartFloats;
           for (int i = 0; i < ti.nrows; ++i) {
-            float gs = __ldcg(all + i * kGemmBMF + fl);
-            float us = __ldcg(all + (128 + i) * kGemmBMF + fl);
-            for (int sk = 1; sk < p.ksplit; ++sk) {
-              gs = __fadd_rn(gs, __ldcg(all + sk * kSplitPartFloats + i * kGemmBMF + fl));
-              us = __fadd_rn(us, __ldcg(all + sk * kSplitPartFloats + (128 + i) * kGemmBMF + fl));
+            float gs = 0.0f, us = 0.0f;
+            for (int c = c_first; c <= c_last; ++c) {
+              const int slot = 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
+              const float* src = p.part + static_cast<int64_t>(slot) * kSplitPartFloats;
+              const float gv = __ldcg(src + i * kGemmBMF + fl);
+              const float uv = __ldcg(src + (128 + i) * kGemmBMF + fl);
+              gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
+              us = (c == c_first) ? uv : __fadd_rn(us, uv);
             }
-            if (fa_ok)
-              p.out[static_cast<int64_t>(ti.row0 + i) * p.n_feat + fa] = bf16_bits(silu_f32(gs) * us);
+            uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
+            if (gemm_is_gate_up(kMode)) {
+              if (fa_ok) orow[fa] = bf16_bits(silu_f32(gs) * us);
+            } else {
+              if (fa_ok) orow[fa] = bf16_bits(gs);
+              if (fb_ok) orow[fb] = bf16_bits(us);
+            }
           }
-          if (lane == 0) p.tickets[ti.bt * 4 + q] = 0u;
+          if (lane == 0) p.tickets[ti.t * 4 + q] = 0u;
         }
         continue;
       }

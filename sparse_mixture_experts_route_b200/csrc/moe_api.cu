@@ -322,21 +322,24 @@ moe_status_t launch_permute(const moe_bf16_t* x, const int32_t* idx, int T, int 
 
 // -------------------------------------------------------------- expert FFN
 
-// K split of the gate/up GEMM when an upper bound on its output tiles is at
-// most half of kSplitTargetCtas (one CTA per SM of a 148-SM part): each tile
-// becomes ksplit CTAs over disjoint K ranges, so a few-token step streams the
-// touched experts' weights with every SM instead of a third of them.
-constexpr int kSplitTargetCtas = 148;
-constexpr int kSplitMaxK = 4;
+// Stream-K for a grouped GEMM whose output tiles (an upper bound from Tk and
+// E) fill at most kStreamKMaxWaves waves of one CTA per SM of a 148-SM part:
+// with that few tiles, whole-tile scheduling leaves SMs idle (a 64-tile
+// one-token step uses 64 of 148 SMs; 448 tiles leave a fourth wave of 4), so
+// the (tile, K block) units are split evenly over kStreamKCtas CTAs instead.
+constexpr int kStreamKCtas = 148;
+constexpr int kStreamKMaxWaves = 4;
 
-// Workspace of the expert FFN: the two tile-prefix arrays, then (only when a K
-// split is possible for this Tk and E, i.e. min(E, Tk) <= kSplitTargetCtas / 2)
-// the split partials (at most kSplitTargetCtas tile-splits) and tickets.
+// Workspace of the expert FFN: the two tile-prefix arrays, then (only when
+// stream-K is possible for this Tk and E, i.e. min(E, Tk) <= the tile limit)
+// the partials (two slots per CTA) and the tickets (four per tile).
 size_t ffn_split_part_bytes() {
-  return align256(static_cast<size_t>(kSplitTargetCtas) * kSplitPartFloats * sizeof(float));
+  return align256(static_cast<size_t>(2 * kStreamKCtas) * kSplitPartFloats * sizeof(float));
 }
-size_t ffn_split_ticket_bytes() { return align256(static_cast<size_t>(kSplitTargetCtas / 2) * 4 * sizeof(unsigned)); }
-bool ffn_split_possible(int Tk, int E) { return (E < Tk ? E : Tk) <= kSplitTargetCtas / 2; }
+size_t ffn_split_ticket_bytes() {
+  return align256(static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * 4 * sizeof(unsigned));
+}
+bool ffn_split_possible(int Tk, int E) { return (E < Tk ? E : Tk) <= kStreamKMaxWaves * kStreamKCtas; }
 size_t ffn_prefix_bytes(int E) { return align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
 size_t ffn_ws(int Tk, int E) {
   size_t b = 2 * ffn_prefix_bytes(E);
@@ -376,7 +379,8 @@ struct FfnPlan {
   int grid0, grid1;
   int mode0;  // gate/up: 0 256-row blocks, 2 128-row blocks
   int mode1;  // down: 1 (128-row blocks)
-  int split_ticket_words;  // K-split tickets the schedule kernel clears (0: no split)
+  int split_ticket_words;     // stream-K tickets the schedule kernel clears (0: none)
+  unsigned int* ticket_buf;   // where they are
 };
 
 moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
@@ -402,33 +406,17 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   fp->mode0 = (static_cast<int64_t>(Tk) > static_cast<int64_t>(E) * 128) ? 0 : 2;
   fp->mode1 = 1;
   const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(fp->mode0)) + min_e_tk) * p0.n_feat_tiles;
-  const int KB0 = d / kGemmBK;
-  int ksplit = 1;
-  if (fp->mode0 == 2 && ffn_split_possible(Tk, E) && 2 * tiles0 <= kSplitTargetCtas) {
-    ksplit = static_cast<int>(kSplitTargetCtas / tiles0);
-    ksplit = ksplit > kSplitMaxK ? kSplitMaxK : ksplit;
-    ksplit = ksplit > KB0 / 8 ? KB0 / 8 : ksplit;
-    if (ksplit < 2) ksplit = 1;
-  }
-  p0.kb_per_split = ceil_div(KB0, ksplit);
-  p0.ksplit = ceil_div(KB0, p0.kb_per_split);  // every split non-empty
-  p0.part = nullptr;
-  p0.tickets = nullptr;
-  fp->split_ticket_words = 0;
-  if (p0.ksplit > 1) {
-    uint8_t* base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
-    p0.part = reinterpret_cast<float*>(base);
-    p0.tickets = reinterpret_cast<unsigned int*>(base + ffn_split_part_bytes());
-    fp->split_ticket_words = static_cast<int>(tiles0) * 4;
-  }
-  const int64_t ctas0 = tiles0 * p0.ksplit;
-  fp->grid0 = static_cast<int>(ctas0 < num_sms ? ctas0 : num_sms);
+  const bool stream_ok = ffn_split_possible(Tk, E);
+  uint8_t* split_base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
+  float* part = stream_ok ? reinterpret_cast<float*>(split_base) : nullptr;
+  unsigned int* tickets = stream_ok ? reinterpret_cast<unsigned int*>(split_base + ffn_split_part_bytes()) : nullptr;
+  p0.stream_k = (stream_ok && fp->mode0 == 2 && tiles0 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
+  p0.part = p0.stream_k ? part : nullptr;
+  p0.tickets = p0.stream_k ? tickets : nullptr;
+  fp->grid0 = p0.stream_k ? (kStreamKCtas < num_sms ? kStreamKCtas : num_sms)
+                          : static_cast<int>(tiles0 < num_sms ? tiles0 : num_sms);
   GemmParams& p1 = fp->p1;
   p1 = p0;
-  p1.ksplit = 1;
-  p1.kb_per_split = f / kGemmBK;
-  p1.part = nullptr;
-  p1.tickets = nullptr;
   p1.tile_prefix = prefix1;
   p1.K = f;
   p1.n_feat = d;
@@ -436,14 +424,24 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p1.a1_offset = kGemmBMF;
   p1.out = y_perm;
   const int64_t tiles1 = (ceil_div64(Tk, gemm_block_rows(fp->mode1)) + min_e_tk) * p1.n_feat_tiles;
-  fp->grid1 = static_cast<int>(tiles1 < num_sms ? tiles1 : num_sms);
+  p1.stream_k = (stream_ok && tiles1 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
+  p1.part = p1.stream_k ? part : nullptr;
+  p1.tickets = p1.stream_k ? tickets : nullptr;
+  fp->grid1 = p1.stream_k ? (kStreamKCtas < num_sms ? kStreamKCtas : num_sms)
+                          : static_cast<int>(tiles1 < num_sms ? tiles1 : num_sms);
+  // the tickets start at zero: the schedule kernel clears them (both GEMMs
+  // share them; each tile's last contributor puts its tickets back to zero)
+  const int64_t max_tiles = (p0.stream_k ? tiles0 : 0) > (p1.stream_k ? tiles1 : 0) ? (p0.stream_k ? tiles0 : 0)
+                                                                                      : (p1.stream_k ? tiles1 : 0);
+  fp->split_ticket_words = static_cast<int>(max_tiles) * 4;
+  fp->ticket_buf = tickets;
   return MOE_OK;
 }
 
 void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
   gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, gemm_block_rows(fp.mode0),
                                                gemm_block_rows(fp.mode1), const_cast<int32_t*>(fp.p0.tile_prefix),
-                                               const_cast<int32_t*>(fp.p1.tile_prefix), fp.p0.tickets,
+                                               const_cast<int32_t*>(fp.p1.tile_prefix), fp.ticket_buf,
                                                fp.split_ticket_words);
 }
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
@@ -650,7 +648,7 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
     dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, gemm_block_rows(fp.mode0), gemm_block_rows(fp.mode1),
                                                   offsets, perm_token, inv_perm,
                                                   const_cast<int32_t*>(fp.p0.tile_prefix),
-                                                  const_cast<int32_t*>(fp.p1.tile_prefix), fp.p0.tickets,
+                                                  const_cast<int32_t*>(fp.p1.tile_prefix), fp.ticket_buf,
                                                   fp.split_ticket_words);
     permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
         reinterpret_cast<const uint4*>(x), perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
