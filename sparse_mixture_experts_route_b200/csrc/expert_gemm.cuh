@@ -97,6 +97,7 @@ struct GemmParams {
   // CTA order, which is ascending K, and finishes the tile. tickets[] start at
   // zero and are put back to zero.
   int stream_k;
+  int b_fixed_row;        // >= 0: every tile's token operand starts at this row (one-token steps read x itself)
   float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
   unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
 };
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_3d(st + Cfg::kABytes + Cfg::kAHalf, &tmA, &full_bar[s], f1 + 64, k0, ti.e, pol_w);
           uint8_t* bdst = st + 2 * Cfg::kABytes;
           if (small_box) {
-            tma_load_2d(bdst, &tmBs, &full_bar[s], k0, ti.row0, pol_x);
+            tma_load_2d(bdst, &tmBs, &full_bar[s], k0, p.b_fixed_row >= 0 ? p.b_fixed_row : ti.row0, pol_x);
           } else {
             for (int b = 0; b < nbox; ++b)
               tma_load_2d(bdst + b * kGemmBoxRows * kGemmBK * 2, &tmB, &full_bar[s], k0, ti.row0 + b * kGemmBoxRows,

@@ -227,8 +227,12 @@ moe_status_t launch_route_tc(const RoutePlan& plan, const moe_bf16_t* x, const f
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// disp (one-token steps in moe_forward only): when the fused one-token router
+// runs, it also writes these dispatch tables and *dispatched is set.
 moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const float* bias, int T, int d, int E, int k,
-                          int32_t* idx, float* w, void* ws, cudaStream_t stream) {
+                          int32_t* idx, float* w, void* ws, cudaStream_t stream,
+                          const RouteDispatch* disp = nullptr, bool* dispatched = nullptr) {
+  if (dispatched != nullptr) *dispatched = false;
   const RoutePlan plan = route_plan(T, d, E);
   if (plan.variant == kRouterTensorCore) return launch_route_tc(plan, x, W_router, bias, T, d, E, k, idx, w, ws, stream);
   float* lg = static_cast<float*>(ws);
@@ -247,15 +251,18 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
       return MOE_ERR_CUDA;
     const dim3 grid(G, plan.nchunks);
     const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
-    if (T == 1)
+    const RouteDispatch none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0};
+    if (T == 1) {
       router_stream_kernel<1><<<grid, kRsThreads, router_stream_smem_bytes(1), stream>>>(
-          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
-    else if (T <= 4)
+          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w, disp != nullptr ? *disp : none);
+      if (dispatched != nullptr && disp != nullptr) *dispatched = true;
+    } else if (T <= 4) {
       router_stream_kernel<4><<<grid, kRsThreads, router_stream_smem_bytes(4), stream>>>(
-          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
-    else
+          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w, none);
+    } else {
       router_stream_kernel<16><<<grid, kRsThreads, router_stream_smem_bytes(16), stream>>>(
-          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w);
+          xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w, none);
+    }
     if (T > 1) router_reduce_topk_kernel<<<T, 256, 0, stream>>>(lg, plan.nchunks, bias, T, E, k, idx, w);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
@@ -410,6 +417,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   uint8_t* split_base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
   float* part = stream_ok ? reinterpret_cast<float*>(split_base) : nullptr;
   unsigned int* tickets = stream_ok ? reinterpret_cast<unsigned int*>(split_base + ffn_split_part_bytes()) : nullptr;
+  p0.b_fixed_row = -1;
   p0.stream_k = (stream_ok && fp->mode0 == 2 && tiles0 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
   p0.part = p0.stream_k ? part : nullptr;
   p0.tickets = p0.stream_k ? tickets : nullptr;
@@ -417,6 +425,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
                           : static_cast<int>(tiles0 < num_sms ? tiles0 : num_sms);
   GemmParams& p1 = fp->p1;
   p1 = p0;
+  p1.b_fixed_row = -1;
   p1.tile_prefix = prefix1;
   p1.K = f;
   p1.n_feat = d;
@@ -639,11 +648,25 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
     if (ev) cudaEventRecord(ev[i], stream);
   };
   mark(0);
-  st = launch_route(x, W_router, router_bias, T, d, E, k, idx, w, ws + L.route, stream);
+  // one token: the router's last CTA also writes the dispatch tables, and the
+  // gate/up GEMM reads its token operand straight from x (every tile is that
+  // one row), so neither the dispatch kernel nor the row copy runs
+  const RouteDispatch disp = {offsets, perm_token, inv_perm, const_cast<int32_t*>(fp.p0.tile_prefix),
+                              const_cast<int32_t*>(fp.p1.tile_prefix), fp.ticket_buf, fp.split_ticket_words};
+  bool dispatched = false;
+  st = launch_route(x, W_router, router_bias, T, d, E, k, idx, w, ws + L.route, stream, T == 1 ? &disp : nullptr,
+                    &dispatched);
   if (st != MOE_OK) return st;
   mark(1);
   mark(2);
-  if (Tk <= kSmallDispatchPairs) {
+  if (dispatched) {
+    if (act_map(&fp.mB0, x, 1, d, kGemmBoxRows) && act_map(&fp.mBs0, x, 1, d, kGemmSmallBox)) {
+      fp.p0.b_fixed_row = 0;
+    } else {  // the maps of the permuted copy stay; make the copy
+      permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
+          reinterpret_cast<const uint4*>(x), perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
+    }
+  } else if (Tk <= kSmallDispatchPairs) {
     // one block: counts, offsets, stable scatter and both GEMM tile prefixes; then the row copy
     dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, gemm_block_rows(fp.mode0), gemm_block_rows(fp.mode1),
                                                   offsets, perm_token, inv_perm,

@@ -44,12 +44,29 @@ __host__ __device__ constexpr int router_stream_smem_bytes(int tmax) {
   return kRsRows * kRsExperts * 4 + kRsRows * tmax * 4;
 }
 
+// The dispatch tables of a one-token step, written by the router's last CTA
+// when offsets != nullptr (the same values the dispatch kernels would write:
+// with one token every selected expert has exactly one row, in ascending
+// expert order): expert offsets and both GEMM token-block prefixes
+// (offsets[e] = prefix[e] = number of selected experts below e), perm_token
+// (all token 0), inv_perm (the row of each slot); zero_n words of zero_buf are
+// cleared (the GEMMs' stream-K tickets).
+struct RouteDispatch {
+  int32_t* offsets;
+  int32_t* perm_token;
+  int32_t* inv_perm;
+  int32_t* prefix0;
+  int32_t* prefix1;
+  unsigned int* zero_buf;
+  int zero_n;
+};
+
 template <int TMAX>
 __global__ void __launch_bounds__(kRsThreads)
     router_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, const float* __restrict__ bias,
                          int T, int d, int E, int k, float* __restrict__ part, float* __restrict__ logits,
                          unsigned int* __restrict__ tickets, int32_t* __restrict__ topk_idx,
-                         float* __restrict__ topk_w) {
+                         float* __restrict__ topk_w, const RouteDispatch disp) {
   static_assert(TMAX == 1 || TMAX == 4 || TMAX == 16, "token tile");
   extern __shared__ __align__(128) uint8_t rs_smem[];
   float* ws = reinterpret_cast<float*>(rs_smem);  // [kRsRows][kRsExperts]
@@ -178,6 +195,27 @@ __global__ void __launch_bounds__(kRsThreads)
   for (int e = tid; e < E; e += kRsThreads) s_l[e] = __ldcg(logits + e);
   __syncthreads();
   cta_softmax_topk_256(s_l, E, k, topk_idx, topk_w);
+  if (disp.offsets == nullptr) return;
+
+  // the dispatch tables of this one-token step
+  __shared__ int32_t s_sel[16];
+  __syncthreads();  // the selection (written by warp 0) is visible to the CTA
+  if (tid < k) s_sel[tid] = __ldcg(topk_idx + tid);
+  for (int i = tid; i < disp.zero_n; i += kRsThreads) disp.zero_buf[i] = 0u;
+  __syncthreads();
+  for (int e = tid; e <= E; e += kRsThreads) {
+    int32_t below = 0;
+    for (int j = 0; j < k; ++j) below += (s_sel[j] < e) ? 1 : 0;
+    disp.offsets[e] = below;
+    disp.prefix0[e] = below;
+    disp.prefix1[e] = below;
+  }
+  if (tid < k) {
+    int32_t row = 0;
+    for (int j = 0; j < k; ++j) row += (s_sel[j] < s_sel[tid]) ? 1 : 0;
+    disp.perm_token[tid] = 0;
+    disp.inv_perm[tid] = row;
+  }
 }
 
 }  // namespace moe

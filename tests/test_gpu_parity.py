@@ -295,8 +295,10 @@ def test_unpermute(lib):
 # 256-row token blocks (N = 256 MMAs) with partial remainders
 # (32, 256, 2, 2, 128) and (33, ...): every expert has exactly T rows, one
 # token block each with N = 32 and N = 48 MMAs
+# (1, 128, 6, 2, 64): one token with E % 4 != 0, so the split-chunk router and
+# the dispatch kernel run instead of the fused one-token path
 @pytest.mark.parametrize("shape", SHAPES + [(300, 128, 8, 2, 128), (600, 128, 4, 2, 128), (32, 256, 2, 2, 128),
-                                            (33, 256, 2, 2, 128)],
+                                            (33, 256, 2, 2, 128), (1, 128, 6, 2, 64)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_forward(lib, shape):
     T, d, E, k, f = shape
