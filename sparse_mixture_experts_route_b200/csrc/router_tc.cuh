@@ -39,6 +39,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "router.cuh"
 
 namespace moe {
 
@@ -347,25 +348,25 @@ __device__ __forceinline__ void stage_x_pairs(const uint16_t* __restrict__ xt, i
 // Chunk partials of the exact-order logit of one expert: lane l runs the fma
 // chains of chunks l and l + 32 (each from +0, offsets j ascending), reading
 // its two chunks of Wc with one 8-byte load and of xs with one 4-byte load per
-// offset; 16 offsets of loads are issued before their fmas. FULL: d % 128 == 0.
+// offset. The Wc loads come from L2, so 32 offsets of them are issued before
+// their fmas (four L2 round trips per expert); the xs loads are shared-memory
+// reads issued in the fma loop. FULL: d % 128 == 0.
 template <bool FULL>
 __device__ __forceinline__ void exact_chunk_pairs(const uint32_t* __restrict__ xs, const float2* __restrict__ wce,
                                                   int d, int lane, float& p0, float& p1) {
+  constexpr int kB = 32;
   const int n0 = FULL ? 128 : max(0, min(128, d - lane * 128));
   const int n1 = FULL ? 128 : max(0, min(128, d - (lane + 32) * 128));
   p0 = 0.0f;
   p1 = 0.0f;
-  for (int j = 0; j < 128; j += 16) {
-    float2 w[16];
-    uint32_t xv[16];
+  for (int j = 0; j < 128; j += kB) {
+    float2 w[kB];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      w[u] = __ldg(wce + (j + u) * 32 + lane);
-      xv[u] = xs[(j + u) * 32 + lane];
-    }
+    for (int u = 0; u < kB; ++u) w[u] = __ldg(wce + (j + u) * 32 + lane);
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const float xa = __uint_as_float(xv[u] << 16), xb = __uint_as_float(xv[u] & 0xFFFF0000u);
+    for (int u = 0; u < kB; ++u) {
+      const uint32_t xv = xs[(j + u) * 32 + lane];
+      const float xa = __uint_as_float(xv << 16), xb = __uint_as_float(xv & 0xFFFF0000u);
       if (FULL || j + u < n0) p0 = __fmaf_rn(xa, w[u].x, p0);
       if (FULL || j + u < n1) p1 = __fmaf_rn(xb, w[u].y, p1);
     }
@@ -450,27 +451,27 @@ __global__ void __launch_bounds__(kRcWarps * 32, 6)
     const int limit = (E <= kMaxCand) ? E : kMaxCand;
     bool overflowed = false;
     while (true) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+      // warp arg-max by (A desc, index asc): a lane's values are in ascending
+      // expert order, so a strict '>' keeps its lowest index among equal
+      // values; across lanes the largest order key wins, then the lowest index
+      float lv = -INFINITY;
+      int li = -1;
 #pragma unroll
       for (int i = 0; i < MAXV; ++i) {
         const int e = i * 32 + lane;
         const bool cand = e < E && !((taken >> i) & 1u);
-        if (cand && (bi == 0x7fffffff || v[i] > bv)) {
-          bv = v[i];
-          bi = e;
+        if (cand && (li < 0 || v[i] > lv)) {
+          lv = v[i];
+          li = e;
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (bi == 0x7fffffff) break;                  // every expert taken
+      const uint32_t key = li < 0 ? 0u : float_order_key(lv + 0.0f);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+      if (kmax == 0u) break;                        // every expert taken
+      const uint32_t win =
+          __reduce_min_sync(0xffffffffu, (li >= 0 && key == kmax) ? static_cast<uint32_t>(li) : 0xffffffffu);
+      const int bi = static_cast<int>(win);
+      const float bv = __shfl_sync(0xffffffffu, lv, bi & 31);
       if (nc == k - 1) tau = bv;
       if (nc >= k && bv < tau - 2.0f * eps) break;  // outside the window
       if (nc == limit) {                            // window too wide: exact fallback
@@ -530,24 +531,17 @@ __global__ void __launch_bounds__(kRcWarps * 32, 6)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, o);
     const float s = s_s + corr;
-    bool used = !mine;
-    for (int j = 0; j < k; ++j) {
-      float bv = used ? -INFINITY : my_l;
-      int bi = used ? 0x7fffffff : my_e;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (!used && bi == my_e) used = true;
-      if (lane == 0) {
-        topk_idx[static_cast<int64_t>(t) * k + j] = bi;
-        topk_w[static_cast<int64_t>(t) * k + j] = expf(bv - m) / s;
-      }
+    // each candidate's slot is its rank among the candidates by (L desc,
+    // index asc); the k best are written
+    int rank = 0;
+    for (int q = 0; q < nc; ++q) {
+      const float lq = s_l[q];
+      const int eq = s_e[q];
+      rank += (lq > my_l || (lq == my_l && eq < my_e)) ? 1 : 0;
+    }
+    if (mine && rank < k) {
+      topk_idx[static_cast<int64_t>(t) * k + rank] = my_e;
+      topk_w[static_cast<int64_t>(t) * k + rank] = expf(my_l - m) / s;
     }
   }
 }
