@@ -81,7 +81,10 @@ const char* moe_status_string(moe_status_t status);
  * Inputs:  x [T, d] bf16; W_router [d, E] fp32; router_bias [E] fp32 or NULL.
  * Outputs: topk_idx [T, k] int32; topk_w [T, k] fp32.
  * Scratch: workspace of at least moe_route_workspace_size(T, d, E) bytes,
- *   256-byte aligned (holds fp32 logits or per-chunk partial sums).
+ *   256-byte aligned (holds fp32 logits or per-chunk partial sums; for T <= 16
+ *   and E % 4 == 0 also the final logits and the completion counters of the
+ *   single-launch few-token router, which the call clears itself; for
+ *   T >= 256 the tensor-core screen's operands and partial sums).
  */
 size_t moe_route_workspace_size(int T, int d, int E);
 moe_status_t moe_route(const moe_bf16_t* x, const float* W_router, const float* router_bias,
@@ -121,7 +124,11 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx,
  * Inputs: x_perm [Tk, d] bf16; expert_offsets [E+1] int32 (device; read on the
  *   device, no host sync); W_gate_up [E, d, 2f] bf16; W_down [E, f, d] bf16.
  * Outputs: h [Tk, f] bf16 (also the operand of the second GEMM); y_perm [Tk, d].
- * Scratch: moe_expert_ffn_workspace_size(Tk, E) bytes, 256-byte aligned.
+ * Scratch: moe_expert_ffn_workspace_size(Tk, E) bytes, 256-byte aligned: the
+ *   GEMM tile schedules and, when min(E, Tk) <= 592 (few output tiles, where
+ *   the GEMMs split (tile, K-block) work evenly over the SMs), fp32 partial
+ *   tiles and completion counters. Results do not depend on the split: every
+ *   partial sum is added in ascending K order.
  */
 size_t moe_expert_ffn_workspace_size(int Tk, int E);
 moe_status_t moe_expert_ffn(const moe_bf16_t* x_perm, const int32_t* expert_offsets,
