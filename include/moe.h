@@ -127,8 +127,8 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx,
  * Scratch: moe_expert_ffn_workspace_size(Tk, E) bytes, 256-byte aligned: the
  *   GEMM tile schedules and, when min(E, Tk) <= 592 (few output tiles, where
  *   the GEMMs split (tile, K-block) work evenly over the SMs), fp32 partial
- *   tiles and completion counters. Results do not depend on the split: every
- *   partial sum is added in ascending K order.
+ *   tiles and completion counters. The split follows from the shapes and the
+ *   partial sums are added in ascending K order, so results are deterministic.
  */
 size_t moe_expert_ffn_workspace_size(int Tk, int E);
 moe_status_t moe_expert_ffn(const moe_bf16_t* x_perm, const int32_t* expert_offsets,
