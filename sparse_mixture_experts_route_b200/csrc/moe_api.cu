@@ -118,13 +118,23 @@ RoutePlan route_plan(int T, int d, int E) {
   const int64_t big_tiles = ceil_div64(T, 128) * ceil_div64(E, 64);
   if (T >= kRouterTcMinTokens && d % 64 == 0 && d <= 8192 && E >= 16) {
     p.variant = kRouterTensorCore;
-    // split K so the screen has about two CTAs per SM of a 148-SM part; every
-    // split keeps at least 8 K blocks
+    // K split of the screen (one CTA per SM: 197 KB of shared memory): the
+    // split count minimising waves x K blocks per CTA on a 148-SM part plus the
+    // cost of each extra partial plane (written by the screen, read by the
+    // reduce: 8 bytes per (token, expert) at about 6.5 TB/s), with a K block
+    // taken as about a microsecond; every split keeps at least 8 K blocks
     const int KB = d / kRtBK;
     const int64_t tiles = ceil_div64(T, kScrT) * ceil_div64(E, kScrE);
-    int ns = static_cast<int>(ceil_div64(296, tiles));
-    ns = ns < 1 ? 1 : ns;
-    ns = ns > KB / 8 ? (KB / 8 > 0 ? KB / 8 : 1) : ns;
+    const double plane_cost = static_cast<double>(T) * E * 8.0 / 6.5e6;  // in K-block times
+    int ns = 1;
+    double best = 1e300;
+    for (int cand = 1; cand <= (KB / 8 > 0 ? KB / 8 : 1); ++cand) {
+      const double cost = static_cast<double>(ceil_div64(tiles * cand, 148)) * ceil_div(KB, cand) + cand * plane_cost;
+      if (cost < best) {
+        best = cost;
+        ns = cand;
+      }
+    }
     p.kb_per_split = ceil_div(KB, ns);
     p.nsplit = ceil_div(KB, p.kb_per_split);  // every split non-empty
     p.nparts = ceil_div(d, 256);
