@@ -57,26 +57,31 @@ constexpr float kRtEpsRel = 1.0f / 2048.0f;
 __global__ void __launch_bounds__(256)
     router_prep_kernel(const float* __restrict__ W, int d, int E, uint16_t* __restrict__ Wt_hi,
                        uint16_t* __restrict__ Wt_lo, double* __restrict__ part) {
-  __shared__ float tile[32][33];
+  __shared__ float tile[256][33];  // the whole 256 (i) x 32 (e) slab, padded
   __shared__ double ssq[8][32];
   const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 256;
   const int tx = threadIdx.x, ty = threadIdx.y;
+  // load the slab, coalesced along e, every load of the thread in flight at once;
+  // thread (tx, ty) sums the squares of rows ty, ty + 8, ... of column e0 + tx
   double acc = 0.0;
-  for (int sub = 0; sub < 8; ++sub) {
-    const int ib = i0 + sub * 32;
-    // load 32 (i) x 32 (e), coalesced along e
-    for (int r = ty; r < 32; r += 8) {
-      const int i = ib + r, e = e0 + tx;
-      const float v = (i < d && e < E) ? __ldg(W + static_cast<int64_t>(i) * E + e) : 0.0f;
-      tile[r][tx] = v;
-      acc += static_cast<double>(v) * static_cast<double>(v);
-    }
-    __syncthreads();
-    // store transposed: rows e, coalesced along i
-    for (int r = ty; r < 32; r += 8) {
-      const int e = e0 + r, i = ib + tx;
-      if (e < E && i < d) {
-        const float v = tile[tx][r];
+#pragma unroll
+  for (int r = ty; r < 256; r += 8) {
+    const int i = i0 + r, e = e0 + tx;
+    const float v = (i < d && e < E) ? __ldg(W + static_cast<int64_t>(i) * E + e) : 0.0f;
+    tile[r][tx] = v;
+    acc += static_cast<double>(v) * static_cast<double>(v);
+  }
+  __syncthreads();
+  // store transposed: rows e, coalesced along i
+#pragma unroll
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r;
+    if (e >= E) continue;
+#pragma unroll
+    for (int sub = 0; sub < 8; ++sub) {
+      const int i = i0 + sub * 32 + tx;
+      if (i < d) {
+        const float v = tile[sub * 32 + tx][r];
         const int64_t at = static_cast<int64_t>(e) * d + i;
         const __nv_bfloat16 hi = __float2bfloat16_rn(v);
         const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
@@ -84,7 +89,6 @@ __global__ void __launch_bounds__(256)
         Wt_lo[at] = *reinterpret_cast<const uint16_t*>(&lo);
       }
     }
-    __syncthreads();
   }
   ssq[ty][tx] = acc;  // column e0 + tx, rows ty, ty + 8, ... of this slab
   __syncthreads();
