@@ -54,7 +54,7 @@ typedef uint16_t moe_bf16_t; /* bfloat16 bit pattern */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1, /* null pointer, size out of range, misalignment */
-  MOE_ERR_UNSUPPORTED = 2, /* valid but beyond this build's limits (k > 16, E > 1024, ...) */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but beyond the library's limits (k > 16, E > 1024, ...) */
   MOE_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than required */
   MOE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
   MOE_ERR_DEVICE = 5       /* a kernel recorded an error (see moe_get_device_error) */
