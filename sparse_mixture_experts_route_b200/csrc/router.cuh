@@ -29,10 +29,6 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
 // Logits of a [BM tokens x BN experts] tile.
 //   SPLIT = false: the CTA walks every chunk in order and writes final logits
 //                  (+ bias) to out[t * E + e].
