@@ -54,8 +54,11 @@ def _load():
             lib.oracle_expert_ffn.argtypes = [P, I, P, P, I, I, P, P]
             lib.oracle_combine.argtypes = [P, P, P, I, I, I, P]
             lib.oracle_forward_tokens.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, P, P]
+            lib.oracle_mxfp4_quantize.argtypes = [P, I, I, P, P]
+            lib.oracle_mxfp4_dequantize.argtypes = [P, P, I, I, P]
             for fn in ("oracle_router_logits", "oracle_topk", "oracle_permute", "oracle_expert_ffn",
-                       "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version"):
+                       "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version",
+                       "oracle_mxfp4_quantize", "oracle_mxfp4_dequantize"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -192,3 +195,36 @@ def forward(x, W_router, bias, W_gate_up, W_down, k: int, tokens=None):
     _check(_load().oracle_forward_tokens(_ptr(xb), _ptr(Wr), _ptr(b), _ptr(Wg), _ptr(Wd), T, d, E, k, f,
                                          _ptr(tok), n, _ptr(out), _ptr(idx), _ptr(w)), "forward")
     return out, idx, w
+
+
+# ---------------------------------------------------------------- MXFP4 weights
+
+def mxfp4_quantize(w):
+    """MXFP4 of a weight matrix w [K, N] (bf16 tensor or uint16 bits, N
+    contiguous, K % 32 == 0) with blocks of 32 along K (the reduction axis).
+    Returns (codes uint8 [K, N]: one E2M1 code per byte, sign in bit 3;
+    scales uint8 [K // 32, N]: E8M0 exponent codes, 2^(code - 127)).
+    Definition and readings: ``oracle_mxfp4_quantize`` in moe_oracle.cpp."""
+    wb = _bf16_bits(w)
+    assert wb.ndim == 2, wb.shape
+    K, N = wb.shape
+    codes = np.empty((K, N), dtype=np.uint8)
+    scales = np.empty((K // 32, N), dtype=np.uint8)
+    st = _load().oracle_mxfp4_quantize(wb.ctypes.data, K, N, codes.ctypes.data, scales.ctypes.data)
+    if st:
+        raise ValueError(f"oracle_mxfp4_quantize: status {st}")
+    return codes, scales
+
+
+def mxfp4_dequantize(codes, scales) -> np.ndarray:
+    """The MXFP4 values as bf16 bits (uint16 [K, N]; every value is exact in
+    bf16): code c, scale code q -> (-1)^(c >> 3) * |E2M1(c & 7)| * 2^(q - 127)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    K, N = codes.shape
+    assert scales.shape == (K // 32, N), (scales.shape, codes.shape)
+    out = np.empty((K, N), dtype=np.uint16)
+    st = _load().oracle_mxfp4_dequantize(codes.ctypes.data, scales.ctypes.data, K, N, out.ctypes.data)
+    if st:
+        raise ValueError(f"oracle_mxfp4_dequantize: status {st}")
+    return out

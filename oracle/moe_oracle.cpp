@@ -284,4 +284,87 @@ int oracle_forward_tokens(const uint16_t* x, const float* Wr, const float* bias,
   return 0;
 }
 
+// ------------------------------------------------ MXFP4 expert weights
+//
+// [P3] section "Systems Optimization, Load Balancing, and Post-Training
+// Alignment": the MoE weights are served as MXFP4 (with MXFP8 activations).
+// The pages do not define the format; reading taken: the published OCP
+// Microscaling (MX) format. Blocks of 32 consecutive values along the
+// reduction axis share one power-of-two scale 2^s, stored as the unsigned
+// 8-bit exponent code s + 127 (E8M0). Each value is a 4-bit E2M1 float: bit 3
+// the sign, bits 2..1 an exponent with bias 1, bit 0 a mantissa bit, so the
+// magnitudes by 3-bit code are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+// Quantisation, the MX conversion: s = floor(log2(max |v|)) - 2 (2 is the
+// exponent of the largest E2M1 magnitude, 6 = 1.5 * 2^2), clamped to
+// [-127, 127]; an all-zero block takes s = -127. Each v / 2^s becomes the
+// nearest E2M1 magnitude (ties to the even code, whose mantissa bit is 0;
+// beyond 6 the nearest is 6, so large values saturate) with the sign of v.
+// Dequantised, code c and scale s give (-1)^(c >> 3) * mag[c & 7] * 2^s,
+// exactly representable in bf16 for every scale a bf16 block can produce.
+
+namespace {
+
+constexpr int64_t kMxBlock = 32;
+const double kE2M1Mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+inline uint8_t e2m1_nearest(double a) {  // a >= 0: code of the nearest magnitude
+  int best = 0;
+  double bd = std::fabs(a - kE2M1Mag[0]);
+  for (int c = 1; c < 8; ++c) {
+    const double dist = std::fabs(a - kE2M1Mag[c]);
+    if (dist < bd || (dist == bd && (c & 1) == 0)) {
+      best = c;
+      bd = dist;
+    }
+  }
+  return static_cast<uint8_t>(best);
+}
+
+}  // namespace
+
+// w [K, N] bf16 (N contiguous), K % 32 == 0: blocks of 32 along K for each
+// column n. codes [K, N] (one E2M1 code per byte), scales [K / 32, N] (E8M0).
+int oracle_mxfp4_quantize(const uint16_t* w, int64_t K, int64_t N, uint8_t* codes, uint8_t* scales) {
+  if (!w || !codes || !scales || K <= 0 || N <= 0 || K % kMxBlock) return 1;
+  for (int64_t b = 0; b < K / kMxBlock; ++b)
+    for (int64_t n = 0; n < N; ++n) {
+      double amax = 0.0;
+      for (int64_t i = 0; i < kMxBlock; ++i) {
+        const double v = bf16_to_double(w[(b * kMxBlock + i) * N + n]);
+        if (!std::isfinite(v)) return 2;
+        amax = std::max(amax, std::fabs(v));
+      }
+      int s = -127;
+      if (amax > 0.0) {
+        int e = 0;
+        std::frexp(amax, &e);  // amax = m * 2^e, m in [0.5, 1): floor(log2 amax) = e - 1
+        s = std::min(127, std::max(-127, e - 1 - 2));
+      }
+      scales[b * N + n] = static_cast<uint8_t>(s + 127);
+      for (int64_t i = 0; i < kMxBlock; ++i) {
+        const double v = bf16_to_double(w[(b * kMxBlock + i) * N + n]);
+        const uint8_t mag = e2m1_nearest(std::ldexp(std::fabs(v), -s));
+        codes[(b * kMxBlock + i) * N + n] = static_cast<uint8_t>((std::signbit(v) ? 8 : 0) | mag);
+      }
+    }
+  return 0;
+}
+
+// The inverse: w_out [K, N] as bf16 bits (every value is exact in bf16).
+int oracle_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t K, int64_t N, uint16_t* w_out) {
+  if (!codes || !scales || !w_out || K <= 0 || N <= 0 || K % kMxBlock) return 1;
+  for (int64_t r = 0; r < K; ++r)
+    for (int64_t n = 0; n < N; ++n) {
+      const uint8_t c = codes[r * N + n];
+      if (c > 15 || scales[(r / kMxBlock) * N + n] == 255) return 1;  // 255: the E8M0 NaN
+      const int s = static_cast<int>(scales[(r / kMxBlock) * N + n]) - 127;
+      const double v = (c & 8 ? -1.0 : 1.0) * std::ldexp(kE2M1Mag[c & 7], s);
+      const float fv = static_cast<float>(v);  // exact: at most two significant bits
+      uint32_t u;
+      std::memcpy(&u, &fv, sizeof(u));
+      w_out[r * N + n] = static_cast<uint16_t>(u >> 16);
+    }
+  return 0;
+}
+
 }  // extern "C"

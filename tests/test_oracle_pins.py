@@ -321,3 +321,98 @@ def test_oracle_rejects_bad_arguments():
         oracle.permute(np.array([[0, 9]], dtype=np.int32), 4)
     with pytest.raises(FloatingPointError):
         oracle.topk(np.array([[0.0, np.nan]], dtype=np.float32), 1)
+
+
+# ------------------------------------------------------------ MXFP4 weights
+#
+# The serving format of the MoE weights on "Kimi K3: Open Frontier
+# Intelligence" (section "Systems Optimization, Load Balancing, and
+# Post-Training Alignment"), read as the OCP MX format. The expected values
+# below are derived here from the bit fields of E2M1 (sign, two exponent bits
+# with bias 1, one mantissa bit) and of the E8M0 scale, not from the oracle's
+# table.
+
+def _e2m1_value(code):
+    sign = -1.0 if code & 8 else 1.0
+    e, m = (code >> 1) & 3, code & 1
+    mag = (m / 2.0) if e == 0 else (2.0 ** (e - 1)) * (1.0 + m / 2.0)  # subnormal when e == 0
+    return sign * mag
+
+
+def _bits_to_f64(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_mxfp4_element_values_from_the_bit_fields():
+    codes = np.arange(16, dtype=np.uint8).reshape(16, 1).repeat(2, axis=0)  # K = 32, N = 1
+    for q, s in ((127, 0), (130, 3), (120, -7)):
+        scales = np.full((1, 1), q, dtype=np.uint8)
+        got = _bits_to_f64(oracle.mxfp4_dequantize(codes, scales))[:, 0]
+        want = np.array([_e2m1_value(int(c)) * 2.0 ** s for c in codes[:, 0]])
+        assert np.array_equal(got, want)
+        assert np.array_equal(np.signbit(got), codes[:, 0] >= 8)  # -0 keeps its sign
+
+
+def _brute_force_mxfp4(block):
+    """Scale exponent and codes of one 32-value block by exhaustive search."""
+    amax = max(abs(v) for v in block)
+    s = -127 if amax == 0 else max(-127, min(127, math.frexp(amax)[1] - 1 - 2))
+    codes = []
+    for v in block:
+        a = abs(v) / 2.0 ** s
+        # the nearest of the eight magnitudes; on a tie the even code
+        best = min(range(8), key=lambda c: (abs(a - abs(_e2m1_value(c))), c & 1))
+        codes.append(best | (8 if math.copysign(1.0, v) < 0 else 0))
+    return s, codes
+
+
+def test_mxfp4_quantize_vs_brute_force_nearest_with_even_ties():
+    g = torch.Generator().manual_seed(7)
+    K, N = 96, 5
+    w = (torch.randn(K, N, generator=g) * torch.tensor([1.0, 1e-3, 30.0, 1.0, 1.0])).to(torch.bfloat16)
+    wf = w.to(torch.float64).numpy()
+    # column 3: exact ties and saturating values on a scale of 2^0 (block max 6)
+    wf[:32, 3] = [6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -2.5, -5.0, 0.0] + [0.1] * 20
+    wf[32:64, 3] = [7.5, 7.0, 6.5] + [1.0] * 29          # max 7.5: scale 2^0, 7.5 and 7.0 saturate to 6
+    wf[64:96, 3] = 0.0                                   # an all-zero block
+    wf[:32, 4] = -0.0                                    # negative zeros
+    w = torch.from_numpy(wf).to(torch.bfloat16)
+    wf = w.to(torch.float64).numpy()
+    codes, scales = oracle.mxfp4_quantize(w)
+    for b in range(K // 32):
+        for n in range(N):
+            s, want = _brute_force_mxfp4(list(wf[32 * b:32 * b + 32, n]))
+            assert int(scales[b, n]) == s + 127, (b, n)
+            assert codes[32 * b:32 * b + 32, n].tolist() == want, (b, n)
+    # the tie and saturation cases by hand: 0.25->0, 0.75->1, 1.25->1, 1.75->2,
+    # 2.5->2, 3.5->4, 5->4 (ties to the even code); 7.5, 7.0, 6.5 -> 6
+    deq = _bits_to_f64(oracle.mxfp4_dequantize(codes, scales))
+    assert deq[:8, 3].tolist() == [6.0, 0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]
+    assert deq[32:35, 3].tolist() == [6.0, 6.0, 6.0]
+    assert int(scales[2, 3]) == 0 and not codes[64:96, 3].any()
+
+
+def test_mxfp4_dequantised_values_requantise_to_themselves():
+    g = np.random.default_rng(11)
+    K, N = 128, 7
+    codes = g.integers(0, 16, size=(K, N), dtype=np.uint8)
+    scales = g.integers(100, 150, size=(K // 32, N), dtype=np.uint8)
+    deq = oracle.mxfp4_dequantize(codes, scales)
+    c2, s2 = oracle.mxfp4_quantize(deq)
+    assert np.array_equal(_bits_to_f64(oracle.mxfp4_dequantize(c2, s2)), _bits_to_f64(deq))
+
+
+def test_mxfp4_error_within_half_a_step():
+    """|v - q(v)| is at most half the E2M1 spacing at |v| (0.25, 0.5 or 1 times
+    the scale), or |v| - 6 * scale where v saturates."""
+    g = torch.Generator().manual_seed(3)
+    w = torch.randn(256, 16, generator=g).to(torch.bfloat16)
+    wf = w.to(torch.float64).numpy()
+    codes, scales = oracle.mxfp4_quantize(w)
+    deq = _bits_to_f64(oracle.mxfp4_dequantize(codes, scales))
+    scale = 2.0 ** (np.repeat(scales.astype(np.int64), 32, axis=0) - 127)
+    a = np.abs(wf) / scale
+    half_step = np.where(a < 2.0, 0.25, np.where(a < 4.0, 0.5, 1.0))
+    bound = np.maximum(half_step, a - 6.0) * scale
+    assert np.all(np.abs(wf - deq) <= bound)
+    assert np.all(np.abs(wf).reshape(8, 32, 16).max(axis=1) / scale[::32] >= 4.0)  # block max lands in [4, 8)
