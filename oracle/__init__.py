@@ -56,9 +56,13 @@ def _load():
             lib.oracle_forward_tokens.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, P, P]
             lib.oracle_mxfp4_quantize.argtypes = [P, I, I, P, P]
             lib.oracle_mxfp4_dequantize.argtypes = [P, P, I, I, P]
+            lib.oracle_mxfp8_quantize.argtypes = [P, I, I, P, P]
+            lib.oracle_mxfp8_dequantize.argtypes = [P, P, I, I, P]
+            lib.oracle_expert_ffn_mx.argtypes = [P, I, P, P, I, I, P, P]
             for fn in ("oracle_router_logits", "oracle_topk", "oracle_permute", "oracle_expert_ffn",
                        "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version",
-                       "oracle_mxfp4_quantize", "oracle_mxfp4_dequantize"):
+                       "oracle_mxfp4_quantize", "oracle_mxfp4_dequantize", "oracle_mxfp8_quantize",
+                       "oracle_mxfp8_dequantize", "oracle_expert_ffn_mx"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -82,6 +86,11 @@ def _bf16_bits(a) -> np.ndarray:
     a = np.asarray(a)
     assert a.dtype == np.uint16, a.dtype
     return np.ascontiguousarray(a)
+
+
+def _bits_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bits (uint16) -> fp64 values, exactly."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def _f32(a) -> np.ndarray:
@@ -228,3 +237,54 @@ def mxfp4_dequantize(codes, scales) -> np.ndarray:
     if st:
         raise ValueError(f"oracle_mxfp4_dequantize: status {st}")
     return out
+
+
+def mxfp8_quantize(v):
+    """MXFP8 (E4M3 elements, E8M0 scales) of v [rows, cols] (anything numpy
+    converts to fp64, cols % 32 == 0) with blocks of 32 along each row.
+    Returns (codes uint8 [rows, cols], scales uint8 [rows, cols // 32]).
+    Definition and readings: ``oracle_mxfp8_quantize`` in moe_oracle.cpp."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    assert v.ndim == 2, v.shape
+    R, C = v.shape
+    codes = np.empty((R, C), dtype=np.uint8)
+    scales = np.empty((R, C // 32), dtype=np.uint8)
+    st = _load().oracle_mxfp8_quantize(v.ctypes.data, R, C, codes.ctypes.data, scales.ctypes.data)
+    if st:
+        raise ValueError(f"oracle_mxfp8_quantize: status {st}")
+    return codes, scales
+
+
+def mxfp8_dequantize(codes, scales) -> np.ndarray:
+    """The MXFP8 values in fp64 [rows, cols]."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    R, C = codes.shape
+    assert scales.shape == (R, C // 32), (scales.shape, codes.shape)
+    out = np.empty((R, C), dtype=np.float64)
+    st = _load().oracle_mxfp8_dequantize(codes.ctypes.data, scales.ctypes.data, R, C, out.ctypes.data)
+    if st:
+        raise ValueError(f"oracle_mxfp8_dequantize: status {st}")
+    return out
+
+
+def expert_ffn_mx(x_rows, gu_codes, gu_scales, dn_codes, dn_scales, want_h: bool = False):
+    """One expert's SwiGLU feed-forward in the MX serving format: the rows of x
+    (bf16 [n, d]) take an MXFP8 round trip along d, the weights are the MXFP4
+    codes/scales of W_gate_up [d, 2f] and W_down [f, d], h takes an MXFP8 round
+    trip along f. Returns y [n, d] fp64 (and h' [n, f] with want_h)."""
+    xb = _bf16_bits(x_rows)
+    n, d = xb.shape
+    x64 = np.ascontiguousarray(_bits_f64(xb))
+    xq = mxfp8_dequantize(*mxfp8_quantize(x64)) if n > 0 else x64
+    wgu = mxfp4_dequantize(gu_codes, gu_scales)
+    wd = mxfp4_dequantize(dn_codes, dn_scales)
+    assert wgu.shape[0] == d and wd.shape[1] == d, (wgu.shape, wd.shape)
+    f = wd.shape[0]
+    y = np.zeros((n, d), dtype=np.float64)
+    h = np.zeros((n, f), dtype=np.float64)
+    st = _load().oracle_expert_ffn_mx(xq.ctypes.data if n else None, n, wgu.ctypes.data, wd.ctypes.data, d, f,
+                                      y.ctypes.data, h.ctypes.data)
+    if st:
+        raise ValueError(f"oracle_expert_ffn_mx: status {st}")
+    return (y, h) if want_h else y

@@ -350,6 +350,120 @@ int oracle_mxfp4_quantize(const uint16_t* w, int64_t K, int64_t N, uint8_t* code
   return 0;
 }
 
+// MXFP8 activations (the same passage): E4M3 elements, the OCP FP8 format
+// without infinities: bit 7 the sign, bits 6..3 an exponent with bias 7,
+// bits 2..0 a mantissa; magnitude (e == 0 ? m / 8 * 2^-6 : (1 + m / 8) *
+// 2^(e - 7)), the largest finite 448 (code 0x7e), 0x7f and 0xff are NaN.
+// Blocks of 32 consecutive values along the contiguous (reduction) axis of
+// each row share an E8M0 scale 2^s, s = floor(log2(max |v|)) - 8 (8 is the
+// exponent of the largest E4M3 magnitude), clamped to [-127, 127]; an
+// all-zero block takes s = -127. Each v / 2^s becomes the nearest E4M3
+// magnitude (ties to the even code; beyond 448 the nearest is 448, so large
+// values saturate) with the sign of v.
+
+namespace {
+
+double e4m3_mag(int c) {  // c in 0..126
+  const int e = c >> 3, m = c & 7;
+  return e == 0 ? std::ldexp(m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
+}
+
+inline uint8_t e4m3_nearest(double a) {  // a >= 0: code of the nearest finite magnitude
+  int best = 0;
+  double bd = a;
+  for (int c = 1; c < 127; ++c) {
+    const double dist = std::fabs(a - e4m3_mag(c));
+    if (dist < bd || (dist == bd && (c & 1) == 0)) {
+      best = c;
+      bd = dist;
+    }
+  }
+  return static_cast<uint8_t>(best);
+}
+
+}  // namespace
+
+// v [rows, cols] fp64 (cols contiguous), cols % 32 == 0: codes [rows, cols],
+// scales [rows, cols / 32].
+int oracle_mxfp8_quantize(const double* v, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales) {
+  if (!v || !codes || !scales || rows <= 0 || cols <= 0 || cols % kMxBlock) return 1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < cols / kMxBlock; ++b) {
+      const double* blk = v + r * cols + b * kMxBlock;
+      double amax = 0.0;
+      for (int64_t i = 0; i < kMxBlock; ++i) {
+        if (!std::isfinite(blk[i])) return 2;
+        amax = std::max(amax, std::fabs(blk[i]));
+      }
+      int s = -127;
+      if (amax > 0.0) {
+        int e = 0;
+        std::frexp(amax, &e);
+        s = std::min(127, std::max(-127, e - 1 - 8));
+      }
+      scales[r * (cols / kMxBlock) + b] = static_cast<uint8_t>(s + 127);
+      for (int64_t i = 0; i < kMxBlock; ++i) {
+        const uint8_t mag = e4m3_nearest(std::ldexp(std::fabs(blk[i]), -s));
+        codes[r * cols + b * kMxBlock + i] = static_cast<uint8_t>((std::signbit(blk[i]) ? 0x80 : 0) | mag);
+      }
+    }
+  return 0;
+}
+
+// The inverse, in fp64.
+int oracle_mxfp8_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, double* out) {
+  if (!codes || !scales || !out || rows <= 0 || cols <= 0 || cols % kMxBlock) return 1;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t i = 0; i < cols; ++i) {
+      const uint8_t c = codes[r * cols + i];
+      const uint8_t q = scales[r * (cols / kMxBlock) + i / kMxBlock];
+      if ((c & 0x7f) == 0x7f || q == 255) return 1;  // NaN codes
+      out[r * cols + i] = (c & 0x80 ? -1.0 : 1.0) * std::ldexp(e4m3_mag(c & 0x7f), static_cast<int>(q) - 127);
+    }
+  return 0;
+}
+
+// The expert feed-forward of step 5 with MXFP8 activations and MXFP4 weights
+// (the serving format above): x_mx [n, d] are the rows after their MXFP8
+// round trip (fp64), Wgu [d, 2f] and Wd [f, d] the dequantised MXFP4 weights
+// (bf16 bits, exact). g, u and h = SiLU(g) * u as in step 5 (fp64); h, the
+// down projection's activation operand, takes its own MXFP8 round trip along
+// f before y = h' Wd. h_out (may be NULL) receives h'. f % 32 == 0.
+int oracle_expert_ffn_mx(const double* x_mx, int64_t n, const uint16_t* Wgu, const uint16_t* Wd, int64_t d,
+                         int64_t f, double* y, double* h_out) {
+  if ((!x_mx && n > 0) || !Wgu || !Wd || !y || n < 0 || d <= 0 || f <= 0 || f % kMxBlock) return 1;
+  const int64_t f2 = 2 * f;
+  int status = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n; ++r) {
+    std::vector<double> gu(f2, 0.0), hrow(f), yy(d, 0.0);
+    std::vector<uint8_t> hc(f), hs(f / kMxBlock);
+    for (int64_t i = 0; i < d; ++i) {
+      const double xi = x_mx[r * d + i];
+      for (int64_t j = 0; j < f2; ++j) gu[j] += xi * bf16_to_double(Wgu[i * f2 + j]);
+    }
+    for (int64_t j = 0; j < f; ++j) {
+      const double g = gu[j], u = gu[f + j];
+      hrow[j] = g / (1.0 + std::exp(-g)) * u;
+    }
+    int st = oracle_mxfp8_quantize(hrow.data(), 1, f, hc.data(), hs.data());
+    if (!st) st = oracle_mxfp8_dequantize(hc.data(), hs.data(), 1, f, hrow.data());
+    if (st) {
+#pragma omp critical
+      status = st;
+      continue;
+    }
+    for (int64_t j = 0; j < f; ++j) {
+      const double hj = hrow[j];
+      for (int64_t c = 0; c < d; ++c) yy[c] += hj * bf16_to_double(Wd[j * d + c]);
+    }
+    for (int64_t c = 0; c < d; ++c) y[r * d + c] = yy[c];
+    if (h_out)
+      for (int64_t j = 0; j < f; ++j) h_out[r * f + j] = hrow[j];
+  }
+  return status;
+}
+
 // The inverse: w_out [K, N] as bf16 bits (every value is exact in bf16).
 int oracle_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t K, int64_t N, uint16_t* w_out) {
   if (!codes || !scales || !w_out || K <= 0 || N <= 0 || K % kMxBlock) return 1;

@@ -41,6 +41,12 @@ MUTATIONS = {
                            "static_cast<uint8_t>(mag);"),
     "mxfp4_subnormal_value": ("const double kE2M1Mag[8] = {0.0, 0.5, 1.0,",
                               "const double kE2M1Mag[8] = {0.0, 0.25, 1.0,"),
+    "mxfp8_scale_one_too_large": ("s = std::min(127, std::max(-127, e - 1 - 8));",
+                                  "s = std::min(127, std::max(-127, e - 1 - 7));"),
+    "mxfp8_subnormal_exponent": ("return e == 0 ? std::ldexp(m / 8.0, -6)", "return e == 0 ? std::ldexp(m / 8.0, -7)"),
+    "mx_ffn_h_not_requantised": ("if (!st) st = oracle_mxfp8_dequantize(hc.data(), hs.data(), 1, f, hrow.data());",
+                                 "if (!st) st = 0;"),
+    "mx_ffn_gate_up_swapped": ("const double g = gu[j], u = gu[f + j];", "const double u = gu[j], g = gu[f + j];"),
 }
 
 

@@ -416,3 +416,78 @@ def test_mxfp4_error_within_half_a_step():
     bound = np.maximum(half_step, a - 6.0) * scale
     assert np.all(np.abs(wf - deq) <= bound)
     assert np.all(np.abs(wf).reshape(8, 32, 16).max(axis=1) / scale[::32] >= 4.0)  # block max lands in [4, 8)
+
+
+# MXFP8 activations: E4M3 elements decoded and rounded by torch's own
+# float8_e4m3fn type (a library implementation of the same format), E8M0 scale
+# from frexp; saturation (which torch's cast does not do) by hand.
+
+def test_mxfp8_element_values_match_torch_e4m3fn():
+    codes = np.array([c for c in range(256) if (c & 0x7f) != 0x7f], dtype=np.uint8)
+    codes = np.concatenate([codes, codes[:2]]).reshape(2, 128)  # 254 + 2 = 256 values, 32-aligned rows
+    for q in (127, 131, 119):
+        scales = np.full((2, 4), q, dtype=np.uint8)
+        got = oracle.mxfp8_dequantize(codes, scales)
+        want = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy() * 2.0 ** (q - 127)
+        assert np.array_equal(got, want)
+        assert np.array_equal(np.signbit(got), codes >= 0x80)
+
+
+def test_mxfp8_quantize_vs_torch_cast_and_saturation():
+    g = torch.Generator().manual_seed(5)
+    v = torch.randn(6, 64, generator=g, dtype=torch.float64)
+    v[1] *= 1e-4
+    v[2] *= 300.0
+    v[3, :32] = 0.0
+    v[4, :8] = torch.tensor([256.0, 0.5 * 2.0 ** -9, 1.5 * 2.0 ** -9, 3.0 * 2.0 ** -10, 452.0, 456.0, -460.0, 511.0])
+    v[5, :32] = -0.0
+    vn = v.numpy()
+    codes, scales = oracle.mxfp8_quantize(vn)
+    deq = oracle.mxfp8_dequantize(codes, scales)
+    for r in range(6):
+        for b in range(2):
+            blk = vn[r, 32 * b:32 * b + 32]
+            amax = np.abs(blk).max()
+            s = -127 if amax == 0 else max(-127, min(127, math.frexp(amax)[1] - 1 - 8))
+            assert int(scales[r, b]) == s + 127, (r, b)
+            a = blk / 2.0 ** s
+            inrange = np.abs(a) <= 448.0
+            ref = torch.from_numpy(a[inrange].copy()).to(torch.float8_e4m3fn).to(torch.float64).numpy() * 2.0 ** s
+            assert np.array_equal(deq[r, 32 * b:32 * b + 32][inrange], ref), (r, b)
+            assert np.all(deq[r, 32 * b:32 * b + 32][~inrange] == np.sign(blk[~inrange]) * 448.0 * 2.0 ** s)
+    # by hand, on a scale of 2^0 (block max 511): ties to the even code, saturation
+    assert deq[4, :8].tolist() == [256.0, 0.0, 2.0 ** -8, 2.0 ** -8, 448.0, 448.0, -448.0, 448.0]
+    assert int(scales[3, 0]) == 0 and not codes[3, :32].any()
+    assert np.all(codes[5, :32] == 0x80)  # -0 keeps its sign
+
+
+def test_mxfp8_dequantised_values_requantise_to_themselves():
+    g = np.random.default_rng(13)
+    codes = g.integers(0, 256, size=(8, 96), dtype=np.uint8)
+    codes[(codes & 0x7f) == 0x7f] = 0x7e
+    scales = g.integers(100, 150, size=(8, 3), dtype=np.uint8)
+    deq = oracle.mxfp8_dequantize(codes, scales)
+    assert np.array_equal(oracle.mxfp8_dequantize(*oracle.mxfp8_quantize(deq)), deq)
+
+
+def test_mx_expert_ffn_vs_numpy_composition():
+    """The MX feed-forward equals its definition assembled here from the pinned
+    pieces and numpy matmuls: x' and h' are MXFP8 round trips, W' the MXFP4
+    dequantised weights, and the gate is the first f columns."""
+    g = torch.Generator().manual_seed(9)
+    n, d, f = 6, 96, 64
+    x = torch.randn(n, d, generator=g).to(torch.bfloat16)
+    Wgu = (torch.randn(d, 2 * f, generator=g) / d ** 0.5).to(torch.bfloat16)
+    Wd = (torch.randn(f, d, generator=g) / f ** 0.5).to(torch.bfloat16)
+    gq = oracle.mxfp4_quantize(Wgu)
+    dq = oracle.mxfp4_quantize(Wd)
+    y, h = oracle.expert_ffn_mx(x, *gq, *dq, want_h=True)
+    xq = oracle.mxfp8_dequantize(*oracle.mxfp8_quantize(x.to(torch.float64).numpy()))
+    wgu = _bits_to_f64(oracle.mxfp4_dequantize(*gq))
+    wd = _bits_to_f64(oracle.mxfp4_dequantize(*dq))
+    gu = xq @ wgu
+    hh = _silu(gu[:, :f]) * gu[:, f:]
+    hq = oracle.mxfp8_dequantize(*oracle.mxfp8_quantize(hh))
+    np.testing.assert_allclose(h, hq, rtol=0, atol=1e-12 * np.abs(hq).max())
+    np.testing.assert_allclose(y, hq @ wd, rtol=0, atol=1e-12 * np.abs(hq @ wd).max())
+    assert not np.allclose(hq, hh)  # the h round trip is not a no-op on these values
