@@ -33,8 +33,10 @@ MUTATIONS = {
     "permute_descending_tokens": ("const int32_t r = cursor[e]++;",
                                   "const int32_t r = offsets[e + 1] - 1 - (cursor[e]++ - offsets[e]);"),
     "bias_dropped": ("l[e] = l[e] + bias[e];", "l[e] = l[e] + 0.0f * bias[e];"),
-    "mxfp4_ties_to_odd_code": ("if (dist < bd || (dist == bd && (c & 1) == 0)) {",
-                               "if (dist < bd || (dist == bd && (c & 1) == 1)) {"),
+    "mxfp4_ties_to_odd_code": ("kE2M1Mag[c]);\n    if (dist < bd || (dist == bd && (c & 1) == 0)) {",
+                               "kE2M1Mag[c]);\n    if (dist < bd || (dist == bd && (c & 1) == 1)) {"),
+    "mxfp8_ties_to_odd_code": ("e4m3_mag(c));\n    if (dist < bd || (dist == bd && (c & 1) == 0)) {",
+                               "e4m3_mag(c));\n    if (dist < bd || (dist == bd && (c & 1) == 1)) {"),
     "mxfp4_scale_one_too_small": ("s = std::min(127, std::max(-127, e - 1 - 2));",
                                   "s = std::min(127, std::max(-127, e - 1 - 1));"),
     "mxfp4_sign_dropped": ("static_cast<uint8_t>((std::signbit(v) ? 8 : 0) | mag);",
