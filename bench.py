@@ -3,6 +3,7 @@ combine) on B200, printing one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+    python bench.py --mx-quant             # the MXFP8 / MXFP4 quantisers alone
 
 A step is one moe_forward over one batch of T synthetic tokens with the
 workload's weights resident in HBM. Timing: W untimed warm-up steps, then K
@@ -453,6 +454,58 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_mx_quant(args):
+    """Throughput of the MX quantisers (the MXFP8 activation and MXFP4 weight
+    formats) on one GPU: the prefill activations widened to 16384 rows
+    [16384, 7168] and 32 experts' W_gate_up [32, 7168, 4096]. Inputs are larger
+    than L2, so no flush is needed; each launch is timed between CUDA events on
+    its stream after W warm-up launches, and the mean over K is reported.
+    Algorithmic bytes per element: 2 read + 1 code + 1/32 scale."""
+    from sparse_mixture_experts_route_b200 import _lib
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    x = torch.randn(16384, 7168, generator=g, device=dev).to(torch.bfloat16)
+    w = torch.empty(32, 7168, 4096, dtype=torch.bfloat16, device=dev)
+    for e in range(32):
+        w[e].copy_(torch.randn(7168, 4096, generator=g, device=dev) / 84.66)
+    cases = {
+        "mxfp8_activations_16384x7168": (lambda c, s_: _lib.moe_mxfp8_quantize(x, codes=c, scales=s_),
+                                        x.numel(), (16384, 7168), (16384, 7168 // 32)),
+        "mxfp4_weights_32x7168x4096": (lambda c, s_: _lib.moe_mxfp4_quantize(w, codes=c, scales=s_),
+                                      w.numel(), (32, 7168, 4096), (32, 7168 // 32, 4096)),
+    }
+    sampler = ClockSampler(0)
+    out = {}
+    sampler.start()
+    for name, (fn, n_el, cshape, sshape) in cases.items():
+        codes = torch.empty(cshape, dtype=torch.uint8, device=dev)
+        scales = torch.empty(sshape, dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            fn(codes, scales)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            a.record(stream)
+            fn(codes, scales)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        gbs = n_el * (2 + 1 + 1 / 32) / (ms * 1e-3) / 1e9
+        out[name] = {"ms_per_launch": ms, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    clocks = sampler.stop()
+    assert _lib.get_device_error() == 0
+    return {"metric": "mx_quantize_bytes_per_s", "unit": "GB/s", "higher_is_better": True,
+            "value": min(v["GB/s"] for v in out.values()), "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "dtype": "bf16->e4m3/e2m1", "data": "synthetic",
+            "kernels": out, "peak": {"hbm_gbs": peaks["hbm_gbs"], "kind": peak_kind},
+            "config": {"workload": "mx_quantize", "l2": "inputs larger than L2"}, "clocks": clocks}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -464,9 +517,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", default="on", choices=["on", "off"],
                     help="time replays of one step captured as a CUDA graph (on) or eager calls (off)")
+    ap.add_argument("--mx-quant", action="store_true",
+                    help="time the MXFP8/MXFP4 quantisers instead of the layer (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.mx_quant:
+        print(json.dumps(run_mx_quant(args)), flush=True)
+        return
     line = run_reference(args) if args.impl == "reference" else run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)

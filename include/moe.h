@@ -231,6 +231,38 @@ moe_status_t moe_route_noalloc(const moe_bf16_t* x, const float* W_router, const
                                int T, int d, int E, int k,
                                int32_t* topk_idx, float* topk_w, cudaStream_t stream);
 
+/* ------------------------------------------------------- MX quantisation --
+ * The serving format of [P3] section "Systems Optimization, Load Balancing,
+ * and Post-Training Alignment": MXFP4 expert weights with MXFP8 activations.
+ * The page names the formats only; the reading taken is the published OCP
+ * Microscaling (MX) format. Blocks of 32 consecutive values along the
+ * reduction axis share a scale 2^s, stored as the E8M0 byte s + 127, with
+ * s = floor(log2(max |v| of the block)) - emax clamped to [-127, 127]
+ * (emax = 2 for E2M1, 8 for E4M3; an all-zero block takes s = -127). Each
+ * element is v / 2^s rounded to the nearest element value (ties to the even
+ * code), saturating at the largest finite magnitude (6 for E2M1, 448 for
+ * E4M3), with the sign bit of v (also when the magnitude rounds to 0).
+ * Codes are one per byte: E2M1 in bits 3..0 (bit 3 the sign), E4M3 in the
+ * whole byte (bit 7 the sign; NaN codes are never produced).
+ * Inputs must be finite (a NaN or infinity gives an unspecified code).
+ * Neither call needs scratch; both only enqueue one kernel on `stream`.
+ *
+ * moe_mxfp8_quantize: x [rows, cols] bf16 (cols % 32 == 0, x 16-byte
+ * aligned), blocks along each row: codes [rows, cols] (16-byte aligned),
+ * scales [rows, cols / 32]. rows >= 1, 32 <= cols <= 2^20.
+ */
+moe_status_t moe_mxfp8_quantize(const moe_bf16_t* x, int rows, int cols,
+                                uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+
+/* moe_mxfp4_quantize: w [K, N] bf16 (N contiguous; an expert's W_gate_up is
+ * [d, 2f], its W_down [f, d]), K % 32 == 0, blocks along K for each column:
+ * codes [K, N], scales [K / 32, N]. 32 <= K <= 2^20, 1 <= N <= 2^20.
+ * A whole stack of experts [E, K, N] is one call with K' = E * K (every
+ * block then lies inside one expert, since K % 32 == 0).
+ */
+moe_status_t moe_mxfp4_quantize(const moe_bf16_t* w, int K, int N,
+                                uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+
 /* ------------------------------------------------------------ diagnostics --
  * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
  * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise

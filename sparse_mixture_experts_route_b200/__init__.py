@@ -9,6 +9,7 @@ is missing: there is no CPU fallback.
 """
 
 __all__ = ["moe_route", "moe_permute", "moe_expert_ffn", "moe_unpermute", "moe_forward",
+           "moe_forward_host", "moe_mxfp8_quantize", "moe_mxfp4_quantize",
            "moe_forward_workspace_size", "MoEError", "inputs"]
 
 

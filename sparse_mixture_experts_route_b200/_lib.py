@@ -38,6 +38,8 @@ EXPORTS = {
     "moe_unpermute": ([P, P, P, I, I, I, P, P], I),
     "moe_forward_workspace_size": ([I, I, I, I, I], Z),
     "moe_forward": ([P, P, P, P, P, I, I, I, I, I, P, P, Z, P], I),
+    "moe_mxfp8_quantize": ([P, I, I, P, P, P], I),
+    "moe_mxfp4_quantize": ([P, I, I, P, P, P], I),
     "moe_get_device_error": ([ctypes.POINTER(ctypes.c_uint32), I], I),
     "moe_selftest_wait_timeout": ([I, P], I),
 }
@@ -182,6 +184,43 @@ def moe_unpermute(y_perm, inv_perm, topk_w, stream=None, out=None):
     _check(_lib.moe_unpermute(_ptr(y_perm), _ptr(inv_perm), _ptr(topk_w), T, d, k, _ptr(out), _stream(stream)),
            "moe_unpermute")
     return out
+
+
+def moe_mxfp8_quantize(x, stream=None, codes=None, scales=None):
+    """MXFP8 (E4M3) of x [rows, cols] bf16, blocks of 32 along each row.
+    Returns (codes uint8 [rows, cols], scales uint8 [rows, cols // 32])."""
+    rows, cols = x.shape
+    _need(x, "x", torch.bfloat16, (rows, cols))
+    if codes is None:
+        codes = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device)
+    _need(codes, "codes", torch.uint8, (rows, cols))
+    _need(scales, "scales", torch.uint8, (rows, cols // 32))
+    _check(_lib.moe_mxfp8_quantize(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _stream(stream)),
+           "moe_mxfp8_quantize")
+    return codes, scales
+
+
+def moe_mxfp4_quantize(w, stream=None, codes=None, scales=None):
+    """MXFP4 (E2M1) of w [K, N] or a stack [E, K, N] bf16, blocks of 32 along K
+    for each column. Returns (codes uint8 shaped like w, scales uint8 with K
+    replaced by K // 32)."""
+    if w.dim() not in (2, 3):
+        raise ValueError("w must be [K, N] or [E, K, N]")
+    K, N = w.shape[-2], w.shape[-1]
+    rows = w.numel() // N
+    _need(w, "w", torch.bfloat16, tuple(w.shape))
+    sshape = tuple(w.shape[:-2]) + (K // 32, N)
+    if codes is None:
+        codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(sshape, dtype=torch.uint8, device=w.device)
+    _need(codes, "codes", torch.uint8, tuple(w.shape))
+    _need(scales, "scales", torch.uint8, sshape)
+    _check(_lib.moe_mxfp4_quantize(_ptr(w), rows, N, _ptr(codes), _ptr(scales), _stream(stream)),
+           "moe_mxfp4_quantize")
+    return codes, scales
 
 
 def moe_forward(x, W_router, router_bias, W_gate_up, W_down, k: int, out=None, workspace=None, stream=None):

@@ -14,6 +14,7 @@
 
 #include "common.cuh"
 #include "expert_gemm.cuh"
+#include "mx_quant.cuh"
 #include "permute.cuh"
 #include "ptx.cuh"
 #include "router.cuh"
@@ -801,6 +802,37 @@ moe_status_t moe_route_noalloc(const moe_bf16_t* x, const float* W_router, const
   const moe_status_t st = noalloc_route_scratch(&scratch);
   if (st != MOE_OK) return st;
   return launch_route(x, W_router, router_bias, T, d, E, k, topk_idx, topk_w, scratch, stream);
+}
+
+moe_status_t moe_mxfp8_quantize(const moe_bf16_t* x, int rows, int cols, uint8_t* codes, uint8_t* scales,
+                                cudaStream_t stream) {
+  if (!x || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || cols < moe::kMxBlock || cols > (1 << 20) || cols % moe::kMxBlock) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes)) return MOE_ERR_INVALID_ARG;
+  const int64_t nblocks = static_cast<int64_t>(rows) * (cols / moe::kMxBlock);
+  const int64_t grid = ceil_div64(nblocks, 256);
+  if (grid > 0x7fffffff) return MOE_ERR_UNSUPPORTED;
+  moe::mxfp8_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x),
+                                                                               nblocks, codes, scales);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_mxfp4_quantize(const moe_bf16_t* w, int K, int N, uint8_t* codes, uint8_t* scales,
+                                cudaStream_t stream) {
+  if (!w || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  if (K < moe::kMxBlock || K > (1 << 20) || K % moe::kMxBlock || N < 1 || N > (1 << 20)) return MOE_ERR_INVALID_ARG;
+  const auto addr = [](const void* p) { return reinterpret_cast<uintptr_t>(p); };
+  const bool x4 = N % 4 == 0 && addr(w) % 8 == 0 && addr(codes) % 4 == 0 && addr(scales) % 4 == 0;
+  const int64_t groups = static_cast<int64_t>(K / moe::kMxBlock) * (x4 ? N / 4 : N);
+  const int64_t grid = ceil_div64(groups, 256);
+  if (grid > 0x7fffffff) return MOE_ERR_UNSUPPORTED;
+  if (x4)
+    moe::mxfp4_quantize_x4_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        reinterpret_cast<const uint2*>(w), K, N / 4, reinterpret_cast<uint32_t*>(codes),
+        reinterpret_cast<uint32_t*>(scales));
+  else
+    moe::mxfp4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(w, K, N, codes, scales);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_get_device_error(uint32_t* code, int clear) {

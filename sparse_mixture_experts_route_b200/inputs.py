@@ -149,3 +149,32 @@ def make_inputs(shape: MoEShape, seed: int = 0, device="cpu") -> MoEInputs:
 
 def custom_shape(T: int, d: int, E: int, k: int, f: int, bias: Optional[str] = None, name: str = "custom") -> MoEShape:
     return MoEShape(name, T, d, E, k, f, bias)
+
+
+def make_mx_values(shape_t, block_axis: int, seed: int = 0, device="cpu") -> torch.Tensor:
+    """bf16 test values for MX block quantisation, blocks of 32 along
+    ``block_axis`` (-1 for activations, -2 for [.., K, N] weights): N(0, 1)
+    draws, a quarter of the blocks shifted by a random power of two in
+    [2^-140, 2^120] (so bf16 subnormals and huge magnitudes occur), one
+    element in eight shrunk by 2^-[0, 24] (a wide range inside a block),
+    one block in 32 set to zero, one element in 64 set to -0. Plain random
+    numbers: no quantisation arithmetic."""
+    g = _gen(seed, 7, "cpu")
+    v = torch.randn(shape_t, generator=g, dtype=torch.float32)
+    ax = block_axis % len(shape_t)
+    vb = v.movedim(ax, -1)
+    bshape = tuple(vb.shape[:-1]) + (vb.shape[-1] // 32, 1)
+    e_blk = torch.randint(-140, 121, bshape, generator=g, dtype=torch.int32)
+    shifted = torch.rand(bshape, generator=g) < 0.25
+    zero_blk = torch.rand(bshape, generator=g) < 1.0 / 32
+    vb = vb.reshape(tuple(vb.shape[:-1]) + (vb.shape[-1] // 32, 32))
+    # ldexp in fp64 so 2^e itself never under- or overflows before rounding
+    vd = vb.to(torch.float64) * torch.pow(2.0, torch.where(shifted, e_blk, 0).to(torch.float64))
+    shrink = torch.rand(vd.shape, generator=g) < 0.125
+    e_el = torch.randint(0, 25, vd.shape, generator=g, dtype=torch.int32).to(torch.float64)
+    vd = torch.where(shrink, vd * torch.pow(2.0, -e_el), vd)
+    vd = torch.where(zero_blk, torch.zeros_like(vd), vd)
+    neg0 = torch.rand(vd.shape, generator=g) < 1.0 / 64
+    vd = torch.where(neg0, torch.full_like(vd, -0.0), vd)
+    out = vd.reshape(tuple(vb.shape[:-2]) + (-1,)).to(torch.bfloat16).movedim(-1, ax).contiguous()
+    return out.to(device)

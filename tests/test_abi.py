@@ -158,3 +158,30 @@ def test_host_buffer_forward_checks(lib):
     assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 32, 17, 256, p, p, 1 << 30, None) == 2  # k > 16
     assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 2, 256, p, p, hw - 256, None) == 3
     assert lib.moe_forward_host(p, p, None, p, p, 64, 128, 8, 2, 256, p, ctypes.c_void_p(FAKE + 8), hw, None) == 3
+
+
+def test_mx_quantize_checks(lib):
+    """moe_mxfp8_quantize / moe_mxfp4_quantize refuse null pointers, a block
+    axis that is not a multiple of 32, sizes out of range and misaligned
+    16-byte operands before any CUDA call."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.moe_mxfp8_quantize.argtypes = [P, I, I, P, P, P]
+    lib.moe_mxfp4_quantize.argtypes = [P, I, I, P, P, P]
+    p = ctypes.c_void_p(FAKE)
+    q8, q4 = lib.moe_mxfp8_quantize, lib.moe_mxfp4_quantize
+    assert q8(None, 4, 64, p, p, None) == 1
+    assert q8(p, 4, 64, None, p, None) == 1
+    assert q8(p, 4, 64, p, None, None) == 1
+    assert q8(p, 0, 64, p, p, None) == 1                          # rows = 0
+    assert q8(p, 4, 48, p, p, None) == 1                          # cols % 32
+    assert q8(p, 4, 16, p, p, None) == 1                          # cols < 32
+    assert q8(p, 4, (1 << 20) + 32, p, p, None) == 1              # cols too large
+    assert q8(ctypes.c_void_p(FAKE + 8), 4, 64, p, p, None) == 1  # x alignment
+    assert q8(p, 4, 64, ctypes.c_void_p(FAKE + 4), p, None) == 1  # codes alignment
+    assert q4(None, 64, 8, p, p, None) == 1
+    assert q4(p, 64, 8, None, p, None) == 1
+    assert q4(p, 64, 8, p, None, None) == 1
+    assert q4(p, 40, 8, p, p, None) == 1                          # K % 32
+    assert q4(p, 0, 8, p, p, None) == 1
+    assert q4(p, 64, 0, p, p, None) == 1                          # N = 0
+    assert q4(p, 64, (1 << 20) + 1, p, p, None) == 1              # N too large
