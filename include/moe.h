@@ -263,6 +263,47 @@ moe_status_t moe_mxfp8_quantize(const moe_bf16_t* x, int rows, int cols,
 moe_status_t moe_mxfp4_quantize(const moe_bf16_t* w, int K, int N,
                                 uint8_t* codes, uint8_t* scales, cudaStream_t stream);
 
+/* ------------------------------------------------ MX expert feed-forward --
+ * The layer with its experts in the serving format above: MXFP4 expert
+ * weights, MXFP8 token activations (x and the SwiGLU output h), on the
+ * block-scaled tensor cores. Routing, dispatch and combine are those of
+ * moe_forward (bit-identical routing); only the expert GEMMs change.
+ * Requires d % 256 == 0 and f % 128 == 0 (128 <= f <= 32768).
+ *
+ * moe_mx_expert_bytes: sizes of the four packed arrays for E experts of
+ * width d and hidden width f (n = E * d * f):
+ *   wq_gate_up n bytes, sf_gate_up n / 16, wq_down n / 2, sf_down n / 32.
+ * moe_mx_pack_experts: quantises W_gate_up [E, d, 2f] and W_down [E, f, d]
+ * (bf16, as moe_forward takes them) with the MXFP4 rule above, blocks of 32
+ * along each matrix's reduction axis (d, resp. f), into
+ *   wq_*: the E2M1 codes of each output feature's column, the reduction axis
+ *         contiguous, two codes per byte (even index in the low nibble):
+ *         [E][2f][d / 2] and [E][d][f / 2];
+ *   sf_*: the E8M0 scales grouped in 512-byte atoms, one per 128 output
+ *         features x 128 reduction elements: [E][2f / 128][d / 128][512]
+ *         and [E][d / 128][f / 128][512]; feature m and block b of an atom
+ *         at byte 16 * (m % 32) + 4 * (m / 32) + b.
+ *   wq_* 32-byte aligned, sf_* 16-byte aligned. One-time preparation of the
+ *   weights; enqueues two kernels on `stream`.
+ * moe_forward_mx: as moe_forward, with the packed experts in place of
+ *   W_gate_up / W_down. x takes an MXFP8 round trip along d before the
+ *   gate/up GEMM and h one along f before the down GEMM (the arithmetic of the
+ *   MX oracle); y is accumulated in fp32 and stored bf16. Workspace:
+ *   moe_forward_mx_workspace_size(T, d, E, k, f) bytes, 256-byte aligned.
+ */
+moe_status_t moe_mx_expert_bytes(int E, int d, int f, size_t* wq_gate_up, size_t* sf_gate_up,
+                                 size_t* wq_down, size_t* sf_down);
+moe_status_t moe_mx_pack_experts(const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, int E, int d, int f,
+                                 uint8_t* wq_gate_up, uint8_t* sf_gate_up, uint8_t* wq_down, uint8_t* sf_down,
+                                 cudaStream_t stream);
+size_t moe_forward_mx_workspace_size(int T, int d, int E, int k, int f);
+moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                            const uint8_t* wq_gate_up, const uint8_t* sf_gate_up,
+                            const uint8_t* wq_down, const uint8_t* sf_down,
+                            int T, int d, int E, int k, int f,
+                            moe_bf16_t* out,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* ------------------------------------------------------------ diagnostics --
  * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
  * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise

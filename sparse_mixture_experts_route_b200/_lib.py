@@ -40,6 +40,11 @@ EXPORTS = {
     "moe_forward": ([P, P, P, P, P, I, I, I, I, I, P, P, Z, P], I),
     "moe_mxfp8_quantize": ([P, I, I, P, P, P], I),
     "moe_mxfp4_quantize": ([P, I, I, P, P, P], I),
+    "moe_mx_expert_bytes": ([I, I, I, ctypes.POINTER(Z), ctypes.POINTER(Z), ctypes.POINTER(Z),
+                             ctypes.POINTER(Z)], I),
+    "moe_mx_pack_experts": ([P, P, I, I, I, P, P, P, P, P], I),
+    "moe_forward_mx_workspace_size": ([I, I, I, I, I], Z),
+    "moe_forward_mx": ([P, P, P, P, P, P, P, I, I, I, I, I, P, P, Z, P], I),
     "moe_get_device_error": ([ctypes.POINTER(ctypes.c_uint32), I], I),
     "moe_selftest_wait_timeout": ([I, P], I),
 }
@@ -221,6 +226,58 @@ def moe_mxfp4_quantize(w, stream=None, codes=None, scales=None):
     _check(_lib.moe_mxfp4_quantize(_ptr(w), rows, N, _ptr(codes), _ptr(scales), _stream(stream)),
            "moe_mxfp4_quantize")
     return codes, scales
+
+
+class MxExperts:
+    """The experts of one layer in the MX serving format (see moe_mx_pack_experts
+    in include/moe.h): packed E2M1 codes and E8M0 scale atoms of W_gate_up and
+    W_down, uint8 tensors on the device."""
+
+    def __init__(self, wq_gate_up, sf_gate_up, wq_down, sf_down, E: int, d: int, f: int):
+        self.wq_gate_up, self.sf_gate_up, self.wq_down, self.sf_down = wq_gate_up, sf_gate_up, wq_down, sf_down
+        self.E, self.d, self.f = E, d, f
+
+
+def moe_mx_expert_bytes(E: int, d: int, f: int):
+    """Bytes of (wq_gate_up, sf_gate_up, wq_down, sf_down)."""
+    vals = [ctypes.c_size_t(0) for _ in range(4)]
+    _check(_lib.moe_mx_expert_bytes(E, d, f, *[ctypes.byref(v) for v in vals]), "moe_mx_expert_bytes")
+    return tuple(v.value for v in vals)
+
+
+def moe_mx_pack_experts(W_gate_up, W_down, stream=None) -> MxExperts:
+    """Quantise and pack W_gate_up [E,d,2f] and W_down [E,f,d] (bf16) to MXFP4."""
+    E, d, f2 = W_gate_up.shape
+    f = f2 // 2
+    _need(W_gate_up, "W_gate_up", torch.bfloat16, (E, d, 2 * f))
+    _need(W_down, "W_down", torch.bfloat16, (E, f, d))
+    sizes = moe_mx_expert_bytes(E, d, f)
+    bufs = [torch.empty(n, dtype=torch.uint8, device=W_gate_up.device) for n in sizes]
+    _check(_lib.moe_mx_pack_experts(_ptr(W_gate_up), _ptr(W_down), E, d, f, *[_ptr(b) for b in bufs],
+                                    _stream(stream)), "moe_mx_pack_experts")
+    return MxExperts(*bufs, E, d, f)
+
+
+def moe_forward_mx(x, W_router, router_bias, experts: MxExperts, k: int, out=None, workspace=None, stream=None):
+    """The whole layer with MX experts. Returns out [T,d] bf16."""
+    T, d = x.shape
+    E, f = experts.E, experts.f
+    _need(x, "x", torch.bfloat16, (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    if d != experts.d:
+        raise ValueError(f"x has width {d}, the experts {experts.d}")
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", torch.bfloat16, (T, d))
+    nbytes = _lib.moe_forward_mx_workspace_size(T, d, E, k, f)
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device, stream)
+    _check(_lib.moe_forward_mx(_ptr(x), _ptr(W_router), _ptr(router_bias), _ptr(experts.wq_gate_up),
+                               _ptr(experts.sf_gate_up), _ptr(experts.wq_down), _ptr(experts.sf_down), T, d, E, k,
+                               f, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_forward_mx")
+    return out
 
 
 def moe_forward(x, W_router, router_bias, W_gate_up, W_down, k: int, out=None, workspace=None, stream=None):

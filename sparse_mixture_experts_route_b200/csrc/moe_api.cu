@@ -14,6 +14,8 @@
 
 #include "common.cuh"
 #include "expert_gemm.cuh"
+#include "mx_gemm.cuh"
+#include "mx_prep.cuh"
 #include "mx_quant.cuh"
 #include "permute.cuh"
 #include "ptx.cuh"
@@ -216,8 +218,8 @@ moe_status_t launch_route_tc(const RoutePlan& plan, const moe_bf16_t* x, const f
   router_prep_kernel<<<dim3(ceil_div(E, 32), plan.nparts), dim3(32, 8), 0, stream>>>(W_router, d, E, hi, lo, part);
   router_interleave_kernel<<<dim3(ceil_div(E, 32), 32), dim3(32, 8), 0, stream>>>(W_router, d, E, C, wt32);
   router_wnorm_kernel<<<1, 1024, 0, stream>>>(part, plan.nparts, E, wnorm);
-  router_xnorm_kernel<<<ceil_div(T * 32, 256), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), T, d / 8, xnorm,
-                                                                 ovf);
+  router_xnorm_kernel<<<static_cast<unsigned>(ceil_div64(T, 8)), 256, 0, stream>>>(reinterpret_cast<const uint4*>(x),
+                                                                                   T, d / 8, xnorm, ovf);
   router_screen_kernel<<<dim3(ceil_div(T, kScrT), ceil_div(E, kScrE), plan.nsplit), kRtThreads, kScrSmemBytes,
                          stream>>>(mX, mHi, mLo, T, d, E, plan.kb_per_split, A);
   // add the K-split planes in order and the bias: A = plane 0
@@ -306,7 +308,7 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
     // ordered sum of the chunk partials, bias, softmax and top-k: one block per token
     router_reduce_topk_kernel<<<T, 256, 0, stream>>>(lg, plan.nchunks, bias, T, E, k, idx, w);
   } else {
-    const int blocks = ceil_div(T, 8);
+    const unsigned blocks = static_cast<unsigned>(ceil_div64(T, 8));
     if (E <= 256)
       router_topk_kernel<8><<<blocks, 256, 0, stream>>>(lg, T, E, k, idx, w);
     else
@@ -832,6 +834,225 @@ moe_status_t moe_mxfp4_quantize(const moe_bf16_t* w, int K, int N, uint8_t* code
         reinterpret_cast<uint32_t*>(scales));
   else
     moe::mxfp4_quantize_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(w, K, N, codes, scales);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------- MX expert FFN path
+
+namespace {
+
+std::mutex g_mx_mutex;
+bool g_mx_ready[kMaxDevices] = {};
+
+// Shared-memory limits of the MX GEMMs (once per device, on first MX use only).
+moe_status_t mx_setup(int* num_sms) {
+  moe_status_t st = device_setup(num_sms);
+  if (st != MOE_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mx_mutex);
+  if (!g_mx_ready[dev]) {
+    if (cudaFuncSetAttribute(mx_grouped_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMxSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(mx_grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMxSmemBytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    g_mx_ready[dev] = true;
+  }
+  return MOE_OK;
+}
+
+bool encode_map_typed(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank, const cuuint64_t* dims,
+                      const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides_bytes,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Packed E2M1 weights Wq[E][rows][K / 2]: boxes of 128 K x 128 rows of one
+// expert, unpacked to one byte per element in shared memory.
+bool mx_weight_map(CUtensorMap* map, const uint8_t* wq, int E, int rows, int K) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) / 2, static_cast<cuuint64_t>(rows) * K / 2};
+  const cuuint32_t box[3] = {128, 128, 1};
+  return encode_map_typed(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wq, 3, dims, strides, box);
+}
+
+// E4M3 token rows [rows][K]: boxes of 128 K x kMxTileRows rows.
+bool mx_token_map(CUtensorMap* map, const uint8_t* q, int rows, int K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kMxTileRows)};
+  return encode_map_typed(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, 2, dims, strides, box);
+}
+
+bool mx_shape_ok(int d, int f) { return d % 256 == 0 && f % 128 == 0 && f >= 128 && f <= 32768; }
+
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+struct MxLayout {
+  size_t route, idx, w, offsets, perm_token, inv_perm, xq, sfx, hq, sfh, y, perm_ws, pre0, pre1, total;
+  int64_t tiles_max;
+};
+
+MxLayout mx_layout(int T, int d, int E, int k, int f) {
+  MxLayout L;
+  const size_t Tk = static_cast<size_t>(T) * k;
+  L.tiles_max = ceil_div64(static_cast<int64_t>(Tk), kMxTileRows) + (E < static_cast<int64_t>(Tk) ? E : Tk);
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t here = at;
+    at += align256(bytes);
+    return here;
+  };
+  L.route = take(route_plan(T, d, E).ws_bytes);
+  L.idx = take(Tk * sizeof(int32_t));
+  L.w = take(Tk * sizeof(float));
+  L.offsets = take((static_cast<size_t>(E) + 1) * sizeof(int32_t));
+  L.perm_token = take(Tk * sizeof(int32_t));
+  L.inv_perm = take(Tk * sizeof(int32_t));
+  L.xq = take(Tk * d);
+  L.sfx = take(static_cast<size_t>(L.tiles_max) * (d / 128) * kMxAtomBytes);
+  L.hq = take(Tk * f);
+  L.sfh = take(static_cast<size_t>(L.tiles_max) * (f / 128) * kMxAtomBytes);
+  L.y = take(Tk * d * 2);
+  L.perm_ws = take(permute_ws(T, E, k));
+  L.pre0 = take((static_cast<size_t>(E) + 1) * sizeof(int32_t));
+  L.pre1 = take((static_cast<size_t>(E) + 1) * sizeof(int32_t));
+  L.total = at;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_mx_expert_bytes(int E, int d, int f, size_t* wq_gate_up, size_t* sf_gate_up, size_t* wq_down,
+                                 size_t* sf_down) {
+  if (!wq_gate_up || !sf_gate_up || !wq_down || !sf_down) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || d < 256 || d > 32768 || !mx_shape_ok(d, f)) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  const size_t n = static_cast<size_t>(E) * d * f;  // elements of W_down; W_gate_up has 2n
+  *wq_gate_up = n;       // 2n codes, two per byte
+  *sf_gate_up = n / 16;  // one scale per 32 codes
+  *wq_down = n / 2;
+  *sf_down = n / 32;
+  return MOE_OK;
+}
+
+moe_status_t moe_mx_pack_experts(const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, int E, int d, int f,
+                                 uint8_t* wq_gate_up, uint8_t* sf_gate_up, uint8_t* wq_down, uint8_t* sf_down,
+                                 cudaStream_t stream) {
+  size_t b0, b1, b2, b3;
+  const moe_status_t st = moe_mx_expert_bytes(E, d, f, &b0, &b1, &b2, &b3);
+  if (st != MOE_OK) return st;
+  if (!W_gate_up || !W_down || !wq_gate_up || !sf_gate_up || !wq_down || !sf_down) return MOE_ERR_INVALID_ARG;
+  if (!aligned32(wq_gate_up) || !aligned32(wq_down) || !aligned16(sf_gate_up) || !aligned16(sf_down))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t g0 = static_cast<int64_t>(E) * (d / kMxBlock) * (2 * f);
+  const int64_t g1 = static_cast<int64_t>(E) * (f / kMxBlock) * d;
+  mx_pack_weights_kernel<<<static_cast<unsigned>(ceil_div64(g0, 256)), 256, 0, stream>>>(W_gate_up, E, d, 2 * f,
+                                                                                        wq_gate_up, sf_gate_up);
+  mx_pack_weights_kernel<<<static_cast<unsigned>(ceil_div64(g1, 256)), 256, 0, stream>>>(W_down, E, f, d, wq_down,
+                                                                                        sf_down);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t moe_forward_mx_workspace_size(int T, int d, int E, int k, int f) {
+  if (T < 1 || d < 1 || E < 1 || k < 1 || f < 1 || !mx_shape_ok(d, f)) return 0;
+  return mx_layout(T, d, E, k, f).total;
+}
+
+moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                            const uint8_t* wq_gate_up, const uint8_t* sf_gate_up, const uint8_t* wq_down,
+                            const uint8_t* sf_down, int T, int d, int E, int k, int f, moe_bf16_t* out,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!x || !W_router || !wq_gate_up || !sf_gate_up || !wq_down || !sf_down || !out) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(T, d, E, k) || !mx_shape_ok(d, f)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out) || !aligned32(wq_gate_up) || !aligned32(wq_down) || !aligned16(sf_gate_up) ||
+      !aligned16(sf_down))
+    return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  const MxLayout L = mx_layout(T, d, E, k, f);
+  if (!workspace || !aligned256(workspace) || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  int sms = 0;
+  moe_status_t st = mx_setup(&sms);
+  if (st != MOE_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_token = reinterpret_cast<int32_t*>(ws + L.perm_token);
+  int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  uint8_t* xq = ws + L.xq;
+  uint8_t* sfx = ws + L.sfx;
+  uint8_t* hq = ws + L.hq;
+  uint8_t* sfh = ws + L.sfh;
+  moe_bf16_t* y = reinterpret_cast<moe_bf16_t*>(ws + L.y);
+  int32_t* pre0 = reinterpret_cast<int32_t*>(ws + L.pre0);
+  int32_t* pre1 = reinterpret_cast<int32_t*>(ws + L.pre1);
+  const int Tk = T * k;
+  CUtensorMap mA0, mB0, mA1, mB1;
+  if (!mx_weight_map(&mA0, wq_gate_up, E, 2 * f, d) || !mx_token_map(&mB0, xq, Tk, d) ||
+      !mx_weight_map(&mA1, wq_down, E, d, f) || !mx_token_map(&mB1, hq, Tk, f))
+    return MOE_ERR_INVALID_ARG;
+
+  // route, then the dispatch tables (counts, offsets, permutation, token tiles
+  // of kMxTileRows rows); no bf16 row copy: the rows are copied as MXFP8 below
+  const RouteDispatch disp = {offsets, perm_token, inv_perm, pre0, pre1, nullptr, 0};
+  bool dispatched = false;
+  st = launch_route(x, W_router, router_bias, T, d, E, k, idx, w, ws + L.route, stream, T == 1 ? &disp : nullptr,
+                    &dispatched);
+  if (st != MOE_OK) return st;
+  if (!dispatched) {
+    if (Tk <= kSmallDispatchPairs) {
+      dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, kMxTileRows, kMxTileRows, offsets, perm_token,
+                                                    inv_perm, pre0, pre1, nullptr, 0);
+    } else {
+      st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, nullptr, ws + L.perm_ws, stream);
+      if (st != MOE_OK) return st;
+      gemm_schedule_kernel<<<1, 1024, 0, stream>>>(offsets, E, kMxTileRows, kMxTileRows, pre0, pre1, nullptr, 0);
+    }
+  }
+  mx_quantize_dispatch_kernel<<<static_cast<unsigned>(T), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), idx, inv_perm, offsets, pre0, d, k, E, xq, sfx);
+
+  MxGemmParams p0;
+  p0.expert_offsets = offsets;
+  p0.tile_prefix = pre0;
+  p0.E = E;
+  p0.K = d;
+  p0.n_feat = f;
+  p0.n_feat_tiles = f / 128;
+  p0.a1_row = f;
+  p0.w_rows = 2 * f;
+  p0.sfw = sf_gate_up;
+  p0.sft = sfx;
+  p0.hq = hq;
+  p0.hs = sfh;
+  p0.out = nullptr;
+  MxGemmParams p1 = p0;
+  p1.K = f;
+  p1.n_feat = d;
+  p1.n_feat_tiles = d / 256;
+  p1.a1_row = 128;
+  p1.w_rows = d;
+  p1.sfw = sf_down;
+  p1.sft = sfh;
+  p1.hq = nullptr;
+  p1.hs = nullptr;
+  p1.out = y;
+  const int64_t g0 = L.tiles_max * p0.n_feat_tiles, g1 = L.tiles_max * p1.n_feat_tiles;
+  mx_grouped_gemm_kernel<0><<<static_cast<unsigned>(g0 < sms ? g0 : sms), kMxThreads, kMxSmemBytes, stream>>>(
+      mA0, mB0, p0);
+  mx_grouped_gemm_kernel<1><<<static_cast<unsigned>(g1 < sms ? g1 : sms), kMxThreads, kMxSmemBytes, stream>>>(
+      mA1, mB1, p1);
+  st = launch_unpermute(y, inv_perm, w, T, d, k, out, stream);
+  if (st != MOE_OK) return st;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -158,6 +158,29 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D[tmem] (+)= (A * 2^SFA) (B * 2^SFB), kind::mxf8f6f4 with E8M0 block scales:
+// A and B from shared-memory descriptors (A E2M1, B E4M3 here, chosen by the
+// instruction descriptor), fp32 accumulate. sfa / sfb are TMEM addresses of
+// the scale columns; their top two bits select the byte (the 32-element K
+// block) within each 32-bit column, and must match the instruction
+// descriptor's scale IDs.
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory (descriptor) to TMEM at `taddr`,
+// the same 32 rows into each of the four 32-lane quadrants. Asynchronous;
+// ordered before the tcgen05.mma instructions this thread issues after it.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -180,6 +203,16 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// The same for 16 columns: r[i] = TMEM[lane_base + laneid][col + i], i < 16.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // --------------------------------------------------- UMMA descriptors (sm_100)
@@ -197,6 +230,28 @@ __device__ __forceinline__ uint64_t umma_smem_desc_sw128(uint32_t saddr, uint32_
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
+}
+
+// The same descriptor for an unswizzled K-major operand (layout 0): 8-row core
+// matrices of 16-byte rows, `sbo_bytes` between core matrices along M/N,
+// `lbo_bytes` between core matrices along K.
+__device__ __forceinline__ uint64_t umma_smem_desc_noswizzle(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with block scales, fp32 D:
+//   [4,6) B scale ID  [7,10) A format (5 = E2M1)  [10,13) B format (0 = E4M3)
+//   [15] A major  [16] B major (0 = K)  [17,23) N >> 3  [23] scale format
+//   (1 = E8M0)  [24,29) M >> 4  [29,31) A scale ID  [31] K size (0 = 32)
+__host__ __device__ constexpr uint32_t umma_idesc_mx_e2m1_e4m3(uint32_t M, uint32_t N, uint32_t sfa_id,
+                                                               uint32_t sfb_id) {
+  return (sfb_id << 4) | (5u << 7) | (0u << 10) | ((N >> 3) << 17) | (1u << 23) | ((M >> 4) << 24) |
+         (sfa_id << 29);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D:

@@ -197,7 +197,7 @@ template <int MAXV>
 __global__ void __launch_bounds__(256)
     router_topk_kernel(const float* __restrict__ lg, int T, int E, int k, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int warp = static_cast<int>(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));  // no overflow for T < 2^31
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
   const int t = warp;

@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(256)
     router_xnorm_kernel(const uint4* __restrict__ x, int T, int vec_per_row, float* __restrict__ xnorm,
                         int32_t* __restrict__ overflow) {
   if (blockIdx.x == 0 && threadIdx.x == 0) overflow[0] = 0;  // the re-check appends to it
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int t = static_cast<int>(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));  // no overflow for T < 2^31
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   float s = 0.0f;

@@ -185,3 +185,51 @@ def test_mx_quantize_checks(lib):
     assert q4(p, 0, 8, p, p, None) == 1
     assert q4(p, 64, 0, p, p, None) == 1                          # N = 0
     assert q4(p, 64, (1 << 20) + 1, p, p, None) == 1              # N too large
+
+
+def test_mx_expert_sizes_and_checks(lib):
+    """MX experts: packed sizes (two E2M1 codes per byte, one E8M0 scale per 32
+    codes), shape limits (d % 256, f % 128), and the host checks of
+    moe_mx_pack_experts / moe_forward_mx, all before any CUDA call."""
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    ZP = ctypes.POINTER(Z)
+    lib.moe_mx_expert_bytes.argtypes = [I, I, I, ZP, ZP, ZP, ZP]
+    lib.moe_mx_pack_experts.argtypes = [P, P, I, I, I, P, P, P, P, P]
+    lib.moe_forward_mx_workspace_size.argtypes = [I, I, I, I, I]
+    lib.moe_forward_mx_workspace_size.restype = Z
+    lib.moe_forward_mx.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, P, Z, P]
+    lib.moe_forward_workspace_size.argtypes = [I, I, I, I, I]
+    lib.moe_forward_workspace_size.restype = Z
+    v = [Z(0) for _ in range(4)]
+    refs = [ctypes.byref(x) for x in v]
+    assert lib.moe_mx_expert_bytes(384, 7168, 2048, *refs) == 0
+    n = 384 * 7168 * 2048
+    assert [x.value for x in v] == [n, n // 16, n // 2, n // 32]
+    # bytes per expert parameter: 4 bits + 8 bits per 32 = 4.25 bits
+    assert (v[0].value + v[1].value + v[2].value + v[3].value) * 8 == 3 * n * 4.25
+    assert lib.moe_mx_expert_bytes(8, 7168 + 128, 512, *refs) == 1   # d % 256
+    assert lib.moe_mx_expert_bytes(8, 7168, 576, *refs) == 1         # f % 128
+    assert lib.moe_mx_expert_bytes(2048, 256, 128, *refs) == 2       # E > 1024
+    assert lib.moe_mx_expert_bytes(8, 256, 128, None, *refs[1:]) == 1
+    for (T, d, E, k, f) in [(1, 7168, 896, 16, 512), (4096, 7168, 384, 8, 2048), (100, 256, 8, 2, 128)]:
+        mw = lib.moe_forward_mx_workspace_size(T, d, E, k, f)
+        Tk = T * k
+        tiles = -(-Tk // 112) + min(E, Tk)
+        assert mw % 256 == 0
+        # MXFP8 x and h rows, their scale atoms, bf16 y, routing tables
+        assert mw >= Tk * d + Tk * f + tiles * (d // 128 + f // 128) * 512 + Tk * d * 2 + Tk * 16
+    assert lib.moe_forward_mx_workspace_size(64, 7168 + 128, 8, 2, 256) == 0
+    p = ctypes.c_void_p(FAKE)
+    p16 = ctypes.c_void_p(FAKE + 16)   # 16- but not 32-byte aligned
+    assert lib.moe_mx_pack_experts(None, p, 8, 256, 128, p, p, p, p, None) == 1
+    assert lib.moe_mx_pack_experts(p, p, 8, 256, 128, p16, p, p, p, None) == 1     # wq alignment
+    assert lib.moe_mx_pack_experts(p, p, 8, 256, 128, p, ctypes.c_void_p(FAKE + 8), p, p, None) == 1
+    assert lib.moe_mx_pack_experts(p, p, 8, 384, 128, p, p, p, p, None) == 1      # d % 256
+    mw = lib.moe_forward_mx_workspace_size(64, 256, 8, 2, 128)
+    args = [p, p, None, p, p, p, p, 64, 256, 8, 2, 128, p, p, mw, None]
+    assert lib.moe_forward_mx(*args[:3], p16, *args[4:]) == 1                     # wq alignment
+    assert lib.moe_forward_mx(*args[:7], 64, 256, 8, 9, 128, *args[12:]) == 1     # k > E
+    assert lib.moe_forward_mx(*args[:7], 64, 256, 32, 17, 128, *args[12:]) == 2   # k > 16
+    assert lib.moe_forward_mx(*args[:11], 192, *args[12:]) == 1                   # f % 128
+    assert lib.moe_forward_mx(*args[:14], mw - 256, None) == 3                    # workspace
+    assert lib.moe_forward_mx(*args[:13], ctypes.c_void_p(FAKE + 64), mw, None) == 3
