@@ -5,6 +5,7 @@
 // (except moe_get_device_error, a documented debug read).
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdint>
 #include <cstring>
@@ -657,8 +658,25 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
   FfnPlan fp;
   st = plan_ffn(x_perm, offsets, W_gate_up, W_down, Tk, d, E, f, h, y_perm, ws + L.ffn_ws, sms, &fp);
   if (st != MOE_OK) return st;
+  // stage boundaries: events (timed calls) and NVTX ranges named for the
+  // stage, which profilers show around the stage's launches (no cost without one)
+  static const char* const kStage[MOE_TIMED_STAGES] = {"moe.route", "moe.dispatch", "moe.gate_up", "moe.down",
+                                                       "moe.combine"};
+  struct NvtxStage {  // closes a range left open by an early return
+    bool open = false;
+    ~NvtxStage() {
+      if (open) nvtxRangePop();
+    }
+  } nv;
   auto mark = [&](int i) {
     if (ev) cudaEventRecord(ev[i], stream);
+    if (i % 2 == 0) {
+      nvtxRangePushA(kStage[i / 2]);
+      nv.open = true;
+    } else {
+      nvtxRangePop();
+      nv.open = false;
+    }
   };
   mark(0);
   // one token: the router's last CTA also writes the dispatch tables, and the
