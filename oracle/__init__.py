@@ -59,10 +59,15 @@ def _load():
             lib.oracle_mxfp8_quantize.argtypes = [P, I, I, P, P]
             lib.oracle_mxfp8_dequantize.argtypes = [P, P, I, I, P]
             lib.oracle_expert_ffn_mx.argtypes = [P, I, P, P, I, I, P, P]
+            lib.oracle_qb_cutoffs.argtypes = [P, P, I, I, I, P]
+            lib.oracle_qb_update.argtypes = [P, P, I, I, I, P]
+            lib.oracle_qb_histogram.argtypes = [P, P, I, I, ctypes.c_double, ctypes.c_double, I, P]
+            lib.oracle_qb_bias_from_histogram.argtypes = [P, I, I, ctypes.c_double, ctypes.c_double, I, I, P]
             for fn in ("oracle_router_logits", "oracle_topk", "oracle_permute", "oracle_expert_ffn",
                        "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version",
                        "oracle_mxfp4_quantize", "oracle_mxfp4_dequantize", "oracle_mxfp8_quantize",
-                       "oracle_mxfp8_dequantize", "oracle_expert_ffn_mx"):
+                       "oracle_mxfp8_dequantize", "oracle_expert_ffn_mx", "oracle_qb_cutoffs", "oracle_qb_update",
+                       "oracle_qb_histogram", "oracle_qb_bias_from_histogram"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -288,3 +293,56 @@ def expert_ffn_mx(x_rows, gu_codes, gu_scales, dn_codes, dn_scales, want_h: bool
     if st:
         raise ValueError(f"oracle_expert_ffn_mx: status {st}")
     return (y, h) if want_h else y
+
+
+# ------------------------------------------------------ Quantile Balancing
+
+def _f64c(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def qb_cutoffs(scores, k: int, bias=None) -> np.ndarray:
+    """alpha [m]: each token's (k+1)-th largest biased score s + b (the cutoff
+    of top-(k+1) routing). Definition and readings: oracle_qb_cutoffs in
+    moe_oracle.cpp."""
+    s = _f64c(scores)
+    m, n = s.shape
+    b = _f64c(bias) if bias is not None else None
+    alpha = np.empty(m, dtype=np.float64)
+    _check(_load().oracle_qb_cutoffs(s.ctypes.data, b.ctypes.data if b is not None else None, m, n, k,
+                                     alpha.ctypes.data), "oracle_qb_cutoffs")
+    return alpha
+
+
+def qb_update(scores, k: int, bias=None) -> np.ndarray:
+    """One Quantile Balancing step with exact quantiles: the new biases [n]."""
+    s = _f64c(scores)
+    m, n = s.shape
+    b = _f64c(bias) if bias is not None else None
+    out = np.empty(n, dtype=np.float64)
+    _check(_load().oracle_qb_update(s.ctypes.data, b.ctypes.data if b is not None else None, m, n, k,
+                                    out.ctypes.data), "oracle_qb_update")
+    return out
+
+
+def qb_histogram(scores, alpha, lo: float, hi: float, bins: int, H=None) -> np.ndarray:
+    """Per-expert margin counts H [n, bins] int64 (added into H if given)."""
+    s = _f64c(scores)
+    m, n = s.shape
+    a = _f64c(alpha)
+    if H is None:
+        H = np.zeros((n, bins), dtype=np.int64)
+    assert H.dtype == np.int64 and H.shape == (n, bins) and H.flags.c_contiguous
+    _check(_load().oracle_qb_histogram(s.ctypes.data, a.ctypes.data, m, n, float(lo), float(hi), bins,
+                                       H.ctypes.data), "oracle_qb_histogram")
+    return H
+
+
+def qb_bias_from_histogram(H, lo: float, hi: float, m_total: int, k: int) -> np.ndarray:
+    """The new biases [n] from (all-reduced) margin histograms."""
+    H = np.ascontiguousarray(H, dtype=np.int64)
+    n, bins = H.shape
+    out = np.empty(n, dtype=np.float64)
+    _check(_load().oracle_qb_bias_from_histogram(H.ctypes.data, n, bins, float(lo), float(hi), m_total, k,
+                                                 out.ctypes.data), "oracle_qb_bias_from_histogram")
+    return out

@@ -39,6 +39,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
 #include <vector>
 
 #ifdef _OPENMP
@@ -478,6 +479,113 @@ int oracle_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t
       std::memcpy(&u, &fv, sizeof(u));
       w_out[r * N + n] = static_cast<uint16_t>(u >> 16);
     }
+  return 0;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------ Quantile Balancing
+//
+// [P3] section "Systems Optimization, Load Balancing, and Post-Training
+// Alignment": Quantile Balancing (QB) sets the router's per-expert biases from
+// the dual of the balanced-assignment linear program. For m tokens, n experts,
+// top-k routing and target load q = m k / n, each expert's bias comes from the
+// (1 - k/n)-quantile, over tokens, of the margins s[i,j] - alpha_i, where
+// alpha_i is token i's cutoff under top-(k+1) routing. The update formula
+// itself is missing from the page; reading taken, from that LP:
+//   maximise sum s[i,j] x[i,j]  s.t.  sum_j x[i,j] = k,  sum_i x[i,j] <= q,
+//   0 <= x <= 1,
+// whose dual has a price alpha_i per token and beta_j per expert. With the
+// current biases b (b = -beta), alpha_i is the (k+1)-th largest of
+// s[i,j] + b_j (the best biased score left out of the top k), and the beta_j
+// minimising the dual objective q beta_j + sum_i max(0, s[i,j] - alpha_i -
+// beta_j) for that alpha is the ceil(q)-th largest margin s[i,j] - alpha_i
+// over tokens: the (1 - k/n)-quantile. The new bias is b_j = -beta_j. The
+// scores s are the router logits, the quantity the bias shifts.
+// Histogram form (the page's per-expert binned counts H[n][B], B = 1000 there,
+// summed over data-parallel ranks by one integer all-reduce): the margins of
+// expert j are counted in B equal bins over [lo, hi) (the range is not given
+// on the page: a parameter here), a margin below lo in bin 0 and one at or
+// above hi in bin B - 1. beta_j is then the lower edge of the bin that holds
+// the ceil(q)-th largest margin, within one bin width (hi - lo) / B of the
+// exact value when every margin lies in [lo, hi).
+
+namespace {
+
+// ceil(m k / n) clamped to [1, m]: the rank, from the top, of the quantile.
+int64_t qb_rank(int64_t m, int64_t n, int64_t k) {
+  int64_t r = (m * k + n - 1) / n;
+  return std::max<int64_t>(1, std::min(r, m));
+}
+
+}  // namespace
+
+extern "C" {
+
+// alpha[i] = (k+1)-th largest of s[i,j] + b[j] over j (b may be NULL: zero).
+// s [m, n] row-major. 1 <= k < n.
+int oracle_qb_cutoffs(const double* s, const double* b, int64_t m, int64_t n, int64_t k, double* alpha) {
+  if (!s || !alpha || m < 1 || n < 2 || k < 1 || k >= n) return 1;
+  std::vector<double> v(n);
+  for (int64_t i = 0; i < m; ++i) {
+    for (int64_t j = 0; j < n; ++j) v[j] = s[i * n + j] + (b ? b[j] : 0.0);
+    std::nth_element(v.begin(), v.begin() + k, v.end(), std::greater<double>());
+    alpha[i] = v[k];
+  }
+  return 0;
+}
+
+// One QB step with exact quantiles: b_new[j] = -(ceil(m k / n)-th largest of
+// s[i,j] - alpha[i] over i), alpha from oracle_qb_cutoffs(s, b).
+int oracle_qb_update(const double* s, const double* b, int64_t m, int64_t n, int64_t k, double* b_new) {
+  if (!b_new) return 1;
+  std::vector<double> alpha(m > 0 ? m : 1);
+  const int st = oracle_qb_cutoffs(s, b, m, n, k, alpha.data());
+  if (st) return st;
+  const int64_t r = qb_rank(m, n, k);
+  std::vector<double> mu(m);
+  for (int64_t j = 0; j < n; ++j) {
+    for (int64_t i = 0; i < m; ++i) mu[i] = s[i * n + j] - alpha[i];
+    std::nth_element(mu.begin(), mu.begin() + (r - 1), mu.end(), std::greater<double>());
+    b_new[j] = -mu[r - 1];
+  }
+  return 0;
+}
+
+// H[j][bin] += 1 for each token's margin s[i,j] - alpha[i] (H [n, B] int64,
+// accumulated into, so several batches or ranks can add up).
+int oracle_qb_histogram(const double* s, const double* alpha, int64_t m, int64_t n, double lo, double hi, int64_t B,
+                        int64_t* H) {
+  if (!s || !alpha || !H || m < 0 || n < 1 || B < 1 || !(hi > lo)) return 1;
+  const double width = (hi - lo) / static_cast<double>(B);
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t j = 0; j < n; ++j) {
+      const double mu = s[i * n + j] - alpha[i];
+      int64_t bin = mu < lo ? 0 : static_cast<int64_t>(std::floor((mu - lo) / width));
+      bin = std::max<int64_t>(0, std::min(bin, B - 1));
+      H[j * B + bin] += 1;
+    }
+  return 0;
+}
+
+// b_new[j] = -(lower edge of the bin of H[j] holding the ceil(m_total k / n)-th
+// largest margin), m_total the number of tokens counted in each row of H.
+int oracle_qb_bias_from_histogram(const int64_t* H, int64_t n, int64_t B, double lo, double hi, int64_t m_total,
+                                  int64_t k, double* b_new) {
+  if (!H || !b_new || n < 2 || B < 1 || !(hi > lo) || m_total < 1 || k < 1 || k >= n) return 1;
+  const int64_t r = qb_rank(m_total, n, k);
+  const double width = (hi - lo) / static_cast<double>(B);
+  for (int64_t j = 0; j < n; ++j) {
+    int64_t total = 0;
+    for (int64_t t = 0; t < B; ++t) total += H[j * B + t];
+    if (total != m_total) return 2;  // every token is counted once per expert
+    int64_t c = 0, bin = B - 1;
+    for (; bin > 0; --bin) {
+      c += H[j * B + bin];
+      if (c >= r) break;
+    }
+    b_new[j] = -(lo + static_cast<double>(bin) * width);
+  }
   return 0;
 }
 

@@ -5,7 +5,10 @@ by tokens; the forward pass has no exchange step), so the only collectives
 are the timing barrier and the max-over-ranks reduction. These tests check
 that logic without a GPU: the max over ranks, the whole-job throughput, that
 replicas draw different tokens from one seeded recipe, and that only rank 0
-of the reference arm does any work.
+of the reference arm does any work. The Quantile Balancing bias update (the
+next row after the forward pass) does have an exchange step, an integer
+all-reduce of per-expert margin histograms; its test checks that the summed
+histograms give every rank the biases of the whole batch.
 """
 import os
 import socket
@@ -87,3 +90,49 @@ def test_reference_arm_rank0_prints_one_line():
     assert d["impl"] == "reference" and d["metric"] == "moe_layer_tokens_per_s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _qb_worker(rank, world, port, q):
+    """Quantile Balancing across data-parallel ranks: each rank counts the
+    margins of its own tokens, one integer all-reduce sums the histograms, and
+    every rank recovers the same biases as one process holding the whole batch."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import numpy as np
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        m, n, k, lo, hi, bins = 600, 16, 2, -10.0, 10.0, 1000
+        rng = np.random.default_rng(11)
+        s = rng.normal(size=(m, n)) + 1.5 * np.log1p(np.arange(n))[::-1]   # the same batch on every rank
+        b0 = np.zeros(n)
+        mine = slice(rank * m // world, (rank + 1) * m // world)
+        a = oracle.qb_cutoffs(s[mine], k, b0)
+        H = torch.from_numpy(oracle.qb_histogram(s[mine], a, lo, hi, bins))
+        dist.all_reduce(H, op=dist.ReduceOp.SUM)
+        b_dist = oracle.qb_bias_from_histogram(H.numpy(), lo, hi, m, k)
+        a_all = oracle.qb_cutoffs(s, k, b0)
+        b_one = oracle.qb_bias_from_histogram(oracle.qb_histogram(s, a_all, lo, hi, bins), lo, hi, m, k)
+        b_exact = oracle.qb_update(s, k, b0)
+        q.put((rank, bool(np.array_equal(b_dist, b_one)),
+               float(np.abs(b_dist - b_exact).max()), (hi - lo) / bins))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_quantile_balancing_histograms_all_reduce_over_two_ranks():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_qb_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, same_as_one_process, err, width in res:
+        assert same_as_one_process
+        assert err <= width + 1e-12

@@ -49,6 +49,12 @@ MUTATIONS = {
     "mx_ffn_h_not_requantised": ("if (!st) st = oracle_mxfp8_dequantize(hc.data(), hs.data(), 1, f, hrow.data());",
                                  "if (!st) st = 0;"),
     "mx_ffn_gate_up_swapped": ("const double g = gu[j], u = gu[f + j];", "const double u = gu[j], g = gu[f + j];"),
+    "qb_cutoff_is_kth_not_k_plus_first": ("std::greater<double>());\n    alpha[i] = v[k];",
+                                          "std::greater<double>());\n    alpha[i] = v[k - 1];"),
+    "qb_quantile_rank_floor": ("int64_t r = (m * k + n - 1) / n;", "int64_t r = (m * k) / n;"),
+    "qb_bias_sign": ("b_new[j] = -mu[r - 1];", "b_new[j] = mu[r - 1];"),
+    "qb_histogram_upper_edge": ("b_new[j] = -(lo + static_cast<double>(bin) * width);",
+                                "b_new[j] = -(lo + static_cast<double>(bin + 1) * width);"),
 }
 
 

@@ -491,3 +491,103 @@ def test_mx_expert_ffn_vs_numpy_composition():
     np.testing.assert_allclose(h, hq, rtol=0, atol=1e-12 * np.abs(hq).max())
     np.testing.assert_allclose(y, hq @ wd, rtol=0, atol=1e-12 * np.abs(hq @ wd).max())
     assert not np.allclose(hq, hh)  # the h round trip is not a no-op on these values
+
+
+# ------------------------------------------------------------ Quantile Balancing
+#
+# The reading of "Kimi K3: Open Frontier Intelligence", section "Systems
+# Optimization, Load Balancing, and Post-Training Alignment" (oracle_qb_* in
+# moe_oracle.cpp): the bias update is the dual step of the balanced-assignment
+# LP. The pins characterise each quantity by what it must satisfy, not by
+# recomputing it the same way.
+
+def _qb_scores(m, n, seed, skew=0.0):
+    rng = np.random.default_rng(seed)
+    return rng.normal(size=(m, n)) + skew * np.log1p(np.arange(n))[::-1]
+
+
+@pytest.mark.parametrize("m,n,k", [(40, 8, 2), (97, 16, 3), (5, 4, 3)])
+def test_qb_cutoff_is_the_k_plus_first_biased_score(m, n, k):
+    s = _qb_scores(m, n, 1)
+    b = np.random.default_rng(2).normal(size=n) * 0.3
+    a = oracle.qb_cutoffs(s, k, b)
+    v = s + b
+    # exactly k biased scores above the cutoff, and the cutoff is one of them
+    assert np.all((v > a[:, None]).sum(1) == k)
+    assert np.all(np.isclose(v, a[:, None], rtol=0, atol=0).sum(1) >= 1)
+
+
+def _dual_obj(beta, mu, q):
+    return q * beta + np.maximum(0.0, mu - beta).sum()
+
+
+@pytest.mark.parametrize("m,n,k", [(40, 8, 2), (50, 8, 2), (97, 16, 3), (64, 64, 8)])
+def test_qb_update_minimises_the_dual_over_each_expert_price(m, n, k):
+    """For the cutoffs alpha, beta_j = -b_new_j minimises the LP dual's
+    expert-j term q * beta + sum_i max(0, s_ij - alpha_i - beta), q = m k / n:
+    a convex piecewise-linear function whose minimum lies at one of the
+    margins, so a brute-force scan over all margins finds its minimum."""
+    s = _qb_scores(m, n, 3, skew=0.5)
+    b0 = np.random.default_rng(4).normal(size=n) * 0.2
+    a = oracle.qb_cutoffs(s, k, b0)
+    beta = -oracle.qb_update(s, k, b0)
+    q = m * k / n
+    for j in range(n):
+        mu = s[:, j] - a
+        best = min(_dual_obj(c, mu, q) for c in mu)
+        assert _dual_obj(beta[j], mu, q) <= best + 1e-12
+        # and beta_j is itself a margin (the quantile is an order statistic)
+        assert np.any(mu == beta[j])
+
+
+def test_qb_update_balances_a_skewed_router():
+    """What the update is for: iterating it on scores with a strong per-expert
+    skew brings the biased top-k loads close to the target m k / n."""
+    m, n, k = 2000, 16, 2
+    s = _qb_scores(m, n, 5, skew=2.0)
+
+    def loads(b):
+        top = np.argsort(-(s + b), axis=1, kind="stable")[:, :k]
+        return np.bincount(top.ravel(), minlength=n)
+
+    b = np.zeros(n)
+    before = loads(b).max() / (m * k / n)
+    for _ in range(20):
+        b = oracle.qb_update(s, k, b)
+    after = loads(b).max() / (m * k / n)
+    assert before > 3.0
+    assert after < 1.15
+
+
+def test_qb_histogram_counts_and_quantile_within_one_bin():
+    m, n, k = 300, 12, 3
+    s = _qb_scores(m, n, 7, skew=0.3)
+    a = oracle.qb_cutoffs(s, k)
+    lo, hi, bins = -8.0, 8.0, 1000
+    H = oracle.qb_histogram(s, a, lo, hi, bins)
+    assert np.all(H.sum(1) == m)
+    mu = s - a[:, None]
+    assert np.all((mu >= lo) & (mu < hi))
+    # bin edges: a margin at a bin's lower edge lands in that bin
+    width = (hi - lo) / bins
+    Hc = oracle.qb_histogram(np.array([[lo + 7 * width, lo], [hi + 1.0, lo - 1.0]]), np.zeros(2), lo, hi, bins)
+    assert Hc[0, 7] == 1 and Hc[0, bins - 1] == 1 and Hc[1, 0] == 2
+    exact = oracle.qb_update(s, k)
+    approx = oracle.qb_bias_from_histogram(H, lo, hi, m, k)
+    # the lower edge of the quantile's bin: beta_hist <= beta <= beta_hist + width
+    assert np.all(approx >= exact - 1e-12)
+    assert np.all(approx <= exact + width + 1e-12)
+
+
+def test_qb_histograms_add_across_batches():
+    """Counts of two halves of a batch add up to the counts of the whole (the
+    property the integer all-reduce over data-parallel ranks relies on)."""
+    m, n, k = 200, 8, 2
+    s = _qb_scores(m, n, 9)
+    a = oracle.qb_cutoffs(s, k)
+    whole = oracle.qb_histogram(s, a, -6, 6, 100)
+    H = oracle.qb_histogram(s[:77], a[:77], -6, 6, 100)
+    oracle.qb_histogram(s[77:], a[77:], -6, 6, 100, H=H)
+    assert np.array_equal(H, whole)
+    assert np.array_equal(oracle.qb_bias_from_histogram(H, -6, 6, m, k),
+                          oracle.qb_bias_from_histogram(whole, -6, 6, m, k))
