@@ -63,11 +63,14 @@ def _load():
             lib.oracle_qb_update.argtypes = [P, P, I, I, I, P]
             lib.oracle_qb_histogram.argtypes = [P, P, I, I, ctypes.c_double, ctypes.c_double, I, P]
             lib.oracle_qb_bias_from_histogram.argtypes = [P, I, I, ctypes.c_double, ctypes.c_double, I, I, P]
+            lib.oracle_qb_histogram_f32.argtypes = [P, P, I, I, I, ctypes.c_float, ctypes.c_float, I, P, P]
+            lib.oracle_qb_quantile_bins.argtypes = [P, I, I, I, I, P]
             for fn in ("oracle_router_logits", "oracle_topk", "oracle_permute", "oracle_expert_ffn",
                        "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version",
                        "oracle_mxfp4_quantize", "oracle_mxfp4_dequantize", "oracle_mxfp8_quantize",
                        "oracle_mxfp8_dequantize", "oracle_expert_ffn_mx", "oracle_qb_cutoffs", "oracle_qb_update",
-                       "oracle_qb_histogram", "oracle_qb_bias_from_histogram"):
+                       "oracle_qb_histogram", "oracle_qb_bias_from_histogram", "oracle_qb_histogram_f32",
+                       "oracle_qb_quantile_bins"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -345,4 +348,31 @@ def qb_bias_from_histogram(H, lo: float, hi: float, m_total: int, k: int) -> np.
     out = np.empty(n, dtype=np.float64)
     _check(_load().oracle_qb_bias_from_histogram(H.ctypes.data, n, bins, float(lo), float(hi), m_total, k,
                                                  out.ctypes.data), "oracle_qb_bias_from_histogram")
+    return out
+
+
+def qb_histogram_f32(scores, k: int, lo: float, hi: float, bins: int, bias=None, H=None):
+    """The margin histogram with every decision in fp32 (scores and bias taken
+    as fp32). Returns (alpha [m] fp32, H [n, bins] int64). Definition:
+    oracle_qb_histogram_f32 in moe_oracle.cpp."""
+    s = np.ascontiguousarray(np.asarray(scores, dtype=np.float32))
+    m, n = s.shape
+    b = np.ascontiguousarray(np.asarray(bias, dtype=np.float32)) if bias is not None else None
+    if H is None:
+        H = np.zeros((n, bins), dtype=np.int64)
+    assert H.dtype == np.int64 and H.shape == (n, bins) and H.flags.c_contiguous
+    alpha = np.empty(m, dtype=np.float32)
+    _check(_load().oracle_qb_histogram_f32(s.ctypes.data, b.ctypes.data if b is not None else None, m, n, k,
+                                           float(lo), float(hi), bins, alpha.ctypes.data, H.ctypes.data),
+           "oracle_qb_histogram_f32")
+    return alpha, H
+
+
+def qb_quantile_bins(H, m_total: int, k: int) -> np.ndarray:
+    """Per expert, the bin holding the ceil(m_total k / n)-th largest margin."""
+    H = np.ascontiguousarray(H, dtype=np.int64)
+    n, bins = H.shape
+    out = np.empty(n, dtype=np.int64)
+    _check(_load().oracle_qb_quantile_bins(H.ctypes.data, n, bins, m_total, k, out.ctypes.data),
+           "oracle_qb_quantile_bins")
     return out

@@ -557,11 +557,13 @@ int oracle_qb_update(const double* s, const double* b, int64_t m, int64_t n, int
 int oracle_qb_histogram(const double* s, const double* alpha, int64_t m, int64_t n, double lo, double hi, int64_t B,
                         int64_t* H) {
   if (!s || !alpha || !H || m < 0 || n < 1 || B < 1 || !(hi > lo)) return 1;
-  const double width = (hi - lo) / static_cast<double>(B);
   for (int64_t i = 0; i < m; ++i)
     for (int64_t j = 0; j < n; ++j) {
       const double mu = s[i * n + j] - alpha[i];
-      int64_t bin = mu < lo ? 0 : static_cast<int64_t>(std::floor((mu - lo) / width));
+      // bin floor(B (mu - lo) / (hi - lo)): exact on the edges that exact
+      // inputs put there (a margin of 0 -- the cutoff expert's own -- with lo
+      // a multiple of the bin width), where dividing by a rounded width is not
+      int64_t bin = mu < lo ? 0 : static_cast<int64_t>(std::floor(static_cast<double>(B) * (mu - lo) / (hi - lo)));
       bin = std::max<int64_t>(0, std::min(bin, B - 1));
       H[j * B + bin] += 1;
     }
@@ -585,6 +587,55 @@ int oracle_qb_bias_from_histogram(const int64_t* H, int64_t n, int64_t B, double
       if (c >= r) break;
     }
     b_new[j] = -(lo + static_cast<double>(bin) * width);
+  }
+  return 0;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+// The histogram with the decisions taken in fp32, as a GPU computing on fp32
+// router logits takes them: v = s + b rounded to fp32, alpha the (k+1)-th
+// largest v, mu = s - alpha rounded to fp32, t = mu - lo rounded to fp32, and
+// the bin floor(t * inv_w) with inv_w = fp32(B) / fp32(hi - lo), both
+// products rounded to fp32; t < 0 counts in bin 0, a bin >= B in bin B - 1.
+// On data with no margin within an fp32 rounding of a bin edge it counts
+// exactly what oracle_qb_histogram counts (from the same fp32 inputs).
+// s [m, n] fp32, b [n] fp32 or NULL; alpha [m] (fp32 values) is written.
+int oracle_qb_histogram_f32(const float* s, const float* b, int64_t m, int64_t n, int64_t k, float lo, float hi,
+                            int64_t B, float* alpha, int64_t* H) {
+  if (!s || !alpha || !H || m < 1 || n < 2 || k < 1 || k >= n || B < 1 || !(hi > lo)) return 1;
+  const float inv_w = static_cast<float>(B) / (hi - lo);
+  std::vector<float> v(n);
+  for (int64_t i = 0; i < m; ++i) {
+    for (int64_t j = 0; j < n; ++j) v[j] = s[i * n + j] + (b ? b[j] : 0.0f);
+    std::nth_element(v.begin(), v.begin() + k, v.end(), std::greater<float>());
+    alpha[i] = v[k];
+    for (int64_t j = 0; j < n; ++j) {
+      const float mu = s[i * n + j] - alpha[i];
+      const float t = mu - lo;
+      const float fbin = t * inv_w;
+      int64_t bin = t < 0.0f ? 0 : (fbin >= static_cast<float>(B) ? B - 1 : static_cast<int64_t>(fbin));
+      H[j * B + bin] += 1;
+    }
+  }
+  return 0;
+}
+
+// The quantile's bin per expert: bins[j] = the bin of H[j] holding the
+// ceil(m_total k / n)-th largest margin (the integer half of
+// oracle_qb_bias_from_histogram).
+int oracle_qb_quantile_bins(const int64_t* H, int64_t n, int64_t B, int64_t m_total, int64_t k, int64_t* bins) {
+  if (!H || !bins || n < 2 || B < 1 || m_total < 1 || k < 1 || k >= n) return 1;
+  const int64_t r = qb_rank(m_total, n, k);
+  for (int64_t j = 0; j < n; ++j) {
+    int64_t c = 0, bin = B - 1;
+    for (; bin > 0; --bin) {
+      c += H[j * B + bin];
+      if (c >= r) break;
+    }
+    bins[j] = bin;
   }
   return 0;
 }

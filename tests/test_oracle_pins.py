@@ -591,3 +591,45 @@ def test_qb_histograms_add_across_batches():
     assert np.array_equal(H, whole)
     assert np.array_equal(oracle.qb_bias_from_histogram(H, -6, 6, m, k),
                           oracle.qb_bias_from_histogram(whole, -6, 6, m, k))
+
+
+def test_qb_fp32_histogram_matches_fp64_away_from_bin_edges():
+    """The fp32-decision histogram (the GPU's arithmetic) counts what the fp64
+    definition counts, except margins within fp32 rounding of a bin edge, which
+    may move to the neighbouring bin."""
+    m, n, k, lo, hi, B = 400, 12, 3, -8.0, 8.0, 1000
+    for seed in range(4):
+        s = np.random.default_rng(seed).normal(size=(m, n)).astype(np.float32)
+        b = (np.random.default_rng(seed + 50).normal(size=n) * 0.25).astype(np.float32)
+        a32, H32 = oracle.qb_histogram_f32(s, k, lo, hi, B, bias=b)
+        # the cutoff: the (k+1)-th largest of the fp32 sums s + b
+        v32 = s + b
+        assert np.all((v32 > a32[:, None]).sum(1) == k) and np.all((v32 == a32[:, None]).sum(1) >= 1)
+        H64 = oracle.qb_histogram(s.astype(np.float64), a32.astype(np.float64), lo, hi, B)
+        assert np.all(H32.sum(1) == m) and np.all(H64.sum(1) == m)
+        mu = s.astype(np.float64) - a32.astype(np.float64)[:, None]
+        pos = B * (mu - lo) / (hi - lo)
+        near = int((np.abs(pos - np.round(pos)) < 1e-4).sum())
+        assert int(np.abs(H32 - H64).sum()) <= 2 * near
+    # without a bias each token's cutoff expert has a margin of exactly 0, on a
+    # bin edge here; both arithmetics put all m of them in the same bin
+    s = np.random.default_rng(9).normal(size=(m, n)).astype(np.float32)
+    a32, H32 = oracle.qb_histogram_f32(s, k, lo, hi, B)
+    H64 = oracle.qb_histogram(s.astype(np.float64), a32.astype(np.float64), lo, hi, B)
+    zero_bin = B // 2
+    assert H32[:, zero_bin].sum() >= m and H64[:, zero_bin].sum() >= m
+    assert H32[:, zero_bin - 1].sum() == H64[:, zero_bin - 1].sum()
+
+
+def test_qb_quantile_bins_are_the_bias_bins():
+    m, n, k, lo, hi, B = 300, 10, 2, -6.0, 6.0, 600
+    s = np.random.default_rng(13).normal(size=(m, n))
+    a = oracle.qb_cutoffs(s, k)
+    H = oracle.qb_histogram(s, a, lo, hi, B)
+    bins = oracle.qb_quantile_bins(H, m, k)
+    bias = oracle.qb_bias_from_histogram(H, lo, hi, m, k)
+    assert np.allclose(-bias, lo + bins * (hi - lo) / B, rtol=0, atol=1e-12)
+    # at least ceil(m k / n) margins lie in or above the bin, fewer strictly above it
+    r = -(-m * k // n)
+    for j in range(n):
+        assert H[j, bins[j]:].sum() >= r and H[j, bins[j] + 1:].sum() < r
