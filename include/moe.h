@@ -304,6 +304,42 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
                             moe_bf16_t* out,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------- Quantile Balancing --
+ * The per-expert bias update of [P3] section "Systems Optimization, Load
+ * Balancing, and Post-Training Alignment" (QB): biases from the (1 - k/n)-
+ * quantile over tokens of the margins s[t,e] - alpha_t, alpha_t the cutoff of
+ * top-(k+1) routing, recovered from per-expert binned histograms that
+ * data-parallel ranks add up with one integer all-reduce. The page's update
+ * formula is garbled; the reading taken, the dual step of the
+ * balanced-assignment LP the page names, is:
+ *   alpha_t = (k+1)-th largest of s[t,e] + b[e];
+ *   beta_e  = the ceil(m k / n)-th largest margin s[t,e] - alpha_t of expert e
+ *             (m tokens over all ranks, n = E experts);
+ *   b_new[e] = -beta_e, beta_e taken at the lower edge of its histogram bin.
+ * All arithmetic is fp32 with every operation rounded as written:
+ *   v = s + b, mu = s - alpha, t = mu - lo, bin = t < 0 ? 0 : (t * inv_w >= B
+ *   ? B - 1 : trunc(t * inv_w)), inv_w = fp32(B) / fp32(hi - lo).
+ *
+ * moe_router_logits: the router logits s = x W_router (+ bias) [T, E] fp32 in
+ *   the canonical order of moe_route (bit-identical to the logits it selects
+ *   on), for every expert. No scratch. T <= 4194240 (64 x 65535).
+ * moe_qb_histogram: from logits [T, E] and the current biases (NULL: zero),
+ *   writes alpha [T] and ADDS this batch's margin counts into H [E][bins]
+ *   (uint64; zero it before the first batch, then all-reduce it over ranks).
+ *   2 <= E <= 1024, 1 <= k < E, k <= 16, 1 <= bins <= 1536, lo < hi finite.
+ * moe_qb_bias: from the (summed) H and m_total, the number of tokens each row
+ *   of H counts, writes bin_out [E] (the quantile's bin: the highest bin whose
+ *   count from the top reaches ceil(m_total k / E), or 0) and bias_out [E] =
+ *   -(lo + bin * w), w = fp32(hi - lo) / fp32(bins), in fp32.
+ * All three only enqueue kernels on `stream`.
+ */
+moe_status_t moe_router_logits(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                               int T, int d, int E, float* logits, cudaStream_t stream);
+moe_status_t moe_qb_histogram(const float* logits, const float* bias, int T, int E, int k,
+                              float lo, float hi, int bins, float* alpha, uint64_t* H, cudaStream_t stream);
+moe_status_t moe_qb_bias(const uint64_t* H, int E, int bins, float lo, float hi, int64_t m_total, int k,
+                         int32_t* bin_out, float* bias_out, cudaStream_t stream);
+
 /* ------------------------------------------------------------ diagnostics --
  * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
  * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise

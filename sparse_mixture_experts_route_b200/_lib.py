@@ -45,6 +45,9 @@ EXPORTS = {
     "moe_mx_pack_experts": ([P, P, I, I, I, P, P, P, P, P], I),
     "moe_forward_mx_workspace_size": ([I, I, I, I, I], Z),
     "moe_forward_mx": ([P, P, P, P, P, P, P, I, I, I, I, I, P, P, Z, P], I),
+    "moe_router_logits": ([P, P, P, I, I, I, P, P], I),
+    "moe_qb_histogram": ([P, P, I, I, I, ctypes.c_float, ctypes.c_float, I, P, P, P], I),
+    "moe_qb_bias": ([P, I, I, ctypes.c_float, ctypes.c_float, ctypes.c_int64, I, P, P, P], I),
     "moe_get_device_error": ([ctypes.POINTER(ctypes.c_uint32), I], I),
     "moe_selftest_wait_timeout": ([I, P], I),
 }
@@ -278,6 +281,50 @@ def moe_forward_mx(x, W_router, router_bias, experts: MxExperts, k: int, out=Non
                                f, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "moe_forward_mx")
     return out
+
+
+def moe_router_logits(x, W_router, router_bias=None, stream=None, out=None):
+    """Router logits [T,E] fp32 for every expert, in the canonical order."""
+    T, d = x.shape
+    E = W_router.shape[1]
+    _need(x, "x", torch.bfloat16, (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    if out is None:
+        out = torch.empty(T, E, dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, (T, E))
+    _check(_lib.moe_router_logits(_ptr(x), _ptr(W_router), _ptr(router_bias), T, d, E, _ptr(out), _stream(stream)),
+           "moe_router_logits")
+    return out
+
+
+def moe_qb_histogram(logits, bias, k: int, lo: float, hi: float, bins: int, H=None, stream=None):
+    """Quantile Balancing, first half: cutoffs alpha [T] and the margin
+    histogram H [E, bins] (int64 tensor; this batch's counts are added into H).
+    All-reduce H over data-parallel ranks before moe_qb_bias."""
+    T, E = logits.shape
+    _need(logits, "logits", torch.float32, (T, E))
+    if bias is not None:
+        _need(bias, "bias", torch.float32, (E,))
+    if H is None:
+        H = torch.zeros(E, bins, dtype=torch.int64, device=logits.device)
+    _need(H, "H", torch.int64, (E, bins))
+    alpha = torch.empty(T, dtype=torch.float32, device=logits.device)
+    _check(_lib.moe_qb_histogram(_ptr(logits), _ptr(bias), T, E, k, float(lo), float(hi), bins, _ptr(alpha), _ptr(H),
+                                 _stream(stream)), "moe_qb_histogram")
+    return alpha, H
+
+
+def moe_qb_bias(H, lo: float, hi: float, m_total: int, k: int, stream=None):
+    """Quantile Balancing, second half: (bins [E] int32, new biases [E] fp32)."""
+    E, bins = H.shape
+    _need(H, "H", torch.int64, (E, bins))
+    bin_out = torch.empty(E, dtype=torch.int32, device=H.device)
+    bias_out = torch.empty(E, dtype=torch.float32, device=H.device)
+    _check(_lib.moe_qb_bias(_ptr(H), E, bins, float(lo), float(hi), int(m_total), k, _ptr(bin_out), _ptr(bias_out),
+                            _stream(stream)), "moe_qb_bias")
+    return bin_out, bias_out
 
 
 def moe_forward(x, W_router, router_bias, W_gate_up, W_down, k: int, out=None, workspace=None, stream=None):

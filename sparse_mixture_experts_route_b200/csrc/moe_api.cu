@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -20,6 +21,7 @@
 #include "mx_quant.cuh"
 #include "permute.cuh"
 #include "ptx.cuh"
+#include "qb.cuh"
 #include "router.cuh"
 #include "router_stream.cuh"
 #include "router_tc.cuh"
@@ -1071,6 +1073,60 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
       mA1, mB1, p1);
   st = launch_unpermute(y, inv_perm, w, T, d, k, out, stream);
   if (st != MOE_OK) return st;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_router_logits(const moe_bf16_t* x, const float* W_router, const float* router_bias, int T, int d,
+                               int E, float* logits, cudaStream_t stream) {
+  if (!x || !W_router || !logits) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || d < 64 || d % 64 || d > 32768 || E < 1 || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || ceil_div64(T, 64) > 65535) return MOE_ERR_UNSUPPORTED;
+  // the whole-chunk-walk variant of the router's logits kernel: final logits
+  // (+ bias) in the canonical order, no scratch
+  const dim3 grid(ceil_div(E, 64), static_cast<unsigned>(ceil_div64(T, 64)), 1);
+  router_logits_kernel<64, 64, 4, 4, false><<<grid, 256, 0, stream>>>(x, W_router, router_bias, T, d, E, logits);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_qb_histogram(const float* logits, const float* bias, int T, int E, int k, float lo, float hi,
+                              int bins, float* alpha, uint64_t* H, cudaStream_t stream) {
+  if (!logits || !alpha || !H) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || E < 2 || k < 1 || k >= E || bins < 1 || !(hi > lo) || !std::isfinite(lo) || !std::isfinite(hi))
+    return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK || bins > kQbMaxBins) return MOE_ERR_UNSUPPORTED;
+  const float inv_w = static_cast<float>(bins) / (hi - lo);
+  if (!std::isfinite(inv_w)) return MOE_ERR_INVALID_ARG;
+  const unsigned cut_blocks = static_cast<unsigned>(ceil_div64(T, 8));
+  if (E <= 256)
+    qb_cutoffs_kernel<8><<<cut_blocks, 256, 0, stream>>>(logits, bias, T, E, k, alpha);
+  else
+    qb_cutoffs_kernel<32><<<cut_blocks, 256, 0, stream>>>(logits, bias, T, E, k, alpha);
+  // about four waves of CTAs on a 148-SM part, each slice at least 32 tokens
+  const int gx = ceil_div(E, kQbExpertsPerCta);
+  int64_t slices = (4 * 148 + gx - 1) / gx;
+  slices = slices < ceil_div64(T, 32) ? slices : ceil_div64(T, 32);
+  if (slices < 1) slices = 1;
+  const int64_t per = ceil_div64(T, slices);
+  const int64_t gy = ceil_div64(T, per);
+  if (gy > 65535) return MOE_ERR_UNSUPPORTED;
+  qb_histogram_kernel<<<dim3(gx, static_cast<unsigned>(gy)), 256,
+                        static_cast<size_t>(kQbExpertsPerCta) * bins * sizeof(uint32_t), stream>>>(
+      logits, alpha, T, E, lo, inv_w, bins, static_cast<int>(per), reinterpret_cast<unsigned long long*>(H));
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_qb_bias(const uint64_t* H, int E, int bins, float lo, float hi, int64_t m_total, int k,
+                         int32_t* bin_out, float* bias_out, cudaStream_t stream) {
+  if (!H || !bin_out || !bias_out) return MOE_ERR_INVALID_ARG;
+  if (E < 2 || k < 1 || k >= E || bins < 1 || m_total < 1 || m_total > (int64_t(1) << 56) || !(hi > lo) ||
+      !std::isfinite(lo) || !std::isfinite(hi))
+    return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK || bins > kQbMaxBins) return MOE_ERR_UNSUPPORTED;
+  int64_t r = (m_total * k + E - 1) / E;
+  r = r < 1 ? 1 : (r > m_total ? m_total : r);
+  const float w = (hi - lo) / static_cast<float>(bins);
+  qb_bias_kernel<<<static_cast<unsigned>(ceil_div(E, 8)), 256, 0, stream>>>(
+      reinterpret_cast<const unsigned long long*>(H), E, bins, lo, w, static_cast<long long>(r), bin_out, bias_out);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -233,3 +233,30 @@ def test_mx_expert_sizes_and_checks(lib):
     assert lib.moe_forward_mx(*args[:11], 192, *args[12:]) == 1                   # f % 128
     assert lib.moe_forward_mx(*args[:14], mw - 256, None) == 3                    # workspace
     assert lib.moe_forward_mx(*args[:13], ctypes.c_void_p(FAKE + 64), mw, None) == 3
+
+
+def test_qb_and_router_logits_checks(lib):
+    """moe_router_logits / moe_qb_histogram / moe_qb_bias refuse bad arguments
+    before any CUDA call."""
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.moe_router_logits.argtypes = [P, P, P, I, I, I, P, P]
+    lib.moe_qb_histogram.argtypes = [P, P, I, I, I, F, F, I, P, P, P]
+    lib.moe_qb_bias.argtypes = [P, I, I, F, F, ctypes.c_int64, I, P, P, P]
+    p = ctypes.c_void_p(FAKE)
+    rl, qh, qbias = lib.moe_router_logits, lib.moe_qb_histogram, lib.moe_qb_bias
+    assert rl(None, p, None, 64, 128, 8, p, None) == 1
+    assert rl(p, p, None, 64, 100, 8, p, None) == 1                   # d % 64
+    assert rl(ctypes.c_void_p(FAKE + 2), p, None, 64, 128, 8, p, None) == 1
+    assert rl(p, p, None, 64, 128, 2048, p, None) == 2                # E > 1024
+    assert rl(p, p, None, 64 * 65535 + 1, 128, 8, p, None) == 2       # grid rows
+    assert qh(None, None, 64, 8, 2, -4.0, 4.0, 1000, p, p, None) == 1
+    assert qh(p, None, 64, 8, 8, -4.0, 4.0, 1000, p, p, None) == 1    # k >= E
+    assert qh(p, None, 64, 8, 2, 4.0, -4.0, 1000, p, p, None) == 1    # hi <= lo
+    assert qh(p, None, 64, 8, 2, -4.0, float("inf"), 1000, p, p, None) == 1
+    assert qh(p, None, 64, 8, 2, -4.0, 4.0, 0, p, p, None) == 1       # no bins
+    assert qh(p, None, 64, 8, 2, -4.0, 4.0, 2000, p, p, None) == 2    # > 1536 bins
+    assert qh(p, None, 64, 64, 17, -4.0, 4.0, 1000, p, p, None) == 2  # k > 16
+    assert qbias(None, 8, 1000, -4.0, 4.0, 64, 2, p, p, None) == 1
+    assert qbias(p, 8, 1000, -4.0, 4.0, 0, 2, p, p, None) == 1        # no tokens
+    assert qbias(p, 8, 1000, -4.0, 4.0, 64, 8, p, p, None) == 1       # k >= E
+    assert qbias(p, 8, 1000, -4.0, 4.0, 64, 2, p, None, None) == 1
