@@ -187,8 +187,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const int ra0 = ti.nb * (kMode == 0 ? 128 : 256);
         const int ra1 = ra0 + p.a1_row;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
-        const uint8_t* sfa0 = p.sfw + ((static_cast<int64_t>(ti.e) * (p.w_rows / 128) + ra0 / 128) * KC) * kMxAtomBytes;
-        const uint8_t* sfa1 = p.sfw + ((static_cast<int64_t>(ti.e) * (p.w_rows / 128) + ra1 / 128) * KC) * kMxAtomBytes;
+        const int64_t wtiles = static_cast<int64_t>(ti.e) * (p.w_rows / 128);
+        const uint8_t* sfa0 = p.sfw + (wtiles + ra0 / 128) * KC * kMxAtomBytes;
+        const uint8_t* sfa1 = p.sfw + (wtiles + ra1 / 128) * KC * kMxAtomBytes;
         const uint8_t* sfb = p.sft + static_cast<int64_t>(ti.tile) * KC * kMxAtomBytes;
         for (int kc = 0; kc < KC; ++kc) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
