@@ -902,11 +902,11 @@ bool mx_weight_map(CUtensorMap* map, const uint8_t* wq, int E, int rows, int K) 
   return encode_map_typed(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, wq, 3, dims, strides, box);
 }
 
-// E4M3 token rows [rows][K]: boxes of 128 K x kMxTileRows rows.
-bool mx_token_map(CUtensorMap* map, const uint8_t* q, int rows, int K) {
+// E4M3 token rows [rows][K]: boxes of 128 K x box_rows rows.
+bool mx_token_map(CUtensorMap* map, const uint8_t* q, int rows, int K, int box_rows) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kMxTileRows)};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
   return encode_map_typed(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, 2, dims, strides, box);
 }
 
@@ -1016,9 +1016,10 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
   int32_t* pre0 = reinterpret_cast<int32_t*>(ws + L.pre0);
   int32_t* pre1 = reinterpret_cast<int32_t*>(ws + L.pre1);
   const int Tk = T * k;
-  CUtensorMap mA0, mB0, mA1, mB1;
-  if (!mx_weight_map(&mA0, wq_gate_up, E, 2 * f, d) || !mx_token_map(&mB0, xq, Tk, d) ||
-      !mx_weight_map(&mA1, wq_down, E, d, f) || !mx_token_map(&mB1, hq, Tk, f))
+  CUtensorMap mA0, mB0, mBs0, mA1, mB1, mBs1;
+  if (!mx_weight_map(&mA0, wq_gate_up, E, 2 * f, d) || !mx_token_map(&mB0, xq, Tk, d, kMxTileRows) ||
+      !mx_token_map(&mBs0, xq, Tk, d, kMxSmallRows) || !mx_weight_map(&mA1, wq_down, E, d, f) ||
+      !mx_token_map(&mB1, hq, Tk, f, kMxTileRows) || !mx_token_map(&mBs1, hq, Tk, f, kMxSmallRows))
     return MOE_ERR_INVALID_ARG;
 
   // route, then the dispatch tables (counts, offsets, permutation, token tiles
@@ -1068,9 +1069,9 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
   p1.out = y;
   const int64_t g0 = L.tiles_max * p0.n_feat_tiles, g1 = L.tiles_max * p1.n_feat_tiles;
   mx_grouped_gemm_kernel<0><<<static_cast<unsigned>(g0 < sms ? g0 : sms), kMxThreads, kMxSmemBytes, stream>>>(
-      mA0, mB0, p0);
+      mA0, mB0, mBs0, p0);
   mx_grouped_gemm_kernel<1><<<static_cast<unsigned>(g1 < sms ? g1 : sms), kMxThreads, kMxSmemBytes, stream>>>(
-      mA1, mB1, p1);
+      mA1, mB1, mBs1, p1);
   st = launch_unpermute(y, inv_perm, w, T, d, k, out, stream);
   if (st != MOE_OK) return st;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -20,7 +20,8 @@
 //   - a stage covers 128 K elements: per A operand a 16U4 TMA box that reads
 //     64 bytes of packed codes per weight row and leaves them in shared memory
 //     with one byte per element (the tensor core's layout for 4-bit operands
-//     next to 8-bit ones); the token box is 128 E4M3 bytes per row;
+//     next to 8-bit ones); the token box is 128 E4M3 bytes per row, 112 rows,
+//     or 16 rows for tiles of at most 16 (decode steps);
 //   - each stage also brings three 512-byte scale atoms (both A operands and
 //     the token tile) by bulk copy; the MMA issuer moves them into TMEM with
 //     tcgen05.cp before the stage's four MMAs (K = 32 each), whose scale IDs
@@ -50,6 +51,8 @@ constexpr int kMxABytes = 128 * kMxBK;            // 16 KB in shared memory (one
 constexpr int kMxATx = 128 * kMxBK / 2;           // 8 KB read from memory (packed)
 constexpr int kMxBBytes = 128 * kMxBK;            // room for 128 token rows of 128 bytes
 constexpr int kMxBTx = kMxTileRows * kMxBK;       // 112 rows are loaded
+constexpr int kMxSmallRows = 16;                  // token box of tiles with <= 16 rows (decode)
+constexpr int kMxBTxSmall = kMxSmallRows * kMxBK;
 constexpr int kMxSfOff = 2 * kMxABytes + kMxBBytes;  // three atoms after the operands
 constexpr int kMxStageBytes = kMxSfOff + 3 * kMxAtomBytes + 512;  // 50 KB (1024-aligned)
 constexpr int kMxSlotCols = 2 * kMxTileRows;      // 224: two accumulators of one tile
@@ -123,7 +126,7 @@ __device__ __forceinline__ void mx_ld_chunk(uint32_t t0, uint32_t t1, int c0, ui
 template <int kMode>
 __global__ void __launch_bounds__(kMxThreads, 1)
     mx_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const MxGemmParams p) {
+                           const __grid_constant__ CUtensorMap tmBs, const MxGemmParams p) {
   constexpr int S = kMxStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -160,6 +163,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBs);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kMxTmemCols);
@@ -191,6 +195,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const uint8_t* sfa0 = p.sfw + (wtiles + ra0 / 128) * KC * kMxAtomBytes;
         const uint8_t* sfa1 = p.sfw + (wtiles + ra1 / 128) * KC * kMxAtomBytes;
         const uint8_t* sfb = p.sft + static_cast<int64_t>(ti.tile) * KC * kMxAtomBytes;
+        // a tile of at most 16 rows loads a 16-row token box (its MMAs have N = 16)
+        const bool small = ti.nrows <= kMxSmallRows;
+        const CUtensorMap* mb = small ? &tmBs : &tmB;
+        const uint32_t tx = 2 * kMxATx + (small ? kMxBTxSmall : kMxBTx) + 3 * kMxAtomBytes;
         for (int kc = 0; kc < KC; ++kc) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
@@ -199,11 +207,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             break;
           }
           uint8_t* st = smem + s * kMxStageBytes;
-          mbar_arrive_expect_tx(&full_bar[s], 2 * kMxATx + kMxBTx + 3 * kMxAtomBytes);
+          mbar_arrive_expect_tx(&full_bar[s], tx);
           const int k0 = kc * kMxBK;
           tma_load_3d(st, &tmA, &full_bar[s], k0, ra0, ti.e, pol_w);
           tma_load_3d(st + kMxABytes, &tmA, &full_bar[s], k0, ra1, ti.e, pol_w);
-          tma_load_2d(st + 2 * kMxABytes, &tmB, &full_bar[s], k0, ti.row0, pol_x);
+          tma_load_2d(st + 2 * kMxABytes, mb, &full_bar[s], k0, ti.row0, pol_x);
           uint8_t* sf = st + kMxSfOff;
           bulk_load(sf, sfa0 + static_cast<int64_t>(kc) * kMxAtomBytes, kMxAtomBytes, &full_bar[s], pol_w);
           bulk_load(sf + kMxAtomBytes, sfa1 + static_cast<int64_t>(kc) * kMxAtomBytes, kMxAtomBytes, &full_bar[s],
