@@ -49,6 +49,9 @@ MUTATIONS = {
     "mx_ffn_h_not_requantised": ("if (!st) st = oracle_mxfp8_dequantize(hc.data(), hs.data(), 1, f, hrow.data());",
                                  "if (!st) st = 0;"),
     "mx_ffn_gate_up_swapped": ("const double g = gu[j], u = gu[f + j];", "const double u = gu[j], g = gu[f + j];"),
+    "mxfp8_nan_code_allowed": ("for (int c = 1; c < 127; ++c) {", "for (int c = 1; c < 128; ++c) {"),
+    "mxfp8_dequant_scale_off_by_one": ("std::ldexp(e4m3_mag(c & 0x7f), static_cast<int>(q) - 127)",
+                                       "std::ldexp(e4m3_mag(c & 0x7f), static_cast<int>(q) - 126)"),
     "qb_cutoff_is_kth_not_k_plus_first": ("std::greater<double>());\n    alpha[i] = v[k];",
                                           "std::greater<double>());\n    alpha[i] = v[k - 1];"),
     "qb_quantile_rank_floor": ("int64_t r = (m * k + n - 1) / n;", "int64_t r = (m * k) / n;"),
