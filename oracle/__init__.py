@@ -5,8 +5,9 @@ and by ``bench.py``'s CPU-baseline leg. The product path (the CUDA library and
 its Python binding) never imports it, and it imports nothing from the product.
 
 The arithmetic lives in ``moe_oracle.cpp`` (plain C++, fp64 except for the fp32
-router whose summation order is stated there). This module only builds that
-file and marshals numpy / torch CPU arrays into it.
+router whose summation order is stated there, and the Quantile Balancing
+histogram's fp32-decision variant, pinned against its fp64 definition). This
+module only builds that file and marshals numpy / torch CPU arrays into it.
 
 Every function cites its passage in ``moe_oracle.cpp``. All oracle functions
 here are pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``
