@@ -915,9 +915,15 @@ bool mx_shape_ok(int d, int f) { return d % 256 == 0 && f % 128 == 0 && f >= 128
 inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 struct MxLayout {
-  size_t route, idx, w, offsets, perm_token, inv_perm, xq, sfx, hq, sfh, y, perm_ws, pre0, pre1, total;
+  size_t route, idx, w, offsets, perm_token, inv_perm, xq, sfx, hq, sfh, y, perm_ws, pre0, pre1, part, tickets, total;
   int64_t tiles_max;
+  bool split0, split1;  // stream-K for the gate/up and the down GEMM
 };
+
+// Stream-K for an MX GEMM whose tile count (an upper bound) fills at most four
+// waves of one CTA per SM on a 148-SM part, as for the bf16 GEMMs.
+constexpr int kMxSplitCtas = 148;
+constexpr int64_t kMxSplitMaxTiles = 4 * kMxSplitCtas;
 
 MxLayout mx_layout(int T, int d, int E, int k, int f) {
   MxLayout L;
@@ -943,6 +949,11 @@ MxLayout mx_layout(int T, int d, int E, int k, int f) {
   L.perm_ws = take(permute_ws(T, E, k));
   L.pre0 = take((static_cast<size_t>(E) + 1) * sizeof(int32_t));
   L.pre1 = take((static_cast<size_t>(E) + 1) * sizeof(int32_t));
+  L.split0 = L.tiles_max * (f / 128) <= kMxSplitMaxTiles;
+  L.split1 = L.tiles_max * (d / 256) <= kMxSplitMaxTiles;
+  const bool split = L.split0 || L.split1;
+  L.part = take(split ? static_cast<size_t>(2 * kMxSplitCtas) * kMxPartFloats * sizeof(float) : 0);
+  L.tickets = take(split ? static_cast<size_t>(kMxSplitMaxTiles) * 4 * sizeof(unsigned int) : 0);
   L.total = at;
   return L;
 }
@@ -1024,7 +1035,11 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
 
   // route, then the dispatch tables (counts, offsets, permutation, token tiles
   // of kMxTileRows rows); no bf16 row copy: the rows are copied as MXFP8 below
-  const RouteDispatch disp = {offsets, perm_token, inv_perm, pre0, pre1, nullptr, 0};
+  // stream-K tickets start at zero: the dispatch step clears them
+  unsigned int* tickets = reinterpret_cast<unsigned int*>(ws + L.tickets);
+  const int ticket_words =
+      static_cast<int>((L.split0 || L.split1) ? static_cast<int64_t>(kMxSplitMaxTiles) * 4 : 0);
+  const RouteDispatch disp = {offsets, perm_token, inv_perm, pre0, pre1, tickets, ticket_words};
   bool dispatched = false;
   st = launch_route(x, W_router, router_bias, T, d, E, k, idx, w, ws + L.route, stream, T == 1 ? &disp : nullptr,
                     &dispatched);
@@ -1032,11 +1047,12 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
   if (!dispatched) {
     if (Tk <= kSmallDispatchPairs) {
       dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, kMxTileRows, kMxTileRows, offsets, perm_token,
-                                                    inv_perm, pre0, pre1, nullptr, 0);
+                                                    inv_perm, pre0, pre1, tickets, ticket_words);
     } else {
       st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, nullptr, ws + L.perm_ws, stream);
       if (st != MOE_OK) return st;
-      gemm_schedule_kernel<<<1, 1024, 0, stream>>>(offsets, E, kMxTileRows, kMxTileRows, pre0, pre1, nullptr, 0);
+      gemm_schedule_kernel<<<1, 1024, 0, stream>>>(offsets, E, kMxTileRows, kMxTileRows, pre0, pre1, tickets,
+                                                   ticket_words);
     }
   }
   mx_quantize_dispatch_kernel<<<static_cast<unsigned>(T), 256, 0, stream>>>(
@@ -1056,6 +1072,9 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
   p0.hq = hq;
   p0.hs = sfh;
   p0.out = nullptr;
+  p0.stream_k = L.split0 ? 1 : 0;
+  p0.part = reinterpret_cast<float*>(ws + L.part);
+  p0.tickets = tickets;
   MxGemmParams p1 = p0;
   p1.K = f;
   p1.n_feat = d;
@@ -1067,7 +1086,13 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
   p1.hq = nullptr;
   p1.hs = nullptr;
   p1.out = y;
-  const int64_t g0 = L.tiles_max * p0.n_feat_tiles, g1 = L.tiles_max * p1.n_feat_tiles;
+  p1.stream_k = L.split1 ? 1 : 0;
+  // stream-K launches one CTA per SM (at most kMxSplitCtas, the partial slots'
+  // count); whole-tile scheduling launches min(tiles, SMs) persistent CTAs
+  const int split_grid = sms < kMxSplitCtas ? sms : kMxSplitCtas;
+  int64_t g0 = L.tiles_max * p0.n_feat_tiles, g1 = L.tiles_max * p1.n_feat_tiles;
+  if (L.split0) g0 = split_grid;
+  if (L.split1) g1 = split_grid;
   mx_grouped_gemm_kernel<0><<<static_cast<unsigned>(g0 < sms ? g0 : sms), kMxThreads, kMxSmemBytes, stream>>>(
       mA0, mB0, mBs0, p0);
   mx_grouped_gemm_kernel<1><<<static_cast<unsigned>(g1 < sms ? g1 : sms), kMxThreads, kMxSmemBytes, stream>>>(

@@ -79,10 +79,24 @@ struct MxGemmParams {
   uint8_t* hq;         // mode 0: h codes [Tk][f]
   uint8_t* hs;         // mode 0: h scale atoms [tiles][f / 128][512]
   uint16_t* out;       // mode 1: y [Tk][d] bf16
+  // Stream-K, as in the bf16 kernel: with few output tiles the (tile, K
+  // chunk) units are split evenly over the CTAs; a CTA's first and last items
+  // may cover part of a tile's K range and leave fp32 partials in part[slot]
+  // (slot 2c for CTA c's first item, 2c + 1 for its last); per (tile, epilogue
+  // warp) the last contributor (a ticket) adds them in CTA order, which is K
+  // order, and finishes the tile. tickets[] start at zero and are put back.
+  int stream_k;
+  float* part;            // [2 * gridDim.x][2][kMxTileRows][128] fp32
+  unsigned int* tickets;  // [tiles][4]
 };
+
+constexpr int kMxPartFloats = 2 * kMxTileRows * 128;
 
 struct MxTile {
   int e, nb, row0, nrows, nblocks, tile;  // tile: global token-tile index (prefix[e] + block)
+  int t, kb0, kb1;                        // output tile index, K-chunk range [kb0, kb1) of this item
+  bool partial;                           // the item covers only part of the tile's K range
+  int slot;                               // partial slot of this CTA's item
 };
 
 __device__ __forceinline__ bool mx_tile(const MxGemmParams& p, const int32_t* pre, const int32_t* off, int t,
@@ -108,6 +122,65 @@ __device__ __forceinline__ bool mx_tile(const MxGemmParams& p, const int32_t* pr
   ti.nrows = min(kMxTileRows, off[e + 1] - ti.row0);
   ti.tile = pre[e] + tb;
   return true;
+}
+
+__device__ __forceinline__ int mx_stream_k_per(int ntiles, int KC) {
+  return (ntiles * KC + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+}
+
+// The it-th work item of this CTA: whole tiles blockIdx.x + it * gridDim.x, or
+// with stream-K the tiles its unit range touches, with their K chunks inside it.
+__device__ __forceinline__ bool mx_work_item(const MxGemmParams& p, const int32_t* pre, const int32_t* off, int it,
+                                             MxTile& ti) {
+  const int KC = p.K / kMxBK;
+  if (!p.stream_k) {
+    const int t = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+    if (!mx_tile(p, pre, off, t, ti)) return false;
+    ti.t = t;
+    ti.kb0 = 0;
+    ti.kb1 = KC;
+    ti.partial = false;
+    ti.slot = -1;
+    return true;
+  }
+  const int ntiles = pre[p.E] * p.n_feat_tiles;
+  const int per = mx_stream_k_per(ntiles, KC);
+  const int u0 = static_cast<int>(blockIdx.x) * per;
+  const int u1 = min(ntiles * KC, u0 + per);
+  const int t = u0 / KC + it;
+  if (u0 >= u1 || t * KC >= u1) return false;
+  mx_tile(p, pre, off, t, ti);
+  ti.t = t;
+  ti.kb0 = max(u0, t * KC) - t * KC;
+  ti.kb1 = min(u1, (t + 1) * KC) - t * KC;
+  ti.partial = ti.kb0 > 0 || ti.kb1 < KC;
+  ti.slot = 2 * static_cast<int>(blockIdx.x) + (it == 0 ? 0 : 1);
+  return true;
+}
+
+// Finishes token row i (0-based in the tile) from this lane's two fp32 sums:
+// mode 0 h = SiLU(g) * u, quantised to MXFP8 over the warp's 32 features (one
+// block), codes to hq and the scale into the tile's atom; mode 1 the two bf16
+// outputs. Warp-uniform: every lane of the warp calls it for the same i.
+template <int kMode>
+__device__ __forceinline__ void mx_finish_row(const MxGemmParams& p, const MxTile& ti, int q, int lane, int i, float g,
+                                              float u) {
+  if (kMode == 0) {
+    const int feat = ti.nb * 128 + q * 32 + lane;
+    const float h = silu_f32(g) * u;
+    const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu);
+    const int sc = mx_scale_exponent(__uint_as_float(amax), 8);
+    const uint32_t code = mx_e4m3_code(h, mx_inverse_scale(sc));
+    p.hq[static_cast<int64_t>(ti.row0 + i) * p.n_feat + feat] = static_cast<uint8_t>(code);
+    if (lane == 0)
+      p.hs[(static_cast<int64_t>(ti.tile) * (p.n_feat / 128) + ti.nb) * kMxAtomBytes + mx_atom_offset(i, q)] =
+          static_cast<uint8_t>(sc + 127);
+  } else {
+    const int fa = ti.nb * 256 + q * 32 + lane;
+    uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
+    orow[fa] = bf16_bits(g);
+    orow[fa + 128] = bf16_bits(u);
+  }
 }
 
 // Columns c0 .. c0 + 31 of both accumulators of a tile (only c0 .. c0 + 15 for
@@ -174,7 +247,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const int KC = p.K / kMxBK;
-  const int first = static_cast<int>(blockIdx.x), step = static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -187,7 +259,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       int issued = 0;
       bool ok = true;
       MxTile ti;
-      for (int t = first; ok && mx_tile(p, s_pre, s_off, t, ti); t += step) {
+      for (int it = 0; ok && mx_work_item(p, s_pre, s_off, it, ti); ++it) {
         const int ra0 = ti.nb * (kMode == 0 ? 128 : 256);
         const int ra1 = ra0 + p.a1_row;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
@@ -199,7 +271,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const bool small = ti.nrows <= kMxSmallRows;
         const CUtensorMap* mb = small ? &tmBs : &tmB;
         const uint32_t tx = 2 * kMxATx + (small ? kMxBTxSmall : kMxBTx) + 3 * kMxAtomBytes;
-        for (int kc = 0; kc < KC; ++kc) {
+        for (int kc = ti.kb0; kc < ti.kb1; ++kc) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
             *abort_flag = 1;
@@ -244,7 +316,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       bool any = false;
       const uint32_t t_sfa0 = tmem_base + kMxSfCol, t_sfa1 = t_sfa0 + 8u, t_sfb = t_sfa0 + 16u;
       MxTile ti;
-      for (int t = first; ok && mx_tile(p, s_pre, s_off, t, ti); t += step) {
+      for (int it = 0; ok && mx_work_item(p, s_pre, s_off, it, ti); ++it) {
         const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
         const int sl = next_slot;
         next_slot ^= 1;
@@ -257,7 +329,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         tc_fence_after_sync();
         const uint32_t d0 = tmem_base + static_cast<uint32_t>(sl * kMxSlotCols);
         const uint32_t d1 = d0 + static_cast<uint32_t>(kMxTileRows);
-        for (int kc = 0; kc < KC; ++kc) {
+        for (int kc = ti.kb0; kc < ti.kb1; ++kc) {
           if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
             record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
             *abort_flag = 1;
@@ -279,7 +351,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             const uint64_t adesc0 = umma_smem_desc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t adesc1 = umma_smem_desc_sw128(a_addr + kMxABytes + kk * 32, 16, 1024);
             const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-            const uint32_t accum = (kc > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t accum = (kc > ti.kb0 || kk > 0) ? 1u : 0u;
             tc_mma_mx(d0, adesc0, bdesc, idesc, t_sfa0 | id, t_sfb | id, accum);
             tc_mma_mx(d1, adesc1, bdesc, idesc, t_sfa1 | id, t_sfb | id, accum);
           }
@@ -306,7 +378,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     uint32_t uses[2] = {0u, 0u};
     int next_slot = 0;
     MxTile ti;
-    for (int t = first; mx_tile(p, s_pre, s_off, t, ti); t += step) {
+    for (int it = 0; mx_work_item(p, s_pre, s_off, it, ti); ++it) {
       const int sl = next_slot;
       next_slot ^= 1;
       if (!mbar_wait_bounded(&acc_full_bar[sl], uses[sl] & 1u, kWaitLimitNs, abort_flag)) {
@@ -317,41 +389,61 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       tc_fence_after_sync();
       const uint32_t t0 = tmem_base + lane_base + static_cast<uint32_t>(sl * kMxSlotCols);
       const uint32_t t1 = t0 + static_cast<uint32_t>(kMxTileRows);
-      if (kMode == 0) {
-        const int feat = ti.nb * 128 + q * 32 + lane;  // < f: f is a multiple of 128
-        uint8_t* hs_atom = p.hs + (static_cast<int64_t>(ti.tile) * (p.n_feat / 128) + ti.nb) * kMxAtomBytes;
+      if (ti.partial) {
+        // stream-K partial item: fp32 accumulators to part[slot]; the TMEM
+        // slot is free as soon as they are read
+        const int fl = q * 32 + lane;
+        float* mine = p.part + static_cast<int64_t>(ti.slot) * kMxPartFloats;
         for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
           uint32_t g[32], u[32];
           mx_ld_chunk(t0, t1, c0, g, u);
-          const int nv = min(32, ti.nrows - c0);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i < nv) {  // warp-uniform
-              const float h = silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-              const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu);
-              const int sc = mx_scale_exponent(__uint_as_float(amax), 8);
-              const uint32_t code = mx_e4m3_code(h, mx_inverse_scale(sc));
-              p.hq[static_cast<int64_t>(ti.row0 + c0 + i) * p.n_feat + feat] = static_cast<uint8_t>(code);
-              if (lane == 0) hs_atom[mx_atom_offset(c0 + i, q)] = static_cast<uint8_t>(sc + 127);
-            }
-          }
-        }
-      } else {
-        const int fa = ti.nb * 256 + q * 32 + lane;  // d is a multiple of 256
-        const int fb = fa + 128;
-        for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
-          uint32_t g[32], u[32];
-          mx_ld_chunk(t0, t1, c0, g, u);
-          uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + c0) * p.n_feat;
           const int nv = min(32, ti.nrows - c0);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             if (i < nv) {
-              orow[static_cast<int64_t>(i) * p.n_feat + fa] = bf16_bits(__uint_as_float(g[i]));
-              orow[static_cast<int64_t>(i) * p.n_feat + fb] = bf16_bits(__uint_as_float(u[i]));
+              __stcg(mine + (c0 + i) * 128 + fl, __uint_as_float(g[i]));
+              __stcg(mine + (kMxTileRows + c0 + i) * 128 + fl, __uint_as_float(u[i]));
             }
           }
         }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty_bar[sl]);
+        ++uses[sl];
+        // contributors of tile t are CTAs c_first..c_last; per (tile, warp) the
+        // last to finish adds their partials in CTA order (K order)
+        const int per = mx_stream_k_per(s_pre[p.E] * p.n_feat_tiles, KC);
+        const int c_first = (ti.t * KC) / per, c_last = ((ti.t + 1) * KC - 1) / per;
+        __threadfence();
+        __syncwarp();
+        unsigned int tk = 0u;
+        if (lane == 0) tk = atomicAdd(&p.tickets[ti.t * 4 + q], 1u);
+        tk = __shfl_sync(0xffffffffu, tk, 0);
+        if (tk == static_cast<unsigned int>(c_last - c_first)) {
+          __threadfence();
+          for (int i = 0; i < ti.nrows; ++i) {
+            float gs = 0.0f, us = 0.0f;
+            for (int c = c_first; c <= c_last; ++c) {
+              const int slot = 2 * c + ((ti.t == (c * per) / KC) ? 0 : 1);
+              const float* src = p.part + static_cast<int64_t>(slot) * kMxPartFloats;
+              const float gv = __ldcg(src + i * 128 + fl);
+              const float uv = __ldcg(src + (kMxTileRows + i) * 128 + fl);
+              gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
+              us = (c == c_first) ? uv : __fadd_rn(us, uv);
+            }
+            mx_finish_row<kMode>(p, ti, q, lane, i, gs, us);
+          }
+          if (lane == 0) p.tickets[ti.t * 4 + q] = 0u;
+        }
+        continue;
+      }
+      for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+        uint32_t g[32], u[32];
+        mx_ld_chunk(t0, t1, c0, g, u);
+        const int nv = min(32, ti.nrows - c0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i < nv) mx_finish_row<kMode>(p, ti, q, lane, c0 + i, __uint_as_float(g[i]), __uint_as_float(u[i]));
       }
       tc_fence_before_sync();
       __syncwarp();
