@@ -317,8 +317,9 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
  *             (m tokens over all ranks, n = E experts);
  *   b_new[e] = -beta_e, beta_e taken at the lower edge of its histogram bin.
  * All arithmetic is fp32 with every operation rounded as written:
- *   v = s + b, mu = s - alpha, t = mu - lo, bin = t < 0 ? 0 : (t * inv_w >= B
- *   ? B - 1 : trunc(t * inv_w)), inv_w = fp32(B) / fp32(hi - lo).
+ *   v = s + b, mu = s - alpha, t = mu - lo, bin = !(t >= 0) ? 0 : (t * inv_w
+ *   >= B ? B - 1 : trunc(t * inv_w)), inv_w = fp32(B) / fp32(hi - lo); a NaN
+ *   margin (from a NaN logit, or infinite ones that cancel) counts in bin 0.
  *
  * moe_router_logits: the router logits s = x W_router (+ bias) [T, E] fp32 in
  *   the canonical order of moe_route (bit-identical to the logits it selects

@@ -563,7 +563,9 @@ int oracle_qb_histogram(const double* s, const double* alpha, int64_t m, int64_t
       // bin floor(B (mu - lo) / (hi - lo)): exact on the edges that exact
       // inputs put there (a margin of 0 -- the cutoff expert's own -- with lo
       // a multiple of the bin width), where dividing by a rounded width is not
-      int64_t bin = mu < lo ? 0 : static_cast<int64_t>(std::floor(static_cast<double>(B) * (mu - lo) / (hi - lo)));
+      // (a NaN margin fails mu >= lo and counts in bin 0, as below lo)
+      int64_t bin =
+          !(mu >= lo) ? 0 : static_cast<int64_t>(std::floor(static_cast<double>(B) * (mu - lo) / (hi - lo)));
       bin = std::max<int64_t>(0, std::min(bin, B - 1));
       H[j * B + bin] += 1;
     }
@@ -599,7 +601,8 @@ extern "C" {
 // router logits takes them: v = s + b rounded to fp32, alpha the (k+1)-th
 // largest v, mu = s - alpha rounded to fp32, t = mu - lo rounded to fp32, and
 // the bin floor(t * inv_w) with inv_w = fp32(B) / fp32(hi - lo), both
-// products rounded to fp32; t < 0 counts in bin 0, a bin >= B in bin B - 1.
+// products rounded to fp32; t < 0 (or NaN) counts in bin 0, a bin >= B in
+// bin B - 1.
 // On data with no margin within an fp32 rounding of a bin edge it counts
 // exactly what oracle_qb_histogram counts (from the same fp32 inputs).
 // s [m, n] fp32, b [n] fp32 or NULL; alpha [m] (fp32 values) is written.
@@ -616,7 +619,7 @@ int oracle_qb_histogram_f32(const float* s, const float* b, int64_t m, int64_t n
       const float mu = s[i * n + j] - alpha[i];
       const float t = mu - lo;
       const float fbin = t * inv_w;
-      int64_t bin = t < 0.0f ? 0 : (fbin >= static_cast<float>(B) ? B - 1 : static_cast<int64_t>(fbin));
+      int64_t bin = !(t >= 0.0f) ? 0 : (fbin >= static_cast<float>(B) ? B - 1 : static_cast<int64_t>(fbin));
       H[j * B + bin] += 1;
     }
   }

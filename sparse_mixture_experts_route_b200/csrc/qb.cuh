@@ -12,7 +12,8 @@
 // Arithmetic (fp32, every operation rounded as written, so that the counts
 // are reproducible bit for bit):
 //   v = s + b;  alpha = (k+1)-th largest v;  mu = s - alpha;  t = mu - lo;
-//   bin = t < 0 ? 0 : (t * inv_w >= B ? B - 1 : trunc(t * inv_w)),
+//   bin = !(t >= 0) ? 0 : (t * inv_w >= B ? B - 1 : trunc(t * inv_w)),
+//   so a NaN margin counts in bin 0 and +inf in bin B - 1,
 //   inv_w = fp32(B) / fp32(hi - lo) (computed on the host).
 // Three kernels: cutoffs (warp per token), histogram (CTA per 8 experts x a
 // token slice, counts in shared memory, then added into H with 64-bit
@@ -93,7 +94,9 @@ __global__ void __launch_bounds__(256)
       const float mu = __fsub_rn(__ldg(s + static_cast<int64_t>(t) * E + e), __ldg(alpha + t));
       const float tt = __fsub_rn(mu, lo);
       const float f = __fmul_rn(tt, inv_w);
-      const int bin = tt < 0.0f ? 0 : (f >= fB ? B - 1 : static_cast<int>(f));
+      // a NaN margin (a NaN logit, or infinities that cancel) fails tt >= 0
+      // and counts in bin 0, like a margin below lo
+      const int bin = !(tt >= 0.0f) ? 0 : (f >= fB ? B - 1 : static_cast<int>(f));
       atomicAdd(&qb_counts[j * B + bin], 1u);
     }
   }
