@@ -341,6 +341,24 @@ moe_status_t moe_qb_histogram(const float* logits, const float* bias, int T, int
 moe_status_t moe_qb_bias(const uint64_t* H, int E, int bins, float lo, float hi, int64_t m_total, int k,
                          int32_t* bin_out, float* bias_out, cudaStream_t stream);
 
+/* ----------------------------------------------- expert parallelism --
+ * [P3] section "Systems Optimization, Load Balancing, and Post-Training
+ * Alignment" (its expert-parallel scheme): the routed experts are split over
+ * ranks, and each rank's dispatched token rows go to the rank that owns their
+ * expert and come back after the expert feed-forward. The exchanges are the
+ * caller's all-to-all collectives (NCCL); on either side of them the rows have
+ * to be put in the order the next step reads, which is a row gather.
+ *
+ * moe_gather_rows: out[i, :] = src[rows[i], :] for 0 <= i < n_out (bf16 rows
+ *   of width d; src [n_src, d], out [n_out, d], row-major, 16-byte aligned,
+ *   d % 8 == 0). rows[i] = -1 writes a zero row (the padding of a
+ *   fixed-capacity exchange buffer); any other index outside [0, n_src)
+ *   writes a zero row and records MOE_DEVERR_BAD_ROUTE in the error word.
+ *   Needs no scratch; n_out = 0 enqueues nothing.
+ */
+moe_status_t moe_gather_rows(const moe_bf16_t* src, int64_t n_src, const int32_t* rows, int64_t n_out, int d,
+                             moe_bf16_t* out, cudaStream_t stream);
+
 /* ------------------------------------------------------------ diagnostics --
  * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
  * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise

@@ -48,6 +48,7 @@ EXPORTS = {
     "moe_router_logits": ([P, P, P, I, I, I, P, P], I),
     "moe_qb_histogram": ([P, P, I, I, I, ctypes.c_float, ctypes.c_float, I, P, P, P], I),
     "moe_qb_bias": ([P, I, I, ctypes.c_float, ctypes.c_float, ctypes.c_int64, I, P, P, P], I),
+    "moe_gather_rows": ([P, ctypes.c_int64, P, ctypes.c_int64, I, P, P], I),
     "moe_get_device_error": ([ctypes.POINTER(ctypes.c_uint32), I], I),
     "moe_selftest_wait_timeout": ([I, P], I),
 }
@@ -390,6 +391,20 @@ def moe_forward_host(x_host, W_router, router_bias, W_gate_up, W_down, k: int, o
                                  T, d, E, k, f, _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward_host")
     return out_host
+
+
+def moe_gather_rows(src, rows, out=None, stream=None):
+    """out[i] = src[rows[i]] (bf16 rows); rows[i] = -1 gives a zero row."""
+    n_src, d = src.shape
+    _need(src, "src", torch.bfloat16, (n_src, d))
+    n_out = rows.shape[0]
+    _need(rows, "rows", torch.int32, (n_out,))
+    if out is None:
+        out = torch.empty(n_out, d, dtype=torch.bfloat16, device=src.device)
+    _need(out, "out", torch.bfloat16, (n_out, d))
+    _check(_lib.moe_gather_rows(_ptr(src), n_src, _ptr(rows), n_out, d, _ptr(out), _stream(stream)),
+           "moe_gather_rows")
+    return out
 
 
 def get_device_error(clear: bool = True) -> int:

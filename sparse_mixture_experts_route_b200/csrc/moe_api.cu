@@ -15,6 +15,7 @@
 #include "moe.h"
 
 #include "common.cuh"
+#include "ep.cuh"
 #include "expert_gemm.cuh"
 #include "mx_gemm.cuh"
 #include "mx_prep.cuh"
@@ -1153,6 +1154,19 @@ moe_status_t moe_qb_bias(const uint64_t* H, int E, int bins, float lo, float hi,
   const float w = (hi - lo) / static_cast<float>(bins);
   qb_bias_kernel<<<static_cast<unsigned>(ceil_div(E, 8)), 256, 0, stream>>>(
       reinterpret_cast<const unsigned long long*>(H), E, bins, lo, w, static_cast<long long>(r), bin_out, bias_out);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_gather_rows(const moe_bf16_t* src, int64_t n_src, const int32_t* rows, int64_t n_out, int d,
+                             moe_bf16_t* out, cudaStream_t stream) {
+  if (n_src < 0 || n_out < 0 || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (n_out == 0) return MOE_OK;
+  if (!rows || !out || (n_src > 0 && !src) || !aligned16(out) || (src && !aligned16(src)))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t blocks = ceil_div64(n_out, 8);  // 8 warps of 256 threads, warp per row
+  if (blocks > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(src), n_src, rows, n_out, d / 8, reinterpret_cast<uint4*>(out));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -260,3 +260,18 @@ def test_qb_and_router_logits_checks(lib):
     assert qbias(p, 8, 1000, -4.0, 4.0, 0, 2, p, p, None) == 1        # no tokens
     assert qbias(p, 8, 1000, -4.0, 4.0, 64, 8, p, p, None) == 1       # k >= E
     assert qbias(p, 8, 1000, -4.0, 4.0, 64, 2, p, None, None) == 1
+
+
+def test_gather_rows_checks(lib):
+    """moe_gather_rows refuses bad sizes and pointers on the host; n_out = 0
+    enqueues nothing and succeeds."""
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.moe_gather_rows.argtypes = [P, I64, P, I64, I, P, P]
+    lib.moe_gather_rows.restype = I
+    p = ctypes.c_void_p(FAKE)
+    assert lib.moe_gather_rows(p, 10, p, 0, 64, p, None) == 0          # nothing to do
+    assert lib.moe_gather_rows(p, 10, p, 5, 60, p, None) == 1          # d % 8
+    assert lib.moe_gather_rows(p, 10, None, 5, 64, p, None) == 1       # no row list
+    assert lib.moe_gather_rows(p, 10, p, 5, 64, None, None) == 1       # no output
+    assert lib.moe_gather_rows(p, -1, p, 5, 64, p, None) == 1
+    assert lib.moe_gather_rows(ctypes.c_void_p(FAKE + 2), 10, p, 5, 64, p, None) == 1   # unaligned rows
