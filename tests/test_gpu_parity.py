@@ -53,9 +53,9 @@ def test_route_bit_exact(lib, shape):
     g = _cuda(inp)
     idx, w = lib.moe_route(g.x, g.W_router, None, k)
     torch.cuda.synchronize()
-    _, ridx, rw = parity.oracle_route(inp, k)
+    lg, ridx, rw = parity.oracle_route(inp, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    parity.assert_route_weights(w, rw, inp.x, inp.W_router, None, k, lg, ridx)
     assert lib.get_device_error() == 0
 
 
@@ -87,9 +87,9 @@ def test_route_few_tokens(lib, shape):
         idx, w = lib.moe_route(g.x, g.W_router, g.bias, k, workspace=ws)
         torch.cuda.synchronize()
         assert lib.get_device_error() == 0
-        _, ridx, rw = parity.oracle_route(inp, k)
+        lg, ridx, rw = parity.oracle_route(inp, k)
         assert np.array_equal(idx.cpu().numpy(), ridx)
-        np.testing.assert_allclose(w.cpu().numpy().astype(np.float64), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+        parity.assert_route_weights(w, rw, inp.x, inp.W_router, inp.bias, k, lg, ridx)
 
 
 @pytest.mark.parametrize("T", [1, 6])
@@ -122,7 +122,7 @@ def test_route_few_tokens_ties_and_unaligned_weights(lib):
     ridx, rw = oracle.topk(lg, k)
     idx, w = lib.moe_route(x.cuda(), Wr.cuda(), bias.cuda(), k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    parity.assert_route_weights(w, rw, x, Wr, bias, k, lg, ridx)
     assert idx[1].tolist() == [5, 0, 1]
     store = torch.empty(d * E + 1, dtype=torch.float32, device="cuda")
     Wr_off = store[1:].view(d, E)
@@ -130,7 +130,7 @@ def test_route_few_tokens_ties_and_unaligned_weights(lib):
     assert Wr_off.data_ptr() % 16 != 0
     idx2, w2 = lib.moe_route(x.cuda(), Wr_off, bias.cuda(), k)
     assert torch.equal(idx2, idx)
-    np.testing.assert_allclose(w2.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    parity.assert_route_weights(w2, rw, x, Wr, bias, k, lg, ridx)
     assert lib.get_device_error() == 0
 
 
@@ -149,7 +149,7 @@ def test_route_bias_ties_zero_rows(lib):
         lg = oracle.router_logits(x, Wr, b)
         ridx, rw = oracle.topk(lg, k)
         assert np.array_equal(idx.cpu().numpy(), ridx)
-        np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+        parity.assert_route_weights(w, rw, x, Wr, b, k, lg, ridx)
     # the zero tokens with a bias on expert 5 pick 5 then 0, 1
     assert idx[10].tolist() == [5, 0, 1]
 
@@ -159,9 +159,9 @@ def test_route_zipf_bias_and_hot_expert(lib):
     inp = _inputs(T, d, E, k, f, bias="zipf")
     g = _cuda(inp)
     idx, w = lib.moe_route(g.x, g.W_router, g.bias, k)
-    _, ridx, rw = parity.oracle_route(inp, k)
+    lg, ridx, rw = parity.oracle_route(inp, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    parity.assert_route_weights(w, rw, inp.x, inp.W_router, inp.bias, k, lg, ridx)
     hot = torch.zeros(E, dtype=torch.float32)
     hot[3] = 100.0
     idx, _ = lib.moe_route(g.x, g.W_router, hot.cuda(), k)
@@ -389,4 +389,4 @@ def test_route_tensor_core_screen_ties_and_fallback(lib, E, k, bias_on):
     lg = oracle.router_logits(x, Wr, inp.bias)
     ridx, rw = oracle.topk(lg, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
-    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=parity.W_RTOL, atol=parity.W_ATOL)
+    parity.assert_route_weights(w, rw, x, Wr, inp.bias, k, lg, ridx)

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from sparse_mixture_experts_route_b200 import inputs as moe_inputs
 
 pytestmark = pytest.mark.gpu
@@ -32,17 +33,29 @@ def _route_both(lib, shape, seed):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == lib.MOE_OK, lib.raw.moe_status_string(st)
     torch.cuda.synchronize()
-    return idx.cpu().numpy(), w.cpu().numpy(), idx_ref.cpu().numpy(), w_ref.cpu().numpy()
+    return inp, idx.cpu().numpy(), w.cpu().numpy(), idx_ref.cpu().numpy(), w_ref.cpu().numpy()
 
 
 def test_route_noalloc_matches_route_on_two_calls_in_a_row():
+    """Consecutive calls with different sizes share the fixed scratch. Each is
+    compared with moe_route (the same routing, bit for bit: same indices, same
+    weight bits) and with the CPU oracle (indices bit-exact, weights within
+    1e-5 relative). The one-token call, whose router keeps its completion
+    tickets in the shared scratch, runs both before and after a 16-token call
+    of the same width."""
     from sparse_mixture_experts_route_b200 import _lib as lib
+    one = moe_inputs.custom_shape(1, 7168, 896, 16, 512, name="decode1")       # few-token router, T = 1
     first = moe_inputs.custom_shape(16, 7168, 896, 16, 512, name="decode16")   # 3.2 MB of scratch
     second = moe_inputs.custom_shape(7, 256, 64, 4, 64, bias="zipf", name="small")  # different sizes, bias
-    for shape, seed in ((first, 0), (second, 1)):
-        idx, w, idx_ref, w_ref = _route_both(lib, shape, seed)
+    for shape, seed in ((one, 2), (first, 0), (one, 3), (second, 1), (one, 2)):
+        inp, idx, w, idx_ref, w_ref = _route_both(lib, shape, seed)
         assert np.array_equal(idx, idx_ref), shape.name
-        np.testing.assert_allclose(w, w_ref, rtol=1e-5, atol=1e-7, err_msg=shape.name)
+        assert np.array_equal(w.view(np.uint32), w_ref.view(np.uint32)), shape.name
+        lg = oracle.router_logits(inp.x.cpu(), inp.W_router.cpu(),
+                                  inp.bias.cpu() if inp.bias is not None else None)
+        ridx, rw = oracle.topk(lg, shape.k)
+        assert np.array_equal(idx, ridx), shape.name
+        np.testing.assert_allclose(w, rw, rtol=1e-5, atol=1e-7, err_msg=shape.name)
     assert lib.get_device_error() == 0
 
 
