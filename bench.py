@@ -120,17 +120,21 @@ def algorithmic(shape: moe_inputs.MoEShape, counts: np.ndarray):
     F_alg = 2*T*d*E (router) + 6*T*k*d*f (experts)
     B_alg = 4*d*E (W_router) + 2*T*d*2 (x in, out) + n_touched*6*d*f (expert
             weights of experts with at least one row) + 4*E (bias, if any)
-    gate/up GEMM kernel (the dominant one): its compulsory bytes per launch =
-            n_touched*4*d*f (gate and up weights) + T*k*d*2 (rows in)
-            + T*k*f*2 (h out)
+    gate/up GEMM kernel (the dominant one), per launch: the per-unit figure of
+            that step, 2*d*f*2 bytes of gate and up weights per touched expert,
+            times the experts one launch touches. The rows it reads and the h
+            it writes (T*k*d*2 + T*k*f*2 bytes) are the materialised
+            intermediates of this implementation, reported beside it.
     """
     T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
     n_touched = int((counts > 0).sum())
     F = 2.0 * T * d * E + 6.0 * T * k * d * f
     B = 4.0 * d * E + 4.0 * T * d + n_touched * 6.0 * d * f + (4.0 * E if shape.bias else 0.0)
-    gu_bytes = n_touched * 4.0 * d * f + 2.0 * T * k * d + 2.0 * T * k * f
+    gu_bytes = n_touched * 4.0 * d * f
+    gu_impl_bytes = 2.0 * T * k * d + 2.0 * T * k * f
     gu_flops = 4.0 * T * k * d * f
-    return {"F": F, "B": B, "n_touched": n_touched, "gu_bytes": gu_bytes, "gu_flops": gu_flops}
+    return {"F": F, "B": B, "n_touched": n_touched, "gu_bytes": gu_bytes, "gu_impl_bytes": gu_impl_bytes,
+            "gu_flops": gu_flops}
 
 
 def count_library_launches(step) -> int:
@@ -167,46 +171,82 @@ def profiled_traffic(workload: str):
 
 # ------------------------------------------------------------ CPU baseline
 
-def cpu_baseline(inp, shape, budget_s: float = 20.0, seed: int = 1):
-    """The oracle, as it stands, on a bounded sample of the workload, on this
-    host's cores. Per-token cost = router+top-k+combine per token + k expert
-    rows; each part is timed on its own sample and scaled to tokens/s."""
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_pass(inp, shape, tokens, threads: int):
+    """The oracle, as it stands, over the listed tokens: router and top-k,
+    every selected (token, expert) row through the expert's SwiGLU block, and
+    the weighted combine. Experts run on a pool of `threads` host threads in
+    groups of `threads`; each group's weights are fetched from the device
+    before its timed region, so only oracle arithmetic is timed. Returns
+    (seconds, expert rows, expert FLOPs, expert seconds)."""
     import oracle
-    rng = np.random.default_rng(seed)
-    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
-    n_route = min(T, 256)
-    toks = np.sort(rng.choice(T, size=n_route, replace=False))
-    xs = inp.x[torch.as_tensor(toks, device=inp.x.device)].cpu()
+    from concurrent.futures import ThreadPoolExecutor
+    d, k, f = shape.d, shape.k, shape.f
+    xs = inp.x[torch.as_tensor(tokens, device=inp.x.device)].cpu()
     Wr = inp.W_router.cpu()
     b = inp.bias.cpu() if inp.bias is not None else None
     t0 = time.perf_counter()
     lg = oracle.router_logits(xs, Wr, b)
     idx, w = oracle.topk(lg, k)
-    t_route = (time.perf_counter() - t0) / n_route
-    # expert rows: rows of a few experts chosen by the sample, until the budget
-    rows_done, t_ffn = 0, 0.0
-    experts = list(dict.fromkeys(idx.ravel().tolist()))
-    deadline = time.perf_counter() + budget_s
-    for e in experts:
-        sel = np.argwhere(idx == e)[:, 0]
-        Wg = inp.W_gate_up[e].cpu()
-        Wd = inp.W_down[e].cpu()
-        t1 = time.perf_counter()
-        y = oracle.expert_ffn(xs[torch.as_tensor(sel)], Wg, Wd)
-        t_ffn += time.perf_counter() - t1
-        rows_done += len(sel)
-        if time.perf_counter() > deadline or rows_done >= n_route * k:
-            break
-    t_row = t_ffn / max(rows_done, 1)
-    yy = np.zeros((n_route * k, d))
+    t_route = time.perf_counter() - t0
+    n = len(tokens)
+    y = np.zeros((n * k, d), dtype=np.float64)
+    experts = np.unique(idx)
+    t_ffn = 0.0
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for g0 in range(0, len(experts), threads):
+            group = experts[g0:g0 + threads]
+            wts = {int(e): (inp.W_gate_up[int(e)].cpu(), inp.W_down[int(e)].cpu()) for e in group}
+
+            def one(e):
+                rows = np.argwhere(idx == e)
+                y[rows[:, 0] * k + rows[:, 1]] = oracle.expert_ffn(xs[torch.as_tensor(rows[:, 0])], *wts[int(e)])
+
+            t1 = time.perf_counter()
+            list(ex.map(one, group))
+            t_ffn += time.perf_counter() - t1
+            del wts
     t2 = time.perf_counter()
-    oracle.combine(yy, np.arange(n_route * k, dtype=np.int32).reshape(n_route, k), w)
-    t_comb = (time.perf_counter() - t2) / n_route
-    per_token = t_route + k * t_row + t_comb
-    return {"value": 1.0 / per_token, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"router+top-k+combine on {n_route} sampled tokens, SwiGLU on {rows_done} routed rows "
-                      f"of {shape.name}; tokens/s = 1/(t_route+k*t_row+t_combine)",
-            "seconds": t_route * n_route + t_ffn + t_comb * n_route}
+    oracle.combine(y, np.arange(n * k, dtype=np.int32).reshape(n, k), w)
+    t_comb = time.perf_counter() - t2
+    return t_route + t_ffn + t_comb, n * k, 6.0 * n * k * d * f, t_ffn
+
+
+def sample_tokens(T: int, n: int, seed: int) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(T, size=min(n, T), replace=False))
+
+
+def calibrate_tokens(inp, shape, budget_s: float, threads: int, cap: int = 1024) -> int:
+    """Tokens per oracle pass so that one pass takes about budget_s: a first
+    untimed pass over 8 tokens sets the per-token cost."""
+    t8, _, _, _ = oracle_pass(inp, shape, sample_tokens(shape.T, 8, 99), threads)
+    per_tok = t8 / min(8, shape.T)
+    return int(max(1, min(shape.T, cap, budget_s / max(per_tok, 1e-9))))
+
+
+def cpu_baseline(inp, shape, budget_s: float = 20.0, seed: int = 1):
+    """The oracle on a bounded sample of the workload, on this host's cores:
+    one complete pass over a seeded sample of tokens sized to take about
+    budget_s; tokens/s = sampled tokens / oracle seconds."""
+    import oracle
+    threads = oracle.num_threads()
+    n = calibrate_tokens(inp, shape, budget_s, threads)
+    secs, rows, ffn_flops, ffn_s = oracle_pass(inp, shape, sample_tokens(shape.T, n, seed), threads)
+    return {"value": n / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"one oracle pass (router, top-k, {rows} expert rows, combine) over {n} seeded tokens "
+                      f"of {shape.name}; tokens/s = {n} / oracle seconds (weights fetched to host untimed)",
+            "seconds": secs, "tokens": n, "cpu_model": cpu_model(),
+            "fp64_gflops": ffn_flops / ffn_s / 1e9 if ffn_s > 0 else None}
 
 
 # ------------------------------------------------------------------ arms
@@ -258,29 +298,32 @@ def aggregate_tokens_per_s(T: int, steps: int, world: int, max_total_ms: float) 
     return world * T * steps / (max_total_ms / 1e3)
 
 
-def run_ours(args):
-    from sparse_mixture_experts_route_b200 import _lib
-    world, rank, local = dist_setup()
-    shape = moe_inputs.WORKLOADS[args.workload]
-    dev = torch.device("cuda", local)
-    peaks, peak_src = load_peaks()
+class L2Flush:
+    """Between timed steps: write a buffer twice the size of L2, then read
+    another one, so the dirty lines are written back here and not inside the
+    next timed step."""
 
-    log(f"[rank {rank}] generating {shape.name} on {dev}")
-    inp = moe_inputs.make_inputs(shape, seed=0, device=dev)
-    if rank != 0:  # each replica routes its own tokens
-        inp.x = moe_inputs.make_x(shape, seed=replica_x_seed(rank), device=dev)
+    def __init__(self, dev):
+        self.w = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self, s):
+        self.w.fill_(float(s))
+        self.r.amax()
+
+
+def time_layer(_lib, shape, inp, steps: int, warmup: int, graph_on: bool, world: int, flush, local: int,
+               count_launches: bool = False):
+    """Times `steps` moe_forward steps of one workload (after `warmup`), each
+    between CUDA events on the launching stream with an L2 flush outside the
+    events; replays of one step captured as a CUDA graph when graph_on. The
+    per-stage times (and so the dominant kernel's duration) come from eager
+    moe_forward_timed steps, since events cannot time nodes inside a replay."""
     T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
-    ws = torch.empty(_lib.moe_forward_workspace_size(T, d, E, k, f), dtype=torch.uint8, device=dev)
-    out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    flush_r = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def flush_l2(s):
-        # write a buffer larger than L2, then read another one so the dirty
-        # lines are written back here and not inside the next timed step
-        flush.fill_(float(s))
-        flush_r.amax()
+    ws = torch.empty(_lib.moe_forward_workspace_size(T, d, E, k, f), dtype=torch.uint8, device=inp.x.device)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=inp.x.device)
     stream = torch.cuda.current_stream()
+    args = (inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
 
     # routing statistics of this batch (for the algorithmic byte counts)
     idx, _ = _lib.moe_route(inp.x, inp.W_router, inp.bias, k)
@@ -289,19 +332,19 @@ def run_ours(args):
     alg = algorithmic(shape, counts)
 
     nst = len(_lib.TIMED_STAGES)
-    launches_per_step = count_library_launches(lambda: _lib.moe_forward(
-        inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws))
-    for _ in range(args.warmup):
-        flush_l2(1)
-        _lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+    launches = count_library_launches(lambda: _lib.moe_forward(*args, out=out, workspace=ws)) \
+        if count_launches else None
+    for _ in range(warmup):
+        flush(1)
+        _lib.moe_forward(*args, out=out, workspace=ws)
     assert _lib.get_device_error() == 0, "device error during warm-up"
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + 2 * nst)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + 2 * nst)] for _ in range(steps)]
     for row in evs:
         for ev in row:
             ev.record(stream)
     graph = None
-    if args.graph == "on":
+    if graph_on:
         # one step captured as a CUDA graph (the library never allocates or
         # synchronises, so its launches capture as they are)
         torch.cuda.synchronize()
@@ -309,46 +352,100 @@ def run_ours(args):
         side = torch.cuda.Stream()
         side.wait_stream(stream)
         with torch.cuda.stream(side):
-            _lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+            _lib.moe_forward(*args, out=out, workspace=ws)
             with torch.cuda.graph(graph, stream=side):
-                _lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, out=out, workspace=ws)
+                _lib.moe_forward(*args, out=out, workspace=ws)
         stream.wait_stream(side)
-        for _ in range(args.warmup):
-            flush_l2(1)
+        for _ in range(warmup):
+            flush(1)
             graph.replay()
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
-    for s in range(args.steps):
-        flush_l2(s)                               # L2 flush, outside the step's events
+    for s in range(steps):
+        flush(s)                                  # L2 flush, outside the step's events
         evs[s][0].record(stream)
         if graph is not None:
             graph.replay()
         else:
-            _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[s][2:], out, ws)
+            _lib.moe_forward_timed(*args, evs[s][2:], out, ws)
         evs[s][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
-    step_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
+    step_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(steps)]
     if graph is not None:
-        # per-kernel-group times (and the roofline kernel's duration) from a few
-        # eager timed steps: events cannot time nodes inside a graph replay
-        n_eager = min(args.steps, 5)
-        _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[0][2:], out, ws)
+        n_eager = min(steps, 5)
+        _lib.moe_forward_timed(*args, evs[0][2:], out, ws)
         for s in range(n_eager):
-            flush_l2(s)
-            _lib.moe_forward_timed(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k, evs[s][2:], out, ws)
+            flush(s)
+            _lib.moe_forward_timed(*args, evs[s][2:], out, ws)
         torch.cuda.synchronize()
         stage_steps = range(n_eager)
     else:
-        stage_steps = range(args.steps)
+        stage_steps = range(steps)
     stage_ms = {name: [evs[s][2 + 2 * i].elapsed_time(evs[s][3 + 2 * i]) for s in stage_steps]
                 for i, name in enumerate(_lib.TIMED_STAGES)}
     total_ms = max_over_ranks(sum(step_ms), world)
     assert _lib.get_device_error() == 0, "device error during timing"
+    del graph
+    return {"total_ms": total_ms, "step_ms": step_ms, "stage_ms": stage_ms, "alg": alg, "clocks": clk,
+            "launches": launches, "out": out, "ws": ws, "counts": counts}
+
+
+def layer_summary(shape, res, steps: int, world: int, peaks: dict) -> dict:
+    """Throughput and roofline figures of one timed workload."""
+    T, k, E = shape.T, shape.k, shape.E
+    alg = res["alg"]
+    ms_per_step = res["total_ms"] / steps
+    t_step = ms_per_step / 1e3
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    gu_ms = statistics.mean(res["stage_ms"]["gemm_gate_up"])
+    layer_roof_s = max(alg["F"] / (tc * 1e12), alg["B"] / (hbm * 1e9))
+    return {
+        "ms_per_step": ms_per_step,
+        "tokens_per_s": aggregate_tokens_per_s(T, steps, world, res["total_ms"]),
+        "tflops": alg["F"] / t_step / 1e12, "hbm_gbs": alg["B"] / t_step / 1e9,
+        "F_alg": alg["F"], "B_alg": alg["B"], "n_touched": alg["n_touched"],
+        "max_rows_per_expert": int(res["counts"].max()),
+        "roofline_frac": layer_roof_s / t_step,
+        "binding_roof": "hbm" if alg["B"] / hbm / 1e9 >= alg["F"] / tc / 1e12 else "tensor",
+        "tensor_frac_of_peak": alg["F"] / t_step / 1e12 / tc,
+        "hbm_frac_of_peak": alg["B"] / t_step / 1e9 / hbm,
+        "stage_ms": {kname: statistics.mean(v) for kname, v in res["stage_ms"].items()},
+        "dominant_kernel": {
+            "kernel": ("grouped_gemm_kernel<0>" if T * k > 128 * E else "grouped_gemm_kernel<2>")
+                      + " (gate/up + SwiGLU)",
+            "ms_per_launch": gu_ms, "alg_bytes_per_launch": alg["gu_bytes"],
+            "achieved_gbs": alg["gu_bytes"] / (gu_ms / 1e3) / 1e9,
+            "achieved_tflops": alg["gu_flops"] / (gu_ms / 1e3) / 1e12},
+        "clocks": res["clocks"],
+    }
+
+
+EXTRA_WORKLOADS = ("decode", "skewed") + tuple(f"sweep_T{t}" for t in moe_inputs.SWEEP_T)
+
+
+def run_ours(args):
+    from sparse_mixture_experts_route_b200 import _lib
+    world, rank, local = dist_setup()
+    shape = moe_inputs.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    flush = L2Flush(dev)
+
+    log(f"[rank {rank}] generating {shape.name} on {dev}")
+    inp = moe_inputs.make_inputs(shape, seed=0, device=dev)
+    if rank != 0:  # each replica routes its own tokens
+        inp.x = moe_inputs.make_x(shape, seed=replica_x_seed(rank), device=dev)
+    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    res = time_layer(_lib, shape, inp, args.steps, args.warmup, args.graph == "on", world, flush, local,
+                     count_launches=True)
+    out = res["out"]
+    stream = torch.cuda.current_stream()
 
     # end to end through the host-buffer call: every step copies x in from
     # pinned host memory, runs the pass and copies the result back, all inside
@@ -385,71 +482,111 @@ def run_ours(args):
     assert torch.equal(e2e_out[(args.steps - 1) % 2], out.cpu()), "host-buffer call disagrees with moe_forward"
     e2e_total = max_over_ranks(sum(e2e_ms), world)
 
+    cpu_line = None
+    if rank == 0 and not args.no_cpu_baseline:
+        log("[rank 0] timing the CPU oracle on a bounded sample")
+        cpu_line = cpu_baseline(inp, shape, budget_s=args.cpu_budget)
+    head = layer_summary(shape, res, args.steps, world, peaks)
+    launches, impl_bytes = res["launches"], res["alg"]["gu_impl_bytes"]
+    del inp, res, e2e_ws, e2e_out, x_host
+    torch.cuda.empty_cache()
+
+    # the other workloads, one after another (every rank runs the same list,
+    # so the timing barriers line up); skewed and the sweep share one set of
+    # expert weights (same shapes and seeds), generated once
+    extra = {}
+    if not args.no_workloads:
+        shared = None
+        for name in EXTRA_WORKLOADS:
+            ws_shape = moe_inputs.WORKLOADS[name]
+            log(f"[rank {rank}] {name}")
+            if shared is not None and shared.W_gate_up.shape == (ws_shape.E, ws_shape.d, 2 * ws_shape.f):
+                x = moe_inputs.make_x(ws_shape, seed=replica_x_seed(rank), device=dev)
+                bias = moe_inputs.zipf_bias(ws_shape.E).to(dev) if ws_shape.bias == "zipf" else None
+                winp = type(shared)(ws_shape, x, shared.W_router, bias, shared.W_gate_up, shared.W_down)
+            else:
+                shared = None
+                torch.cuda.empty_cache()
+                winp = moe_inputs.make_inputs(ws_shape, seed=0, device=dev)
+                if rank != 0:
+                    winp.x = moe_inputs.make_x(ws_shape, seed=replica_x_seed(rank), device=dev)
+                shared = winp
+            steps = args.workload_steps
+            r = time_layer(_lib, ws_shape, winp, steps, args.warmup, args.graph == "on", world, flush, local)
+            extra[name] = {**{kk: v for kk, v in ws_shape.as_dict().items() if kk != "workload"},
+                           "steps": steps, **layer_summary(ws_shape, r, steps, world, peaks)}
+            del r, winp
+        del shared
+        torch.cuda.empty_cache()
+
     if rank != 0:
         return None
     n = world
-    value = aggregate_tokens_per_s(T, args.steps, n, total_ms)
-    ms_per_step = total_ms / args.steps
-    t_step = ms_per_step / 1e3
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    gu_ms = statistics.mean(stage_ms["gemm_gate_up"])
-    gu_achieved = alg["gu_bytes"] / (gu_ms / 1e3) / 1e9
-    traffic = profiled_traffic(shape.name)
-    layer_roof_s = max(alg["F"] / (tc * 1e12), alg["B"] / (hbm * 1e9))
+    dom = head["dominant_kernel"]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": n, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
+        "metric": METRIC, "value": head["tokens_per_s"], "unit": UNIT, "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {**shape.as_dict(), "seed": 0, "parallelism": f"replicas{n}",
-                   "launch": "cuda_graph_replay" if graph is not None else "eager",
+                   "launch": "cuda_graph_replay" if args.graph == "on" else "eager",
                    "l2": "flushed between steps (2x L2 write, then 2x L2 read, outside the step events)",
                    "weights_gb": round(E * 6.0 * d * f / 1e9, 3)},
-        "roofline": {"bound": "hbm",
-                     "kernel": ("grouped_gemm_kernel<0>" if T * k > 128 * E else "grouped_gemm_kernel<2>")
-                               + " (gate/up + SwiGLU)",
-                     "achieved": gu_achieved, "peak": hbm, "unit": "GB/s", "frac": gu_achieved / hbm,
-                     "traffic": traffic, "peak_source": f"{peak_src} hbm_gbs (burst copy)",
-                     "alg_bytes_per_launch": alg["gu_bytes"], "ms_per_launch": gu_ms},
-        "layer": {"tflops": alg["F"] / t_step / 1e12, "hbm_gbs": alg["B"] / t_step / 1e9,
-                  "F_alg": alg["F"], "B_alg": alg["B"], "n_touched": alg["n_touched"],
-                  "roofline_frac": layer_roof_s / t_step,
-                  "binding_roof": "hbm" if alg["B"] / hbm / 1e9 >= alg["F"] / tc / 1e12 else "tensor",
-                  "tensor_frac_of_peak": alg["F"] / t_step / 1e12 / tc,
-                  "stage_ms": {kname: statistics.mean(v) for kname, v in stage_ms.items()}},
+        "roofline": {"bound": "hbm", "kernel": dom["kernel"],
+                     "achieved": dom["achieved_gbs"], "peak": hbm, "unit": "GB/s", "frac": dom["achieved_gbs"] / hbm,
+                     "traffic": profiled_traffic(shape.name), "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+                     "alg_bytes_per_launch": dom["alg_bytes_per_launch"],
+                     "alg_bytes_rule": "touched experts x 4*d*f (gate and up weights, bf16)",
+                     "impl_bytes_per_launch": impl_bytes,
+                     "ms_per_launch": dom["ms_per_launch"]},
+        "layer": {kk: v for kk, v in head.items() if kk not in ("ms_per_step", "tokens_per_s", "clocks",
+                                                                 "dominant_kernel")},
         "e2e": {"value": aggregate_tokens_per_s(T, args.steps, n, e2e_total), "unit": UNIT,
                 "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * d * 2,
                 "call": "moe_forward_host, steps alternating over 2 streams"},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
+        "gpu_launches": launches * args.steps,
+        "clocks": head["clocks"],
     }
-    if not args.no_cpu_baseline:
-        log("[rank 0] timing the CPU oracle on a bounded sample")
-        line["cpu_baseline"] = cpu_baseline(inp, shape, budget_s=args.cpu_budget)
+    if extra:
+        line["workloads"] = extra
+    if cpu_line is not None:
+        line["cpu_baseline"] = cpu_line
     return line
 
 
 def run_reference(args):
-    """The oracle on the host cores, each step a bounded sample of the workload."""
+    """The oracle on the host cores, each step one oracle pass over a bounded,
+    seeded sample of the workload's tokens (sized so the whole run takes about
+    two and a half minutes)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
+    import oracle
     shape = moe_inputs.WORKLOADS[args.workload]
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = moe_inputs.make_inputs(shape, seed=0, device=dev)
-    budget = max(2.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
-    for _ in range(args.warmup):
-        cpu_baseline(inp, shape, budget_s=budget)
-    vals = [cpu_baseline(inp, shape, budget_s=budget) for _ in range(args.steps)]
-    tps = [v["value"] for v in vals]
-    value = statistics.mean(tps)
-    cb = dict(vals[-1])
-    cb["value"] = value
+    threads = oracle.num_threads()
+    budget = max(1.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
+    n = calibrate_tokens(inp, shape, budget, threads)
+    for w_ in range(args.warmup):
+        oracle_pass(inp, shape, sample_tokens(shape.T, n, 500 + w_), threads)
+    secs, ffn = [], []
+    for s in range(args.steps):
+        t, rows, fl, fs = oracle_pass(inp, shape, sample_tokens(shape.T, n, 1 + s), threads)
+        secs.append(t)
+        ffn.append((fl, fs))
+    ms_per_step = 1e3 * statistics.mean(secs)
+    value = n * args.steps / sum(secs)
+    cb = {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+          "sample": f"each step: one oracle pass (router, top-k, {n * shape.k} expert rows, combine) over {n} "
+                    f"seeded tokens of {shape.name} (weights fetched to host untimed)",
+          "tokens": n, "cpu_model": cpu_model(),
+          "fp64_gflops": sum(a for a, _ in ffn) / max(sum(b for _, b in ffn), 1e-9) / 1e9}
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * shape.T / value,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {**shape.as_dict(), "seed": 0, "parallelism": "host cores"},
+            "config": {**shape.as_dict(), "seed": 0, "parallelism": "host cores", "tokens_per_step": n},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -515,6 +652,10 @@ def main():
     ap.add_argument("--workload", default="prefill", choices=sorted(moe_inputs.WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only --workload (skip the decode, skewed and sweep entries of the line)")
+    ap.add_argument("--workload-steps", type=int, default=10,
+                    help="timed steps of each of the other workloads")
     ap.add_argument("--graph", default="on", choices=["on", "off"],
                     help="time replays of one step captured as a CUDA graph (on) or eager calls (off)")
     ap.add_argument("--mx-quant", action="store_true",
