@@ -9,10 +9,13 @@ router whose summation order is stated there, and the Quantile Balancing
 histogram's fp32-decision variant, pinned against its fp64 definition). This
 module only builds that file and marshals numpy / torch CPU arrays into it.
 
-Every function cites its passage in ``moe_oracle.cpp``. All oracle functions
+Every function cites its passage in ``moe_oracle.cpp``. The oracle functions
 here are pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``
-(brute-force sorts, closed forms, invariants, and library routines); none is
-parity-unpinned.
+(brute-force sorts, closed forms, invariants, and library routines), with one
+exception: SiTU-GLU's own formula (``glu_ffn`` / ``latent_forward`` with
+``ACT_SITU``) is parity unpinned, because the page lost it; what is pinned
+there is its stated bound, its SwiGLU limit for large caps, and the latent
+layer's reductions to the pinned plain layer.
 """
 from __future__ import annotations
 
@@ -66,12 +69,17 @@ def _load():
             lib.oracle_qb_bias_from_histogram.argtypes = [P, I, I, ctypes.c_double, ctypes.c_double, I, I, P]
             lib.oracle_qb_histogram_f32.argtypes = [P, P, I, I, I, ctypes.c_float, ctypes.c_float, I, P, P]
             lib.oracle_qb_quantile_bins.argtypes = [P, I, I, I, I, P]
+            D = ctypes.c_double
+            lib.oracle_glu_ffn.argtypes = [P, I, P, P, I, I, I, ctypes.c_int, D, D, P, P]
+            lib.oracle_rmsnorm.argtypes = [P, I, I, P, D, P]
+            lib.oracle_latent_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                                  ctypes.c_int, D, D, D, P, P]
             for fn in ("oracle_router_logits", "oracle_topk", "oracle_permute", "oracle_expert_ffn",
                        "oracle_combine", "oracle_forward_tokens", "oracle_num_threads", "oracle_version",
                        "oracle_mxfp4_quantize", "oracle_mxfp4_dequantize", "oracle_mxfp8_quantize",
                        "oracle_mxfp8_dequantize", "oracle_expert_ffn_mx", "oracle_qb_cutoffs", "oracle_qb_update",
                        "oracle_qb_histogram", "oracle_qb_bias_from_histogram", "oracle_qb_histogram_f32",
-                       "oracle_qb_quantile_bins"):
+                       "oracle_qb_quantile_bins", "oracle_glu_ffn", "oracle_rmsnorm", "oracle_latent_forward"):
                 getattr(lib, fn).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -377,3 +385,88 @@ def qb_quantile_bins(H, m_total: int, k: int) -> np.ndarray:
     _check(_load().oracle_qb_quantile_bins(H.ctypes.data, n, bins, m_total, k, out.ctypes.data),
            "oracle_qb_quantile_bins")
     return out
+
+
+# ------------------------------------------------------ Stable LatentMoE
+
+#: SiTU-GLU soft caps stated on the page (its bound is beta1 * beta2 = 100).
+SITU_BETA1 = 4.0
+SITU_BETA2 = 25.0
+ACT_SWIGLU, ACT_SITU = 0, 1
+
+
+def glu_ffn(x_rows, W_gu, W_d, act: int = ACT_SITU, beta1: float = SITU_BETA1, beta2: float = SITU_BETA2,
+            want_h: bool = False):
+    """One GLU feed-forward in fp64: x_rows [n, K] (anything numpy widens to
+    fp64, or a bf16 tensor), W_gu [K, 2F] and W_d [F, N] bf16. act
+    ACT_SWIGLU or ACT_SITU (SiTU-GLU with the given caps). Returns y [n, N]
+    (and h [n, F] with want_h). Definition and readings: oracle_glu_ffn and the
+    Stable LatentMoE notes in moe_oracle.cpp."""
+    try:
+        import torch
+        if isinstance(x_rows, torch.Tensor) and x_rows.dtype == torch.bfloat16:
+            x_rows = _bits_f64(_bf16_bits(x_rows))
+    except ImportError:  # pragma: no cover
+        pass
+    x = _f64c(x_rows)
+    n, K = x.shape
+    wg = _bf16_bits(W_gu)
+    wd = _bf16_bits(W_d)
+    assert wg.shape[0] == K and wg.shape[1] % 2 == 0, (wg.shape, K)
+    F = wg.shape[1] // 2
+    N = wd.shape[1]
+    assert wd.shape[0] == F, (wd.shape, F)
+    y = np.zeros((n, N), dtype=np.float64)
+    h = np.zeros((n, F), dtype=np.float64)
+    _check(_load().oracle_glu_ffn(x.ctypes.data if n else None, n, wg.ctypes.data, wd.ctypes.data, K, F, N, act,
+                                  float(beta1), float(beta2), y.ctypes.data, h.ctypes.data), "oracle_glu_ffn")
+    return (y, h) if want_h else y
+
+
+def rmsnorm(u, gamma=None, eps: float = 1e-6) -> np.ndarray:
+    """gamma * u / sqrt(mean(u^2) + eps) per row, fp64 [n, l]."""
+    u = _f64c(u)
+    n, l = u.shape
+    g = _f32(gamma) if gamma is not None else None
+    out = np.empty_like(u)
+    _check(_load().oracle_rmsnorm(u.ctypes.data if n else None, n, l, _ptr(g), float(eps), out.ctypes.data),
+           "oracle_rmsnorm")
+    return out
+
+
+def latent_forward(x, W_router, bias, W_dn, W_up, W_gate_up, W_down, gamma, Ws_gate_up, Ws_down, k: int,
+                   act: int = ACT_SITU, beta1: float = SITU_BETA1, beta2: float = SITU_BETA2, eps: float = 1e-6,
+                   want_u: bool = False):
+    """The Stable LatentMoE layer in fp64: out [T, d] (and the routed sum u
+    [T, l] before the RMSNorm with want_u). x [T, d] bf16; W_router [d, E] fp32;
+    bias [E] or None; W_dn [d, l], W_up [l, d]; routed W_gate_up [E, l, 2f],
+    W_down [E, f, l]; gamma [l] or None; shared Ws_gate_up [S, d, 2fs],
+    Ws_down [S, fs, d] (S may be 0, then both None). Definition and readings:
+    oracle_latent_forward in moe_oracle.cpp."""
+    xb = _bf16_bits(x)
+    T, d = xb.shape
+    Wr = _f32(W_router)
+    E = Wr.shape[1]
+    b = _f32(bias) if bias is not None else None
+    wdn = _bf16_bits(W_dn)
+    l = wdn.shape[1]
+    wup = _bf16_bits(W_up)
+    wgu = _bf16_bits(W_gate_up)
+    wd = _bf16_bits(W_down)
+    f = wd.shape[1]
+    assert wgu.shape == (E, l, 2 * f) and wd.shape == (E, f, l) and wup.shape == (l, d), (wgu.shape, wd.shape)
+    g = _f32(gamma) if gamma is not None else None
+    if Ws_gate_up is not None:
+        wsg = _bf16_bits(Ws_gate_up)
+        wsd = _bf16_bits(Ws_down)
+        S, fs = wsd.shape[0], wsd.shape[1]
+    else:
+        wsg = wsd = None
+        S, fs = 0, 0
+    out = np.zeros((T, d), dtype=np.float64)
+    u = np.zeros((T, l), dtype=np.float64)
+    _check(_load().oracle_latent_forward(xb.ctypes.data, Wr.ctypes.data, _ptr(b), wdn.ctypes.data, wup.ctypes.data,
+                                         wgu.ctypes.data, wd.ctypes.data, _ptr(g), _ptr(wsg), _ptr(wsd), T, d, l, E,
+                                         k, f, S, fs, act, float(beta1), float(beta2), float(eps), out.ctypes.data,
+                                         u.ctypes.data), "oracle_latent_forward")
+    return (out, u) if want_u else out

@@ -644,3 +644,154 @@ int oracle_qb_quantile_bins(const int64_t* H, int64_t n, int64_t B, int64_t m_to
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ Stable LatentMoE (next row)
+//
+// [P3] section "Operational Execution Flow": two full-width shared experts act
+// on x directly; the routed path projects x down to a latent z = x W_dn of
+// width l (3584 on the page); the k active routed experts act on z; their
+// probability-weighted sum u = sum_{i in top-k} p_i E_i(z) passes an explicit
+// RMSNorm and W_up brings it back to width d. The experts' GLU is SiTU-GLU
+// ("Sigmoid Tanh Unit GLU"), a soft-capped SwiGLU with beta1 = 4, beta2 = 25,
+// for which the page states |SiTU-GLU| <= beta1 beta2 = 100. The page's
+// formulas for SiTU-GLU and for the layer output did not survive. Readings:
+//   SiTU-GLU(g, v) = beta1 tanh(SiLU(g) / beta1) * beta2 tanh(v / beta2):
+//     SiLU's sigmoid, a tanh soft cap on each factor, so the product is
+//     bounded by beta1 beta2, and it equals SwiGLU's SiLU(g) v wherever
+//     |SiLU(g)| << beta1 and |v| << beta2 (SwiGLU's linear regime);
+//   out = sum_s S_s(x) + RMSNorm(u) W_up, RMSNorm(u) = gamma u / sqrt(mean(u^2) + eps);
+//   the router reads x (width d), as the plain layer's does; no biases.
+// SiTU-GLU's own formula is therefore parity-unpinned: what pins it is the
+// stated bound, its limit SwiGLU as beta1, beta2 -> infinity, and the layer's
+// reduction to the RMSNorm of the plain layer.
+
+namespace {
+
+inline double silu(double a) { return a / (1.0 + std::exp(-a)); }
+
+// act 0: SwiGLU SiLU(g) v; act 1: SiTU-GLU with caps b1, b2.
+inline double glu(double g, double v, int act, double b1, double b2) {
+  if (act == 0) return silu(g) * v;
+  return b1 * std::tanh(silu(g) / b1) * (b2 * std::tanh(v / b2));
+}
+
+}  // namespace
+
+extern "C" {
+
+// One GLU feed-forward on fp64 rows: x [n, K], W_gu [K, 2F] (columns 0..F-1
+// gate, F..2F-1 the second factor), W_d [F, N], bf16 weights; y [n, N] fp64;
+// h (optional) [n, F] the activation. act 0 SwiGLU, 1 SiTU-GLU (b1, b2).
+int oracle_glu_ffn(const double* x, int64_t n, const uint16_t* Wgu, const uint16_t* Wd, int64_t K, int64_t F,
+                   int64_t N, int act, double b1, double b2, double* y, double* h_out) {
+  if ((!x && n > 0) || !Wgu || !Wd || !y || n < 0 || K <= 0 || F <= 0 || N <= 0 || (act != 0 && act != 1))
+    return 1;
+  if (act == 1 && !(b1 > 0.0 && b2 > 0.0)) return 1;
+  const int64_t F2 = 2 * F;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n; ++r) {
+    std::vector<double> gv(F2, 0.0), h(F), yy(N, 0.0);
+    for (int64_t i = 0; i < K; ++i) {
+      const double xi = x[r * K + i];
+      for (int64_t j = 0; j < F2; ++j) gv[j] += xi * bf16_to_double(Wgu[i * F2 + j]);
+    }
+    for (int64_t j = 0; j < F; ++j) h[j] = glu(gv[j], gv[F + j], act, b1, b2);
+    for (int64_t j = 0; j < F; ++j)
+      for (int64_t c = 0; c < N; ++c) yy[c] += h[j] * bf16_to_double(Wd[j * N + c]);
+    for (int64_t c = 0; c < N; ++c) y[r * N + c] = yy[c];
+    if (h_out)
+      for (int64_t j = 0; j < F; ++j) h_out[r * F + j] = h[j];
+  }
+  return 0;
+}
+
+// RMSNorm of each row: out = gamma * u / sqrt(mean(u^2) + eps); gamma [l]
+// fp32 or NULL (ones). u, out [n, l] fp64 (may alias).
+int oracle_rmsnorm(const double* u, int64_t n, int64_t l, const float* gamma, double eps, double* out) {
+  if ((!u && n > 0) || !out || n < 0 || l <= 0 || !(eps >= 0.0)) return 1;
+  for (int64_t r = 0; r < n; ++r) {
+    double ss = 0.0;
+    for (int64_t c = 0; c < l; ++c) ss += u[r * l + c] * u[r * l + c];
+    const double den = std::sqrt(ss / static_cast<double>(l) + eps);
+    for (int64_t c = 0; c < l; ++c)
+      out[r * l + c] = (gamma ? static_cast<double>(gamma[c]) : 1.0) * (den > 0.0 ? u[r * l + c] / den : 0.0);
+  }
+  return 0;
+}
+
+// The Stable LatentMoE layer for T tokens (readings above). x [T, d] bf16;
+// W_router [d, E] fp32, bias [E] or NULL; W_dn [d, l] and W_up [l, d] bf16;
+// routed experts W_gu [E, l, 2f], W_d [E, f, l] bf16; gamma [l] fp32 or NULL;
+// shared experts Ws_gu [S, d, 2fs], Ws_d [S, fs, d] bf16 (S may be 0); act,
+// b1, b2 the experts' GLU; eps the RMSNorm's. out [T, d] fp64; u_out
+// (optional) [T, l] the routed sum before the RMSNorm.
+int oracle_latent_forward(const uint16_t* x, const float* Wr, const float* bias, const uint16_t* Wdn,
+                          const uint16_t* Wup, const uint16_t* Wgu, const uint16_t* Wd, const float* gamma,
+                          const uint16_t* Wsgu, const uint16_t* Wsd, int64_t T, int64_t d, int64_t l, int64_t E,
+                          int64_t k, int64_t f, int64_t S, int64_t fs, int act, double b1, double b2, double eps,
+                          double* out, double* u_out) {
+  if (!x || !Wr || !Wdn || !Wup || !Wgu || !Wd || !out || T < 0 || d <= 0 || l <= 0 || E <= 0 || k <= 0 || k > E ||
+      f <= 0 || S < 0 || (S > 0 && (!Wsgu || !Wsd || fs <= 0)))
+    return 1;
+  // 1-3. route on x
+  std::vector<float> logits(T * E);
+  int st = oracle_router_logits(x, Wr, bias, T, d, E, logits.data());
+  if (st) return st;
+  std::vector<int32_t> idx(T * k);
+  std::vector<double> w(T * k);
+  st = oracle_topk(logits.data(), T, E, k, idx.data(), w.data(), nullptr);
+  if (st) return st;
+  // z = x W_dn (fp64)
+  std::vector<double> xd(T * d), z(T * l, 0.0);
+  for (int64_t q = 0; q < T * d; ++q) xd[q] = bf16_to_double(x[q]);
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t i = 0; i < d; ++i) {
+      const double xi = xd[t * d + i];
+      for (int64_t c = 0; c < l; ++c) z[t * l + c] += xi * bf16_to_double(Wdn[i * l + c]);
+    }
+  // routed experts on z, rows grouped by expert; u = sum_j p_j E_j(z) in slot order
+  std::vector<int32_t> counts(E), offsets(E + 1), perm(T * k), inv(T * k);
+  st = oracle_permute(idx.data(), T, E, k, counts.data(), offsets.data(), perm.data(), inv.data());
+  if (st) return st;
+  std::vector<double> y(T * k * l);
+  for (int64_t e = 0; e < E; ++e) {
+    const int64_t n = counts[e];
+    if (n == 0) continue;
+    std::vector<double> rows(n * l);
+    for (int64_t r = 0; r < n; ++r)
+      std::memcpy(&rows[r * l], &z[static_cast<int64_t>(perm[offsets[e] + r]) * l], sizeof(double) * l);
+    st = oracle_glu_ffn(rows.data(), n, Wgu + e * l * 2 * f, Wd + e * f * l, l, f, l, act, b1, b2,
+                        &y[static_cast<int64_t>(offsets[e]) * l], nullptr);
+    if (st) return st;
+  }
+  std::vector<double> u(T * l, 0.0);
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t j = 0; j < k; ++j) {
+      const double* yr = &y[static_cast<int64_t>(inv[t * k + j]) * l];
+      for (int64_t c = 0; c < l; ++c) u[t * l + c] += w[t * k + j] * yr[c];
+    }
+  if (u_out) std::memcpy(u_out, u.data(), sizeof(double) * T * l);
+  // RMSNorm, then W_up back to width d
+  std::vector<double> un(T * l);
+  st = oracle_rmsnorm(u.data(), T, l, gamma, eps, un.data());
+  if (st) return st;
+  for (int64_t q = 0; q < T * d; ++q) out[q] = 0.0;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t c = 0; c < l; ++c) {
+      const double v = un[t * l + c];
+      for (int64_t o = 0; o < d; ++o) out[t * d + o] += v * bf16_to_double(Wup[c * d + o]);
+    }
+  // shared experts on x, added after
+  std::vector<double> ys(T * d);
+  for (int64_t s = 0; s < S; ++s) {
+    st = oracle_glu_ffn(xd.data(), T, Wsgu + s * d * 2 * fs, Wsd + s * fs * d, d, fs, d, act, b1, b2, ys.data(),
+                        nullptr);
+    if (st) return st;
+    for (int64_t q = 0; q < T * d; ++q) out[q] += ys[q];
+  }
+  return 0;
+}
+
+}  // extern "C"

@@ -58,6 +58,16 @@ MUTATIONS = {
     "qb_bias_sign": ("b_new[j] = -mu[r - 1];", "b_new[j] = mu[r - 1];"),
     "qb_histogram_upper_edge": ("b_new[j] = -(lo + static_cast<double>(bin) * width);",
                                 "b_new[j] = -(lo + static_cast<double>(bin + 1) * width);"),
+    "situ_cap_ignored": ("if (act == 0) return silu(g) * v;", "if (act >= 0) return silu(g) * v;"),
+    "situ_gate_without_sigmoid": ("return b1 * std::tanh(silu(g) / b1) * (b2 * std::tanh(v / b2));",
+                                  "return b1 * std::tanh(g / b1) * (b2 * std::tanh(v / b2));"),
+    "rmsnorm_without_sqrt": ("const double den = std::sqrt(ss / static_cast<double>(l) + eps);",
+                             "const double den = ss / static_cast<double>(l) + eps;"),
+    "latent_down_projection_shifted": ("z[t * l + c] += xi * bf16_to_double(Wdn[i * l + c]);",
+                                       "z[t * l + c] += xi * bf16_to_double(Wdn[((i + 1) % d) * l + c]);"),
+    "latent_combine_unweighted": ("u[t * l + c] += w[t * k + j] * yr[c];", "u[t * l + c] += yr[c];"),
+    "latent_shared_experts_dropped": ("for (int64_t q = 0; q < T * d; ++q) out[q] += ys[q];",
+                                      "for (int64_t q = 0; q < T * d; ++q) out[q] += 0.0 * ys[q];"),
 }
 
 

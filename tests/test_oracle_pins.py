@@ -633,3 +633,124 @@ def test_qb_quantile_bins_are_the_bias_bins():
     r = -(-m * k // n)
     for j in range(n):
         assert H[j, bins[j]:].sum() >= r and H[j, bins[j] + 1:].sum() < r
+
+
+# ------------------------------------------------------------ Stable LatentMoE
+# "Kimi K3: Open Frontier Intelligence", section "Operational Execution Flow":
+# shared experts on x, routed experts on a latent z = x W_dn, RMSNorm of the
+# routed sum, W_up back to width d; SiTU-GLU with beta1 = 4, beta2 = 25 and
+# |SiTU-GLU| <= 100. The page lost SiTU-GLU's formula (parity unpinned beyond
+# what follows): pinned are the stated bound, the SwiGLU limit of large caps,
+# RMSNorm's invariants, and the layer's reductions to the plain layer.
+
+def _bf(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+def test_glu_ffn_swiglu_matches_expert_ffn_and_numpy():
+    g = torch.Generator().manual_seed(21)
+    n, K, F = 5, 96, 40
+    x = torch.randn(n, K, generator=g).to(torch.bfloat16)
+    Wgu = (torch.randn(K, 2 * F, generator=g) / K ** 0.5).to(torch.bfloat16)
+    Wd = (torch.randn(F, K, generator=g) / F ** 0.5).to(torch.bfloat16)
+    y = oracle.glu_ffn(x, Wgu, Wd, act=oracle.ACT_SWIGLU)
+    assert np.array_equal(y, oracle.expert_ffn(x, Wgu, Wd))          # the pinned step 5, same arithmetic
+    xd, wg, wd = (t.to(torch.float64).numpy() for t in (x, Wgu, Wd))
+    gu = xd @ wg
+    ref = (gu[:, :F] / (1 + np.exp(-gu[:, :F])) * gu[:, F:]) @ wd
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_situ_glu_bound_and_swiglu_limit():
+    g = torch.Generator().manual_seed(22)
+    n, K, F, N = 64, 32, 48, 16
+    x = (torch.randn(n, K, generator=g, dtype=torch.float64) * 40.0).numpy()    # far past both caps
+    Wgu = (torch.randn(K, 2 * F, generator=g) * 3.0).to(torch.bfloat16)
+    Wd = torch.eye(F, N).to(torch.bfloat16)
+    _, h = oracle.glu_ffn(x, Wgu, Wd, act=oracle.ACT_SITU, want_h=True)
+    assert np.abs(h).max() <= oracle.SITU_BETA1 * oracle.SITU_BETA2           # the stated bound, 100
+    assert np.abs(h).max() > 0.99 * 100.0                                       # and it is reached
+    # huge caps: SiTU-GLU is SwiGLU (beta tanh(v / beta) -> v)
+    x2 = torch.randn(n, K, generator=g, dtype=torch.float64).numpy()
+    big = 1e150
+    y_s = oracle.glu_ffn(x2, Wgu, Wd, act=oracle.ACT_SITU, beta1=big, beta2=big)
+    y_w = oracle.glu_ffn(x2, Wgu, Wd, act=oracle.ACT_SWIGLU)
+    np.testing.assert_allclose(y_s, y_w, rtol=1e-12, atol=1e-300)
+    # zero gate row or zero second factor: exactly zero; sign follows SiLU(g) * v
+    x0 = np.zeros((1, K))
+    assert not np.any(oracle.glu_ffn(x0, Wgu, Wd, act=oracle.ACT_SITU))
+    _, hs = oracle.glu_ffn(x2, Wgu, Wd, act=oracle.ACT_SITU, want_h=True)
+    _, hw = oracle.glu_ffn(x2, Wgu, Wd, act=oracle.ACT_SWIGLU, want_h=True)
+    assert np.array_equal(np.sign(hs), np.sign(hw))
+    assert np.all(np.abs(hs) <= np.abs(hw) + 1e-15)                           # a cap never enlarges
+
+
+def test_rmsnorm_invariants():
+    rng = np.random.default_rng(23)
+    u = rng.normal(size=(6, 40)) * rng.uniform(0.1, 10, size=(6, 1))
+    r = oracle.rmsnorm(u, eps=0.0)
+    np.testing.assert_allclose((r ** 2).mean(axis=1), 1.0, rtol=1e-12)       # unit RMS
+    np.testing.assert_allclose(oracle.rmsnorm(7.25 * u, eps=0.0), r, rtol=1e-12)  # scale invariant
+    assert np.array_equal(np.sign(r), np.sign(u))
+    gamma = rng.uniform(0.5, 2.0, size=40).astype(np.float32)
+    np.testing.assert_allclose(oracle.rmsnorm(u, gamma, eps=0.0), r * gamma.astype(np.float64), rtol=1e-12)
+    assert not np.any(oracle.rmsnorm(np.zeros((2, 40)), eps=1e-6))            # zero row stays zero
+    # eps: the denominator is sqrt(mean(u^2) + eps), so a row of RMS s shrinks by s / sqrt(s^2 + eps)
+    s = np.sqrt((u[0] ** 2).mean())
+    np.testing.assert_allclose(oracle.rmsnorm(u[:1], eps=0.5), r[:1] * s / np.sqrt(s * s + 0.5), rtol=1e-12)
+
+
+def _latent_inputs(T, d, l, E, k, f, S, fs, seed, bias=None):
+    shape = moe_inputs.custom_shape(T, d, E, k, f, bias=bias)
+    inp = moe_inputs.make_inputs(shape, seed=seed)
+    g = torch.Generator().manual_seed(seed + 100)
+    Wdn = (torch.randn(d, l, generator=g) / d ** 0.5).to(torch.bfloat16)
+    Wup = (torch.randn(l, d, generator=g) / l ** 0.5).to(torch.bfloat16)
+    Wgu = (torch.randn(E, l, 2 * f, generator=g) / l ** 0.5).to(torch.bfloat16)
+    Wd = (torch.randn(E, f, l, generator=g) / f ** 0.5).to(torch.bfloat16)
+    Wsg = (torch.randn(S, d, 2 * fs, generator=g) / d ** 0.5).to(torch.bfloat16) if S else None
+    Wsd = (torch.randn(S, fs, d, generator=g) / fs ** 0.5).to(torch.bfloat16) if S else None
+    return inp, Wdn, Wup, Wgu, Wd, Wsg, Wsd
+
+
+def test_latent_layer_with_identity_projections_is_rmsnorm_of_the_plain_layer():
+    T, d, E, k, f = 40, 64, 8, 3, 32
+    inp, *_ = _latent_inputs(T, d, d, E, k, f, 0, 0, seed=24, bias="zipf")
+    eye = torch.eye(d).to(torch.bfloat16)
+    out, u = oracle.latent_forward(inp.x, inp.W_router, inp.bias, eye, eye, inp.W_gate_up, inp.W_down, None,
+                                   None, None, k, act=oracle.ACT_SWIGLU, eps=0.0, want_u=True)
+    plain, _, _ = oracle.forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    np.testing.assert_allclose(u, plain, rtol=1e-12, atol=1e-14)              # the routed sum is the plain layer
+    np.testing.assert_allclose(out, oracle.rmsnorm(plain, eps=0.0), rtol=1e-12, atol=1e-14)
+
+
+def test_latent_layer_against_numpy_composition():
+    """Projection, dispatch, combine, RMSNorm, W_up and the shared experts'
+    sum, composed in numpy around the pinned pieces (router, top-k, GLU)."""
+    T, d, l, E, k, f, S, fs = 33, 64, 48, 6, 2, 32, 2, 40
+    inp, Wdn, Wup, Wgu, Wd, Wsg, Wsd = _latent_inputs(T, d, l, E, k, f, S, fs, seed=25)
+    gamma = np.linspace(0.5, 1.5, l).astype(np.float32)
+    out = oracle.latent_forward(inp.x, inp.W_router, None, Wdn, Wup, Wgu, Wd, gamma, Wsg, Wsd, k)
+    x = inp.x.to(torch.float64).numpy()
+    lg = oracle.router_logits(inp.x, inp.W_router, None)
+    idx, w = oracle.topk(lg, k)
+    z = x @ Wdn.to(torch.float64).numpy()
+    u = np.zeros((T, l))
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            u[t] += w[t, j] * oracle.glu_ffn(z[t:t + 1], Wgu[e], Wd[e])[0]
+    un = u / np.sqrt((u ** 2).mean(axis=1, keepdims=True) + 1e-6) * gamma.astype(np.float64)
+    ref = un @ Wup.to(torch.float64).numpy()
+    for s in range(S):
+        ref += oracle.glu_ffn(x, Wsg[s], Wsd[s])
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_latent_layer_with_silent_routed_experts_is_the_shared_experts():
+    T, d, l, E, k, f, S, fs = 20, 64, 32, 4, 2, 32, 2, 48
+    inp, Wdn, Wup, Wgu, Wd, Wsg, Wsd = _latent_inputs(T, d, l, E, k, f, S, fs, seed=26)
+    out = oracle.latent_forward(inp.x, inp.W_router, None, Wdn, Wup, torch.zeros_like(Wgu), Wd, None, Wsg, Wsd, k,
+                                act=oracle.ACT_SWIGLU)
+    ref = sum(oracle.expert_ffn(inp.x, Wsg[s], Wsd[s]) for s in range(S))   # pinned step 5 per shared expert
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
