@@ -373,6 +373,8 @@ moe_status_t moe_gather_rows(const moe_bf16_t* src, int64_t n_src, const int32_t
 #define MOE_DEVERR_SELFTEST_TIMEOUT 4u      /* moe_selftest_wait_timeout fired as intended */
 #define MOE_DEVERR_BAD_ROUTE 5u             /* an expert index outside [0, E) reached the dispatch */
 #define MOE_DEVERR_WAIT_TIMEOUT_ROUTER 6u   /* few-token router gave up waiting for its W tile */
+#define MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY 7u /* one-launch feed-forward gave up waiting for an expert's h rows */
+#define MOE_DEVERR_INDEX_CHECK 8u           /* index-checking build only: a row or expert offset out of range, skipped */
 moe_status_t moe_get_device_error(uint32_t* code, int clear);
 
 /* moe_selftest_wait_timeout: launches one tiny kernel that waits, with a

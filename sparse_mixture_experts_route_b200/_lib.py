@@ -5,6 +5,8 @@ contiguity, their ``data_ptr()`` and torch's current CUDA stream are passed to
 the C entry point of the same name, and a non-OK status raises ``MoEError``.
 Every step of the layer runs in the library's kernels. Importing this module
 loads the library and raises if it is missing: there is no fallback.
+MOE_LIBRARY=checks in the environment loads the index-checking build
+``libmoe_checks.so`` instead (same entry points, see build.py).
 """
 from __future__ import annotations
 
@@ -15,10 +17,14 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+_VARIANT = os.environ.get("MOE_LIBRARY", "")
+if _VARIANT not in ("", "checks"):
+    raise ImportError(f"MOE_LIBRARY={_VARIANT!r}: expected 'checks' or unset")
+LIB_PATH = os.path.join(_HERE, "libmoe_checks.so" if _VARIANT == "checks" else "libmoe.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run python -m sparse_mixture_experts_route_b200.build")
+    raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
+                      f"python -m sparse_mixture_experts_route_b200.build{' --checks' if _VARIANT else ''}")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -59,6 +65,9 @@ for _name, (_args, _res) in EXPORTS.items():
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
 DEVERR_SELFTEST_TIMEOUT = 4
+DEVERR_BAD_ROUTE = 5
+DEVERR_WAIT_TIMEOUT_DEPENDENCY = 7
+DEVERR_INDEX_CHECK = 8  # index-checking build only
 
 
 class MoEError(RuntimeError):

@@ -13,6 +13,23 @@ __device__ unsigned int g_device_error = 0u;
 
 __device__ __forceinline__ void record_device_error(unsigned int code) { atomicCAS(&g_device_error, 0u, code); }
 
+// The MOE_CHECKS build (libmoe_checks.so) checks every data-dependent index
+// before it is used -- rows read or written through a permutation, expert
+// offsets handed to the GEMMs -- and on a bad one records
+// MOE_DEVERR_INDEX_CHECK (8) and skips the access instead of faulting. In the
+// normal build the checks are constant true and compile away.
+#ifdef MOE_CHECKS
+constexpr bool kIndexChecks = true;
+#else
+constexpr bool kIndexChecks = false;
+#endif
+
+__device__ __forceinline__ bool index_ok(bool ok) {
+  if (!kIndexChecks) return true;
+  if (!ok) record_device_error(8u /* MOE_DEVERR_INDEX_CHECK */);
+  return ok;
+}
+
 // Bounded waits give up after this long. A healthy pipeline stage waits
 // microseconds; the limit only ends waits that can no longer complete.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s

@@ -97,6 +97,13 @@ struct GemmParams {
   // CTA order, which is ascending K, and finishes the tile. tickets[] start at
   // zero and are put back to zero.
   int stream_k;
+  // Whole-tile scheduling takes the tiles in the order 0, n-1, 1, n-2, ...
+  // instead of 0, 1, 2, ... (interleave != 0). Tiles are expert-major, so
+  // when a few experts hold most rows (compute-bound tiles at the front) and
+  // many hold few (weight-streaming tiles at the back) every wave mixes both;
+  // a heavy expert's consecutive tiles still run in the same wave and share
+  // its weight tile in L2. Results do not depend on the order.
+  int interleave;
   int b_fixed_row;        // >= 0: every tile's token operand starts at this row (one-token steps read x itself)
   float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
   unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
@@ -154,8 +161,9 @@ __device__ __forceinline__ bool work_item(const GemmParams& p, const int32_t* pr
   const int KB = p.K / kGemmBK;
   const int ntiles = pre[p.E] * p.n_feat_tiles;
   if (!p.stream_k) {
-    const int t = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
-    if (t >= ntiles) return false;
+    const int u = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+    if (u >= ntiles) return false;
+    const int t = p.interleave ? ((u & 1) ? ntiles - 1 - (u >> 1) : (u >> 1)) : u;
     decode_tile<kMode>(p, pre, off, t, ti);
     ti.kb0 = 0;
     ti.kb1 = KB;
@@ -199,6 +207,242 @@ __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
   const __nv_bfloat16 b = __float2bfloat16_rn(v);
   return *reinterpret_cast<const uint16_t*>(&b);
+}
+
+// ------------------------------------------------------- pipeline pieces
+// One K block of a work item: both A operands (four 64-feature boxes), then the
+// token rows (one small box, or one to two 128-row boxes), into stage `st`,
+// completing on `bar`.
+
+template <int kMode>
+__device__ __forceinline__ uint32_t gemm_b_bytes(const TileInfo& ti) {
+  if (ti.nrows <= kGemmSmallBox) return kGemmSmallBox * kGemmBK * 2;
+  return static_cast<uint32_t>((ti.nrows + kGemmBoxRows - 1) / kGemmBoxRows) * kGemmBoxRows * kGemmBK * 2;
+}
+
+template <int kMode>
+__device__ __forceinline__ void gemm_load_a(uint8_t* st, const CUtensorMap* tmA, uint64_t* bar, const GemmParams& p,
+                                            const TileInfo& ti, int k0, uint64_t pol_w) {
+  using Cfg = GemmCfg<kMode>;
+  const int f0 = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF);
+  const int f1 = f0 + p.a1_offset;
+  tma_load_3d(st, tmA, bar, f0, k0, ti.e, pol_w);
+  tma_load_3d(st + Cfg::kAHalf, tmA, bar, f0 + 64, k0, ti.e, pol_w);
+  tma_load_3d(st + Cfg::kABytes, tmA, bar, f1, k0, ti.e, pol_w);
+  tma_load_3d(st + Cfg::kABytes + Cfg::kAHalf, tmA, bar, f1 + 64, k0, ti.e, pol_w);
+}
+
+template <int kMode>
+__device__ __forceinline__ void gemm_load_b(uint8_t* st, const CUtensorMap* tmB, const CUtensorMap* tmBs,
+                                            uint64_t* bar, const GemmParams& p, int row0, int nrows, int k0,
+                                            uint64_t pol_x) {
+  using Cfg = GemmCfg<kMode>;
+  uint8_t* bdst = st + 2 * Cfg::kABytes;
+  if (nrows <= kGemmSmallBox) {
+    tma_load_2d(bdst, tmBs, bar, k0, p.b_fixed_row >= 0 ? p.b_fixed_row : row0, pol_x);
+  } else {
+    const int nbox = (nrows + kGemmBoxRows - 1) / kGemmBoxRows;
+    for (int b = 0; b < nbox; ++b)
+      tma_load_2d(bdst + b * kGemmBoxRows * kGemmBK * 2, tmB, bar, k0, row0 + b * kGemmBoxRows, pol_x);
+  }
+}
+
+// The shared-memory ring and TMEM state of one CTA's pipeline.
+struct GemmRing {
+  uint8_t* smem;
+  uint64_t* full_bar;
+  uint64_t* empty_bar;
+  uint64_t* acc_full_bar;   // [2] one per TMEM slot
+  uint64_t* acc_empty_bar;  // [2]
+  volatile int* abort_flag;
+  uint32_t tmem_base;
+};
+
+// MMA issuer, one work item: waits for its TMEM slot(s) to be free, then for
+// each K block for the stage to be full, issues the stage's MMAs (two A
+// operands into two accumulators) and frees the stage; finally marks the
+// accumulators complete. Returns false if a wait gave up.
+template <int kMode>
+__device__ __forceinline__ bool gemm_mma_item(const GemmRing& r, const TileInfo& ti, int& s, uint32_t& ph,
+                                              uint32_t (&uses)[2], int& next_slot, bool& any) {
+  using Cfg = GemmCfg<kMode>;
+  constexpr int S = Cfg::kStages;
+  const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
+  const uint32_t idesc = umma_idesc_bf16_f32(128u, n_mma, 1u, 0u);
+  const SlotPlan sp = slot_plan(ti.nrows, next_slot);
+  for (int j = 0; j < sp.count; ++j) {
+    const int sl = sp.first + j;
+    if (!mbar_wait_bounded(&r.acc_empty_bar[sl], (uses[sl] & 1u) ^ 1u, kWaitLimitNs, r.abort_flag)) {
+      record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+      *r.abort_flag = 1;
+      return false;
+    }
+  }
+  tc_fence_after_sync();
+  // accumulator 0 at the slot start; accumulator 1 after N columns (128 or 256)
+  const uint32_t d0 = r.tmem_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
+  const uint32_t d1 = d0 + (sp.count == 2 ? 256u : 128u);
+  for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+    if (!mbar_wait_bounded(&r.full_bar[s], ph, kWaitLimitNs, r.abort_flag)) {
+      record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+      *r.abort_flag = 1;
+      return false;
+    }
+    tc_fence_after_sync();
+    const uint32_t a_addr = smem_u32(r.smem + s * Cfg::kStageBytes);
+    const uint32_t b_addr = a_addr + 2 * Cfg::kABytes;
+#pragma unroll
+    for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+      const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+      const uint64_t adesc0 = umma_smem_desc_sw128(a_addr + kk * 2048, Cfg::kAHalf, 1024);
+      const uint64_t adesc1 = umma_smem_desc_sw128(a_addr + Cfg::kABytes + kk * 2048, Cfg::kAHalf, 1024);
+      const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
+      tc_mma_bf16(d0, adesc0, bdesc, idesc, accum);
+      tc_mma_bf16(d1, adesc1, bdesc, idesc, accum);
+    }
+    tc_commit(&r.empty_bar[s]);  // stage s is free once these MMAs have read it
+    any = true;
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  for (int j = 0; j < sp.count; ++j) {
+    tc_commit(&r.acc_full_bar[sp.first + j]);  // accumulators complete
+    ++uses[sp.first + j];
+  }
+  return true;
+}
+
+// One count per (gate/up tile, epilogue warp) once that warp's 32-feature
+// slice of h is stored, published with release semantics for a CTA that will
+// read h with TMA loads (the fused one-launch feed-forward below).
+__device__ __forceinline__ void signal_h_slice(unsigned int* ready, int e, int lane) {
+  fence_proxy_async_global();
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(ready + e, 1u);
+}
+
+// Epilogue warp q (TMEM lanes 32q..32q+31 = features), one work item: waits
+// for the accumulators, then either stores the finished rows (mode 0/2: h =
+// SiLU(g) * u; mode 1: the two 128-feature halves of y), or, for a stream-K
+// partial item, writes its fp32 partials and, if it is the last of the tile's
+// contributors, adds them in K order and stores the rows. With kSignal, a
+// finished gate/up slice is counted in ready[e]. Returns false if a wait gave up.
+template <int kMode, bool kSignal>
+__device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const GemmParams& p, const int32_t* pre,
+                                                   const TileInfo& ti, int q, int lane, uint32_t (&uses)[2],
+                                                   int& next_slot, unsigned int* ready) {
+  const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+  const SlotPlan sp = slot_plan(ti.nrows, next_slot);
+  for (int j = 0; j < sp.count; ++j) {
+    const int sl = sp.first + j;
+    if (!mbar_wait_bounded(&r.acc_full_bar[sl], uses[sl] & 1u, kWaitLimitNs, r.abort_flag)) {
+      record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
+      *r.abort_flag = 1;
+      return false;
+    }
+  }
+  tc_fence_after_sync();
+  const uint32_t t0 = r.tmem_base + lane_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
+  const uint32_t t1 = t0 + (sp.count == 2 ? 256u : 128u);
+  const int fa = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF) + q * 32 + lane;
+  const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
+  const bool fa_ok = fa < p.n_feat;
+  const bool fb_ok = !gemm_is_gate_up(kMode) && fb < p.n_feat;
+  if (kMode != 0 && ti.partial) {
+    // stream-K partial item: fp32 accumulators to part[slot]; the TMEM
+    // slot is free as soon as it is read
+    const int fl = q * 32 + lane;
+    float* mine = p.part + static_cast<int64_t>(ti.slot) * kSplitPartFloats;
+    for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+      uint32_t g[32], u[32];
+      tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
+      tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
+      tmem_ld_wait();
+      const int nv = min(32, ti.nrows - c0);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (i < nv) {
+          __stcg(mine + (c0 + i) * kGemmBMF + fl, __uint_as_float(g[i]));
+          __stcg(mine + (128 + c0 + i) * kGemmBMF + fl, __uint_as_float(u[i]));
+        }
+      }
+    }
+    tc_fence_before_sync();
+    __syncwarp();
+    for (int j = 0; j < sp.count; ++j) {
+      if (lane == 0) mbar_arrive(&r.acc_empty_bar[sp.first + j]);
+      ++uses[sp.first + j];
+    }
+    // the tile's contributors are CTAs c_first..c_last; per (tile, warp),
+    // the last one to finish adds their partials in CTA order (K order)
+    const int KB = p.K / kGemmBK;
+    const int per = stream_k_per(pre[p.E] * p.n_feat_tiles, KB);
+    const int c_first = (ti.t * KB) / per, c_last = ((ti.t + 1) * KB - 1) / per;
+    __threadfence();
+    __syncwarp();
+    unsigned int tk = 0u;
+    if (lane == 0) tk = atomicAdd(&p.tickets[ti.t * 4 + q], 1u);
+    tk = __shfl_sync(0xffffffffu, tk, 0);
+    if (tk == static_cast<unsigned int>(c_last - c_first)) {
+      __threadfence();
+      for (int i = 0; i < ti.nrows; ++i) {
+        float gs = 0.0f, us = 0.0f;
+        for (int c = c_first; c <= c_last; ++c) {
+          const int slot = 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
+          const float* src = p.part + static_cast<int64_t>(slot) * kSplitPartFloats;
+          const float gv = __ldcg(src + i * kGemmBMF + fl);
+          const float uv = __ldcg(src + (128 + i) * kGemmBMF + fl);
+          gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
+          us = (c == c_first) ? uv : __fadd_rn(us, uv);
+        }
+        uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
+        if (gemm_is_gate_up(kMode)) {
+          if (fa_ok) orow[fa] = bf16_bits(silu_f32(gs) * us);
+        } else {
+          if (fa_ok) orow[fa] = bf16_bits(gs);
+          if (fb_ok) orow[fb] = bf16_bits(us);
+        }
+      }
+      if (lane == 0) p.tickets[ti.t * 4 + q] = 0u;
+      if (kSignal) signal_h_slice(ready, ti.e, lane);
+    }
+    return true;
+  }
+  for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+    uint32_t g[32], u[32];
+    tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
+    tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
+    tmem_ld_wait();
+    uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + c0) * p.n_feat;
+    const int nv = min(32, ti.nrows - c0);
+    if (gemm_is_gate_up(kMode)) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (fa_ok && i < nv)
+          orow[static_cast<int64_t>(i) * p.n_feat + fa] =
+              bf16_bits(silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (i < nv) {
+          if (fa_ok) orow[static_cast<int64_t>(i) * p.n_feat + fa] = bf16_bits(__uint_as_float(g[i]));
+          if (fb_ok) orow[static_cast<int64_t>(i) * p.n_feat + fb] = bf16_bits(__uint_as_float(u[i]));
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncwarp();
+  for (int j = 0; j < sp.count; ++j) {
+    if (lane == 0) mbar_arrive(&r.acc_empty_bar[sp.first + j]);
+    ++uses[sp.first + j];
+  }
+  if (kSignal) signal_h_slice(ready, ti.e, lane);
+  return true;
 }
 
 template <int kMode>
@@ -252,7 +496,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem_base = *tmem_slot;
+  const GemmRing ring{smem, full_bar, empty_bar, acc_full_bar, acc_empty_bar, abort_flag, *tmem_slot};
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -268,12 +512,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       TileInfo ti;
       for (int it = 0; ok && work_item<kMode>(p, s_pre, s_off, it, ti); ++it) {
-        const int f0 = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF);
-        const int f1 = f0 + p.a1_offset;
         const uint64_t pol_w = (ti.nblocks == 1) ? pol_w_once : pol_w_shared;
-        const bool small_box = ti.nrows <= kGemmSmallBox;
-        const int nbox = small_box ? 1 : (ti.nrows + kGemmBoxRows - 1) / kGemmBoxRows;
-        const uint32_t b_bytes = small_box ? kGemmSmallBox * kGemmBK * 2 : nbox * kGemmBoxRows * kGemmBK * 2;
+        const uint32_t tx = 2 * Cfg::kABytes + gemm_b_bytes<kMode>(ti);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
@@ -282,20 +522,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           uint8_t* st = smem + s * Cfg::kStageBytes;
-          mbar_arrive_expect_tx(&full_bar[s], 2 * Cfg::kABytes + b_bytes);
+          mbar_arrive_expect_tx(&full_bar[s], tx);
           const int k0 = kb * kGemmBK;
-          tma_load_3d(st, &tmA, &full_bar[s], f0, k0, ti.e, pol_w);
-          tma_load_3d(st + Cfg::kAHalf, &tmA, &full_bar[s], f0 + 64, k0, ti.e, pol_w);
-          tma_load_3d(st + Cfg::kABytes, &tmA, &full_bar[s], f1, k0, ti.e, pol_w);
-          tma_load_3d(st + Cfg::kABytes + Cfg::kAHalf, &tmA, &full_bar[s], f1 + 64, k0, ti.e, pol_w);
-          uint8_t* bdst = st + 2 * Cfg::kABytes;
-          if (small_box) {
-            tma_load_2d(bdst, &tmBs, &full_bar[s], k0, p.b_fixed_row >= 0 ? p.b_fixed_row : ti.row0, pol_x);
-          } else {
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d(bdst + b * kGemmBoxRows * kGemmBK * 2, &tmB, &full_bar[s], k0, ti.row0 + b * kGemmBoxRows,
-                          pol_x);
-          }
+          gemm_load_a<kMode>(st, &tmA, &full_bar[s], p, ti, k0, pol_w);
+          gemm_load_b<kMode>(st, &tmB, &tmBs, &full_bar[s], p, ti.row0, ti.nrows, k0, pol_x);
           ++issued;
           if (++s == S) {
             s = 0;
@@ -319,58 +549,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ph = 0;
       uint32_t uses[2] = {0u, 0u};  // completed uses of each TMEM slot
       int next_slot = 0;
-      bool ok = true;
       bool any = false;
       TileInfo ti;
-      for (int it = 0; ok && work_item<kMode>(p, s_pre, s_off, it, ti); ++it) {
-        const uint32_t n_mma = static_cast<uint32_t>(max(16, (ti.nrows + 15) & ~15));
-        const uint32_t idesc = umma_idesc_bf16_f32(128u, n_mma, 1u, 0u);
-        const SlotPlan sp = slot_plan(ti.nrows, next_slot);
-        for (int j = 0; j < sp.count && ok; ++j) {
-          const int sl = sp.first + j;
-          if (!mbar_wait_bounded(&acc_empty_bar[sl], (uses[sl] & 1u) ^ 1u, kWaitLimitNs, abort_flag)) {
-            record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
-            *abort_flag = 1;
-            ok = false;
-          }
-        }
-        if (!ok) break;
-        tc_fence_after_sync();
-        // accumulator 0 at the slot start; accumulator 1 after N columns (128 or 256)
-        const uint32_t d0 = tmem_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
-        const uint32_t d1 = d0 + (sp.count == 2 ? 256u : 128u);
-        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
-          if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
-            record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(smem + s * Cfg::kStageBytes);
-          const uint32_t b_addr = a_addr + 2 * Cfg::kABytes;
-#pragma unroll
-          for (int kk = 0; kk < kGemmBK / 16; ++kk) {
-            const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-            const uint64_t adesc0 = umma_smem_desc_sw128(a_addr + kk * 2048, Cfg::kAHalf, 1024);
-            const uint64_t adesc1 = umma_smem_desc_sw128(a_addr + Cfg::kABytes + kk * 2048, Cfg::kAHalf, 1024);
-            const uint32_t accum = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
-            tc_mma_bf16(d0, adesc0, bdesc, idesc, accum);
-            tc_mma_bf16(d1, adesc1, bdesc, idesc, accum);
-          }
-          tc_commit(&empty_bar[s]);  // stage s is free once these MMAs have read it
-          any = true;
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-        if (!ok) break;
-        for (int j = 0; j < sp.count; ++j) {
-          tc_commit(&acc_full_bar[sp.first + j]);  // accumulators complete
-          ++uses[sp.first + j];
-        }
-      }
+      for (int it = 0; work_item<kMode>(p, s_pre, s_off, it, ti); ++it)
+        if (!gemm_mma_item<kMode>(ring, ti, s, ph, uses, next_slot, any)) break;
       if (any) {
         // make sure no MMA is still running before TMEM is released
         tc_commit(drain_bar);
@@ -380,118 +562,248 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
-    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     uint32_t uses[2] = {0u, 0u};
     int next_slot = 0;
-    bool ok = true;
     TileInfo ti;
-    for (int it = 0; ok && work_item<kMode>(p, s_pre, s_off, it, ti); ++it) {
-      const SlotPlan sp = slot_plan(ti.nrows, next_slot);
-      for (int j = 0; j < sp.count && ok; ++j) {
-        const int sl = sp.first + j;
-        if (!mbar_wait_bounded(&acc_full_bar[sl], uses[sl] & 1u, kWaitLimitNs, abort_flag)) {
-          record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
-          *abort_flag = 1;
-          ok = false;
+    for (int it = 0; work_item<kMode>(p, s_pre, s_off, it, ti); ++it)
+      if (!gemm_epilogue_item<kMode, false>(ring, p, s_pre, ti, q, lane, uses, next_slot, nullptr)) break;
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(ring.tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ------------------------------------------- one launch for both GEMMs
+//
+// For steps in which no expert has more than 32 rows (T <= 32), the gate/up
+// GEMM (mode 2 items) and the down GEMM (mode 1 items) run in one persistent
+// cooperative launch: each CTA takes its gate/up work items, then its down
+// work items, in one pipeline. A down item of expert e needs all of e's h
+// rows, which other CTAs' gate/up items write: each epilogue warp that
+// finishes a 32-feature slice of an h tile counts it in h_ready[e], and the
+// producer loads a down item's token rows (h) only once h_ready[e] reaches
+// 4 * (gate/up feature tiles). Its weight boxes do not depend on h, so the
+// producer issues them at once and keeps up to a ring of stages whose token
+// rows are still pending: the down weights stream while the last gate/up
+// tiles finish, and neither GEMM pays its own launch, ramp-up and drain. The
+// launch is cooperative (every CTA resident), so a wait on another CTA always
+// ends; it is bounded anyway, recording MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY.
+// Stream-K partial slots and tickets of the two phases are disjoint
+// (p0.part / p1.part, p0.tickets / p1.tickets).
+
+constexpr int kFusedSmemBytes = GemmCfg<1>::kStages * GemmCfg<1>::kStageBytes + GemmCfg<1>::kBarrierBytes +
+                                3 * (1024 + 1) * 4 + 8 + 1024;
+static_assert(GemmCfg<1>::kStageBytes == GemmCfg<2>::kStageBytes && GemmCfg<1>::kStages == GemmCfg<2>::kStages,
+              "the fused launch runs mode 2 and mode 1 items in one ring");
+static_assert(kFusedSmemBytes <= 232448, "shared memory per CTA");
+
+// Items of one CTA: its gate/up work items, then its down work items.
+struct FusedIter {
+  int phase = 0, it = 0;
+};
+__device__ __forceinline__ bool fused_next(const GemmParams& p0, const GemmParams& p1, const int32_t* pre0,
+                                           const int32_t* pre1, const int32_t* off, FusedIter& f, TileInfo& ti) {
+  if (f.phase == 0) {
+    if (work_item<2>(p0, pre0, off, f.it, ti)) {
+      ++f.it;
+      return true;
+    }
+    f.phase = 1;
+    f.it = 0;
+  }
+  if (work_item<1>(p1, pre1, off, f.it, ti)) {
+    ++f.it;
+    return true;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_ffn_fused_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmBs0,
+                             const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmBs1,
+                             const GemmParams p0, const GemmParams p1, unsigned int* __restrict__ h_ready) {
+  using Cfg = GemmCfg<1>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
+  uint64_t* empty_bar = full_bar + S;
+  uint64_t* acc_full_bar = empty_bar + S;
+  uint64_t* acc_empty_bar = acc_full_bar + 2;
+  uint64_t* drain_bar = acc_empty_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_pre0 = reinterpret_cast<int32_t*>(smem + S * Cfg::kStageBytes + Cfg::kBarrierBytes);
+  int32_t* s_pre1 = s_pre0 + (p0.E + 1);
+  int32_t* s_off = s_pre1 + (p0.E + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= p0.E; i += blockDim.x) {
+    s_pre0[i] = __ldg(p0.tile_prefix + i);
+    s_pre1[i] = __ldg(p1.tile_prefix + i);
+    s_off[i] = __ldg(p0.expert_offsets + i);
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full_bar[b], 1);
+      mbar_init(&acc_empty_bar[b], 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmBs0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmBs1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const GemmRing ring{smem, full_bar, empty_bar, acc_full_bar, acc_empty_bar, abort_flag, *tmem_slot};
+  const unsigned int h_target = 4u * static_cast<unsigned int>(p0.n_feat_tiles);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();  // every expert has one token block: weights read once
+      const uint64_t pol_x = l2_policy_evict_last();
+      constexpr uint32_t kTx = 2 * Cfg::kABytes + kGemmSmallBox * kGemmBK * 2;  // every tile fits the small box
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      // down stages whose weight boxes are issued and whose h rows are not yet:
+      // a FIFO of (stage, K offset, first row, expert), at most S long
+      int q_stage[S], q_k0[S], q_row[S], q_e[S];
+      int q_head = 0, q_n = 0;
+      int ready_e = -1;  // an expert whose h is known complete
+      auto h_is_ready = [&](int e) -> bool {
+        if (e == ready_e) return true;
+        if (ld_acquire_gpu(h_ready + e) >= h_target) {
+          ready_e = e;
+          return true;
+        }
+        return false;
+      };
+      // issue the pending h loads in order; with `block`, wait (bounded) for
+      // each one's expert. After an abort they are issued without waiting, so
+      // that every stage's barrier completes and the drain below ends.
+      auto flush = [&](bool block) {
+        while (q_n > 0) {
+          const int e = q_e[q_head];
+          if (!*abort_flag && !h_is_ready(e)) {
+            if (!block) return;
+            const uint64_t t0 = global_timer_ns();
+            while (!h_is_ready(e)) {
+              if (*abort_flag) break;
+              if (global_timer_ns() - t0 > kWaitLimitNs) {
+                record_device_error(7u /* MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY */);
+                *abort_flag = 1;
+                break;
+              }
+            }
+          }
+          fence_proxy_async_global();
+          const int st_i = q_stage[q_head];
+          gemm_load_b<1>(smem + st_i * Cfg::kStageBytes, &tmBs1, &tmBs1, &full_bar[st_i], p1, q_row[q_head], 1,
+                         q_k0[q_head], pol_x);
+          q_head = (q_head + 1) % S;
+          --q_n;
+        }
+      };
+      FusedIter fi;
+      TileInfo ti;
+      while (ok && fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
+        const bool down = fi.phase == 1;
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
+          if (q_n == S) flush(true);  // the ring holds only stages waiting for h
+          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
+            record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * Cfg::kStageBytes;
+          mbar_arrive_expect_tx(&full_bar[s], kTx);
+          const int k0 = kb * kGemmBK;
+          if (!down) {
+            gemm_load_a<2>(st, &tmA0, &full_bar[s], p0, ti, k0, pol_w);
+            gemm_load_b<2>(st, &tmBs0, &tmBs0, &full_bar[s], p0, ti.row0, 1, k0, pol_x);
+          } else {
+            gemm_load_a<1>(st, &tmA1, &full_bar[s], p1, ti, k0, pol_w);
+            const int qi = (q_head + q_n) % S;
+            q_stage[qi] = s;
+            q_k0[qi] = k0;
+            q_row[qi] = ti.row0;
+            q_e[qi] = ti.e;
+            ++q_n;
+            flush(false);
+          }
+          ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
+      if (!ok) *abort_flag = 1;
+      flush(true);
+      if (!ok) {
+        for (int i = 0; i < S && i < issued; ++i) {
+          s = (s == 0) ? S - 1 : s - 1;
+          if (s == S - 1) ph ^= 1u;
+          mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t uses[2] = {0u, 0u};
+      int next_slot = 0;
+      bool any = false;
+      FusedIter fi;
+      TileInfo ti;
+      while (fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
+        const bool ok = (fi.phase == 0) ? gemm_mma_item<2>(ring, ti, s, ph, uses, next_slot, any)
+                                        : gemm_mma_item<1>(ring, ti, s, ph, uses, next_slot, any);
+        if (!ok) break;
+      }
+      if (any) {
+        tc_commit(drain_bar);
+        mbar_wait_bounded(drain_bar, 0u, kWaitLimitNs, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    uint32_t uses[2] = {0u, 0u};
+    int next_slot = 0;
+    FusedIter fi;
+    TileInfo ti;
+    while (fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
+      const bool ok = (fi.phase == 0)
+                          ? gemm_epilogue_item<2, true>(ring, p0, s_pre0, ti, q, lane, uses, next_slot, h_ready)
+                          : gemm_epilogue_item<1, false>(ring, p1, s_pre1, ti, q, lane, uses, next_slot, nullptr);
       if (!ok) break;
-      tc_fence_after_sync();
-      const uint32_t t0 = tmem_base + lane_base + static_cast<uint32_t>(sp.first * kTmemSlotCols);
-      const uint32_t t1 = t0 + (sp.count == 2 ? 256u : 128u);
-      const int fa = ti.nb * (gemm_is_gate_up(kMode) ? kGemmBMF : 2 * kGemmBMF) + q * 32 + lane;
-      const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
-      const bool fa_ok = fa < p.n_feat;
-      const bool fb_ok = !gemm_is_gate_up(kMode) && fb < p.n_feat;
-      if (kMode != 0 && ti.partial) {
-        // stream-K partial item: fp32 accumulators to part[slot]; the TMEM
-        // slot is free as soon as it is read
-        const int fl = q * 32 + lane;
-        float* mine = p.part + static_cast<int64_t>(ti.slot) * kSplitPartFloats;
-        for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
-          uint32_t g[32], u[32];
-          tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
-          tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
-          tmem_ld_wait();
-          const int nv = min(32, ti.nrows - c0);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i < nv) {
-              __stcg(mine + (c0 + i) * kGemmBMF + fl, __uint_as_float(g[i]));
-              __stcg(mine + (128 + c0 + i) * kGemmBMF + fl, __uint_as_float(u[i]));
-            }
-          }
-        }
-        tc_fence_before_sync();
-        __syncwarp();
-        for (int j = 0; j < sp.count; ++j) {
-          if (lane == 0) mbar_arrive(&acc_empty_bar[sp.first + j]);
-          ++uses[sp.first + j];
-        }
-        // the tile's contributors are CTAs c_first..c_last; per (tile, warp),
-        // the last one to finish adds their partials in CTA order (K order)
-        const int KB = p.K / kGemmBK;
-        const int per = stream_k_per(s_pre[p.E] * p.n_feat_tiles, KB);
-        const int c_first = (ti.t * KB) / per, c_last = ((ti.t + 1) * KB - 1) / per;
-        __threadfence();
-        __syncwarp();
-        unsigned int tk = 0u;
-        if (lane == 0) tk = atomicAdd(&p.tickets[ti.t * 4 + q], 1u);
-        tk = __shfl_sync(0xffffffffu, tk, 0);
-        if (tk == static_cast<unsigned int>(c_last - c_first)) {
-          __threadfence();
-          for (int i = 0; i < ti.nrows; ++i) {
-            float gs = 0.0f, us = 0.0f;
-            for (int c = c_first; c <= c_last; ++c) {
-              const int slot = 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
-              const float* src = p.part + static_cast<int64_t>(slot) * kSplitPartFloats;
-              const float gv = __ldcg(src + i * kGemmBMF + fl);
-              const float uv = __ldcg(src + (128 + i) * kGemmBMF + fl);
-              gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
-              us = (c == c_first) ? uv : __fadd_rn(us, uv);
-            }
-            uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
-            if (gemm_is_gate_up(kMode)) {
-              if (fa_ok) orow[fa] = bf16_bits(silu_f32(gs) * us);
-            } else {
-              if (fa_ok) orow[fa] = bf16_bits(gs);
-              if (fb_ok) orow[fb] = bf16_bits(us);
-            }
-          }
-          if (lane == 0) p.tickets[ti.t * 4 + q] = 0u;
-        }
-        continue;
-      }
-      for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
-        uint32_t g[32], u[32];
-        tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
-        tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
-        tmem_ld_wait();
-        uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + c0) * p.n_feat;
-        const int nv = min(32, ti.nrows - c0);
-        if (gemm_is_gate_up(kMode)) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (fa_ok && i < nv)
-              orow[static_cast<int64_t>(i) * p.n_feat + fa] =
-                  bf16_bits(silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]));
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i < nv) {
-              if (fa_ok) orow[static_cast<int64_t>(i) * p.n_feat + fa] = bf16_bits(__uint_as_float(g[i]));
-              if (fb_ok) orow[static_cast<int64_t>(i) * p.n_feat + fb] = bf16_bits(__uint_as_float(u[i]));
-            }
-          }
-        }
-      }
-      tc_fence_before_sync();
-      __syncwarp();
-      for (int j = 0; j < sp.count; ++j) {
-        if (lane == 0) mbar_arrive(&acc_empty_bar[sp.first + j]);
-        ++uses[sp.first + j];
-      }
     }
   }
 
@@ -499,20 +811,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    tmem_dealloc(ring.tmem_base, Cfg::kTmemCols);
   }
 }
 
 // Token blocks per expert for both GEMMs:
 //   prefix0[e] = sum_{e' < e} ceil(count_e' / rows0)  (gate/up, rows0 = 256 or 128)
 //   prefix1[e] = sum_{e' < e} ceil(count_e' / rows1)  (down, rows1 = 128)
+// The MOE_CHECKS build first checks the offsets (offsets[0] = 0, never
+// decreasing, offsets[E] <= rows_total); on bad ones it records
+// MOE_DEVERR_INDEX_CHECK and schedules no tile at all.
 __global__ void __launch_bounds__(1024)
-    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int rows0, int rows1, int32_t* __restrict__ prefix0,
-                         int32_t* __restrict__ prefix1, unsigned int* __restrict__ zero_buf, int zero_n) {
+    gemm_schedule_kernel(const int32_t* __restrict__ offsets, int E, int rows_total, int rows0, int rows1,
+                         int32_t* __restrict__ prefix0, int32_t* __restrict__ prefix1, unsigned int* __restrict__ zero_buf,
+                         int zero_n) {
   __shared__ int32_t warp_sums[2][32];
   const int e = threadIdx.x;
   for (int i = e; i < zero_n; i += 1024) zero_buf[i] = 0u;  // K-split tickets of the gate/up GEMM
-  const int32_t cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
+  int32_t cnt = (e < E) ? (offsets[e + 1] - offsets[e]) : 0;
+  if (kIndexChecks) {
+    const bool bad = (e < E && cnt < 0) || (e == 0 && offsets[0] != 0) || (e == E - 1 && offsets[E] > rows_total);
+    if (__syncthreads_or(bad)) {
+      if (e == 0) index_ok(false);
+      cnt = 0;
+    }
+  }
   const int32_t nb[2] = {(cnt + rows0 - 1) / rows0, (cnt + rows1 - 1) / rows1};
   const int lane = e & 31, w = e >> 5;
   int32_t incl[2];

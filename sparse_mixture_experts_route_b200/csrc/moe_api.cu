@@ -36,6 +36,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  bool fused_ffn = false;  // the one-launch feed-forward fits one CTA on every SM (a cooperative launch)
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -74,6 +75,14 @@ moe_status_t device_setup(int* num_sms) {
     if (cudaFuncSetAttribute(router_screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScrSmemBytes) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
+    int coop = 0, per_sm = 0;
+    if (cudaFuncSetAttribute(grouped_ffn_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kFusedSmemBytes) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, grouped_ffn_fused_kernel, kGemmThreads,
+                                                      kFusedSmemBytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    di.fused_ffn = coop != 0 && per_sm >= 1;
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -403,6 +412,7 @@ struct FfnPlan {
   int grid0, grid1;
   int mode0;  // gate/up: 0 256-row blocks, 2 128-row blocks
   int mode1;  // down: 1 (128-row blocks)
+  int rows;                   // Tk: rows of x_perm, h and y_perm
   int split_ticket_words;     // stream-K tickets the schedule kernel clears (0: none)
   unsigned int* ticket_buf;   // where they are
 };
@@ -416,6 +426,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
     return MOE_ERR_INVALID_ARG;
   int32_t* prefix0 = static_cast<int32_t*>(ws);
   int32_t* prefix1 = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ffn_prefix_bytes(E));
+  fp->rows = Tk;
   const int64_t min_e_tk = E < Tk ? E : Tk;
   GemmParams& p0 = fp->p0;
   p0.expert_offsets = offsets;
@@ -435,6 +446,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   float* part = stream_ok ? reinterpret_cast<float*>(split_base) : nullptr;
   unsigned int* tickets = stream_ok ? reinterpret_cast<unsigned int*>(split_base + ffn_split_part_bytes()) : nullptr;
   p0.b_fixed_row = -1;
+  p0.interleave = fp->mode0 == 0 ? 1 : 0;  // heavily loaded experts: mix compute- and weight-bound tiles per wave
   p0.stream_k = (stream_ok && fp->mode0 == 2 && tiles0 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
   p0.part = p0.stream_k ? part : nullptr;
   p0.tickets = p0.stream_k ? tickets : nullptr;
@@ -465,7 +477,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
 }
 
 void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
-  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, gemm_block_rows(fp.mode0),
+  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(fp.p0.expert_offsets, fp.p0.E, fp.rows, gemm_block_rows(fp.mode0),
                                                gemm_block_rows(fp.mode1), const_cast<int32_t*>(fp.p0.tile_prefix),
                                                const_cast<int32_t*>(fp.p1.tile_prefix), fp.ticket_buf,
                                                fp.split_ticket_words);
@@ -478,6 +490,33 @@ void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
 }
 void launch_gemm_down(const FfnPlan& fp, cudaStream_t stream) {
   grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
+}
+
+bool device_fused_ffn() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return g_devices[dev].ready && g_devices[dev].fused_ffn;
+}
+
+// Both GEMMs in one cooperative launch of min(148, SMs) CTAs (one per SM), so
+// that every CTA whose down items wait for another CTA's h rows is resident.
+// Both phases' stream-K splits use that grid.
+moe_status_t launch_ffn_fused(FfnPlan& fp, unsigned int* h_ready, int num_sms, cudaStream_t stream) {
+  const int grid = kStreamKCtas < num_sms ? kStreamKCtas : num_sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kFusedSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_ffn_fused_kernel, fp.mA0, fp.mBs0, fp.mA1, fp.mBs1, fp.p0,
+                                           fp.p1, h_ready);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t launch_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const moe_bf16_t* Wgu, const moe_bf16_t* Wd,
@@ -521,8 +560,23 @@ moe_status_t launch_unpermute(const moe_bf16_t* y_perm, const int32_t* inv_perm,
 // ----------------------------------------------------------------- forward
 
 struct ForwardLayout {
-  size_t route, idx, w, offsets, perm_token, inv_perm, x_perm, h, y_perm, perm_ws, ffn_ws, total;
+  size_t route, idx, w, offsets, perm_token, inv_perm, x_perm, h, y_perm, perm_ws, ffn_ws, fused_ws, total;
 };
+
+// Steps in which no expert can hold more than this many rows (T <= 32) run
+// both GEMMs in one cooperative launch (grouped_ffn_fused_kernel).
+constexpr int kFusedMaxTokens = kGemmSmallBox;
+bool ffn_fused_shape(int T) { return T <= kFusedMaxTokens; }
+
+// The fused launch's down phase has its own stream-K tickets (four per tile)
+// and partial slots (two per CTA), plus the h_ready counters [E]. They sit
+// right after the gate/up GEMM's tickets, which end the feed-forward
+// workspace, so one zeroing pass clears both phases' tickets and the counters:
+// [tickets0][tickets1][h_ready][part1].
+size_t fused_ticket_words() { return static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * 4; }
+size_t fused_ws(int E) {
+  return align256((fused_ticket_words() + static_cast<size_t>(E)) * sizeof(unsigned)) + ffn_split_part_bytes();
+}
 
 ForwardLayout forward_layout(int T, int d, int E, int k, int f) {
   ForwardLayout L;
@@ -544,6 +598,7 @@ ForwardLayout forward_layout(int T, int d, int E, int k, int f) {
   L.y_perm = take(Tk * d * 2);
   L.perm_ws = take(permute_ws(T, E, k));
   L.ffn_ws = take(ffn_ws(T * k, E));
+  L.fused_ws = ffn_fused_shape(T) ? take(fused_ws(E)) : 0;
   L.total = at;
   return L;
 }
@@ -661,6 +716,21 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
   FfnPlan fp;
   st = plan_ffn(x_perm, offsets, W_gate_up, W_down, Tk, d, E, f, h, y_perm, ws + L.ffn_ws, sms, &fp);
   if (st != MOE_OK) return st;
+  // few tokens: both GEMMs in one cooperative launch, the down phase with its
+  // own tickets and partial slots; the zeroing that clears the gate/up
+  // tickets (router or dispatch kernel) covers the down tickets and h_ready too
+  unsigned int* h_ready = nullptr;
+  const bool fused = ffn_fused_shape(T) && device_fused_ffn() && fp.ticket_buf != nullptr &&
+                     reinterpret_cast<uint8_t*>(fp.ticket_buf) + ffn_split_ticket_bytes() == ws + L.fused_ws;
+  if (fused) {
+    unsigned int* tickets1 = fp.ticket_buf + fused_ticket_words();
+    h_ready = tickets1 + fused_ticket_words();
+    fp.p0.tickets = fp.ticket_buf;
+    fp.p0.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(fp.ticket_buf) - ffn_split_part_bytes());
+    fp.p1.tickets = tickets1;
+    fp.p1.part = reinterpret_cast<float*>(ws + L.fused_ws + align256((fused_ticket_words() + E) * sizeof(unsigned)));
+    fp.split_ticket_words = static_cast<int>(2 * fused_ticket_words()) + E;
+  }
   // stage boundaries: events (timed calls) and NVTX ranges named for the
   // stage, which profilers show around the stage's launches (no cost without one)
   static const char* const kStage[MOE_TIMED_STAGES] = {"moe.route", "moe.dispatch", "moe.gate_up", "moe.down",
@@ -698,7 +768,7 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
       fp.p0.b_fixed_row = 0;
     } else {  // the maps of the permuted copy stay; make the copy
       permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
-          reinterpret_cast<const uint4*>(x), perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
+          reinterpret_cast<const uint4*>(x), T, perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
     }
   } else if (Tk <= kSmallDispatchPairs) {
     // one block: counts, offsets, stable scatter and both GEMM tile prefixes; then the row copy
@@ -708,7 +778,7 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
                                                   const_cast<int32_t*>(fp.p1.tile_prefix), fp.ticket_buf,
                                                   fp.split_ticket_words);
     permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(x), perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
+        reinterpret_cast<const uint4*>(x), T, perm_token, Tk, d / 8, reinterpret_cast<uint4*>(x_perm));
   } else {
     st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, x_perm, ws + L.perm_ws, stream);
     if (st != MOE_OK) return st;
@@ -716,10 +786,15 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
   }
   mark(3);
   mark(4);
-  launch_gemm_gate_up(fp, stream);
+  if (fused) {
+    st = launch_ffn_fused(fp, h_ready, sms, stream);
+    if (st != MOE_OK) return st;
+  } else {
+    launch_gemm_gate_up(fp, stream);
+  }
   mark(5);
   mark(6);
-  launch_gemm_down(fp, stream);
+  if (!fused) launch_gemm_down(fp, stream);
   mark(7);
   mark(8);
   st = launch_unpermute(y_perm, inv_perm, w, T, d, k, out, stream);
@@ -1052,7 +1127,7 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
     } else {
       st = launch_permute(x, idx, T, d, E, k, offsets, perm_token, inv_perm, nullptr, ws + L.perm_ws, stream);
       if (st != MOE_OK) return st;
-      gemm_schedule_kernel<<<1, 1024, 0, stream>>>(offsets, E, kMxTileRows, kMxTileRows, pre0, pre1, tickets,
+      gemm_schedule_kernel<<<1, 1024, 0, stream>>>(offsets, E, Tk, kMxTileRows, kMxTileRows, pre0, pre1, tickets,
                                                    ticket_words);
     }
   }

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256)
     const int64_t pr = static_cast<int64_t>(t) * k + threadIdx.x;
     const int e = __ldg(idx + pr);
     const int r = __ldg(inv_perm + pr);
-    const bool ok = e >= 0 && e < E;
+    const bool ok = e >= 0 && e < E && index_ok(r >= 0 && r < static_cast<int64_t>(gridDim.x) * k);
     const int local = ok ? r - __ldg(offsets + e) : 0;
     s_row[threadIdx.x] = ok ? r : -1;
     s_tile[threadIdx.x] = ok ? __ldg(prefix + e) + local / kMxTileRows : 0;

@@ -133,14 +133,17 @@ __global__ void __launch_bounds__(32)
 }
 
 // x_perm[row, :] = x[perm_token[row], :], 16-byte vectors, one warp per row;
-// each lane keeps 4 loads in flight.
+// each lane keeps 4 loads in flight. x has n_src rows (checked in the
+// MOE_CHECKS build).
 __global__ void __launch_bounds__(256)
-    permute_copy_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_token, int64_t n_rows,
-                             int vec_per_row, uint4* __restrict__ x_perm) {
+    permute_copy_rows_kernel(const uint4* __restrict__ x, int64_t n_src, const int32_t* __restrict__ perm_token,
+                             int64_t n_rows, int vec_per_row, uint4* __restrict__ x_perm) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= n_rows) return;
   const int lane = threadIdx.x & 31;
-  const uint4* src = x + static_cast<int64_t>(__ldg(perm_token + row)) * vec_per_row;
+  const int32_t tok = __ldg(perm_token + row);
+  if (!index_ok(tok >= 0 && tok < n_src)) return;
+  const uint4* src = x + static_cast<int64_t>(tok) * vec_per_row;
   uint4* dst = x_perm + row * vec_per_row;
   int v = lane;
   for (; v + 96 < vec_per_row; v += 128) {
@@ -164,8 +167,12 @@ __global__ void __launch_bounds__(128)
   const int64_t t = blockIdx.x;
   const int tid = threadIdx.x;
   int32_t dst_row[16];
+  const int64_t n_rows = static_cast<int64_t>(gridDim.x) * k;  // x_perm has T k rows
 #pragma unroll
-  for (int j = 0; j < 16; ++j) dst_row[j] = (j < k) ? __ldg(inv_perm + t * k + j) : 0;
+  for (int j = 0; j < 16; ++j) {
+    dst_row[j] = (j < k) ? __ldg(inv_perm + t * k + j) : 0;
+    if (j < k && !index_ok(dst_row[j] >= 0 && dst_row[j] < n_rows)) dst_row[j] = -1;
+  }
   const uint4* src = x + t * vec_per_row;
   for (int v0 = 0; v0 < vec_per_row; v0 += 128 * kVec) {
     uint4 r[kVec];
@@ -177,6 +184,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       if (j >= k) break;
+      if (kIndexChecks && dst_row[j] < 0) continue;
       uint4* dst = x_perm + static_cast<int64_t>(dst_row[j]) * vec_per_row;
 #pragma unroll
       for (int u = 0; u < kVec; ++u) {
@@ -205,7 +213,9 @@ __global__ void __launch_bounds__(256)
   for (int j = 0; j < K; ++j) {
     const int32_t row = __ldg(inv_perm + t * K + j);
     ws[j] = __ldg(topk_w + t * K + j);
-    y[j] = __ldg(y_perm + static_cast<int64_t>(row) * vec_per_row + v);
+    // y_perm has T K rows; the MOE_CHECKS build skips (adds zero for) a bad one
+    y[j] = index_ok(row >= 0 && row < T * K) ? __ldg(y_perm + static_cast<int64_t>(row) * vec_per_row + v)
+                                              : make_uint4(0u, 0u, 0u, 0u);
   }
   float acc[8];
 #pragma unroll

@@ -390,3 +390,29 @@ def test_route_tensor_core_screen_ties_and_fallback(lib, E, k, bias_on):
     ridx, rw = oracle.topk(lg, k)
     assert np.array_equal(idx.cpu().numpy(), ridx)
     parity.assert_route_weights(w, rw, x, Wr, inp.bias, k, lg, ridx)
+
+
+# Steps of at most 32 tokens run both GEMMs in one cooperative launch (down
+# items wait for their expert's h rows). The staged entry points run the same
+# GEMMs as two launches with the same stream-K splits, so the results must be
+# identical bit for bit; both are checked against the oracle too.
+@pytest.mark.parametrize("shape", [(1, 7168, 896, 16, 512, None), (3, 1024, 8, 2, 192, "zipf"),
+                                   (8, 2048, 64, 8, 256, None), (32, 512, 16, 4, 320, None),
+                                   (17, 256, 4, 4, 128, None)],
+                         ids=lambda s: "x".join(map(str, s[:5])) + (f"_{s[5]}" if s[5] else ""))
+def test_forward_one_launch_ffn_matches_staged_steps(lib, shape):
+    T, d, E, k, f, bias = shape
+    inp = _inputs(T, d, E, k, f, bias=bias)
+    g = _cuda(inp)
+    out = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k)
+    idx, w = lib.moe_route(g.x, g.W_router, g.bias, k)
+    offs, perm, inv, xp = lib.moe_permute(g.x, idx, E)
+    _, y = lib.moe_expert_ffn(xp, offs, g.W_gate_up, g.W_down)
+    staged = lib.moe_unpermute(y, inv, w)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    assert torch.equal(out.view(torch.int16), staged.view(torch.int16))
+    ref, _, _ = oracle.forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(out, ref, "one-launch feed-forward")
+    out2 = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k)
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
