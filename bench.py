@@ -440,6 +440,165 @@ def layer_summary(shape, res, steps: int, world: int, peaks: dict) -> dict:
 
 
 EXTRA_WORKLOADS = ("decode", "skewed") + tuple(f"sweep_T{t}" for t in moe_inputs.SWEEP_T)
+# workloads also timed with the experts in the MX serving format
+MX_WORKLOADS = ("decode",) + tuple(f"sweep_T{t}" for t in moe_inputs.SWEEP_T)
+
+
+def time_layer_mx(_lib, shape, inp, experts, steps: int, warmup: int, graph_on: bool, world: int, flush,
+                  local: int):
+    """Times moe_forward_mx steps (MXFP4 expert weights packed once, MXFP8
+    activations) like time_layer, without per-stage times."""
+    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    ws = torch.empty(_lib.raw.moe_forward_mx_workspace_size(T, d, E, k, f), dtype=torch.uint8, device=inp.x.device)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=inp.x.device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        _lib.moe_forward_mx(inp.x, inp.W_router, inp.bias, experts, k, out=out, workspace=ws)
+
+    idx, _ = _lib.moe_route(inp.x, inp.W_router, inp.bias, k)
+    offs, _, _, _ = _lib.moe_permute(None, idx, E, with_rows=False)
+    counts = np.diff(offs.cpu().numpy())
+    for _ in range(warmup):
+        flush(1)
+        step()
+    graph = None
+    if graph_on:
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+            with torch.cuda.graph(graph, stream=side):
+                step()
+        stream.wait_stream(side)
+        for _ in range(warmup):
+            flush(1)
+            graph.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for s_, (a, b) in enumerate(evs):
+        flush(s_)
+        a.record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
+    assert _lib.get_device_error() == 0, "device error during MX timing"
+    del graph
+    return total_ms, counts, clk
+
+
+def time_latent(_lib, li, steps: int, warmup: int, graph_on: bool, world: int, flush, local: int):
+    """Times moe_latent_forward steps like time_layer_mx (no per-stage times)."""
+    k = li.shape.k
+    args = (li.x, li.W_router, li.bias, li.W_dn, li.W_up, li.W_gate_up, li.W_down, li.gamma, li.Ws_gate_up,
+            li.Ws_down, k)
+    T, d, E, f = li.shape.T, li.shape.d, li.shape.E, li.shape.f
+    S = li.Ws_down.shape[0] if li.Ws_down is not None else 0
+    fs = li.Ws_down.shape[1] if li.Ws_down is not None else 0
+    ws = torch.empty(_lib.raw.moe_latent_workspace_size(T, d, li.l, E, k, f, S, fs), dtype=torch.uint8,
+                     device=li.x.device)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=li.x.device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        _lib.moe_latent_forward(*args, out=out, workspace=ws)
+
+    idx, _ = _lib.moe_route(li.x, li.W_router, li.bias, k)
+    offs, _, _, _ = _lib.moe_permute(None, idx, E, with_rows=False)
+    counts = np.diff(offs.cpu().numpy())
+    for _ in range(warmup):
+        flush(1)
+        step()
+    graph = None
+    if graph_on:
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+            with torch.cuda.graph(graph, stream=side):
+                step()
+        stream.wait_stream(side)
+        for _ in range(warmup):
+            flush(1)
+            graph.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for s_, (a, b) in enumerate(evs):
+        flush(s_)
+        a.record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
+    assert _lib.get_device_error() == 0, "device error during latent timing"
+    del graph
+    return total_ms, counts, clk, S, fs
+
+
+def latent_summary(li, total_ms, counts, clk, S, fs, steps, world, peaks) -> dict:
+    """Throughput and roofline of a Stable LatentMoE step. F_alg: router
+    2 T d E, the two projections 2 * 2 T d l, routed experts 6 T k l f, shared
+    experts 6 T S d fs. B_alg: W_router 4 d E, x in and out 4 T d, W_dn and W_up
+    2 * 2 d l, the touched routed experts 6 l f each, the shared experts
+    S * 6 d fs, gamma 4 l (+ 4 E with a bias)."""
+    T, d, E, k, f = li.shape.T, li.shape.d, li.shape.E, li.shape.k, li.shape.f
+    l = li.l
+    n_touched = int((counts > 0).sum())
+    F = 2.0 * T * d * E + 4.0 * T * d * l + 6.0 * T * k * l * f + 6.0 * T * S * d * fs
+    B = (4.0 * d * E + 4.0 * T * d + 4.0 * d * l + n_touched * 6.0 * l * f + S * 6.0 * d * fs + 4.0 * l
+         + (4.0 * E if li.bias is not None else 0.0))
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    ms = total_ms / steps
+    t = ms / 1e3
+    return {"T": T, "d": d, "l": l, "E": E, "k": k, "f": f, "S": S, "fs": fs, "steps": steps,
+            "ms_per_step": ms, "tokens_per_s": aggregate_tokens_per_s(T, steps, world, total_ms),
+            "F_alg": F, "B_alg": B, "n_touched": n_touched, "tflops": F / t / 1e12, "hbm_gbs": B / t / 1e9,
+            "roofline_frac": max(F / (tc * 1e12), B / (hbm * 1e9)) / t,
+            "binding_roof": "hbm" if B / hbm / 1e9 >= F / tc / 1e12 else "tensor",
+            "glu": "SiTU-GLU beta1=4 beta2=25", "clocks": clk}
+
+
+def mx_summary(shape, total_ms: float, counts, clk, steps: int, world: int, peaks: dict) -> dict:
+    """Throughput and roofline of an MX step: expert weights at 4.25 bits
+    (E2M1 codes plus one E8M0 scale per 32), the rest as in the bf16 layer."""
+    T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    n_touched = int((counts > 0).sum())
+    F = 2.0 * T * d * E + 6.0 * T * k * d * f
+    B = 4.0 * d * E + 4.0 * T * d + n_touched * 3.0 * d * f * (0.5 + 1.0 / 32) + (4.0 * E if shape.bias else 0.0)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    ms = total_ms / steps
+    t = ms / 1e3
+    return {"ms_per_step": ms, "tokens_per_s": aggregate_tokens_per_s(T, steps, world, total_ms),
+            "F_alg": F, "B_alg": B, "n_touched": n_touched, "hbm_gbs": B / t / 1e9,
+            "roofline_frac": max(F / (tc * 1e12), B / (hbm * 1e9)) / t,
+            "binding_roof": "hbm" if B / hbm / 1e9 >= F / tc / 1e12 else "tensor",
+            "bytes_rule": "expert weights at 4.25 bits (E2M1 + E8M0 per 32); router fp32; x, out bf16",
+            "clocks": clk}
 
 
 def run_ours(args):
@@ -508,6 +667,7 @@ def run_ours(args):
     # so the timing barriers line up); skewed and the sweep share one set of
     # expert weights (same shapes and seeds), generated once
     extra = {}
+    mx_packed = {}
     if not args.no_workloads:
         shared = None
         for name in EXTRA_WORKLOADS:
@@ -528,9 +688,31 @@ def run_ours(args):
             r = time_layer(_lib, ws_shape, winp, steps, args.warmup, args.graph == "on", world, flush, local)
             extra[name] = {**{kk: v for kk, v in ws_shape.as_dict().items() if kk != "workload"},
                            "steps": steps, **layer_summary(ws_shape, r, steps, world, peaks)}
-            del r, winp
+            del r
+            if name in MX_WORKLOADS and not args.no_mx:
+                if mx_packed.get("src") is not shared.W_gate_up:
+                    mx_packed["experts"] = _lib.moe_mx_pack_experts(winp.W_gate_up, winp.W_down)
+                    mx_packed["src"] = shared.W_gate_up
+                tm, cnt, clk = time_layer_mx(_lib, ws_shape, winp, mx_packed["experts"], steps, args.warmup,
+                                             args.graph == "on", world, flush, local)
+                extra[name + "_mx"] = {**{kk: v for kk, v in ws_shape.as_dict().items() if kk != "workload"},
+                                       "steps": steps, "experts": "MXFP4 (E2M1, E8M0 per 32), activations MXFP8",
+                                       **mx_summary(ws_shape, tm, cnt, clk, steps, world, peaks)}
+            del winp
         del shared
+        mx_packed.clear()
         torch.cuda.empty_cache()
+        if not args.no_latent:
+            log(f"[rank {rank}] latent_prefill")
+            lat = moe_inputs.LATENT
+            li = moe_inputs.make_latent_inputs(lat["shape"], lat["l"], lat["S"], lat["fs"], seed=0, device=dev)
+            if rank != 0:
+                li.x = moe_inputs.make_x(lat["shape"], seed=replica_x_seed(rank), device=dev)
+            tm, cnt, clk, S, fs = time_latent(_lib, li, args.workload_steps, args.warmup, args.graph == "on", world,
+                                              flush, local)
+            extra["latent_prefill"] = latent_summary(li, tm, cnt, clk, S, fs, args.workload_steps, world, peaks)
+            del li
+            torch.cuda.empty_cache()
 
     if rank != 0:
         return None
@@ -666,6 +848,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="time only --workload (skip the decode, skewed and sweep entries of the line)")
+    ap.add_argument("--no-mx", action="store_true", help="skip the MX-format entries of the workloads")
+    ap.add_argument("--no-latent", action="store_true", help="skip the Stable LatentMoE entry of the workloads")
     ap.add_argument("--workload-steps", type=int, default=10,
                     help="timed steps of each of the other workloads")
     ap.add_argument("--graph", default="on", choices=["on", "off"],

@@ -359,6 +359,38 @@ moe_status_t moe_qb_bias(const uint64_t* H, int E, int bins, float lo, float hi,
 moe_status_t moe_gather_rows(const moe_bf16_t* src, int64_t n_src, const int32_t* rows, int64_t n_out, int d,
                              moe_bf16_t* out, cudaStream_t stream);
 
+/* --------------------------------------------------- Stable LatentMoE --
+ * [P3] section "Operational Execution Flow": two full-width shared experts
+ * act on x; the routed path projects x down to a latent z = x W_dn of width l
+ * (3584 on the page), the k routed experts chosen by the router (on x, as in
+ * moe_route) act on z, their probability-weighted sum u passes an explicit
+ * RMSNorm, and W_up brings it back to width d. The experts' GLU is SiTU-GLU,
+ * a soft-capped SwiGLU with beta1 = 4, beta2 = 25 on the page and
+ * |SiTU-GLU| <= beta1 beta2. The page lost the formulas; readings taken:
+ *   SiTU-GLU(g, v) = beta1 tanh(SiLU(g) / beta1) * beta2 tanh(v / beta2);
+ *   out = sum_s S_s(x) + RMSNorm(u) W_up, RMSNorm(u) = gamma u / sqrt(mean(u^2) + eps).
+ *
+ * moe_latent_forward: x [T, d] bf16; W_router [d, E] fp32, router_bias [E] or
+ *   NULL; W_dn [d, l], W_up [l, d] bf16; routed W_gate_up [E, l, 2f] (columns
+ *   0..f-1 gate, f..2f-1 the second factor), W_down [E, f, l] bf16; gamma [l]
+ *   fp32 or NULL (ones); shared Ws_gate_up [S, d, 2fs], Ws_down [S, fs, d]
+ *   bf16 (S = 0: none, both may be NULL); act 0 SwiGLU, 1 SiTU-GLU with
+ *   beta1, beta2 > 0; eps >= 0. out [T, d] bf16. Intermediates (z, the
+ *   routed rows, h, y, RMSNorm(u), the shared experts' outputs) are carved
+ *   from `workspace` (moe_latent_workspace_size bytes, 256-byte aligned) and
+ *   rounded to bf16 between the GEMMs; the routed sum, the RMSNorm and the
+ *   final sum are fp32. d, l, f, fs multiples of 64; l <= 8192; S <= 8;
+ *   other limits as moe_forward. Asynchronous on `stream`, no host sync.
+ */
+size_t moe_latent_workspace_size(int T, int d, int l, int E, int k, int f, int S, int fs);
+moe_status_t moe_latent_forward(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                                const moe_bf16_t* W_dn, const moe_bf16_t* W_up,
+                                const moe_bf16_t* W_gate_up, const moe_bf16_t* W_down, const float* gamma,
+                                const moe_bf16_t* Ws_gate_up, const moe_bf16_t* Ws_down,
+                                int T, int d, int l, int E, int k, int f, int S, int fs,
+                                int act, float beta1, float beta2, float eps,
+                                moe_bf16_t* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* ------------------------------------------------------------ diagnostics --
  * moe_get_device_error: reads (and, if clear != 0, resets) the error word of
  * the CURRENT device. *code is 0 when no kernel recorded an error, otherwise

@@ -55,6 +55,9 @@ EXPORTS = {
     "moe_qb_histogram": ([P, P, I, I, I, ctypes.c_float, ctypes.c_float, I, P, P, P], I),
     "moe_qb_bias": ([P, I, I, ctypes.c_float, ctypes.c_float, ctypes.c_int64, I, P, P, P], I),
     "moe_gather_rows": ([P, ctypes.c_int64, P, ctypes.c_int64, I, P, P], I),
+    "moe_latent_workspace_size": ([I, I, I, I, I, I, I, I], Z),
+    "moe_latent_forward": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, ctypes.c_float,
+                            ctypes.c_float, ctypes.c_float, P, P, Z, P], I),
     "moe_get_device_error": ([ctypes.POINTER(ctypes.c_uint32), I], I),
     "moe_selftest_wait_timeout": ([I, P], I),
 }
@@ -413,6 +416,49 @@ def moe_gather_rows(src, rows, out=None, stream=None):
     _need(out, "out", torch.bfloat16, (n_out, d))
     _check(_lib.moe_gather_rows(_ptr(src), n_src, _ptr(rows), n_out, d, _ptr(out), _stream(stream)),
            "moe_gather_rows")
+    return out
+
+
+ACT_SWIGLU, ACT_SITU = 0, 1
+SITU_BETA1, SITU_BETA2 = 4.0, 25.0
+
+
+def moe_latent_forward(x, W_router, router_bias, W_dn, W_up, W_gate_up, W_down, gamma, Ws_gate_up, Ws_down, k: int,
+                       act: int = ACT_SITU, beta1: float = SITU_BETA1, beta2: float = SITU_BETA2, eps: float = 1e-6,
+                       out=None, workspace=None, stream=None):
+    """The Stable LatentMoE layer (include/moe.h, moe_latent_forward). Returns out [T, d] bf16."""
+    T, d = x.shape
+    E = W_router.shape[1]
+    l = W_dn.shape[1]
+    f = W_down.shape[1]
+    _need(x, "x", torch.bfloat16, (T, d))
+    _need(W_router, "W_router", torch.float32, (d, E))
+    if router_bias is not None:
+        _need(router_bias, "router_bias", torch.float32, (E,))
+    _need(W_dn, "W_dn", torch.bfloat16, (d, l))
+    _need(W_up, "W_up", torch.bfloat16, (l, d))
+    _need(W_gate_up, "W_gate_up", torch.bfloat16, (E, l, 2 * f))
+    _need(W_down, "W_down", torch.bfloat16, (E, f, l))
+    if gamma is not None:
+        _need(gamma, "gamma", torch.float32, (l,))
+    if Ws_gate_up is not None:
+        S, fs = Ws_down.shape[0], Ws_down.shape[1]
+        _need(Ws_gate_up, "Ws_gate_up", torch.bfloat16, (S, d, 2 * fs))
+        _need(Ws_down, "Ws_down", torch.bfloat16, (S, fs, d))
+    else:
+        S, fs = 0, 0
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", torch.bfloat16, (T, d))
+    nbytes = _lib.moe_latent_workspace_size(T, d, l, E, k, f, S, fs)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_INVALID_ARG, "moe_latent_workspace_size")
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device, stream)
+    _check(_lib.moe_latent_forward(_ptr(x), _ptr(W_router), _ptr(router_bias), _ptr(W_dn), _ptr(W_up),
+                                   _ptr(W_gate_up), _ptr(W_down), _ptr(gamma), _ptr(Ws_gate_up), _ptr(Ws_down),
+                                   T, d, l, E, k, f, S, fs, int(act), float(beta1), float(beta2), float(eps),
+                                   _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_latent_forward")
     return out
 
 

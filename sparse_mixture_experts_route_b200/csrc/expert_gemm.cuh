@@ -57,18 +57,21 @@ constexpr int kTmemSlotCols = 256;
 
 // Modes: 0 gate/up with 256-row token blocks (3 stages of 64 KB), 2 gate/up
 // with 128-row token blocks (4 stages of 48 KB: more stages in flight when no
-// expert fills a 256-row block), 1 down (128-row blocks, 4 stages of 48 KB).
-__host__ __device__ constexpr bool gemm_is_gate_up(int mode) { return mode != 1; }
-__host__ __device__ constexpr int gemm_block_rows(int mode) { return mode == 0 ? 256 : 128; }
+// expert fills a 256-row block), 1 down with 128-row blocks (4 stages of
+// 48 KB), 3 down with 256-row blocks (3 stages of 64 KB: for heavily loaded
+// experts, each weight tile is read once per 256 rows and every stage carries
+// twice the MMA work). The 256-row modes never take the stream-K split.
+__host__ __device__ constexpr bool gemm_is_gate_up(int mode) { return mode == 0 || mode == 2; }
+__host__ __device__ constexpr int gemm_block_rows(int mode) { return (mode == 0 || mode == 3) ? 256 : 128; }
 
 template <int kMode>
 struct GemmCfg {
   static constexpr int kABytes = kGemmBK * kGemmBMF * 2;         // 16 KB per A operand
   static constexpr int kAHalf = kABytes / 2;                     // one 64-feature box (8 KB)
   static constexpr int kBRows = gemm_block_rows(kMode);          // 256 / 128
-  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB (mode 0) / 16 KB
+  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB (256-row modes) / 16 KB
   static constexpr int kStageBytes = 2 * kABytes + kBBytes;      // 64 KB / 48 KB
-  static constexpr int kStages = (kMode == 0) ? 3 : 4;
+  static constexpr int kStages = (kBRows == 256) ? 3 : 4;
   static constexpr int kTmemCols = 2 * kTmemSlotCols;            // 512
   static constexpr int kBarrierBytes = 256;
   static constexpr int kTableBytes = 2 * (1024 + 1) * 4 + 8;  // shared copies of tile_prefix and expert_offsets
@@ -107,6 +110,7 @@ struct GemmParams {
   int b_fixed_row;        // >= 0: every tile's token operand starts at this row (one-token steps read x itself)
   float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
   unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
+  float beta1, beta2;     // SiTU-GLU soft caps (gate/up kernels with kAct = 1 only)
 };
 
 // fp32 elements of one partial: two accumulators, 128 rows x 128 features
@@ -203,6 +207,17 @@ __device__ __forceinline__ SlotPlan slot_plan(int nrows, int& next_slot) {
 }
 
 __device__ __forceinline__ float silu_f32(float a) { return a / (1.0f + expf(-a)); }
+
+// The gate/up epilogue's GLU: kAct 0 SwiGLU, SiLU(g) * u; kAct 1 SiTU-GLU
+// (the soft-capped GLU of "Kimi K3: Open Frontier Intelligence", section
+// "Operational Execution Flow"; its formula is lost on the page, the reading
+// taken is beta1 tanh(SiLU(g) / beta1) * beta2 tanh(u / beta2), bounded by
+// beta1 beta2).
+template <int kAct>
+__device__ __forceinline__ float glu_f32(float g, float u, const GemmParams& p) {
+  if (kAct == 0) return silu_f32(g) * u;
+  return p.beta1 * tanhf(silu_f32(g) / p.beta1) * (p.beta2 * tanhf(u / p.beta2));
+}
 
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
   const __nv_bfloat16 b = __float2bfloat16_rn(v);
@@ -330,7 +345,7 @@ __device__ __forceinline__ void signal_h_slice(unsigned int* ready, int e, int l
 // partial item, writes its fp32 partials and, if it is the last of the tile's
 // contributors, adds them in K order and stores the rows. With kSignal, a
 // finished gate/up slice is counted in ready[e]. Returns false if a wait gave up.
-template <int kMode, bool kSignal>
+template <int kMode, bool kSignal, int kAct = 0>
 __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const GemmParams& p, const int32_t* pre,
                                                    const TileInfo& ti, int q, int lane, uint32_t (&uses)[2],
                                                    int& next_slot, unsigned int* ready) {
@@ -351,7 +366,7 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
   const int fb = fa + kGemmBMF;  // mode 1: the second 128 output features
   const bool fa_ok = fa < p.n_feat;
   const bool fb_ok = !gemm_is_gate_up(kMode) && fb < p.n_feat;
-  if (kMode != 0 && ti.partial) {
+  if (gemm_block_rows(kMode) == 128 && ti.partial) {
     // stream-K partial item: fp32 accumulators to part[slot]; the TMEM
     // slot is free as soon as it is read
     const int fl = q * 32 + lane;
@@ -400,7 +415,7 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
         }
         uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
         if (gemm_is_gate_up(kMode)) {
-          if (fa_ok) orow[fa] = bf16_bits(silu_f32(gs) * us);
+          if (fa_ok) orow[fa] = bf16_bits(glu_f32<kAct>(gs, us, p));
         } else {
           if (fa_ok) orow[fa] = bf16_bits(gs);
           if (fb_ok) orow[fb] = bf16_bits(us);
@@ -423,7 +438,7 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
       for (int i = 0; i < 32; ++i) {
         if (fa_ok && i < nv)
           orow[static_cast<int64_t>(i) * p.n_feat + fa] =
-              bf16_bits(silu_f32(__uint_as_float(g[i])) * __uint_as_float(u[i]));
+              bf16_bits(glu_f32<kAct>(__uint_as_float(g[i]), __uint_as_float(u[i]), p));
       }
     } else {
 #pragma unroll
@@ -445,7 +460,7 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
   return true;
 }
 
-template <int kMode>
+template <int kMode, int kAct = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBs, const GemmParams p) {
@@ -566,7 +581,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int next_slot = 0;
     TileInfo ti;
     for (int it = 0; work_item<kMode>(p, s_pre, s_off, it, ti); ++it)
-      if (!gemm_epilogue_item<kMode, false>(ring, p, s_pre, ti, q, lane, uses, next_slot, nullptr)) break;
+      if (!gemm_epilogue_item<kMode, false, kAct>(ring, p, s_pre, ti, q, lane, uses, next_slot, nullptr)) break;
   }
 
   tc_fence_before_sync();

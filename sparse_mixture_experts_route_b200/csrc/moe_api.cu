@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "ep.cuh"
 #include "expert_gemm.cuh"
+#include "latent.cuh"
 #include "mx_gemm.cuh"
 #include "mx_prep.cuh"
 #include "mx_quant.cuh"
@@ -63,7 +64,13 @@ moe_status_t device_setup(int* num_sms) {
                              GemmCfg<2>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<1>::kSmemBytes) != cudaSuccess)
+                             GemmCfg<1>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<3>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<0>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(grouped_gemm_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<2>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(router_stream_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              router_stream_smem_bytes(1)) != cudaSuccess ||
@@ -411,7 +418,8 @@ struct FfnPlan {
   GemmParams p0, p1;
   int grid0, grid1;
   int mode0;  // gate/up: 0 256-row blocks, 2 128-row blocks
-  int mode1;  // down: 1 (128-row blocks)
+  int mode1;  // down: 1 128-row blocks, 3 256-row blocks
+  int act = 0;  // gate/up GLU: 0 SwiGLU, 1 SiTU-GLU (p0.beta1, p0.beta2)
   int rows;                   // Tk: rows of x_perm, h and y_perm
   int split_ticket_words;     // stream-K tickets the schedule kernel clears (0: none)
   unsigned int* ticket_buf;   // where they are
@@ -439,7 +447,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p0.out = h;
   // 256-row blocks pay off only when experts average more than 128 rows
   fp->mode0 = (static_cast<int64_t>(Tk) > static_cast<int64_t>(E) * 128) ? 0 : 2;
-  fp->mode1 = 1;
+  fp->mode1 = fp->mode0 == 0 ? 3 : 1;
   const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(fp->mode0)) + min_e_tk) * p0.n_feat_tiles;
   const bool stream_ok = ffn_split_possible(Tk, E);
   uint8_t* split_base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
@@ -462,7 +470,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p1.a1_offset = kGemmBMF;
   p1.out = y_perm;
   const int64_t tiles1 = (ceil_div64(Tk, gemm_block_rows(fp->mode1)) + min_e_tk) * p1.n_feat_tiles;
-  p1.stream_k = (stream_ok && tiles1 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
+  p1.stream_k = (stream_ok && fp->mode1 == 1 && tiles1 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
   p1.part = p1.stream_k ? part : nullptr;
   p1.tickets = p1.stream_k ? tickets : nullptr;
   fp->grid1 = p1.stream_k ? (kStreamKCtas < num_sms ? kStreamKCtas : num_sms)
@@ -483,13 +491,25 @@ void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
                                                fp.split_ticket_words);
 }
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
+  if (fp.act == 1) {
+    if (fp.mode0 == 0)
+      grouped_gemm_kernel<0, 1><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0,
+                                                                                             fp.p0);
+    else
+      grouped_gemm_kernel<2, 1><<<fp.grid0, kGemmThreads, GemmCfg<2>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0,
+                                                                                             fp.p0);
+    return;
+  }
   if (fp.mode0 == 0)
     grouped_gemm_kernel<0><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
   else
     grouped_gemm_kernel<2><<<fp.grid0, kGemmThreads, GemmCfg<2>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
 }
 void launch_gemm_down(const FfnPlan& fp, cudaStream_t stream) {
-  grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
+  if (fp.mode1 == 3)
+    grouped_gemm_kernel<3><<<fp.grid1, kGemmThreads, GemmCfg<3>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
+  else
+    grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
 }
 
 bool device_fused_ffn() {
@@ -1261,6 +1281,241 @@ moe_status_t moe_get_device_error(uint32_t* code, int clear) {
 moe_status_t moe_selftest_wait_timeout(int timeout_us, cudaStream_t stream) {
   if (timeout_us < 1 || timeout_us > 1000000) return MOE_ERR_INVALID_ARG;
   moe::selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<unsigned long long>(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------- Stable LatentMoE
+
+namespace {
+
+// A linear layer out = A W on the down-GEMM kernel (mode 1): n experts that
+// each take `rows` consecutive rows of A [n rows, K] through their own W [n, K,
+// N] into out [n rows, N] (bf16). The expert offsets and token-block prefixes
+// are written on the device by launch_linear_schedule.
+struct LinearPlan {
+  CUtensorMap mA, mB, mBs;
+  GemmParams p;
+  int grid;
+  int32_t* offsets;
+  int32_t* prefix0;
+  int rows, n;
+};
+
+moe_status_t plan_linear(const moe_bf16_t* A, const moe_bf16_t* W, moe_bf16_t* out, int rows, int n, int K, int N,
+                         int32_t* offsets, int32_t* prefix0, int32_t* prefix1, int num_sms, LinearPlan* lp) {
+  if (!weight_map(&lp->mA, W, n, K, N) || !act_map(&lp->mB, A, n * rows, K, kGemmBoxRows) ||
+      !act_map(&lp->mBs, A, n * rows, K, kGemmSmallBox))
+    return MOE_ERR_INVALID_ARG;
+  GemmParams& p = lp->p;
+  p = GemmParams{};
+  p.expert_offsets = offsets;
+  p.tile_prefix = prefix1;
+  p.E = n;
+  p.K = K;
+  p.n_feat = N;
+  p.n_feat_tiles = ceil_div(N, 2 * kGemmBMF);
+  p.a1_offset = kGemmBMF;
+  p.out = reinterpret_cast<uint16_t*>(out);
+  p.stream_k = 0;
+  p.interleave = 0;
+  p.b_fixed_row = -1;
+  const int64_t tiles = static_cast<int64_t>(n) * ceil_div64(rows, 128) * p.n_feat_tiles;
+  lp->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  lp->offsets = offsets;
+  lp->prefix0 = prefix0;
+  lp->rows = rows;
+  lp->n = n;
+  return MOE_OK;
+}
+
+void launch_linear_schedule(const LinearPlan& lp, cudaStream_t stream) {
+  uniform_offsets_kernel<<<1, 64, 0, stream>>>(lp.rows, lp.n, lp.offsets);
+  gemm_schedule_kernel<<<1, 1024, 0, stream>>>(lp.offsets, lp.n, lp.n * lp.rows, 128, 128, lp.prefix0,
+                                               const_cast<int32_t*>(lp.p.tile_prefix), nullptr, 0);
+}
+
+void launch_linear(const LinearPlan& lp, cudaStream_t stream) {
+  grouped_gemm_kernel<1><<<lp.grid, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(lp.mA, lp.mB, lp.mBs, lp.p);
+}
+
+constexpr int kLatentMaxShared = 8;
+
+struct LatentLayout {
+  size_t route, idx, w, offsets, perm_token, inv_perm, z, z_perm, h, y_perm, n, o, perm_ws, ffn_ws, lin, x_rep, hs,
+      ys, sh_offsets, ffn_ws_sh, total;
+};
+
+LatentLayout latent_layout(int T, int d, int l, int E, int k, int f, int S, int fs) {
+  LatentLayout L{};
+  const size_t Tk = static_cast<size_t>(T) * k;
+  const size_t ST = static_cast<size_t>(S) * T;
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t here = at;
+    at += align256(bytes);
+    return here;
+  };
+  L.route = take(route_plan(T, d, E).ws_bytes);
+  L.idx = take(Tk * 4);
+  L.w = take(Tk * 4);
+  L.offsets = take((static_cast<size_t>(E) + 1) * 4);
+  L.perm_token = take(Tk * 4);
+  L.inv_perm = take(Tk * 4);
+  L.z = take(static_cast<size_t>(T) * l * 2);
+  L.z_perm = take(Tk * l * 2);
+  L.h = take(Tk * f * 2);
+  L.y_perm = take(Tk * l * 2);
+  L.n = take(static_cast<size_t>(T) * l * 2);
+  L.o = take(static_cast<size_t>(T) * d * 2);
+  L.perm_ws = take(permute_ws(T, E, k));
+  L.ffn_ws = take(ffn_ws(T * k, E));
+  L.lin = take(3 * align256(2 * 4));  // offsets, prefix0, prefix1 of the one-expert projections
+  if (S > 0) {
+    L.x_rep = take(ST * d * 2);
+    L.hs = take(ST * fs * 2);
+    L.ys = take(ST * d * 2);
+    L.sh_offsets = take((static_cast<size_t>(S) + 1) * 4);
+    L.ffn_ws_sh = take(ffn_ws(S * T, S));
+  }
+  L.total = at;
+  return L;
+}
+
+bool latent_shape_ok(int T, int d, int l, int E, int k, int f, int S, int fs) {
+  const bool dims = d >= 64 && d % 64 == 0 && d <= 32768 && l >= 64 && l % 64 == 0 && l <= 8192 && f >= 64 &&
+                    f % 64 == 0 && f <= 32768 && S >= 0 && S <= kLatentMaxShared &&
+                    (S == 0 || (fs >= 64 && fs % 64 == 0 && fs <= 32768));
+  return dims && shape_ok(T, d, E, k) && static_cast<int64_t>(T) * (S > 0 ? S : 1) < (int64_t(1) << 31);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_latent_workspace_size(int T, int d, int l, int E, int k, int f, int S, int fs) {
+  if (!latent_shape_ok(T, d, l, E, k, f, S, fs)) return 0;
+  return latent_layout(T, d, l, E, k, f, S, fs).total;
+}
+
+moe_status_t moe_latent_forward(const moe_bf16_t* x, const float* W_router, const float* router_bias,
+                                const moe_bf16_t* W_dn, const moe_bf16_t* W_up, const moe_bf16_t* W_gate_up,
+                                const moe_bf16_t* W_down, const float* gamma, const moe_bf16_t* Ws_gate_up,
+                                const moe_bf16_t* Ws_down, int T, int d, int l, int E, int k, int f, int S, int fs,
+                                int act, float beta1, float beta2, float eps, moe_bf16_t* out, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream) {
+  if (!x || !W_router || !W_dn || !W_up || !W_gate_up || !W_down || !out) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!Ws_gate_up || !Ws_down)) return MOE_ERR_INVALID_ARG;
+  if (!latent_shape_ok(T, d, l, E, k, f, S, fs)) return MOE_ERR_INVALID_ARG;
+  if (act != 0 && act != 1) return MOE_ERR_INVALID_ARG;
+  if (act == 1 && !(beta1 > 0.0f && beta2 > 0.0f && std::isfinite(beta1) && std::isfinite(beta2)))
+    return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !std::isfinite(eps)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {static_cast<const void*>(x), static_cast<const void*>(W_dn), static_cast<const void*>(W_up),
+                        static_cast<const void*>(W_gate_up), static_cast<const void*>(W_down),
+                        static_cast<const void*>(out)})
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!aligned16(Ws_gate_up) || !aligned16(Ws_down))) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  const LatentLayout L = latent_layout(T, d, l, E, k, f, S, fs);
+  if (!workspace || !aligned256(workspace) || workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  int sms = 0;
+  moe_status_t st = device_setup(&sms);
+  if (st != MOE_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm_token = reinterpret_cast<int32_t*>(ws + L.perm_token);
+  int32_t* inv_perm = reinterpret_cast<int32_t*>(ws + L.inv_perm);
+  moe_bf16_t* z = reinterpret_cast<moe_bf16_t*>(ws + L.z);
+  moe_bf16_t* z_perm = reinterpret_cast<moe_bf16_t*>(ws + L.z_perm);
+  moe_bf16_t* h = reinterpret_cast<moe_bf16_t*>(ws + L.h);
+  moe_bf16_t* y_perm = reinterpret_cast<moe_bf16_t*>(ws + L.y_perm);
+  moe_bf16_t* nrm = reinterpret_cast<moe_bf16_t*>(ws + L.n);
+  moe_bf16_t* o = reinterpret_cast<moe_bf16_t*>(ws + L.o);
+  int32_t* lin_off = reinterpret_cast<int32_t*>(ws + L.lin);
+  int32_t* lin_pre0 = reinterpret_cast<int32_t*>(ws + L.lin + align256(8));
+  int32_t* lin_pre1 = reinterpret_cast<int32_t*>(ws + L.lin + 2 * align256(8));
+  const int Tk = T * k;
+
+  // plans (host only: tensor maps and parameters)
+  LinearPlan down_proj, up_proj;
+  st = plan_linear(x, W_dn, z, T, 1, d, l, lin_off, lin_pre0, lin_pre1, sms, &down_proj);
+  if (st != MOE_OK) return st;
+  st = plan_linear(nrm, W_up, o, T, 1, l, d, lin_off, lin_pre0, lin_pre1, sms, &up_proj);
+  if (st != MOE_OK) return st;
+  FfnPlan fr;
+  st = plan_ffn(z_perm, offsets, W_gate_up, W_down, Tk, l, E, f, h, y_perm, ws + L.ffn_ws, sms, &fr);
+  if (st != MOE_OK) return st;
+  fr.act = act;
+  fr.p0.beta1 = beta1;
+  fr.p0.beta2 = beta2;
+  FfnPlan fsh;
+  moe_bf16_t* x_rep = nullptr;
+  moe_bf16_t* ys = nullptr;
+  if (S > 0) {
+    x_rep = reinterpret_cast<moe_bf16_t*>(ws + L.x_rep);
+    ys = reinterpret_cast<moe_bf16_t*>(ws + L.ys);
+    st = plan_ffn(x_rep, reinterpret_cast<int32_t*>(ws + L.sh_offsets), Ws_gate_up, Ws_down, S * T, d, S, fs,
+                  reinterpret_cast<moe_bf16_t*>(ws + L.hs), ys, ws + L.ffn_ws_sh, sms, &fsh);
+    if (st != MOE_OK) return st;
+    fsh.act = act;
+    fsh.p0.beta1 = beta1;
+    fsh.p0.beta2 = beta2;
+  }
+
+  // 1-3. route on x
+  st = launch_route(x, W_router, router_bias, T, d, E, k, idx, w, ws + L.route, stream);
+  if (st != MOE_OK) return st;
+  // z = x W_dn (one-expert GEMM)
+  launch_linear_schedule(down_proj, stream);
+  launch_linear(down_proj, stream);
+  // dispatch z rows, the routed SiTU-GLU experts on z
+  if (Tk <= kSmallDispatchPairs) {
+    dispatch_small_kernel<<<1, 1024, 0, stream>>>(idx, Tk, E, k, gemm_block_rows(fr.mode0), gemm_block_rows(fr.mode1),
+                                                  offsets, perm_token, inv_perm,
+                                                  const_cast<int32_t*>(fr.p0.tile_prefix),
+                                                  const_cast<int32_t*>(fr.p1.tile_prefix), fr.ticket_buf,
+                                                  fr.split_ticket_words);
+    permute_copy_rows_kernel<<<static_cast<unsigned>(ceil_div64(Tk, 8)), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(z), T, perm_token, Tk, l / 8, reinterpret_cast<uint4*>(z_perm));
+  } else {
+    st = launch_permute(z, idx, T, l, E, k, offsets, perm_token, inv_perm, z_perm, ws + L.perm_ws, stream);
+    if (st != MOE_OK) return st;
+    launch_schedule(fr, stream);
+  }
+  launch_gemm_gate_up(fr, stream);
+  launch_gemm_down(fr, stream);
+  // u = sum_j p_j E_j(z), RMSNorm -> n; o = n W_up
+  const int vpr_l = l / 8;
+  switch (k) {
+#define MOE_LATENT_RMS_CASE(K)                                                                            \
+  case K:                                                                                                 \
+    combine_rmsnorm_kernel<K><<<static_cast<unsigned>(T), 256, 0, stream>>>(                             \
+        reinterpret_cast<const uint4*>(y_perm), inv_perm, w, gamma, eps, T, vpr_l, reinterpret_cast<uint4*>(nrm)); \
+    break;
+    MOE_LATENT_RMS_CASE(1) MOE_LATENT_RMS_CASE(2) MOE_LATENT_RMS_CASE(3) MOE_LATENT_RMS_CASE(4)
+    MOE_LATENT_RMS_CASE(5) MOE_LATENT_RMS_CASE(6) MOE_LATENT_RMS_CASE(7) MOE_LATENT_RMS_CASE(8)
+    MOE_LATENT_RMS_CASE(9) MOE_LATENT_RMS_CASE(10) MOE_LATENT_RMS_CASE(11) MOE_LATENT_RMS_CASE(12)
+    MOE_LATENT_RMS_CASE(13) MOE_LATENT_RMS_CASE(14) MOE_LATENT_RMS_CASE(15) MOE_LATENT_RMS_CASE(16)
+#undef MOE_LATENT_RMS_CASE
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+  launch_linear(up_proj, stream);  // same one-expert tables as the down projection
+  // shared experts on x, then out = o + sum_s y_s
+  const int64_t nvec = static_cast<int64_t>(T) * d / 8;
+  if (S > 0) {
+    repeat_rows_kernel<<<static_cast<unsigned>(ceil_div64(nvec, 256)), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(x), nvec, S, reinterpret_cast<uint4*>(x_rep));
+    uniform_offsets_kernel<<<1, 64, 0, stream>>>(T, S, const_cast<int32_t*>(fsh.p0.expert_offsets));
+    launch_schedule(fsh, stream);
+    launch_gemm_gate_up(fsh, stream);
+    launch_gemm_down(fsh, stream);
+  }
+  sum_rows_kernel<<<static_cast<unsigned>(ceil_div64(nvec, 256)), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(o), reinterpret_cast<const uint4*>(ys), S, nvec, reinterpret_cast<uint4*>(out));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

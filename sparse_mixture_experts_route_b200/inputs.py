@@ -178,3 +178,51 @@ def make_mx_values(shape_t, block_axis: int, seed: int = 0, device="cpu") -> tor
     vd = torch.where(neg0, torch.full_like(vd, -0.0), vd)
     out = vd.reshape(tuple(vb.shape[:-2]) + (-1,)).to(torch.bfloat16).movedim(-1, ax).contiguous()
     return out.to(device)
+
+
+@dataclass
+class LatentInputs:
+    """One seeded draw of the Stable LatentMoE layer's operands."""
+
+    shape: MoEShape                  # T, d (model width), E, k, f (routed expert width), bias
+    l: int                           # latent width
+    x: torch.Tensor                  # [T, d] bf16
+    W_router: torch.Tensor           # [d, E] fp32
+    bias: Optional[torch.Tensor]     # [E] fp32 or None
+    W_dn: torch.Tensor               # [d, l] bf16
+    W_up: torch.Tensor               # [l, d] bf16
+    W_gate_up: torch.Tensor          # [E, l, 2f] bf16
+    W_down: torch.Tensor             # [E, f, l] bf16
+    gamma: torch.Tensor              # [l] fp32
+    Ws_gate_up: Optional[torch.Tensor]   # [S, d, 2fs] bf16
+    Ws_down: Optional[torch.Tensor]      # [S, fs, d] bf16
+
+
+def make_latent_inputs(shape: MoEShape, l: int, S: int, fs: int, seed: int = 0, device="cpu") -> LatentInputs:
+    """x and W_router as make_inputs (streams 0 and 1); W_dn ~ N(0, 1/d),
+    W_up ~ N(0, 1/l), routed W_gate_up ~ N(0, 1/l) and W_down ~ N(0, 1/f),
+    shared Ws_gate_up ~ N(0, 1/d) and Ws_down ~ N(0, 1/fs), all rounded to
+    bf16; gamma = 1 + N(0, 0.1^2) fp32. Streams 4..10 of the seed."""
+    d, E, f = shape.d, shape.E, shape.f
+    x = make_x(shape, seed, device)
+    W_router = make_router(shape, seed, device)
+    bias = zipf_bias(E).to(device) if shape.bias == "zipf" else None
+    W_dn = _randn_bf16((d, l), 1.0 / math.sqrt(d), _gen(seed, 4, device), device)
+    W_up = _randn_bf16((l, d), 1.0 / math.sqrt(l), _gen(seed, 5, device), device)
+    W_gate_up = _randn_bf16((E, l, 2 * f), 1.0 / math.sqrt(l), _gen(seed, 6, device), device)
+    W_down = _randn_bf16((E, f, l), 1.0 / math.sqrt(f), _gen(seed, 7, device), device)
+    gamma = 1.0 + 0.1 * torch.randn(l, generator=_gen(seed, 8, device), device=device, dtype=torch.float32)
+    if S > 0:
+        Ws_gate_up = _randn_bf16((S, d, 2 * fs), 1.0 / math.sqrt(d), _gen(seed, 9, device), device)
+        Ws_down = _randn_bf16((S, fs, d), 1.0 / math.sqrt(fs), _gen(seed, 10, device), device)
+    else:
+        Ws_gate_up = Ws_down = None
+    return LatentInputs(shape, l, x, W_router, bias, W_dn, W_up, W_gate_up, W_down, gamma, Ws_gate_up, Ws_down)
+
+
+#: The Stable LatentMoE layer at the page's widths (d = 7168, l = 3584, 896
+#: routed experts, 16 active, two shared experts); the expert widths are not
+#: on the page: f = 512 for the routed experts (as in the other 896-expert
+#: workloads) and fs = 2048 for the shared ones.
+LATENT = {"shape": MoEShape("latent_prefill", 4096, 7168, 896, 16, 512, note="Stable LatentMoE"),
+          "l": 3584, "S": 2, "fs": 2048}
