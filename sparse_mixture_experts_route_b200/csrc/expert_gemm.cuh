@@ -58,18 +58,16 @@ constexpr int kTmemSlotCols = 256;
 // Modes: 0 gate/up with 256-row token blocks (3 stages of 64 KB), 2 gate/up
 // with 128-row token blocks (4 stages of 48 KB: more stages in flight when no
 // expert fills a 256-row block), 1 down with 128-row blocks (4 stages of
-// 48 KB), 3 down with 256-row blocks (3 stages of 64 KB: for heavily loaded
-// experts, each weight tile is read once per 256 rows and every stage carries
-// twice the MMA work). The 256-row modes never take the stream-K split.
-__host__ __device__ constexpr bool gemm_is_gate_up(int mode) { return mode == 0 || mode == 2; }
-__host__ __device__ constexpr int gemm_block_rows(int mode) { return (mode == 0 || mode == 3) ? 256 : 128; }
+// 48 KB). Mode 0 never takes the stream-K split.
+__host__ __device__ constexpr bool gemm_is_gate_up(int mode) { return mode != 1; }
+__host__ __device__ constexpr int gemm_block_rows(int mode) { return mode == 0 ? 256 : 128; }
 
 template <int kMode>
 struct GemmCfg {
   static constexpr int kABytes = kGemmBK * kGemmBMF * 2;         // 16 KB per A operand
   static constexpr int kAHalf = kABytes / 2;                     // one 64-feature box (8 KB)
   static constexpr int kBRows = gemm_block_rows(kMode);          // 256 / 128
-  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB (256-row modes) / 16 KB
+  static constexpr int kBBytes = kBRows * kGemmBK * 2;           // 32 KB (mode 0) / 16 KB
   static constexpr int kStageBytes = 2 * kABytes + kBBytes;      // 64 KB / 48 KB
   static constexpr int kStages = (kBRows == 256) ? 3 : 4;
   static constexpr int kTmemCols = 2 * kTmemSlotCols;            // 512
@@ -100,13 +98,6 @@ struct GemmParams {
   // CTA order, which is ascending K, and finishes the tile. tickets[] start at
   // zero and are put back to zero.
   int stream_k;
-  // Whole-tile scheduling takes the tiles in the order 0, n-1, 1, n-2, ...
-  // instead of 0, 1, 2, ... (interleave != 0). Tiles are expert-major, so
-  // when a few experts hold most rows (compute-bound tiles at the front) and
-  // many hold few (weight-streaming tiles at the back) every wave mixes both;
-  // a heavy expert's consecutive tiles still run in the same wave and share
-  // its weight tile in L2. Results do not depend on the order.
-  int interleave;
   int b_fixed_row;        // >= 0: every tile's token operand starts at this row (one-token steps read x itself)
   float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
   unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
@@ -165,9 +156,8 @@ __device__ __forceinline__ bool work_item(const GemmParams& p, const int32_t* pr
   const int KB = p.K / kGemmBK;
   const int ntiles = pre[p.E] * p.n_feat_tiles;
   if (!p.stream_k) {
-    const int u = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
-    if (u >= ntiles) return false;
-    const int t = p.interleave ? ((u & 1) ? ntiles - 1 - (u >> 1) : (u >> 1)) : u;
+    const int t = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+    if (t >= ntiles) return false;
     decode_tile<kMode>(p, pre, off, t, ti);
     ti.kb0 = 0;
     ti.kb1 = KB;

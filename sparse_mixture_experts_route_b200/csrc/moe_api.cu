@@ -65,8 +65,6 @@ moe_status_t device_setup(int* num_sms) {
       return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(grouped_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<1>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(grouped_gemm_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<3>::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(grouped_gemm_kernel<0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<0>::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(grouped_gemm_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -418,7 +416,7 @@ struct FfnPlan {
   GemmParams p0, p1;
   int grid0, grid1;
   int mode0;  // gate/up: 0 256-row blocks, 2 128-row blocks
-  int mode1;  // down: 1 128-row blocks, 3 256-row blocks
+  int mode1;  // down: 1 (128-row blocks)
   int act = 0;  // gate/up GLU: 0 SwiGLU, 1 SiTU-GLU (p0.beta1, p0.beta2)
   int rows;                   // Tk: rows of x_perm, h and y_perm
   int split_ticket_words;     // stream-K tickets the schedule kernel clears (0: none)
@@ -447,14 +445,13 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p0.out = h;
   // 256-row blocks pay off only when experts average more than 128 rows
   fp->mode0 = (static_cast<int64_t>(Tk) > static_cast<int64_t>(E) * 128) ? 0 : 2;
-  fp->mode1 = fp->mode0 == 0 ? 3 : 1;
+  fp->mode1 = 1;
   const int64_t tiles0 = (ceil_div64(Tk, gemm_block_rows(fp->mode0)) + min_e_tk) * p0.n_feat_tiles;
   const bool stream_ok = ffn_split_possible(Tk, E);
   uint8_t* split_base = static_cast<uint8_t*>(ws) + 2 * ffn_prefix_bytes(E);
   float* part = stream_ok ? reinterpret_cast<float*>(split_base) : nullptr;
   unsigned int* tickets = stream_ok ? reinterpret_cast<unsigned int*>(split_base + ffn_split_part_bytes()) : nullptr;
   p0.b_fixed_row = -1;
-  p0.interleave = fp->mode0 == 0 ? 1 : 0;  // heavily loaded experts: mix compute- and weight-bound tiles per wave
   p0.stream_k = (stream_ok && fp->mode0 == 2 && tiles0 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
   p0.part = p0.stream_k ? part : nullptr;
   p0.tickets = p0.stream_k ? tickets : nullptr;
@@ -470,7 +467,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   p1.a1_offset = kGemmBMF;
   p1.out = y_perm;
   const int64_t tiles1 = (ceil_div64(Tk, gemm_block_rows(fp->mode1)) + min_e_tk) * p1.n_feat_tiles;
-  p1.stream_k = (stream_ok && fp->mode1 == 1 && tiles1 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
+  p1.stream_k = (stream_ok && tiles1 <= kStreamKMaxWaves * kStreamKCtas) ? 1 : 0;
   p1.part = p1.stream_k ? part : nullptr;
   p1.tickets = p1.stream_k ? tickets : nullptr;
   fp->grid1 = p1.stream_k ? (kStreamKCtas < num_sms ? kStreamKCtas : num_sms)
@@ -506,10 +503,7 @@ void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
     grouped_gemm_kernel<2><<<fp.grid0, kGemmThreads, GemmCfg<2>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0, fp.p0);
 }
 void launch_gemm_down(const FfnPlan& fp, cudaStream_t stream) {
-  if (fp.mode1 == 3)
-    grouped_gemm_kernel<3><<<fp.grid1, kGemmThreads, GemmCfg<3>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
-  else
-    grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
+  grouped_gemm_kernel<1><<<fp.grid1, kGemmThreads, GemmCfg<1>::kSmemBytes, stream>>>(fp.mA1, fp.mB1, fp.mBs1, fp.p1);
 }
 
 bool device_fused_ffn() {
@@ -1319,7 +1313,6 @@ moe_status_t plan_linear(const moe_bf16_t* A, const moe_bf16_t* W, moe_bf16_t* o
   p.a1_offset = kGemmBMF;
   p.out = reinterpret_cast<uint16_t*>(out);
   p.stream_k = 0;
-  p.interleave = 0;
   p.b_fixed_row = -1;
   const int64_t tiles = static_cast<int64_t>(n) * ceil_div64(rows, 128) * p.n_feat_tiles;
   lp->grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
