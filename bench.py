@@ -614,6 +614,17 @@ def run_ours(args):
     if rank != 0:  # each replica routes its own tokens
         inp.x = moe_inputs.make_x(shape, seed=replica_x_seed(rank), device=dev)
     T, d, E, k, f = shape.T, shape.d, shape.E, shape.k, shape.f
+    if args.mx:
+        # the MX serving format alone, on this workload (for profiling runs)
+        experts = _lib.moe_mx_pack_experts(inp.W_gate_up, inp.W_down)
+        tm, cnt, clk = time_layer_mx(_lib, shape, inp, experts, args.steps, args.warmup, args.graph == "on", world,
+                                     flush, local)
+        if rank != 0:
+            return None
+        summ = mx_summary(shape, tm, cnt, clk, args.steps, world, peaks)
+        return {"metric": METRIC + "_mx", "value": summ["tokens_per_s"], "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": "e4m3 x e2m1",
+                "data": "synthetic", "config": {**shape.as_dict(), "experts": "MXFP4, activations MXFP8"}, **summ}
     res = time_layer(_lib, shape, inp, args.steps, args.warmup, args.graph == "on", world, flush, local,
                      count_launches=True)
     out = res["out"]
@@ -849,6 +860,7 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="time only --workload (skip the decode, skewed and sweep entries of the line)")
     ap.add_argument("--no-mx", action="store_true", help="skip the MX-format entries of the workloads")
+    ap.add_argument("--mx", action="store_true", help="time only moe_forward_mx on --workload (profiling runs)")
     ap.add_argument("--no-latent", action="store_true", help="skip the Stable LatentMoE entry of the workloads")
     ap.add_argument("--workload-steps", type=int, default=10,
                     help="timed steps of each of the other workloads")

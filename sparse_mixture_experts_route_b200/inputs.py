@@ -75,6 +75,9 @@ WORKLOADS = {
 WORKLOADS["prefill_small"] = MoEShape("prefill_small", 1024, 7168, 32, 8, 2048, note="profiling size")
 #: Skewed-shaped (Zipf-like bias, top-16) with 128 experts: 2.8 GB of weights.
 WORKLOADS["skewed_small"] = MoEShape("skewed_small", 2048, 7168, 128, 16, 512, bias="zipf", note="profiling size")
+#: Decode-shaped (T=128, top-4, f=2048) with 32 experts: 2.8 GB of bf16
+#: weights, 0.75 GB in the MX format (both more than L2), for full ncu captures.
+WORKLOADS["decode_small"] = MoEShape("decode_small", 128, 7168, 32, 4, 2048, note="profiling size")
 #: One token, 16 of 64 experts at the sweep's widths: 1.4 GB of weights (more
 #: than L2) for full ncu captures of the one-token step's kernels.
 WORKLOADS["onetoken_small"] = MoEShape("onetoken_small", 1, 7168, 64, 16, 512, note="profiling size")

@@ -28,8 +28,8 @@ MUTATIONS = {
                   "const double silu = g / (1.0 + std::exp(g));"),
     "down_transposed": ("wrow[c] = bf16_to_double(Wd[j * d + c]);",
                         "wrow[c] = bf16_to_double(Wd[(c % f) * d + (j + c / f) % d]);"),
-    "combine_drops_last_slot": ("for (int64_t j = 0; j < k; ++j) {\n      const double* yr",
-                                "for (int64_t j = 0; j < k - 1; ++j) {\n      const double* yr"),
+    "combine_drops_last_slot": ("for (int64_t j = 0; j < k; ++j) {\n      const double* yr = y_rows",
+                                "for (int64_t j = 0; j < k - 1; ++j) {\n      const double* yr = y_rows"),
     "permute_descending_tokens": ("const int32_t r = cursor[e]++;",
                                   "const int32_t r = offsets[e + 1] - 1 - (cursor[e]++ - offsets[e]);"),
     "bias_dropped": ("l[e] = l[e] + bias[e];", "l[e] = l[e] + 0.0f * bias[e];"),
