@@ -28,10 +28,14 @@
 // TMEM holds two 256-column slots: a tile with N <= 128 uses one slot (the
 // epilogue of one tile overlaps the MMAs of the next), a tile with N > 128 both.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+// Warp roles (320 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one lane): smem ring of kStages stages;
 //   warp 1      TMEM allocator and MMA issuer (one lane);
-//   warps 2..5  epilogue: tcgen05.ld -> fp32 math -> bf16 stores.
+//   warps 2..9  epilogue: tcgen05.ld -> fp32 math -> bf16 stores. A warp may
+//               read only the TMEM lane quadrant warp % 4, so each quadrant
+//               (32 features) has two epilogue warps, which take alternate
+//               32-token chunks of the tile: the epilogue's 2-byte stores and
+//               GLU math then keep up with the MMAs of the next tile.
 // Tiles are (expert, feature block, token block), enumerated from the device
 // copy of the expert offsets, so there is no host synchronisation; consecutive
 // tiles share a weight tile when an expert has several token blocks.
@@ -50,7 +54,8 @@ namespace moe {
 
 constexpr int kGemmBK = 64;         // K per stage: one 128-byte swizzle row of bf16
 constexpr int kGemmBMF = 128;       // output features per A operand (UMMA M)
-constexpr int kGemmThreads = 192;
+constexpr int kGemmEpiWarps = 8;                   // two per TMEM lane quadrant
+constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
 constexpr int kGemmBoxRows = 128;   // rows of the large B box
 constexpr int kGemmSmallBox = 32;   // rows of the small B box (tiles of <= 32 rows)
 constexpr int kTmemSlotCols = 256;
@@ -100,7 +105,7 @@ struct GemmParams {
   int stream_k;
   int b_fixed_row;        // >= 0: every tile's token operand starts at this row (one-token steps read x itself)
   float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
-  unsigned int* tickets;  // [tiles][4]: one per epilogue warp (32 features)
+  unsigned int* tickets;  // [tiles][kGemmEpiWarps]: one per epilogue warp (32 features x alternate chunks)
   float beta1, beta2;     // SiTU-GLU soft caps (gate/up kernels with kAct = 1 only)
 };
 
@@ -329,15 +334,18 @@ __device__ __forceinline__ void signal_h_slice(unsigned int* ready, int e, int l
   if (lane == 0) atomicAdd(ready + e, 1u);
 }
 
-// Epilogue warp q (TMEM lanes 32q..32q+31 = features), one work item: waits
-// for the accumulators, then either stores the finished rows (mode 0/2: h =
+// Epilogue warp (q, h): TMEM lanes 32q..32q+31 (features) and the 32-token
+// chunks h, h + 2, ... of the tile's columns. One work item: waits for the
+// accumulators, then either stores the finished rows (mode 0/2: h =
 // SiLU(g) * u; mode 1: the two 128-feature halves of y), or, for a stream-K
 // partial item, writes its fp32 partials and, if it is the last of the tile's
-// contributors, adds them in K order and stores the rows. With kSignal, a
-// finished gate/up slice is counted in ready[e]. Returns false if a wait gave up.
+// contributors for this warp's rows, adds them in K order and stores the
+// rows. With kSignal, a finished gate/up slice is counted in ready[e].
+// Returns false if a wait gave up.
+constexpr int kGemmEpiHalves = kGemmEpiWarps / 4;
 template <int kMode, bool kSignal, int kAct = 0>
 __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const GemmParams& p, const int32_t* pre,
-                                                   const TileInfo& ti, int q, int lane, uint32_t (&uses)[2],
+                                                   const TileInfo& ti, int q, int h, int lane, uint32_t (&uses)[2],
                                                    int& next_slot, unsigned int* ready) {
   const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
   const SlotPlan sp = slot_plan(ti.nrows, next_slot);
@@ -361,7 +369,7 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
     // slot is free as soon as it is read
     const int fl = q * 32 + lane;
     float* mine = p.part + static_cast<int64_t>(ti.slot) * kSplitPartFloats;
-    for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+    for (int c0 = 32 * h; c0 < ti.nrows; c0 += 32 * kGemmEpiHalves) {
       uint32_t g[32], u[32];
       tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
       tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
@@ -382,41 +390,46 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
       ++uses[sp.first + j];
     }
     // the tile's contributors are CTAs c_first..c_last; per (tile, warp),
-    // the last one to finish adds their partials in CTA order (K order)
+    // the last one to finish adds their partials in CTA order (K order) for
+    // this warp's rows
     const int KB = p.K / kGemmBK;
     const int per = stream_k_per(pre[p.E] * p.n_feat_tiles, KB);
     const int c_first = (ti.t * KB) / per, c_last = ((ti.t + 1) * KB - 1) / per;
     __threadfence();
     __syncwarp();
     unsigned int tk = 0u;
-    if (lane == 0) tk = atomicAdd(&p.tickets[ti.t * 4 + q], 1u);
+    const int wslot = ti.t * kGemmEpiWarps + h * 4 + q;
+    if (lane == 0) tk = atomicAdd(&p.tickets[wslot], 1u);
     tk = __shfl_sync(0xffffffffu, tk, 0);
     if (tk == static_cast<unsigned int>(c_last - c_first)) {
       __threadfence();
-      for (int i = 0; i < ti.nrows; ++i) {
-        float gs = 0.0f, us = 0.0f;
-        for (int c = c_first; c <= c_last; ++c) {
-          const int slot = 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
-          const float* src = p.part + static_cast<int64_t>(slot) * kSplitPartFloats;
-          const float gv = __ldcg(src + i * kGemmBMF + fl);
-          const float uv = __ldcg(src + (128 + i) * kGemmBMF + fl);
-          gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
-          us = (c == c_first) ? uv : __fadd_rn(us, uv);
-        }
-        uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
-        if (gemm_is_gate_up(kMode)) {
-          if (fa_ok) orow[fa] = bf16_bits(glu_f32<kAct>(gs, us, p));
-        } else {
-          if (fa_ok) orow[fa] = bf16_bits(gs);
-          if (fb_ok) orow[fb] = bf16_bits(us);
+      for (int c0 = 32 * h; c0 < ti.nrows; c0 += 32 * kGemmEpiHalves) {
+        const int c1 = min(c0 + 32, ti.nrows);
+        for (int i = c0; i < c1; ++i) {
+          float gs = 0.0f, us = 0.0f;
+          for (int c = c_first; c <= c_last; ++c) {
+            const int slot = 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
+            const float* src = p.part + static_cast<int64_t>(slot) * kSplitPartFloats;
+            const float gv = __ldcg(src + i * kGemmBMF + fl);
+            const float uv = __ldcg(src + (128 + i) * kGemmBMF + fl);
+            gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
+            us = (c == c_first) ? uv : __fadd_rn(us, uv);
+          }
+          uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
+          if (gemm_is_gate_up(kMode)) {
+            if (fa_ok) orow[fa] = bf16_bits(glu_f32<kAct>(gs, us, p));
+          } else {
+            if (fa_ok) orow[fa] = bf16_bits(gs);
+            if (fb_ok) orow[fb] = bf16_bits(us);
+          }
         }
       }
-      if (lane == 0) p.tickets[ti.t * 4 + q] = 0u;
+      if (lane == 0) p.tickets[wslot] = 0u;
       if (kSignal) signal_h_slice(ready, ti.e, lane);
     }
     return true;
   }
-  for (int c0 = 0; c0 < ti.nrows; c0 += 32) {
+  for (int c0 = 32 * h; c0 < ti.nrows; c0 += 32 * kGemmEpiHalves) {
     uint32_t g[32], u[32];
     tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
     tmem_ld_32x32b_x32(t1 + static_cast<uint32_t>(c0), u);
@@ -482,7 +495,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full_bar[b], 1);
-      mbar_init(&acc_empty_bar[b], 4);
+      mbar_init(&acc_empty_bar[b], kGemmEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -566,12 +579,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int q = warp & 3;         // TMEM lane quadrant this warp may access
+    const int h = (warp - 2) >> 2;  // its share of the token chunks
     uint32_t uses[2] = {0u, 0u};
     int next_slot = 0;
     TileInfo ti;
     for (int it = 0; work_item<kMode>(p, s_pre, s_off, it, ti); ++it)
-      if (!gemm_epilogue_item<kMode, false, kAct>(ring, p, s_pre, ti, q, lane, uses, next_slot, nullptr)) break;
+      if (!gemm_epilogue_item<kMode, false, kAct>(ring, p, s_pre, ti, q, h, lane, uses, next_slot, nullptr)) break;
   }
 
   tc_fence_before_sync();
@@ -589,9 +603,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // cooperative launch: each CTA takes its gate/up work items, then its down
 // work items, in one pipeline. A down item of expert e needs all of e's h
 // rows, which other CTAs' gate/up items write: each epilogue warp that
-// finishes a 32-feature slice of an h tile counts it in h_ready[e], and the
-// producer loads a down item's token rows (h) only once h_ready[e] reaches
-// 4 * (gate/up feature tiles). Its weight boxes do not depend on h, so the
+// finishes its slice of an h tile counts it in h_ready[e], and the producer
+// loads a down item's token rows (h) only once h_ready[e] reaches
+// kGemmEpiWarps * (gate/up feature tiles). Its weight boxes do not depend on h, so the
 // producer issues them at once and keeps up to a ring of stages whose token
 // rows are still pending: the down weights stream while the last gate/up
 // tiles finish, and neither GEMM pays its own launch, ramp-up and drain. The
@@ -660,7 +674,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full_bar[b], 1);
-      mbar_init(&acc_empty_bar[b], 4);
+      mbar_init(&acc_empty_bar[b], kGemmEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -681,7 +695,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const GemmRing ring{smem, full_bar, empty_bar, acc_full_bar, acc_empty_bar, abort_flag, *tmem_slot};
-  const unsigned int h_target = 4u * static_cast<unsigned int>(p0.n_feat_tiles);
+  const unsigned int h_target = static_cast<unsigned int>(kGemmEpiWarps * p0.n_feat_tiles);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -800,14 +814,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
     uint32_t uses[2] = {0u, 0u};
     int next_slot = 0;
     FusedIter fi;
     TileInfo ti;
     while (fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
       const bool ok = (fi.phase == 0)
-                          ? gemm_epilogue_item<2, true>(ring, p0, s_pre0, ti, q, lane, uses, next_slot, h_ready)
-                          : gemm_epilogue_item<1, false>(ring, p1, s_pre1, ti, q, lane, uses, next_slot, nullptr);
+                          ? gemm_epilogue_item<2, true>(ring, p0, s_pre0, ti, q, h, lane, uses, next_slot, h_ready)
+                          : gemm_epilogue_item<1, false>(ring, p1, s_pre1, ti, q, h, lane, uses, next_slot, nullptr);
       if (!ok) break;
     }
   }

@@ -370,12 +370,12 @@ constexpr int kStreamKMaxWaves = 4;
 
 // Workspace of the expert FFN: the two tile-prefix arrays, then (only when
 // stream-K is possible for this Tk and E, i.e. min(E, Tk) <= the tile limit)
-// the partials (two slots per CTA) and the tickets (four per tile).
+// the partials (two slots per CTA) and the tickets (one per tile and epilogue warp).
 size_t ffn_split_part_bytes() {
   return align256(static_cast<size_t>(2 * kStreamKCtas) * kSplitPartFloats * sizeof(float));
 }
 size_t ffn_split_ticket_bytes() {
-  return align256(static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * 4 * sizeof(unsigned));
+  return align256(static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * kGemmEpiWarps * sizeof(unsigned));
 }
 bool ffn_split_possible(int Tk, int E) { return (E < Tk ? E : Tk) <= kStreamKMaxWaves * kStreamKCtas; }
 size_t ffn_prefix_bytes(int E) { return align256(static_cast<size_t>(E + 1) * sizeof(int32_t)); }
@@ -476,7 +476,7 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
   // share them; each tile's last contributor puts its tickets back to zero)
   const int64_t max_tiles = (p0.stream_k ? tiles0 : 0) > (p1.stream_k ? tiles1 : 0) ? (p0.stream_k ? tiles0 : 0)
                                                                                       : (p1.stream_k ? tiles1 : 0);
-  fp->split_ticket_words = static_cast<int>(max_tiles) * 4;
+  fp->split_ticket_words = static_cast<int>(max_tiles) * kGemmEpiWarps;
   fp->ticket_buf = tickets;
   return MOE_OK;
 }
@@ -582,12 +582,12 @@ struct ForwardLayout {
 constexpr int kFusedMaxTokens = kGemmSmallBox;
 bool ffn_fused_shape(int T) { return T <= kFusedMaxTokens; }
 
-// The fused launch's down phase has its own stream-K tickets (four per tile)
+// The fused launch's down phase has its own stream-K tickets (one per tile and epilogue warp)
 // and partial slots (two per CTA), plus the h_ready counters [E]. They sit
 // right after the gate/up GEMM's tickets, which end the feed-forward
 // workspace, so one zeroing pass clears both phases' tickets and the counters:
 // [tickets0][tickets1][h_ready][part1].
-size_t fused_ticket_words() { return static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * 4; }
+size_t fused_ticket_words() { return static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * kGemmEpiWarps; }
 size_t fused_ws(int E) {
   return align256((fused_ticket_words() + static_cast<size_t>(E)) * sizeof(unsigned)) + ffn_split_part_bytes();
 }
