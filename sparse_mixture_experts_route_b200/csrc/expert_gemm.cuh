@@ -104,9 +104,10 @@ struct GemmParams {
   // zero and are put back to zero.
   int stream_k;
   int b_fixed_row;        // >= 0: every tile's token operand starts at this row (one-token steps read x itself)
-  float* part;            // [2 * gridDim.x][2][128 rows][128 features] fp32
+  float* part;            // [slots][2][part_rows rows][128 features] fp32
   unsigned int* tickets;  // [tiles][kGemmEpiWarps]: one per epilogue warp (32 features x alternate chunks)
   float beta1, beta2;     // SiTU-GLU soft caps (gate/up kernels with kAct = 1 only)
+  int part_rows = 128;    // rows of one partial's accumulators (32 when no tile has more)
 };
 
 // fp32 elements of one partial: two accumulators, 128 rows x 128 features
@@ -117,6 +118,9 @@ struct TileInfo {
   int t, kb0, kb1;                  // tile index, K-block range [kb0, kb1) of this item
   bool partial;                     // the item covers only part of the tile's K range
   int slot;                         // partial slot of this CTA's item
+  // chunked items (the one-launch feed-forward): the tile's partials are the
+  // slots chunk_first .. chunk_first + chunk_count - 1, in K order
+  int chunk_first = 0, chunk_count = 0;
 };
 
 // Tile t -> (expert, feature block, token block), from shared-memory copies of
@@ -368,7 +372,8 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
     // stream-K partial item: fp32 accumulators to part[slot]; the TMEM
     // slot is free as soon as it is read
     const int fl = q * 32 + lane;
-    float* mine = p.part + static_cast<int64_t>(ti.slot) * kSplitPartFloats;
+    const int64_t slot_floats = 2 * static_cast<int64_t>(p.part_rows) * kGemmBMF;
+    float* mine = p.part + ti.slot * slot_floats;
     for (int c0 = 32 * h; c0 < ti.nrows; c0 += 32 * kGemmEpiHalves) {
       uint32_t g[32], u[32];
       tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
@@ -379,7 +384,7 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
       for (int i = 0; i < 32; ++i) {
         if (i < nv) {
           __stcg(mine + (c0 + i) * kGemmBMF + fl, __uint_as_float(g[i]));
-          __stcg(mine + (128 + c0 + i) * kGemmBMF + fl, __uint_as_float(u[i]));
+          __stcg(mine + (p.part_rows + c0 + i) * kGemmBMF + fl, __uint_as_float(u[i]));
         }
       }
     }
@@ -389,12 +394,20 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
       if (lane == 0) mbar_arrive(&r.acc_empty_bar[sp.first + j]);
       ++uses[sp.first + j];
     }
-    // the tile's contributors are CTAs c_first..c_last; per (tile, warp),
-    // the last one to finish adds their partials in CTA order (K order) for
-    // this warp's rows
+    // the tile's contributors: CTAs c_first..c_last (stream-K; slot 2c for a
+    // CTA's first item, 2c + 1 for its last) or, for a chunked item, chunks
+    // chunk_first..; per (tile, warp), the last one to finish adds their
+    // partials in that order (K order) for this warp's rows
+    int c_first, c_last, per = 0;
     const int KB = p.K / kGemmBK;
-    const int per = stream_k_per(pre[p.E] * p.n_feat_tiles, KB);
-    const int c_first = (ti.t * KB) / per, c_last = ((ti.t + 1) * KB - 1) / per;
+    if (ti.chunk_count > 0) {
+      c_first = ti.chunk_first;
+      c_last = ti.chunk_first + ti.chunk_count - 1;
+    } else {
+      per = stream_k_per(pre[p.E] * p.n_feat_tiles, KB);
+      c_first = (ti.t * KB) / per;
+      c_last = ((ti.t + 1) * KB - 1) / per;
+    }
     __threadfence();
     __syncwarp();
     unsigned int tk = 0u;
@@ -406,14 +419,29 @@ __device__ __forceinline__ bool gemm_epilogue_item(const GemmRing& r, const Gemm
       for (int c0 = 32 * h; c0 < ti.nrows; c0 += 32 * kGemmEpiHalves) {
         const int c1 = min(c0 + 32, ti.nrows);
         for (int i = c0; i < c1; ++i) {
+          // the contributors' partials, eight loads in flight at a time, added
+          // one after another in contributor order
           float gs = 0.0f, us = 0.0f;
-          for (int c = c_first; c <= c_last; ++c) {
-            const int slot = 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
-            const float* src = p.part + static_cast<int64_t>(slot) * kSplitPartFloats;
-            const float gv = __ldcg(src + i * kGemmBMF + fl);
-            const float uv = __ldcg(src + (128 + i) * kGemmBMF + fl);
-            gs = (c == c_first) ? gv : __fadd_rn(gs, gv);
-            us = (c == c_first) ? uv : __fadd_rn(us, uv);
+          for (int cb = c_first; cb <= c_last; cb += 8) {
+            float gv[8], uv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = cb + j;
+              if (c <= c_last) {
+                const int slot = ti.chunk_count > 0 ? c : 2 * c + ((ti.t == (c * per) / KB) ? 0 : 1);
+                const float* src = p.part + slot * slot_floats;
+                gv[j] = __ldcg(src + i * kGemmBMF + fl);
+                uv[j] = __ldcg(src + (p.part_rows + i) * kGemmBMF + fl);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = cb + j;
+              if (c <= c_last) {
+                gs = (c == c_first) ? gv[j] : __fadd_rn(gs, gv[j]);
+                us = (c == c_first) ? uv[j] : __fadd_rn(us, uv[j]);
+              }
+            }
           }
           uint16_t* orow = p.out + static_cast<int64_t>(ti.row0 + i) * p.n_feat;
           if (gemm_is_gate_up(kMode)) {
@@ -599,54 +627,89 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ------------------------------------------- one launch for both GEMMs
 //
 // For steps in which no expert has more than 32 rows (T <= 32), the gate/up
-// GEMM (mode 2 items) and the down GEMM (mode 1 items) run in one persistent
-// cooperative launch: each CTA takes its gate/up work items, then its down
-// work items, in one pipeline. A down item of expert e needs all of e's h
-// rows, which other CTAs' gate/up items write: each epilogue warp that
-// finishes its slice of an h tile counts it in h_ready[e], and the producer
-// loads a down item's token rows (h) only once h_ready[e] reaches
-// kGemmEpiWarps * (gate/up feature tiles). Its weight boxes do not depend on h, so the
-// producer issues them at once and keeps up to a ring of stages whose token
-// rows are still pending: the down weights stream while the last gate/up
-// tiles finish, and neither GEMM pays its own launch, ramp-up and drain. The
-// launch is cooperative (every CTA resident), so a wait on another CTA always
-// ends; it is bounded anyway, recording MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY.
-// Stream-K partial slots and tickets of the two phases are disjoint
-// (p0.part / p1.part, p0.tickets / p1.tickets).
+// GEMM (mode 2) and the down GEMM (mode 1) run in one persistent cooperative
+// launch whose CTAs take their work from a shared queue: chunk ids are handed
+// out one at a time by an atomic counter, gate/up chunks first, then down
+// chunks, both in expert-major tile order. A chunk is one tile's K-block range
+// [j * ck, (j + 1) * ck); a GEMM with few tiles cuts each of them into up to
+// kFusedTargetChunks / tiles chunks (about four per SM) so that every SM stays busy, one with many
+// tiles hands out whole tiles. Because the queue is shared, a CTA that streams
+// its weights faster simply takes more chunks: no SM waits at the end of the
+// gate/up chunks for a slower one, and the experts' h tiles are finished in
+// expert order, well before the down chunks that read them are handed out.
+//
+// A chunk's fp32 accumulators go to the partial slot of its chunk id; the
+// last chunk of a tile to finish (a ticket per tile and epilogue warp) adds
+// the tile's partials in chunk order, which is ascending K, and stores the
+// rows. Which CTA takes which chunk depends on timing, but every sum is taken
+// in the fixed order, so results are deterministic. A down chunk of expert e
+// needs all of e's h rows: each epilogue warp that finishes its slice of an h
+// tile counts it in h_ready[e], and the producer loads a down chunk's token
+// rows (h) only once h_ready[e] reaches kGemmEpiWarps * (gate/up feature
+// tiles); its weight boxes do not depend on h, so the producer issues them at
+// once and keeps up to a ring of stages whose token rows are still pending.
+// The producer lane claims the chunks and passes each id to the MMA lane and
+// the epilogue warps through a small shared-memory queue (kFusedQueue entries,
+// one mbarrier pair each). The launch is cooperative (every CTA resident), so
+// a wait on another CTA always ends; it is bounded anyway, recording
+// MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY. The claim counter, the tickets and
+// h_ready start at zero (the dispatch step clears them).
 
-constexpr int kFusedSmemBytes = GemmCfg<1>::kStages * GemmCfg<1>::kStageBytes + GemmCfg<1>::kBarrierBytes +
-                                3 * (1024 + 1) * 4 + 8 + 1024;
+// Partial slots per GEMM: one per chunk, of 2 x 32 rows x 128 features fp32.
+// A tile is cut into at most kFusedMaxCpt chunks (the partials its last chunk
+// adds).
+constexpr int kFusedSlots = 2 * 148 * (128 / kGemmSmallBox);
+constexpr int kFusedMaxCpt = 16;
+constexpr int kFusedTargetChunks = 4 * 148;  // per GEMM: about four chunks per SM
+constexpr int kFusedQueue = 16;
+constexpr int kFusedBarrierBytes = 512;
+constexpr int kFusedSmemBytes = GemmCfg<1>::kStages * GemmCfg<1>::kStageBytes + kFusedBarrierBytes +
+                                kFusedQueue * 4 + 3 * (1024 + 1) * 4 + 8 + 1024;
 static_assert(GemmCfg<1>::kStageBytes == GemmCfg<2>::kStageBytes && GemmCfg<1>::kStages == GemmCfg<2>::kStages,
-              "the fused launch runs mode 2 and mode 1 items in one ring");
+              "the fused launch runs mode 2 and mode 1 chunks in one ring");
 static_assert(kFusedSmemBytes <= 232448, "shared memory per CTA");
+static_assert((2 * GemmCfg<1>::kStages + 5 + 2 * kFusedQueue) * 8 + 8 <= kFusedBarrierBytes, "fused barriers");
 
-// Items of one CTA: its gate/up work items, then its down work items.
-struct FusedIter {
-  int phase = 0, it = 0;
+// How one GEMM of the fused launch is cut into chunks (the same in every CTA).
+struct FusedPlan {
+  int KB;      // K blocks per tile
+  int ck;      // K blocks per chunk
+  int cpt;     // chunks per tile
+  int chunks;  // tiles * cpt
 };
-__device__ __forceinline__ bool fused_next(const GemmParams& p0, const GemmParams& p1, const int32_t* pre0,
-                                           const int32_t* pre1, const int32_t* off, FusedIter& f, TileInfo& ti) {
-  if (f.phase == 0) {
-    if (work_item<2>(p0, pre0, off, f.it, ti)) {
-      ++f.it;
-      return true;
-    }
-    f.phase = 1;
-    f.it = 0;
-  }
-  if (work_item<1>(p1, pre1, off, f.it, ti)) {
-    ++f.it;
-    return true;
-  }
-  return false;
+__device__ __forceinline__ FusedPlan fused_plan(const GemmParams& p, int tiles) {
+  FusedPlan f;
+  f.KB = p.K / kGemmBK;
+  int cpt = tiles > 0 ? kFusedTargetChunks / tiles : 1;
+  cpt = max(1, min(min(cpt, kFusedMaxCpt), f.KB));
+  f.ck = (f.KB + cpt - 1) / cpt;
+  f.cpt = (f.KB + f.ck - 1) / f.ck;  // no empty chunk
+  f.chunks = tiles * f.cpt;
+  return f;
+}
+
+// Chunk c of one GEMM -> its work item.
+template <int kMode>
+__device__ __forceinline__ void fused_chunk(const GemmParams& p, const int32_t* pre, const int32_t* off,
+                                            const FusedPlan& f, int c, TileInfo& ti) {
+  const int t = c / f.cpt, j = c - (c / f.cpt) * f.cpt;
+  decode_tile<kMode>(p, pre, off, t, ti);
+  ti.kb0 = j * f.ck;
+  ti.kb1 = min(f.KB, ti.kb0 + f.ck);
+  ti.partial = f.cpt > 1;
+  ti.slot = c;
+  ti.chunk_first = t * f.cpt;
+  ti.chunk_count = f.cpt;
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_ffn_fused_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmBs0,
                              const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmBs1,
-                             const GemmParams p0, const GemmParams p1, unsigned int* __restrict__ h_ready) {
+                             const GemmParams p0, const GemmParams p1, unsigned int* __restrict__ h_ready,
+                             unsigned int* __restrict__ claim) {
   using Cfg = GemmCfg<1>;
   constexpr int S = Cfg::kStages;
+  constexpr int Q = kFusedQueue;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
@@ -654,9 +717,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full_bar = empty_bar + S;
   uint64_t* acc_empty_bar = acc_full_bar + 2;
   uint64_t* drain_bar = acc_empty_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* q_full = drain_bar + 1;   // [Q] the producer has written entry i
+  uint64_t* q_empty = q_full + Q;     // [Q] the MMA lane and every epilogue warp have read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + Q);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_pre0 = reinterpret_cast<int32_t*>(smem + S * Cfg::kStageBytes + Cfg::kBarrierBytes);
+  volatile int* s_chunk = reinterpret_cast<volatile int*>(smem + S * Cfg::kStageBytes + kFusedBarrierBytes);
+  int32_t* s_pre0 = reinterpret_cast<int32_t*>(smem + S * Cfg::kStageBytes + kFusedBarrierBytes + Q * 4);
   int32_t* s_pre1 = s_pre0 + (p0.E + 1);
   int32_t* s_off = s_pre1 + (p0.E + 1);
 
@@ -677,6 +743,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty_bar[b], kGemmEpiWarps);
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < Q; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1 + kGemmEpiWarps);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_shared();
@@ -696,6 +766,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after_sync();
   const GemmRing ring{smem, full_bar, empty_bar, acc_full_bar, acc_empty_bar, abort_flag, *tmem_slot};
   const unsigned int h_target = static_cast<unsigned int>(kGemmEpiWarps * p0.n_feat_tiles);
+  const FusedPlan f0 = fused_plan(p0, s_pre0[p0.E] * p0.n_feat_tiles);
+  const FusedPlan f1 = fused_plan(p1, s_pre1[p0.E] * p1.n_feat_tiles);
+  const int total = f0.chunks + f1.chunks;
+  // chunk id -> work item of the gate/up (true) or the down GEMM
+  auto decode = [&](int c, TileInfo& ti) -> bool {
+    if (c < f0.chunks) {
+      fused_chunk<2>(p0, s_pre0, s_off, f0, c, ti);
+      return true;
+    }
+    fused_chunk<1>(p1, s_pre1, s_off, f1, c - f0.chunks, ti);
+    return false;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -705,6 +787,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr uint32_t kTx = 2 * Cfg::kABytes + kGemmSmallBox * kGemmBK * 2;  // every tile fits the small box
       int s = 0;
       uint32_t ph = 0;
+      int qi = 0;
+      uint32_t qph = 0;
       int issued = 0;
       bool ok = true;
       // down stages whose weight boxes are issued and whose h rows are not yet:
@@ -746,15 +830,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           --q_n;
         }
       };
-      FusedIter fi;
-      TileInfo ti;
-      while (ok && fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
-        const bool down = fi.phase == 1;
+      while (ok) {
+        const unsigned int id = atomicAdd(claim, 1u);
+        const int c = id < static_cast<unsigned int>(total) ? static_cast<int>(id) : -1;
+        // hand the id to the MMA lane and the epilogue warps
+        if (!mbar_wait_bounded(&q_empty[qi], qph ^ 1u, kWaitLimitNs, abort_flag)) {
+          record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
+          ok = false;
+          break;
+        }
+        s_chunk[qi] = c;
+        mbar_arrive(&q_full[qi]);
+        if (++qi == Q) {
+          qi = 0;
+          qph ^= 1u;
+        }
+        if (c < 0) break;
+        TileInfo ti;
+        const bool down = !decode(c, ti);
         for (int kb = ti.kb0; kb < ti.kb1; ++kb) {
           if (q_n == S) flush(true);  // the ring holds only stages waiting for h
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
             record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
-            *abort_flag = 1;
             ok = false;
             break;
           }
@@ -766,11 +863,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             gemm_load_b<2>(st, &tmBs0, &tmBs0, &full_bar[s], p0, ti.row0, 1, k0, pol_x);
           } else {
             gemm_load_a<1>(st, &tmA1, &full_bar[s], p1, ti, k0, pol_w);
-            const int qi = (q_head + q_n) % S;
-            q_stage[qi] = s;
-            q_k0[qi] = k0;
-            q_row[qi] = ti.row0;
-            q_e[qi] = ti.e;
+            const int qj = (q_head + q_n) % S;
+            q_stage[qj] = s;
+            q_k0[qj] = k0;
+            q_row[qj] = ti.row0;
+            q_e[qj] = ti.e;
             ++q_n;
             flush(false);
           }
@@ -796,14 +893,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
+      int qi = 0;
+      uint32_t qph = 0;
       uint32_t uses[2] = {0u, 0u};
       int next_slot = 0;
       bool any = false;
-      FusedIter fi;
-      TileInfo ti;
-      while (fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
-        const bool ok = (fi.phase == 0) ? gemm_mma_item<2>(ring, ti, s, ph, uses, next_slot, any)
-                                        : gemm_mma_item<1>(ring, ti, s, ph, uses, next_slot, any);
+      while (true) {
+        if (!mbar_wait_bounded(&q_full[qi], qph, kWaitLimitNs, abort_flag)) {
+          if (!*abort_flag) record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+          *abort_flag = 1;
+          break;
+        }
+        const int c = s_chunk[qi];
+        mbar_arrive(&q_empty[qi]);
+        if (++qi == Q) {
+          qi = 0;
+          qph ^= 1u;
+        }
+        if (c < 0) break;
+        TileInfo ti;
+        const bool ok = decode(c, ti) ? gemm_mma_item<2>(ring, ti, s, ph, uses, next_slot, any)
+                                      : gemm_mma_item<1>(ring, ti, s, ph, uses, next_slot, any);
         if (!ok) break;
       }
       if (any) {
@@ -815,12 +925,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
+    int qi = 0;
+    uint32_t qph = 0;
     uint32_t uses[2] = {0u, 0u};
     int next_slot = 0;
-    FusedIter fi;
-    TileInfo ti;
-    while (fused_next(p0, p1, s_pre0, s_pre1, s_off, fi, ti)) {
-      const bool ok = (fi.phase == 0)
+    while (true) {
+      if (!mbar_wait_bounded(&q_full[qi], qph, kWaitLimitNs, abort_flag)) {
+        if (!*abort_flag) record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
+        *abort_flag = 1;
+        break;
+      }
+      const int c = s_chunk[qi];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[qi]);
+      if (++qi == Q) {
+        qi = 0;
+        qph ^= 1u;
+      }
+      if (c < 0) break;
+      TileInfo ti;
+      const bool ok = decode(c, ti)
                           ? gemm_epilogue_item<2, true>(ring, p0, s_pre0, ti, q, h, lane, uses, next_slot, h_ready)
                           : gemm_epilogue_item<1, false>(ring, p1, s_pre1, ti, q, h, lane, uses, next_slot, nullptr);
       if (!ok) break;

@@ -514,9 +514,10 @@ bool device_fused_ffn() {
 }
 
 // Both GEMMs in one cooperative launch of min(148, SMs) CTAs (one per SM), so
-// that every CTA whose down items wait for another CTA's h rows is resident.
-// Both phases' stream-K splits use that grid.
-moe_status_t launch_ffn_fused(FfnPlan& fp, unsigned int* h_ready, int num_sms, cudaStream_t stream) {
+// that every CTA whose down chunks wait for another CTA's h rows is resident.
+// claim: the chunk counter (zero at launch).
+moe_status_t launch_ffn_fused(FfnPlan& fp, unsigned int* h_ready, unsigned int* claim, int num_sms,
+                              cudaStream_t stream) {
   const int grid = kStreamKCtas < num_sms ? kStreamKCtas : num_sms;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -529,7 +530,7 @@ moe_status_t launch_ffn_fused(FfnPlan& fp, unsigned int* h_ready, int num_sms, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_ffn_fused_kernel, fp.mA0, fp.mBs0, fp.mA1, fp.mBs1, fp.p0,
-                                           fp.p1, h_ready);
+                                           fp.p1, h_ready, claim);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -582,15 +583,21 @@ struct ForwardLayout {
 constexpr int kFusedMaxTokens = kGemmSmallBox;
 bool ffn_fused_shape(int T) { return T <= kFusedMaxTokens; }
 
-// The fused launch's down phase has its own stream-K tickets (one per tile and epilogue warp)
-// and partial slots (two per CTA), plus the h_ready counters [E]. They sit
-// right after the gate/up GEMM's tickets, which end the feed-forward
-// workspace, so one zeroing pass clears both phases' tickets and the counters:
-// [tickets0][tickets1][h_ready][part1].
+// The fused launch's down GEMM has its own tickets (one per tile and epilogue
+// warp) and partial slots, plus the h_ready counters [E] and the chunk
+// counter. They sit right after the gate/up GEMM's tickets, which end the
+// feed-forward workspace, so one zeroing pass clears both GEMMs' tickets and
+// the counters: [tickets0][tickets1][h_ready][claim][part1]. Each GEMM's
+// partials are kFusedSlots compact slots (2 x 32 rows x 128 features fp32),
+// which fill exactly the stream-K partial area of the two-launch path.
 size_t fused_ticket_words() { return static_cast<size_t>(kStreamKMaxWaves * kStreamKCtas) * kGemmEpiWarps; }
-size_t fused_ws(int E) {
-  return align256((fused_ticket_words() + static_cast<size_t>(E)) * sizeof(unsigned)) + ffn_split_part_bytes();
-}
+size_t fused_counter_words(int E) { return fused_ticket_words() + static_cast<size_t>(E) + 1; }
+static_assert(static_cast<size_t>(kFusedSlots) * 2 * kGemmSmallBox * kGemmBMF <=
+                  static_cast<size_t>(2 * kStreamKCtas) * kSplitPartFloats,
+              "fused partial slots");
+static_assert(kFusedSlots / 2 <= kStreamKMaxWaves * kStreamKCtas,
+              "a GEMM cut into chunks has at most kFusedSlots / 2 tiles, each with its tickets");
+size_t fused_ws(int E) { return align256(fused_counter_words(E) * sizeof(unsigned)) + ffn_split_part_bytes(); }
 
 ForwardLayout forward_layout(int T, int d, int E, int k, int f) {
   ForwardLayout L;
@@ -742,8 +749,10 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
     fp.p0.tickets = fp.ticket_buf;
     fp.p0.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(fp.ticket_buf) - ffn_split_part_bytes());
     fp.p1.tickets = tickets1;
-    fp.p1.part = reinterpret_cast<float*>(ws + L.fused_ws + align256((fused_ticket_words() + E) * sizeof(unsigned)));
-    fp.split_ticket_words = static_cast<int>(2 * fused_ticket_words()) + E;
+    fp.p1.part = reinterpret_cast<float*>(ws + L.fused_ws + align256(fused_counter_words(E) * sizeof(unsigned)));
+    fp.p0.part_rows = kGemmSmallBox;  // no tile of a step of <= 32 tokens has more rows
+    fp.p1.part_rows = kGemmSmallBox;
+    fp.split_ticket_words = static_cast<int>(fused_ticket_words() + fused_counter_words(E));
   }
   // stage boundaries: events (timed calls) and NVTX ranges named for the
   // stage, which profilers show around the stage's launches (no cost without one)
@@ -801,7 +810,7 @@ moe_status_t forward_impl(const moe_bf16_t* x, const float* W_router, const floa
   mark(3);
   mark(4);
   if (fused) {
-    st = launch_ffn_fused(fp, h_ready, sms, stream);
+    st = launch_ffn_fused(fp, h_ready, h_ready + E, sms, stream);
     if (st != MOE_OK) return st;
   } else {
     launch_gemm_gate_up(fp, stream);

@@ -103,10 +103,10 @@ def test_workspace_sizes(lib):
         Tk = T * k
         inter = Tk * 4 * 4 + (E + 1) * 4 + Tk * d * 2 * 2 + Tk * f * 2
         # steps of <= 32 tokens run both GEMMs in one launch: a second set of
-        # stream-K tickets (592 tiles x 8 epilogue warps) and h_ready [E] (int32), and 296
+        # stream-K tickets (592 tiles x 8 epilogue warps), h_ready [E] and the chunk counter (int32), and 296
         # partial slots of 2 x 128 x 128 fp32
         a256 = lambda n: (n + 255) // 256 * 256
-        fused = a256((592 * 8 + E) * 4) + a256(296 * 2 * 128 * 128 * 4) if T <= 32 else 0
+        fused = a256((592 * 8 + E + 1) * 4) + a256(296 * 2 * 128 * 128 * 4) if T <= 32 else 0
         assert fw >= rw + pw + ew + inter + fused
         assert fw % 256 == 0 and rw % 256 == 0 and pw % 256 == 0 and ew % 256 == 0
         assert rw >= T * E * 4

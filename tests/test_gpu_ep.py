@@ -5,7 +5,8 @@ device). With one rank every exchange is a local copy, but the whole path
 runs -- count and row all-to-alls through NCCL, the index maps on the device,
 the gathers, the grouped feed-forward of the rank's experts and the combine,
 all in this library's kernels -- and must match the oracle within the layer
-tolerance and moe_forward bit for bit. The protocol across several ranks is
+tolerance and the staged entry points (route, permute, expert_ffn,
+unpermute) bit for bit. The protocol across several ranks is
 tested on CPU ranks in test_ep_gloo.py."""
 import datetime
 import os
@@ -80,6 +81,10 @@ def test_ep_forward_one_rank(lib, nccl_group, shape, mode):
     ref, _, _ = oracle.forward(inp.x.cpu(), inp.W_router.cpu(), inp.bias.cpu() if inp.bias is not None else None,
                                inp.W_gate_up.cpu(), inp.W_down.cpu(), k)
     parity.assert_layer_close(out, ref, f"ep_forward {shape} {mode}")
-    fused = lib.moe_forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    # one rank runs the staged steps on its rows: the same bits as those steps
+    idx, w = lib.moe_route(inp.x, inp.W_router, inp.bias, k)
+    offs, _, inv, xp = lib.moe_permute(inp.x, idx, E)
+    _, y = lib.moe_expert_ffn(xp, offs, inp.W_gate_up, inp.W_down)
+    staged = lib.moe_unpermute(y, inv, w)
     torch.cuda.synchronize()
-    assert torch.equal(out.view(torch.int16), fused.view(torch.int16))
+    assert torch.equal(out.view(torch.int16), staged.view(torch.int16))
