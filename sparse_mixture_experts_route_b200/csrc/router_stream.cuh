@@ -50,7 +50,7 @@ __host__ __device__ constexpr int router_stream_smem_bytes(int tmax) {
 // expert order): expert offsets and both GEMM token-block prefixes
 // (offsets[e] = prefix[e] = number of selected experts below e), perm_token
 // (all token 0), inv_perm (the row of each slot); zero_n words of zero_buf are
-// cleared (the GEMMs' stream-K tickets).
+// cleared (the feed-forward's tickets and counters), by all CTAs at the start.
 struct RouteDispatch {
   int32_t* offsets;
   int32_t* perm_token;
@@ -85,6 +85,13 @@ __global__ void __launch_bounds__(kRsThreads)
   if (tid == 0) {
     mbar_init(&bar, 1);
     fence_barrier_init();
+  }
+  if (TMAX == 1 && disp.zero_buf != nullptr) {
+    // the feed-forward's counters, cleared by all CTAs at once (only the next
+    // launch reads them)
+    const int64_t nth = static_cast<int64_t>(G) * C * kRsThreads;
+    for (int64_t i = (static_cast<int64_t>(c) * G + g) * kRsThreads + tid; i < disp.zero_n; i += nth)
+      disp.zero_buf[i] = 0u;
   }
   __syncthreads();
   if (tid == 0) mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nr * ne * 4));
@@ -201,7 +208,6 @@ __global__ void __launch_bounds__(kRsThreads)
   __shared__ int32_t s_sel[16];
   __syncthreads();  // the selection (written by warp 0) is visible to the CTA
   if (tid < k) s_sel[tid] = __ldcg(topk_idx + tid);
-  for (int i = tid; i < disp.zero_n; i += kRsThreads) disp.zero_buf[i] = 0u;
   __syncthreads();
   for (int e = tid; e <= E; e += kRsThreads) {
     int32_t below = 0;
