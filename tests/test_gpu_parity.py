@@ -323,6 +323,31 @@ def test_forward_zipf_bias(lib):
     parity.assert_layer_close(out, ref, "forward zipf")
 
 
+# Experts average more than 128 rows, so the gate/up GEMM takes 256-row
+# blocks (both TMEM slots per tile), and the dispatch is the multi-block one.
+# The Zipf-like bias gives experts with several full blocks and experts with
+# a few rows side by side; f = 384 makes the down K six blocks, d = 320 a
+# half-empty second output tile.
+@pytest.mark.parametrize("shape", [(1500, 256, 16, 4, 384), (2100, 320, 12, 2, 128)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_forward_heavy_and_light_experts(lib, shape):
+    T, d, E, k, f = shape
+    inp = _inputs(T, d, E, k, f, bias="zipf")
+    _, ridx, _ = parity.oracle_route(inp, k)
+    counts = np.bincount(ridx.ravel(), minlength=E)
+    assert T * k > 2048 and T * k > 128 * E
+    assert (counts >= 256).any() and ((counts > 0) & (counts < 256)).any(), counts
+    g = _cuda(inp)
+    out = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k)
+    out2 = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    assert torch.equal(out, out2)
+    ref, _, _ = oracle.forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(out, ref, "forward heavy and light experts")
+    _ffn_check(lib, inp, k)
+
+
 @pytest.mark.parametrize("shape", [(333, 320, 20, 3, 192), (600, 128, 4, 2, 128)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_forward_host_buffers(lib, shape):
