@@ -624,6 +624,246 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------- gate/up on CTA pairs
+//
+// The gate/up GEMM when experts average more than 128 rows (256-row token
+// blocks; the skewed loads, whose heavily loaded experts make the tensor core
+// the limit). A cluster of two CTAs (one TPC) shares each MMA (tcgen05
+// .cta_group::2, M = 256): a pair tile is 256 gate features and the 256
+// matching up features of one expert times one token block of up to 256
+// rows, N = the block's rows rounded up to 16. CTA r (rank in the pair) loads
+// gate and up features f0 + 128 r .. f0 + 128 r + 127 and token rows
+// row0 + r N/2 .. of each 64-wide K block: 48 KB per stage per SM, 8.4 MFLOP
+// of its MMA work on a full block (the single-CTA 256-row kernel loads 64 KB
+// for the same work), and four stages in flight instead of three for the
+// weight-streaming tiles of lightly loaded experts. Each CTA's TMEM receives
+// its 128 features x N tokens of both accumulators, so each CTA's epilogue
+// finishes its own features. The even CTA (rank 0) posts the stage's expected
+// bytes (both CTAs' loads complete on its barrier), issues the MMAs, and
+// frees the stage in both CTAs with one multicast commit; both CTAs' epilogue
+// warps arrive on its accumulator-empty barrier. No load uses cluster
+// multicast. Token blocks: the schedule kernel's 256-row prefix (prefix0).
+constexpr int kPairStages = 4;
+constexpr int kPairABytes = 128 * kGemmBK * 2;                     // one A operand half: 16 KB
+constexpr int kPairBBytes = 128 * kGemmBK * 2;                     // 128 token rows: 16 KB
+constexpr int kPairStageBytes = 2 * kPairABytes + kPairBBytes;     // 48 KB
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 256 + 2 * (1024 + 1) * 4 + 8 + 1024;
+static_assert(kPairSmemBytes <= 232448, "shared memory per CTA");
+
+template <int kAct>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const GemmParams p) {
+  constexpr int S = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S * kPairStageBytes);
+  uint64_t* empty_bar = full_bar + S;
+  uint64_t* acc_full_bar = empty_bar + S;
+  uint64_t* acc_empty_bar = acc_full_bar + 1;
+  uint64_t* drain_bar = acc_empty_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_pre = reinterpret_cast<int32_t*>(smem + S * kPairStageBytes + 256);
+  int32_t* s_off = s_pre + (p.E + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const int pair = static_cast<int>(blockIdx.x) >> 1, npairs = static_cast<int>(gridDim.x) >> 1;
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+    s_pre[i] = __ldg(p.tile_prefix + i);
+    s_off[i] = __ldg(p.expert_offsets + i);
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(acc_full_bar, 1);
+    mbar_init(acc_empty_bar, 2 * kGemmEpiWarps);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrive or load
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const int NP = p.n_feat_tiles;  // pair tiles per token block: ceil(f / 256)
+  const int KB = p.K / kGemmBK;
+  const int ntiles = s_pre[p.E] * NP;
+  // pair tile t -> expert, 256-feature block, 256-row token block
+  auto decode = [&](int t, int& e, int& np, int& row0, int& nrows) {
+    int lo = 0, hi = p.E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] * NP <= t)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    e = lo;
+    const int tbc = s_pre[e + 1] - s_pre[e];
+    const int local = t - s_pre[e] * NP;
+    np = local / tbc;
+    row0 = s_off[e] + (local % tbc) * 256;
+    nrows = min(256, s_off[e + 1] - row0);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_normal();  // a heavy expert's weights serve several token blocks
+      const uint64_t pol_x = l2_policy_evict_last();
+      uint32_t full_lead[S];
+#pragma unroll
+      for (int s = 0; s < S; ++s) full_lead[s] = smem_peer_u32(&full_bar[s], 0);
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < ntiles; t += npairs) {
+        int e, np, row0, nrows;
+        decode(t, e, np, row0, nrows);
+        const int f0 = np * 256 + static_cast<int>(rank) * 128;
+        const int half_n = max(16, (nrows + 15) & ~15) / 2;  // token rows of each CTA's B half
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, kWaitLimitNs, abort_flag)) {
+            record_device_error(1u /* MOE_DEVERR_WAIT_TIMEOUT_PRODUCER */);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kPairStageBytes;
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * kPairStageBytes);
+          const int k0 = kb * kGemmBK;
+          tma_load_3d_pair(st, &tmA, full_lead[s], f0, k0, e, pol_w);
+          tma_load_3d_pair(st + kPairABytes / 2, &tmA, full_lead[s], f0 + 64, k0, e, pol_w);
+          tma_load_3d_pair(st + kPairABytes, &tmA, full_lead[s], p.a1_offset + f0, k0, e, pol_w);
+          tma_load_3d_pair(st + kPairABytes + kPairABytes / 2, &tmA, full_lead[s], p.a1_offset + f0 + 64, k0, e,
+                           pol_w);
+          tma_load_2d_pair(st + 2 * kPairABytes, &tmB, full_lead[s], k0, row0 + static_cast<int>(rank) * half_n,
+                           pol_x);
+          ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      (void)issued;
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && rank == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t uses = 0;
+      bool any = false, ok = true;
+      for (int t = pair; ok && t < ntiles; t += npairs) {
+        int e, np, row0, nrows;
+        decode(t, e, np, row0, nrows);
+        const uint32_t idesc = umma_idesc_bf16_f32(256u, static_cast<uint32_t>(max(16, (nrows + 15) & ~15)), 1u, 0u);
+        if (!mbar_wait_bounded(acc_empty_bar, (uses & 1u) ^ 1u, kWaitLimitNs, abort_flag)) {
+          record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after_sync();
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[s], ph, kWaitLimitNs, abort_flag)) {
+            record_device_error(2u /* MOE_DEVERR_WAIT_TIMEOUT_MMA */);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(smem + s * kPairStageBytes);
+          const uint32_t b_addr = a_addr + 2 * kPairABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+            const uint64_t bdesc = umma_smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            const uint64_t adesc0 = umma_smem_desc_sw128(a_addr + kk * 2048, kPairABytes / 2, 1024);
+            const uint64_t adesc1 = umma_smem_desc_sw128(a_addr + kPairABytes + kk * 2048, kPairABytes / 2, 1024);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            tc_mma_bf16_pair(tmem_base, adesc0, bdesc, idesc, accum);
+            tc_mma_bf16_pair(tmem_base + 256u, adesc1, bdesc, idesc, accum);
+          }
+          tc_commit_pair_mc(&empty_bar[s], 0x3);  // stage s is free in both CTAs
+          any = true;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(acc_full_bar, 0x3);  // both CTAs' accumulators complete
+        ++uses;
+      }
+      if (any) {
+        tc_commit_pair_mc(drain_bar, 0x1);
+        mbar_wait_bounded(drain_bar, 0u, kWaitLimitNs, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t acc_empty_lead = smem_peer_u32(acc_empty_bar, 0);
+    uint32_t uses = 0;
+    for (int t = pair; t < ntiles; t += npairs) {
+      int e, np, row0, nrows;
+      decode(t, e, np, row0, nrows);
+      if (!mbar_wait_bounded(acc_full_bar, uses & 1u, kWaitLimitNs, abort_flag)) {
+        record_device_error(3u /* MOE_DEVERR_WAIT_TIMEOUT_EPILOGUE */);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after_sync();
+      const int fa = np * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      const bool fa_ok = fa < p.n_feat;
+      const uint32_t t0 = tmem_base + lane_base;
+      for (int c0 = 32 * h; c0 < nrows; c0 += 32 * kGemmEpiHalves) {
+        uint32_t g[32], u[32];
+        tmem_ld_32x32b_x32(t0 + static_cast<uint32_t>(c0), g);
+        tmem_ld_32x32b_x32(t0 + 256u + static_cast<uint32_t>(c0), u);
+        tmem_ld_wait();
+        uint16_t* orow = p.out + static_cast<int64_t>(row0 + c0) * p.n_feat;
+        const int nv = min(32, nrows - c0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (fa_ok && i < nv)
+            orow[static_cast<int64_t>(i) * p.n_feat + fa] =
+                bf16_bits(glu_f32<kAct>(__uint_as_float(g[i]), __uint_as_float(u[i]), p));
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_lead);
+      ++uses;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its pair may still use its barriers or TMEM
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
 // ------------------------------------------- one launch for both GEMMs
 //
 // For steps in which no expert has more than 32 rows (T <= 32), the gate/up

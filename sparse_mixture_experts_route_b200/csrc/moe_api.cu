@@ -38,6 +38,7 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   bool fused_ffn = false;  // the one-launch feed-forward fits one CTA on every SM (a cooperative launch)
+  int pair_grid = 0;       // CTAs of the CTA-pair gate/up kernel (two per cluster); 0: not available
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -88,6 +89,28 @@ moe_status_t device_setup(int* num_sms) {
                                                       kFusedSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
     di.fused_ffn = coop != 0 && per_sm >= 1;
+    // the CTA-pair gate/up kernel: clusters of two CTAs, as many as fit
+    di.pair_grid = 0;
+    if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPairSmemBytes) == cudaSuccess &&
+        cudaFuncSetAttribute(grouped_gemm_pair_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPairSmemBytes) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(sms - sms % 2));
+      cfg.blockDim = dim3(kGemmThreads);
+      cfg.dynamicSmemBytes = kPairSmemBytes;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<0>, &cfg) == cudaSuccess && clusters > 0)
+        di.pair_grid = 2 * (clusters < sms / 2 ? clusters : sms / 2);
+    }
+    cudaGetLastError();  // a device without cluster launches only loses the pair kernel
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -199,6 +222,14 @@ RoutePlan route_plan(int T, int d, int E) {
   const int64_t planes = (p.variant == kRouterFullBig) ? 1 : p.nchunks;
   p.ws_bytes = align256(static_cast<size_t>(planes) * T * E * sizeof(float));
   return p;
+}
+
+// CTAs of the CTA-pair gate/up kernel on the current device (0: none).
+int device_pair_grid() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return g_devices[dev].ready ? g_devices[dev].pair_grid : 0;
 }
 
 bool shape_ok(int T, int d, int E, int k) {
@@ -414,6 +445,9 @@ bool act_map(CUtensorMap* map, const moe_bf16_t* A, int rows, int K, int box_row
 struct FfnPlan {
   CUtensorMap mA0, mB0, mBs0, mA1, mB1, mBs1;
   GemmParams p0, p1;
+  // gate/up on CTA pairs (pairs0, 256-row blocks; p0 with 256-feature tiles)
+  bool pairs0 = false;
+  int pair_grid = 0;
   int grid0, grid1;
   int mode0;  // gate/up: 0 256-row blocks, 2 128-row blocks
   int mode1;  // down: 1 (128-row blocks)
@@ -478,6 +512,10 @@ moe_status_t plan_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const mo
                                                                                       : (p1.stream_k ? tiles1 : 0);
   fp->split_ticket_words = static_cast<int>(max_tiles) * kGemmEpiWarps;
   fp->ticket_buf = tickets;
+  // experts average more than 128 rows (256-row blocks): the gate/up GEMM
+  // runs on CTA pairs
+  fp->pair_grid = device_pair_grid();
+  fp->pairs0 = fp->mode0 == 0 && fp->pair_grid >= 2;
   return MOE_OK;
 }
 
@@ -487,7 +525,34 @@ void launch_schedule(const FfnPlan& fp, cudaStream_t stream) {
                                                const_cast<int32_t*>(fp.p1.tile_prefix), fp.ticket_buf,
                                                fp.split_ticket_words);
 }
+// The gate/up GEMM on CTA pairs (clusters of two): p0 as it stands at launch
+// (callers set the GLU's caps after planning), with 256-feature tiles.
+void launch_gemm_gate_up_pairs(const FfnPlan& fp, cudaStream_t stream) {
+  GemmParams ph = fp.p0;
+  ph.n_feat_tiles = ceil_div(ph.n_feat, 2 * kGemmBMF);
+  ph.stream_k = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(fp.pair_grid));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (fp.act == 1)
+    cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<1>, fp.mA0, fp.mB0, ph);
+  else
+    cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<0>, fp.mA0, fp.mB0, ph);
+}
 void launch_gemm_gate_up(const FfnPlan& fp, cudaStream_t stream) {
+  if (fp.pairs0) {
+    launch_gemm_gate_up_pairs(fp, stream);
+    return;
+  }
   if (fp.act == 1) {
     if (fp.mode0 == 0)
       grouped_gemm_kernel<0, 1><<<fp.grid0, kGemmThreads, GemmCfg<0>::kSmemBytes, stream>>>(fp.mA0, fp.mB0, fp.mBs0,
