@@ -415,7 +415,7 @@ def layer_summary(shape, res, steps: int, world: int, peaks: dict) -> dict:
                "bytes": alg["ffn_bytes"], "flops": alg["ffn_flops"],
                "rule": "touched experts x 6*d*f (gate, up and down weights, bf16)"}
     else:
-        dom = {"kernel": ("grouped_gemm_kernel<0>" if T * k > 128 * E else "grouped_gemm_kernel<2>")
+        dom = {"kernel": ("grouped_gemm_pair_kernel (CTA pairs)" if T * k > 128 * E else "grouped_gemm_kernel<2>")
                          + " (gate/up + SwiGLU)",
                "bytes": alg["gu_bytes"], "flops": alg["gu_flops"],
                "rule": "touched experts x 4*d*f (gate and up weights, bf16)"}
