@@ -71,6 +71,9 @@ moe_status_t device_setup(int* num_sms) {
         cudaFuncSetAttribute(grouped_gemm_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              GemmCfg<2>::kSmemBytes) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(router_one_token_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             router_one_smem_bytes()) != cudaSuccess)
+      return MOE_ERR_CUDA;
     if (cudaFuncSetAttribute(router_stream_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              router_stream_smem_bytes(1)) != cudaSuccess ||
         cudaFuncSetAttribute(router_stream_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -239,6 +242,7 @@ bool shape_ok(int T, int d, int E, int k) {
 
 bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
                 const cuuint32_t* box);
+bool router_w_map(CUtensorMap* map, const float* W, int d, int E);
 
 moe_status_t launch_route_tc(const RoutePlan& plan, const moe_bf16_t* x, const float* W_router, const float* bias,
                              int T, int d, int E, int k, int32_t* idx, float* w, void* ws, cudaStream_t stream) {
@@ -314,7 +318,14 @@ moe_status_t launch_route(const moe_bf16_t* x, const float* W_router, const floa
     const dim3 grid(G, plan.nchunks);
     const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
     const RouteDispatch none = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0};
-    if (T == 1) {
+    CUtensorMap wmap;
+    if (T == 1 && d <= kR1MaxD && router_w_map(&wmap, W_router, d, E)) {
+      // one CTA per 8 experts over all of d: no cross-CTA chunk sums
+      router_one_token_kernel<<<static_cast<unsigned>(ceil_div(E, kR1Experts)), 256, router_one_smem_bytes(),
+                                stream>>>(wmap, xb, bias, d, E, k, logits, tickets, idx, w,
+                                          disp != nullptr ? *disp : none);
+      if (dispatched != nullptr && disp != nullptr) *dispatched = true;
+    } else if (T == 1) {
       router_stream_kernel<1><<<grid, kRsThreads, router_stream_smem_bytes(1), stream>>>(
           xb, W_router, bias, T, d, E, k, lg, logits, tickets, idx, w, disp != nullptr ? *disp : none);
       if (dispatched != nullptr && disp != nullptr) *dispatched = true;
@@ -414,6 +425,19 @@ size_t ffn_ws(int Tk, int E) {
   size_t b = 2 * ffn_prefix_bytes(E);
   if (ffn_split_possible(Tk, E)) b += ffn_split_part_bytes() + ffn_split_ticket_bytes();
   return b;
+}
+
+// W_router [d][E] fp32 (E contiguous) in boxes of kR1Experts experts x
+// kR1BoxRows rows, unswizzled, for the one-token router.
+bool router_w_map(CUtensorMap* map, const float* W, int d, int E) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(E), static_cast<cuuint64_t>(d)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(E) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kR1Experts), static_cast<cuuint32_t>(kR1BoxRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(W), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 bool encode_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,

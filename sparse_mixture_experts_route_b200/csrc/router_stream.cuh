@@ -61,6 +61,36 @@ struct RouteDispatch {
   int zero_n;
 };
 
+// The end of a one-token route, by one CTA of 256 threads once all E logits
+// are in global memory: softmax and top-k, and, when disp.offsets != nullptr,
+// the dispatch tables of the step.
+__device__ __forceinline__ void one_token_finish(const float* logits, int E, int k, int32_t* topk_idx,
+                                                 float* topk_w, const RouteDispatch& disp) {
+  __shared__ float s_l[1024];
+  __shared__ int32_t s_sel[16];
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += 256) s_l[e] = __ldcg(logits + e);
+  __syncthreads();
+  cta_softmax_topk_256(s_l, E, k, topk_idx, topk_w);
+  if (disp.offsets == nullptr) return;
+  __syncthreads();  // the selection (written by warp 0) is visible to the CTA
+  if (tid < k) s_sel[tid] = __ldcg(topk_idx + tid);
+  __syncthreads();
+  for (int e = tid; e <= E; e += 256) {
+    int32_t below = 0;
+    for (int j = 0; j < k; ++j) below += (s_sel[j] < e) ? 1 : 0;
+    disp.offsets[e] = below;
+    disp.prefix0[e] = below;
+    disp.prefix1[e] = below;
+  }
+  if (tid < k) {
+    int32_t row = 0;
+    for (int j = 0; j < k; ++j) row += (s_sel[j] < s_sel[tid]) ? 1 : 0;
+    disp.perm_token[tid] = 0;
+    disp.inv_perm[tid] = row;
+  }
+}
+
 template <int TMAX>
 __global__ void __launch_bounds__(kRsThreads)
     router_stream_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W, const float* __restrict__ bias,
@@ -188,7 +218,6 @@ __global__ void __launch_bounds__(kRsThreads)
   }
 
   // the last group to finish takes softmax and top-k with the whole CTA
-  __shared__ float s_l[1024];
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -199,29 +228,124 @@ __global__ void __launch_bounds__(kRsThreads)
   if (s_ticket != static_cast<unsigned int>(G - 1)) return;
   __threadfence();
   if (tid == 0) tickets[G] = 0u;
-  for (int e = tid; e < E; e += kRsThreads) s_l[e] = __ldcg(logits + e);
-  __syncthreads();
-  cta_softmax_topk_256(s_l, E, k, topk_idx, topk_w);
-  if (disp.offsets == nullptr) return;
+  one_token_finish(logits, E, k, topk_idx, topk_w, disp);
+}
 
-  // the dispatch tables of this one-token step
-  __shared__ int32_t s_sel[16];
-  __syncthreads();  // the selection (written by warp 0) is visible to the CTA
-  if (tid < k) s_sel[tid] = __ldcg(topk_idx + tid);
+
+// One-token router without cross-CTA partial sums, for d <= kR1MaxD: CTA g
+// owns experts [8 g, 8 g + 8) and streams all d rows of W_router for them
+// (TMA boxes of 8 experts x 256 rows, fp32, 32 KB stages of 1024 rows in a
+// ring of four). The 256 threads form four groups of 64; group q takes the
+// stages q, q + 4, ... (ring slot q), and thread (c, e) of a group runs the
+// fma chain of chunk c (128 rows) of that stage for expert e, in the stated
+// order. When a group has read its slot it loads the slot's next stage
+// itself. Each CTA then adds its experts' C chunk sums in chunk order (+ bias)
+// and writes the final logits; the last CTA to finish (a ticket) takes the
+// softmax, the top-k and the dispatch tables. Same arithmetic and order as
+// the other router kernels, so the logits are bit-identical; two dependent
+// rounds of global partial sums fewer than router_stream_kernel<1>.
+constexpr int kR1Experts = 8;
+constexpr int kR1StageRows = 1024;
+constexpr int kR1BoxRows = 256;
+constexpr int kR1Slots = 4;
+constexpr int kR1MaxD = 8192;
+// x is widened into shared memory with 8 floats of padding after every
+// 128-value chunk, so the four chunks a warp reads at once sit in different
+// banks.
+__host__ __device__ constexpr int router_one_x_floats() { return kR1MaxD + (kR1MaxD / 128) * 8; }
+__host__ __device__ constexpr int router_one_smem_bytes() {
+  return kR1Slots * kR1StageRows * kR1Experts * 4 + router_one_x_floats() * 4 + (kR1MaxD / 128) * kR1Experts * 4;
+}
+
+__global__ void __launch_bounds__(256)
+    router_one_token_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ x,
+                            const float* __restrict__ bias, int d, int E, int k, float* __restrict__ logits,
+                            unsigned int* __restrict__ tickets, int32_t* __restrict__ topk_idx,
+                            float* __restrict__ topk_w, const RouteDispatch disp) {
+  extern __shared__ __align__(128) uint8_t r1_smem[];
+  float* ws = reinterpret_cast<float*>(r1_smem);                 // [slot][1024 rows][8 experts]
+  float* xs = ws + kR1Slots * kR1StageRows * kR1Experts;         // x widened, chunk c at 136 c
+  float* part = xs + router_one_x_floats();                      // chunk sums [C][8]
+  __shared__ __align__(8) uint64_t full[kR1Slots];
+  __shared__ unsigned int s_ticket;
+  const int g = blockIdx.x, G = gridDim.x, tid = threadIdx.x;
+  const int e0 = g * kR1Experts;
+  const int nst = (d + kR1StageRows - 1) / kR1StageRows;
+  const int C = (d + 127) / 128;
+  if (disp.zero_buf != nullptr) {
+    // the feed-forward's counters, cleared by all CTAs at once (only the next
+    // launch reads them)
+    for (int64_t i = static_cast<int64_t>(g) * 256 + tid; i < disp.zero_n; i += static_cast<int64_t>(G) * 256)
+      disp.zero_buf[i] = 0u;
+  }
+  // stage j into slot j % 4: its boxes of 256 rows that start inside d
+  auto issue = [&](int j) {
+    const int slot = j % kR1Slots;
+    const int r0 = j * kR1StageRows;
+    const int nbox = min(kR1StageRows / kR1BoxRows, (d - r0 + kR1BoxRows - 1) / kR1BoxRows);
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nbox * kR1BoxRows * kR1Experts * 4));
+    for (int b = 0; b < nbox; ++b)
+      tma_load_2d(ws + (slot * kR1StageRows + b * kR1BoxRows) * kR1Experts, &tmW, &full[slot], e0,
+                  r0 + b * kR1BoxRows, l2_policy_evict_first());
+  };
+  if (tid == 0) {
+    for (int s = 0; s < kR1Slots; ++s) mbar_init(&full[s], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+  }
   __syncthreads();
-  for (int e = tid; e <= E; e += kRsThreads) {
-    int32_t below = 0;
-    for (int j = 0; j < k; ++j) below += (s_sel[j] < e) ? 1 : 0;
-    disp.offsets[e] = below;
-    disp.prefix0[e] = below;
-    disp.prefix1[e] = below;
+  if (tid == 0)
+    for (int j = 0; j < kR1Slots && j < nst; ++j) issue(j);
+  for (int v = tid; v < d / 8; v += 256) {
+    const uint4 u = *reinterpret_cast<const uint4*>(x + v * 8);
+    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    float* dst = xs + v * 8 + (v >> 4) * 8;  // 16 vectors of 8 per 128-value chunk
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      dst[2 * h] = __uint_as_float(w4[h] << 16);
+      dst[2 * h + 1] = __uint_as_float(w4[h] & 0xFFFF0000u);
+    }
   }
-  if (tid < k) {
-    int32_t row = 0;
-    for (int j = 0; j < k; ++j) row += (s_sel[j] < s_sel[tid]) ? 1 : 0;
-    disp.perm_token[tid] = 0;
-    disp.inv_perm[tid] = row;
+  __syncthreads();
+  const int grp = tid >> 6, t = tid & 63, cl = t >> 3, e = t & 7;
+  bool ok = true;
+  for (int j = grp; j < nst; j += kR1Slots) {
+    if (ok && !mbar_wait_bounded(&full[grp], static_cast<uint32_t>((j / kR1Slots) & 1), kWaitLimitNs, nullptr)) {
+      record_device_error(6u /* MOE_DEVERR_WAIT_TIMEOUT_ROUTER */);
+      ok = false;
+    }
+    const int row0 = j * kR1StageRows + cl * 128;
+    if (ok && row0 < d) {
+      const int nr = min(128, d - row0);
+      const float* wp = ws + (grp * kR1StageRows + cl * 128) * kR1Experts + e;
+      const float* xp = xs + row0 + (row0 >> 7) * 8;
+      float acc = 0.0f;
+#pragma unroll 8
+      for (int i = 0; i < nr; ++i) acc = __fmaf_rn(xp[i], wp[i * kR1Experts], acc);
+      part[(j * (kR1StageRows / 128) + cl) * kR1Experts + e] = acc;
+    }
+    // the group has read its slot: load the slot's next stage
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(64) : "memory");
+    if (t == 0 && j + kR1Slots < nst) {
+      fence_proxy_async_shared();
+      issue(j + kR1Slots);
+    }
   }
+  __syncthreads();
+  if (tid < kR1Experts && e0 + tid < E) {
+    float l = part[tid];
+    for (int c = 1; c < C; ++c) l = __fadd_rn(l, part[c * kR1Experts + tid]);
+    if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e0 + tid));
+    logits[e0 + tid] = l;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_ticket = atomicAdd(&tickets[0], 1u);
+  __syncthreads();
+  if (s_ticket != static_cast<unsigned int>(G - 1)) return;
+  __threadfence();
+  if (tid == 0) tickets[0] = 0u;
+  one_token_finish(logits, E, k, topk_idx, topk_w, disp);
 }
 
 }  // namespace moe

@@ -60,7 +60,8 @@ def test_route_bit_exact(lib, shape):
 
 
 # The few-token router (T <= 16, E % 4 == 0): one launch that streams every
-# chunk of W_router at once and reduces in the last CTAs. Ragged last chunk
+# chunk of W_router at once and reduces in the last CTAs (for one token with
+# d <= 8192 a CTA per 8 experts walks all of d instead). Ragged last chunk
 # (d % 128 == 64), partial last expert group (E % 128 != 0), one chunk only,
 # k = E, 1024 experts, the full-width decode shape, and a bias.
 STREAM_SHAPES = [
@@ -74,6 +75,7 @@ STREAM_SHAPES = [
     (16, 64, 8, 8, None),
     (9, 7168, 384, 8, "zipf"),
     (2, 128, 6, 1, None),     # E % 4 != 0: the split-chunk router instead
+    (1, 9216, 64, 4, "zipf"),  # one token with d > 8192: the chunk-partial one-token router
 ]
 
 
@@ -427,7 +429,8 @@ def test_route_tensor_core_screen_ties_and_fallback(lib, E, k, bias_on):
 # staged result only by the order of the fp32 partial sums.
 @pytest.mark.parametrize("shape", [(1, 7168, 896, 16, 512, None), (3, 1024, 8, 2, 192, "zipf"),
                                    (8, 2048, 64, 8, 256, None), (32, 512, 16, 4, 320, None),
-                                   (17, 256, 4, 4, 128, None), (1, 256, 16, 4, 2048, None)],
+                                   (17, 256, 4, 4, 128, None), (1, 256, 16, 4, 2048, None),
+                                   (1, 9216, 16, 4, 128, None)],
                          ids=lambda s: "x".join(map(str, s[:5])) + (f"_{s[5]}" if s[5] else ""))
 def test_forward_one_launch_ffn_matches_staged_steps(lib, shape):
     T, d, E, k, f, bias = shape
