@@ -903,12 +903,18 @@ constexpr int kFusedMaxCpt = 16;
 constexpr int kFusedTargetChunks = 4 * 148;  // per GEMM: about four chunks per SM
 constexpr int kFusedQueue = 16;
 constexpr int kFusedBarrierBytes = 512;
+constexpr int kFusedAuxBars = 12;
+// The claim order's lag L (below): half the experts with rows when there are
+// at least kFusedLagMin of them, else all of them (no interleaving), the
+// better of the two as measured on one-token, 8-token and 32-token steps.
+constexpr int kFusedLagMin = 64;
 constexpr int kFusedSmemBytes = GemmCfg<1>::kStages * GemmCfg<1>::kStageBytes + kFusedBarrierBytes +
                                 kFusedQueue * 4 + 3 * (1024 + 1) * 4 + 8 + 1024;
 static_assert(GemmCfg<1>::kStageBytes == GemmCfg<2>::kStageBytes && GemmCfg<1>::kStages == GemmCfg<2>::kStages,
               "the fused launch runs mode 2 and mode 1 chunks in one ring");
 static_assert(kFusedSmemBytes <= 232448, "shared memory per CTA");
-static_assert((2 * GemmCfg<1>::kStages + 5 + 2 * kFusedQueue) * 8 + 8 <= kFusedBarrierBytes, "fused barriers");
+static_assert((2 * GemmCfg<1>::kStages + 5 + 2 * kFusedQueue + kFusedAuxBars) * 8 + 8 <= kFusedBarrierBytes,
+              "fused barriers");
 
 // How one GEMM of the fused launch is cut into chunks (the same in every CTA).
 struct FusedPlan {
@@ -942,80 +948,144 @@ __device__ __forceinline__ void fused_chunk(const GemmParams& p, const int32_t* 
   ti.chunk_count = f.cpt;
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    grouped_ffn_fused_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmBs0,
-                             const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmBs1,
-                             const GemmParams p0, const GemmParams p1, unsigned int* __restrict__ h_ready,
-                             unsigned int* __restrict__ claim) {
+// One CTA's state in the chunk-queue feed-forward: the stage ring, its
+// mbarriers, the chunk queue and the shared tables (tile prefixes of both
+// GEMMs and the expert offsets, E + 1 entries each).
+struct FusedCta {
+  uint8_t* smem;  // 1024-aligned: the ring (kStages stages), then the barriers and tables
+  uint64_t* full_bar;
+  uint64_t* empty_bar;
+  uint64_t* acc_full_bar;
+  uint64_t* acc_empty_bar;
+  uint64_t* drain_bar;
+  uint64_t* q_full;   // [Q] the producer has written entry i
+  uint64_t* q_empty;  // [Q] the MMA lane and every epilogue warp have read it
+  uint64_t* aux_bar;  // [kFusedAuxBars] free for the caller (the one-token router's W ring)
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  volatile int* s_chunk;
+  int32_t* s_pre0;
+  int32_t* s_pre1;
+  int32_t* s_off;
+};
+
+__device__ __forceinline__ FusedCta fused_cta_layout(uint8_t* smem_raw, int E) {
   using Cfg = GemmCfg<1>;
   constexpr int S = Cfg::kStages;
-  constexpr int Q = kFusedQueue;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
-  uint64_t* empty_bar = full_bar + S;
-  uint64_t* acc_full_bar = empty_bar + S;
-  uint64_t* acc_empty_bar = acc_full_bar + 2;
-  uint64_t* drain_bar = acc_empty_bar + 2;
-  uint64_t* q_full = drain_bar + 1;   // [Q] the producer has written entry i
-  uint64_t* q_empty = q_full + Q;     // [Q] the MMA lane and every epilogue warp have read it
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + Q);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_chunk = reinterpret_cast<volatile int*>(smem + S * Cfg::kStageBytes + kFusedBarrierBytes);
-  int32_t* s_pre0 = reinterpret_cast<int32_t*>(smem + S * Cfg::kStageBytes + kFusedBarrierBytes + Q * 4);
-  int32_t* s_pre1 = s_pre0 + (p0.E + 1);
-  int32_t* s_off = s_pre1 + (p0.E + 1);
+  FusedCta c;
+  c.smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  c.full_bar = reinterpret_cast<uint64_t*>(c.smem + S * Cfg::kStageBytes);
+  c.empty_bar = c.full_bar + S;
+  c.acc_full_bar = c.empty_bar + S;
+  c.acc_empty_bar = c.acc_full_bar + 2;
+  c.drain_bar = c.acc_empty_bar + 2;
+  c.q_full = c.drain_bar + 1;
+  c.q_empty = c.q_full + kFusedQueue;
+  c.aux_bar = c.q_empty + kFusedQueue;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(c.aux_bar + kFusedAuxBars);
+  c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
+  c.s_chunk = reinterpret_cast<volatile int*>(c.smem + S * Cfg::kStageBytes + kFusedBarrierBytes);
+  c.s_pre0 = reinterpret_cast<int32_t*>(c.smem + S * Cfg::kStageBytes + kFusedBarrierBytes + kFusedQueue * 4);
+  c.s_pre1 = c.s_pre0 + (E + 1);
+  c.s_off = c.s_pre1 + (E + 1);
+  return c;
+}
 
+// Barrier initialisation (thread 0), tensor-map prefetch (warp 0) and the TMEM
+// allocation (warp 1); the caller then fences and synchronises the CTA.
+__device__ __forceinline__ void fused_cta_setup(const FusedCta& c, const CUtensorMap* tmA0, const CUtensorMap* tmBs0,
+                                                const CUtensorMap* tmA1, const CUtensorMap* tmBs1) {
+  using Cfg = GemmCfg<1>;
+  constexpr int S = Cfg::kStages;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i <= p0.E; i += blockDim.x) {
-    s_pre0[i] = __ldg(p0.tile_prefix + i);
-    s_pre1[i] = __ldg(p1.tile_prefix + i);
-    s_off[i] = __ldg(p0.expert_offsets + i);
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
+      mbar_init(&c.full_bar[s], 1);
+      mbar_init(&c.empty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full_bar[b], 1);
-      mbar_init(&acc_empty_bar[b], kGemmEpiWarps);
+      mbar_init(&c.acc_full_bar[b], 1);
+      mbar_init(&c.acc_empty_bar[b], kGemmEpiWarps);
     }
-    mbar_init(drain_bar, 1);
-    for (int i = 0; i < Q; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1 + kGemmEpiWarps);
+    mbar_init(c.drain_bar, 1);
+    for (int i = 0; i < kFusedQueue; ++i) {
+      mbar_init(&c.q_full[i], 1);
+      mbar_init(&c.q_empty[i], 1 + kGemmEpiWarps);
     }
-    *abort_flag = 0;
+    for (int i = 0; i < kFusedAuxBars; ++i) mbar_init(&c.aux_bar[i], 1);
+    *c.abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_shared();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA0);
-    tma_prefetch_desc(&tmBs0);
-    tma_prefetch_desc(&tmA1);
-    tma_prefetch_desc(&tmBs1);
+    tma_prefetch_desc(tmA0);
+    tma_prefetch_desc(tmBs0);
+    tma_prefetch_desc(tmA1);
+    tma_prefetch_desc(tmBs1);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_alloc(c.tmem_slot, GemmCfg<1>::kTmemCols);
     tmem_relinquish();
   }
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const GemmRing ring{smem, full_bar, empty_bar, acc_full_bar, acc_empty_bar, abort_flag, *tmem_slot};
+}
+
+// The CTA's part of the feed-forward: claims chunks until the queue is empty
+// (producer lane of warp 0), issues their MMAs (lane 0 of warp 1) and runs
+// their epilogues (warps 2..9). The shared tables must be loaded.
+__device__ __forceinline__ void fused_cta_run(const FusedCta& fc, const CUtensorMap* tmA0, const CUtensorMap* tmBs0,
+                                              const CUtensorMap* tmA1, const CUtensorMap* tmBs1, const GemmParams& p0,
+                                              const GemmParams& p1, unsigned int* __restrict__ h_ready,
+                                              unsigned int* __restrict__ claim) {
+  using Cfg = GemmCfg<1>;
+  constexpr int S = Cfg::kStages;
+  constexpr int Q = kFusedQueue;
+  uint8_t* smem = fc.smem;
+  uint64_t* full_bar = fc.full_bar;
+  uint64_t* empty_bar = fc.empty_bar;
+  uint64_t* drain_bar = fc.drain_bar;
+  uint64_t* q_full = fc.q_full;
+  uint64_t* q_empty = fc.q_empty;
+  volatile int* abort_flag = fc.abort_flag;
+  volatile int* s_chunk = fc.s_chunk;
+  const int32_t* s_pre0 = fc.s_pre0;
+  const int32_t* s_pre1 = fc.s_pre1;
+  const int32_t* s_off = fc.s_off;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const GemmRing ring{smem, full_bar, empty_bar, fc.acc_full_bar, fc.acc_empty_bar, abort_flag, *fc.tmem_slot};
   const unsigned int h_target = static_cast<unsigned int>(kGemmEpiWarps * p0.n_feat_tiles);
   const FusedPlan f0 = fused_plan(p0, s_pre0[p0.E] * p0.n_feat_tiles);
   const FusedPlan f1 = fused_plan(p1, s_pre1[p0.E] * p1.n_feat_tiles);
   const int total = f0.chunks + f1.chunks;
-  // chunk id -> work item of the gate/up (true) or the down GEMM
+  // Claim order. Every expert with rows has one token block in each GEMM (no
+  // step of this launch gives an expert more than 32 rows), so it has G
+  // gate/up and D down chunks. The gate/up chunks of the first L experts come
+  // first; then, for each later expert i, its gate/up chunks followed by the
+  // down chunks of expert i - L; then the down chunks of the last L experts.
+  // A down chunk is thus claimed L experts' worth of work after the gate/up
+  // chunks whose h rows it reads, instead of right behind the last of them.
+  const int nsel = s_pre0[p0.E];
+  const int G = nsel > 0 ? f0.chunks / nsel : 0;
+  const int D = nsel > 0 ? f1.chunks / nsel : 0;
+  const int L = nsel >= kFusedLagMin ? (nsel + 1) / 2 : nsel;
+  const int seg_a = L * G, seg_b = (nsel - L) * (G + D);
+  // claim id -> work item of the gate/up (true) or the down GEMM
   auto decode = [&](int c, TileInfo& ti) -> bool {
-    if (c < f0.chunks) {
-      fused_chunk<2>(p0, s_pre0, s_off, f0, c, ti);
+    int gate_up = 1, loc = c;
+    if (c >= seg_a && c < seg_a + seg_b) {
+      const int i = (c - seg_a) / (G + D), r = (c - seg_a) - i * (G + D);
+      gate_up = r < G;
+      loc = gate_up ? (L + i) * G + r : i * D + (r - G);
+    } else if (c >= seg_a + seg_b) {
+      gate_up = 0;
+      loc = (nsel - L) * D + (c - seg_a - seg_b);
+    }
+    if (gate_up) {
+      fused_chunk<2>(p0, s_pre0, s_off, f0, loc, ti);
       return true;
     }
-    fused_chunk<1>(p1, s_pre1, s_off, f1, c - f0.chunks, ti);
+    fused_chunk<1>(p1, s_pre1, s_off, f1, loc, ti);
     return false;
   };
 
@@ -1064,7 +1134,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           fence_proxy_async_global();
           const int st_i = q_stage[q_head];
-          gemm_load_b<1>(smem + st_i * Cfg::kStageBytes, &tmBs1, &tmBs1, &full_bar[st_i], p1, q_row[q_head], 1,
+          gemm_load_b<1>(smem + st_i * Cfg::kStageBytes, tmBs1, tmBs1, &full_bar[st_i], p1, q_row[q_head], 1,
                          q_k0[q_head], pol_x);
           q_head = (q_head + 1) % S;
           --q_n;
@@ -1099,10 +1169,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full_bar[s], kTx);
           const int k0 = kb * kGemmBK;
           if (!down) {
-            gemm_load_a<2>(st, &tmA0, &full_bar[s], p0, ti, k0, pol_w);
-            gemm_load_b<2>(st, &tmBs0, &tmBs0, &full_bar[s], p0, ti.row0, 1, k0, pol_x);
+            gemm_load_a<2>(st, tmA0, &full_bar[s], p0, ti, k0, pol_w);
+            gemm_load_b<2>(st, tmBs0, tmBs0, &full_bar[s], p0, ti.row0, 1, k0, pol_x);
           } else {
-            gemm_load_a<1>(st, &tmA1, &full_bar[s], p1, ti, k0, pol_w);
+            gemm_load_a<1>(st, tmA1, &full_bar[s], p1, ti, k0, pol_w);
             const int qj = (q_head + q_n) % S;
             q_stage[qj] = s;
             q_k0[qj] = k0;
@@ -1190,13 +1260,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) break;
     }
   }
+}
 
+__device__ __forceinline__ void fused_cta_teardown(const FusedCta& fc) {
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if ((threadIdx.x >> 5) == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(ring.tmem_base, Cfg::kTmemCols);
+    tmem_dealloc(*fc.tmem_slot, GemmCfg<1>::kTmemCols);
   }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_ffn_fused_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmBs0,
+                             const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmBs1,
+                             const GemmParams p0, const GemmParams p1, unsigned int* __restrict__ h_ready,
+                             unsigned int* __restrict__ claim) {
+  extern __shared__ uint8_t smem_raw[];
+  const FusedCta fc = fused_cta_layout(smem_raw, p0.E);
+  for (int i = threadIdx.x; i <= p0.E; i += blockDim.x) {
+    fc.s_pre0[i] = __ldg(p0.tile_prefix + i);
+    fc.s_pre1[i] = __ldg(p1.tile_prefix + i);
+    fc.s_off[i] = __ldg(p0.expert_offsets + i);
+  }
+  fused_cta_setup(fc, &tmA0, &tmBs0, &tmA1, &tmBs1);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  fused_cta_run(fc, &tmA0, &tmBs0, &tmA1, &tmBs1, p0, p1, h_ready, claim);
+  fused_cta_teardown(fc);
 }
 
 // Token blocks per expert for both GEMMs:

@@ -252,18 +252,36 @@ __global__ void __launch_bounds__(256)
 
 namespace moe {
 
+// The barrier of the threads that run the CTA-wide helpers below: the whole
+// CTA, or, in a CTA of more than 256 threads, threads 0..255 alone (named
+// barrier 5).
+struct CtaSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct FirstWarps8Sync {
+  __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 5, 256;" ::: "memory"); }
+};
+
+// The probability of a logit l given the softmax statistics of its token:
+// exp(l - M) / S. The CTA-wide top-k helpers below and the one-launch
+// one-token kernel (which takes the weights after the selection) share this
+// expression, so both give the same bits.
+__device__ __forceinline__ float softmax_weight(float l, float M, float S) { return expf(l - M) / S; }
+
 // Softmax statistics of one token's E <= 1024 logits held in shared memory,
 // by a CTA of 256 threads: M = max_e l_e and S = sum_e exp(l_e - M), the sum
 // taken per warp in a fixed shuffle order and then over the warps in order.
-__device__ __forceinline__ void cta_softmax_stats_256(const float* s_l, int E, float* M, float* S) {
+template <class Sync = CtaSync>
+__device__ __forceinline__ void cta_softmax_stats_256(const float* s_l, int E, float* M, float* S, Sync sync = Sync(),
+                                                      int tid = threadIdx.x) {
   __shared__ float s_wm[8], s_ws[8];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int lane = tid & 31, w = tid >> 5;
   float m = -INFINITY;
   for (int e = tid; e < E; e += 256) m = fmaxf(m, s_l[e]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) s_wm[w] = m;
-  __syncthreads();
+  sync();
   float gm = s_wm[0];
 #pragma unroll
   for (int q = 1; q < 8; ++q) gm = fmaxf(gm, s_wm[q]);
@@ -272,7 +290,7 @@ __device__ __forceinline__ void cta_softmax_stats_256(const float* s_l, int E, f
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) s_ws[w] = s;
-  __syncthreads();
+  sync();
   float gs = s_ws[0];
 #pragma unroll
   for (int q = 1; q < 8; ++q) gs += s_ws[q];
@@ -280,7 +298,7 @@ __device__ __forceinline__ void cta_softmax_stats_256(const float* s_l, int E, f
   *S = gs;
 }
 
-// For warp 0: the bin of a 256-bin histogram (hist, bins ascending) that
+// For one warp: the bin of a 256-bin histogram (hist, bins ascending) that
 // holds the kk-th largest element, and how many elements lie in higher bins.
 __device__ __forceinline__ void warp_find_bin_from_top(const unsigned* hist, unsigned kk, unsigned* bin,
                                                        unsigned* above) {
@@ -317,9 +335,10 @@ __device__ __forceinline__ void warp_find_bin_from_top(const unsigned* hist, uns
 // candidates by the key (order key of the logit, -0 taken as +0; then the
 // complemented index), a total order. Returns false, writing nothing, when
 // more than 64 logits are candidates (heavy ties); the caller then takes
-// cta_topk_rounds_256.
+// cta_topk_rounds_256. out_w may be null (indices only).
+template <class Sync = CtaSync>
 __device__ __forceinline__ bool cta_topk_histogram_256(const float* s_l, int E, int k, float M, float S,
-                                                       int32_t* out_idx, float* out_w) {
+                                                       int32_t* out_idx, float* out_w, Sync sync = Sync()) {
   __shared__ unsigned s_hist[256];
   __shared__ unsigned s_sel[4];
   __shared__ unsigned s_ncand;
@@ -334,23 +353,23 @@ __device__ __forceinline__ bool cta_topk_histogram_256(const float* s_l, int E, 
   // pass 1: the top byte of the key
   s_hist[tid] = 0u;
   if (tid == 0) s_ncand = 0u;
-  __syncthreads();
+  sync();
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (tid + 256 * i < E) atomicAdd(&s_hist[key[i] >> 24], 1u);
-  __syncthreads();
+  sync();
   if (w == 0) warp_find_bin_from_top(s_hist, static_cast<unsigned>(k), &s_sel[0], &s_sel[1]);
-  __syncthreads();
+  sync();
   const unsigned b1 = s_sel[0], above1 = s_sel[1];
   // pass 2: the second byte, within that bin
   s_hist[tid] = 0u;
-  __syncthreads();
+  sync();
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     if (tid + 256 * i < E && (key[i] >> 24) == b1) atomicAdd(&s_hist[(key[i] >> 16) & 255u], 1u);
-  __syncthreads();
+  sync();
   if (w == 0) warp_find_bin_from_top(s_hist, static_cast<unsigned>(k) - above1, &s_sel[2], &s_sel[3]);
-  __syncthreads();
+  sync();
   const unsigned thr = (b1 << 8) | s_sel[2];
   const unsigned ncand = above1 + s_sel[3] + s_hist[s_sel[2]];
   if (ncand > 64u) return false;  // the same for every thread: all read the same shared values
@@ -363,7 +382,7 @@ __device__ __forceinline__ bool cta_topk_histogram_256(const float* s_l, int E, 
       s_ckey[slot] = (static_cast<uint64_t>(key[i]) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(e));
     }
   }
-  __syncthreads();
+  sync();
   if (w == 0) {
     for (unsigned r = lane; r < ncand; r += 32) {
       const uint64_t kk = s_ckey[r];
@@ -372,7 +391,7 @@ __device__ __forceinline__ bool cta_topk_histogram_256(const float* s_l, int E, 
       if (rank < k) {
         const int e = static_cast<int>(~static_cast<uint32_t>(kk & 0xffffffffu));
         out_idx[rank] = e;
-        out_w[rank] = expf(s_l[e] - M) / S;
+        if (out_w != nullptr) out_w[rank] = softmax_weight(s_l[e], M, S);
       }
     }
   }
@@ -381,9 +400,10 @@ __device__ __forceinline__ bool cta_topk_histogram_256(const float* s_l, int E, 
 
 // Top-k by k rounds of arg-max (the general case, any ties): warp w takes the
 // experts e with (e / 32) % 8 == w and finds its local top-k; warp 0 merges
-// the 8 local lists. Weights exp(l - M) / S.
+// the 8 local lists. Weights exp(l - M) / S (out_w may be null).
+template <class Sync = CtaSync>
 __device__ __forceinline__ void cta_topk_rounds_256(const float* s_l, int E, int k, float M, float S,
-                                                    int32_t* out_idx, float* out_w) {
+                                                    int32_t* out_idx, float* out_w, Sync sync = Sync()) {
   __shared__ float s_cv[8][16];
   __shared__ int s_ci[8][16];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -420,7 +440,7 @@ __device__ __forceinline__ void cta_topk_rounds_256(const float* s_l, int E, int
       s_ci[w][j] = wi >= 0 ? wi : 0x7fffffff;
     }
   }
-  __syncthreads();
+  sync();
 
   // merge
   if (w == 0) {
@@ -459,20 +479,23 @@ __device__ __forceinline__ void cta_topk_rounds_256(const float* s_l, int E, int
       }
       if (lane == 0) {
         out_idx[j] = wb;
-        out_w[j] = expf(wv - M) / S;
+        if (out_w != nullptr) out_w[j] = softmax_weight(wv, M, S);
       }
     }
   }
 }
 
 // Softmax over one token's E <= 1024 final logits, held in shared memory, and
-// their top-k by (logit desc, index asc), by a CTA of 256 threads. Writes
-// out_idx[0..k) and out_w[0..k) = exp(l - M) / S. Every thread of the CTA
-// must call it.
-__device__ __forceinline__ void cta_softmax_topk_256(const float* s_l, int E, int k, int32_t* out_idx, float* out_w) {
+// their top-k by (logit desc, index asc), by 256 threads (threads 0..255 of
+// the CTA, all of which must call it; `sync` is their barrier). Writes
+// out_idx[0..k) and out_w[0..k) = exp(l - M) / S.
+template <class Sync = CtaSync>
+__device__ __forceinline__ void cta_softmax_topk_256(const float* s_l, int E, int k, int32_t* out_idx, float* out_w,
+                                                     Sync sync = Sync()) {
   float M, S;
-  cta_softmax_stats_256(s_l, E, &M, &S);
-  if (!cta_topk_histogram_256(s_l, E, k, M, S, out_idx, out_w)) cta_topk_rounds_256(s_l, E, k, M, S, out_idx, out_w);
+  cta_softmax_stats_256(s_l, E, &M, &S, sync);
+  if (!cta_topk_histogram_256(s_l, E, k, M, S, out_idx, out_w, sync))
+    cta_topk_rounds_256(s_l, E, k, M, S, out_idx, out_w, sync);
 }
 
 // Small-T router, second half, one block of 256 threads per token:

@@ -257,27 +257,24 @@ __host__ __device__ constexpr int router_one_smem_bytes() {
   return kR1Slots * kR1StageRows * kR1Experts * 4 + router_one_x_floats() * 4 + (kR1MaxD / 128) * kR1Experts * 4;
 }
 
-__global__ void __launch_bounds__(256)
-    router_one_token_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ x,
-                            const float* __restrict__ bias, int d, int E, int k, float* __restrict__ logits,
-                            unsigned int* __restrict__ tickets, int32_t* __restrict__ topk_idx,
-                            float* __restrict__ topk_w, const RouteDispatch disp) {
-  extern __shared__ __align__(128) uint8_t r1_smem[];
-  float* ws = reinterpret_cast<float*>(r1_smem);                 // [slot][1024 rows][8 experts]
+// The logits of experts [e0, e0 + 8) of one token, by threads 0..255 of the
+// calling CTA (every one of them calls it; tid = threadIdx.x). `sm` holds
+// router_one_smem_bytes() of shared memory (W ring, widened x, chunk sums) and
+// full[kR1Slots] are mbarriers initialised to count 1 and fenced by the caller.
+// Named barriers 1..5 are used. A warp's 32 threads are four chunks x eight
+// experts, and chunk c of a group starts its chain c steps after chunk 0, so at
+// each step the four chunks read rows in four different bank groups (every
+// chain still runs over its rows in ascending order). Returns false when a
+// wait for W gave up (MOE_DEVERR_WAIT_TIMEOUT_ROUTER recorded).
+__device__ __forceinline__ bool router_one_token_logits(const CUtensorMap* tmW, const uint16_t* __restrict__ x,
+                                                        const float* __restrict__ bias, int d, int E, int e0,
+                                                        uint8_t* sm, uint64_t* full, float* __restrict__ logits) {
+  float* ws = reinterpret_cast<float*>(sm);                      // [slot][1024 rows][8 experts]
   float* xs = ws + kR1Slots * kR1StageRows * kR1Experts;         // x widened, chunk c at 136 c
   float* part = xs + router_one_x_floats();                      // chunk sums [C][8]
-  __shared__ __align__(8) uint64_t full[kR1Slots];
-  __shared__ unsigned int s_ticket;
-  const int g = blockIdx.x, G = gridDim.x, tid = threadIdx.x;
-  const int e0 = g * kR1Experts;
+  const int tid = threadIdx.x;
   const int nst = (d + kR1StageRows - 1) / kR1StageRows;
   const int C = (d + 127) / 128;
-  if (disp.zero_buf != nullptr) {
-    // the feed-forward's counters, cleared by all CTAs at once (only the next
-    // launch reads them)
-    for (int64_t i = static_cast<int64_t>(g) * 256 + tid; i < disp.zero_n; i += static_cast<int64_t>(G) * 256)
-      disp.zero_buf[i] = 0u;
-  }
   // stage j into slot j % 4: its boxes of 256 rows that start inside d
   auto issue = [&](int j) {
     const int slot = j % kR1Slots;
@@ -285,15 +282,9 @@ __global__ void __launch_bounds__(256)
     const int nbox = min(kR1StageRows / kR1BoxRows, (d - r0 + kR1BoxRows - 1) / kR1BoxRows);
     mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nbox * kR1BoxRows * kR1Experts * 4));
     for (int b = 0; b < nbox; ++b)
-      tma_load_2d(ws + (slot * kR1StageRows + b * kR1BoxRows) * kR1Experts, &tmW, &full[slot], e0,
+      tma_load_2d(ws + (slot * kR1StageRows + b * kR1BoxRows) * kR1Experts, tmW, &full[slot], e0,
                   r0 + b * kR1BoxRows, l2_policy_evict_first());
   };
-  if (tid == 0) {
-    for (int s = 0; s < kR1Slots; ++s) mbar_init(&full[s], 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&tmW);
-  }
-  __syncthreads();
   if (tid == 0)
     for (int j = 0; j < kR1Slots && j < nst; ++j) issue(j);
   for (int v = tid; v < d / 8; v += 256) {
@@ -306,8 +297,9 @@ __global__ void __launch_bounds__(256)
       dst[2 * h + 1] = __uint_as_float(w4[h] & 0xFFFF0000u);
     }
   }
-  __syncthreads();
+  FirstWarps8Sync()();
   const int grp = tid >> 6, t = tid & 63, cl = t >> 3, e = t & 7;
+  const int skew = cl & 3;  // the chunk's place among the warp's four
   bool ok = true;
   for (int j = grp; j < nst; j += kR1Slots) {
     if (ok && !mbar_wait_bounded(&full[grp], static_cast<uint32_t>((j / kR1Slots) & 1), kWaitLimitNs, nullptr)) {
@@ -319,9 +311,15 @@ __global__ void __launch_bounds__(256)
       const int nr = min(128, d - row0);
       const float* wp = ws + (grp * kR1StageRows + cl * 128) * kR1Experts + e;
       const float* xp = xs + row0 + (row0 >> 7) * 8;
+      // step s reads row s - skew: steps skew..2, then 3..nr-1 for every
+      // chunk of the warp at once, then nr..nr+skew-1
+      const float* xq = xp - skew;
+      const float* wq = wp - skew * kR1Experts;
       float acc = 0.0f;
+      for (int s = skew; s < 3; ++s) acc = __fmaf_rn(xq[s], wq[s * kR1Experts], acc);
 #pragma unroll 8
-      for (int i = 0; i < nr; ++i) acc = __fmaf_rn(xp[i], wp[i * kR1Experts], acc);
+      for (int s = 3; s < nr; ++s) acc = __fmaf_rn(xq[s], wq[s * kR1Experts], acc);
+      for (int s = nr; s < nr + skew; ++s) acc = __fmaf_rn(xq[s], wq[s * kR1Experts], acc);
       part[(j * (kR1StageRows / 128) + cl) * kR1Experts + e] = acc;
     }
     // the group has read its slot: load the slot's next stage
@@ -331,13 +329,38 @@ __global__ void __launch_bounds__(256)
       issue(j + kR1Slots);
     }
   }
-  __syncthreads();
+  FirstWarps8Sync()();
   if (tid < kR1Experts && e0 + tid < E) {
     float l = part[tid];
     for (int c = 1; c < C; ++c) l = __fadd_rn(l, part[c * kR1Experts + tid]);
     if (bias != nullptr) l = __fadd_rn(l, __ldg(bias + e0 + tid));
     logits[e0 + tid] = l;
   }
+  return ok;
+}
+
+__global__ void __launch_bounds__(256)
+    router_one_token_kernel(const __grid_constant__ CUtensorMap tmW, const uint16_t* __restrict__ x,
+                            const float* __restrict__ bias, int d, int E, int k, float* __restrict__ logits,
+                            unsigned int* __restrict__ tickets, int32_t* __restrict__ topk_idx,
+                            float* __restrict__ topk_w, const RouteDispatch disp) {
+  extern __shared__ __align__(128) uint8_t r1_smem[];
+  __shared__ __align__(8) uint64_t full[kR1Slots];
+  __shared__ unsigned int s_ticket;
+  const int g = blockIdx.x, G = gridDim.x, tid = threadIdx.x;
+  if (disp.zero_buf != nullptr) {
+    // the feed-forward's counters, cleared by all CTAs at once (only the next
+    // launch reads them)
+    for (int64_t i = static_cast<int64_t>(g) * 256 + tid; i < disp.zero_n; i += static_cast<int64_t>(G) * 256)
+      disp.zero_buf[i] = 0u;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kR1Slots; ++s) mbar_init(&full[s], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+  }
+  __syncthreads();
+  router_one_token_logits(&tmW, x, bias, d, E, g * kR1Experts, r1_smem, full, logits);
   __threadfence();
   __syncthreads();
   if (tid == 0) s_ticket = atomicAdd(&tickets[0], 1u);

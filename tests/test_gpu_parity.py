@@ -458,3 +458,33 @@ def test_forward_one_launch_ffn_matches_staged_steps(lib, shape):
     torch.cuda.synchronize()
     assert lib.get_device_error() == 0
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+@pytest.mark.parametrize("shape", [(1, 7168, 896, 16, 512, None), (1, 7168, 896, 16, 512, "zipf"),
+                                   (1, 8192, 64, 1, 128, None), (1, 64, 20, 3, 64, None),
+                                   (1, 1024, 12, 12, 192, None), (1, 2048, 1024, 16, 256, "zipf")],
+                         ids=lambda s: "x".join(map(str, s[:5])) + (f"_{s[5]}" if s[5] else ""))
+def test_one_token_single_launch_matches_separate_launches(lib, shape):
+    """One token: moe_forward runs router, dispatch, both GEMMs and the combine
+    in one cooperative launch; moe_forward_timed runs them as three launches
+    (router, one-launch feed-forward, combine). Same arithmetic in the same
+    order, so the same bits; both within the layer tolerance of the oracle.
+    Shapes: the one-token decode step with and without a router bias, the
+    largest d of the one-token router, a single 64-row chunk with E not a
+    multiple of 8, k = E, and the most experts (128 router CTAs). A second
+    call gives the same bits (the launch's counters are cleared each call)."""
+    T, d, E, k, f, bias = shape
+    inp = _inputs(T, d, E, k, f, bias=bias, seed=4)
+    g = _cuda(inp)
+    ws = torch.zeros(lib.moe_forward_workspace_size(T, d, E, k, f), dtype=torch.uint8, device="cuda")
+    one = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k, workspace=ws).clone()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(lib.TIMED_STAGES))]
+    three = torch.empty_like(one)
+    lib.moe_forward_timed(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k, evs, three, ws)
+    again = lib.moe_forward(g.x, g.W_router, g.bias, g.W_gate_up, g.W_down, k, workspace=ws)
+    torch.cuda.synchronize()
+    assert lib.get_device_error() == 0
+    ref, _, _ = oracle.forward(inp.x, inp.W_router, inp.bias, inp.W_gate_up, inp.W_down, k)
+    parity.assert_layer_close(one, ref, "one-token single launch")
+    assert torch.equal(one.view(torch.int16), three.view(torch.int16)), "single launch differs from three launches"
+    assert torch.equal(one.view(torch.int16), again.view(torch.int16))
