@@ -152,6 +152,11 @@ moe_status_t moe_unpermute(const moe_bf16_t* y_perm, const int32_t* inv_perm, co
  * stream, with no host synchronisation. All intermediates are carved from
  * `workspace` (at least moe_forward_workspace_size(T, d, E, k, f) bytes,
  * 256-byte aligned). out [T, d] bf16.
+ * Launch shapes: T <= 32 runs both expert GEMMs as one cooperative launch
+ * (its own K split, so its sums may differ from moe_expert_ffn's in rounding
+ * order); T = 1 with d <= 8192 runs the whole layer as one cooperative launch
+ * (after an 8-byte memset of its barrier counts), bit-identical to the
+ * separate stages that moe_forward_timed runs.
  */
 size_t moe_forward_workspace_size(int T, int d, int E, int k, int f);
 moe_status_t moe_forward(const moe_bf16_t* x, const float* W_router, const float* router_bias,
@@ -168,7 +173,9 @@ moe_status_t moe_forward(const moe_bf16_t* x, const float* W_router, const float
  *   row copy, GEMM tile schedule)       2 gate/up grouped GEMM (one kernel)
  *   3 down grouped GEMM (one kernel)    4 combine (one kernel)
  * Same arguments, results and errors as moe_forward otherwise; events == NULL
- * is MOE_ERR_INVALID_ARG.
+ * is MOE_ERR_INVALID_ARG. The stages always run as separate launches (for
+ * T = 1 the router, the feed-forward and the combine, where moe_forward runs
+ * one launch).
  */
 #define MOE_TIMED_STAGES 5
 moe_status_t moe_forward_timed(const moe_bf16_t* x, const float* W_router, const float* router_bias,
