@@ -140,6 +140,7 @@ def algorithmic(shape: moe_inputs.MoEShape, counts: np.ndarray):
 # Steps of at most this many tokens run both expert GEMMs in one launch
 # (the library's one-launch feed-forward): the gate/up stage then times both.
 FUSED_FFN_MAX_TOKENS = 32
+ONE_TOKEN_MAX_D = 8192  # one-token steps up to this width run the whole layer in one launch
 
 
 def count_library_launches(step) -> int:
@@ -410,7 +411,15 @@ def layer_summary(shape, res, steps: int, world: int, peaks: dict) -> dict:
     tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     gu_ms = statistics.mean(res["stage_ms"]["gemm_gate_up"])
     layer_roof_s = max(alg["F"] / (tc * 1e12), alg["B"] / (hbm * 1e9))
-    if T <= FUSED_FFN_MAX_TOKENS:
+    if T == 1 and shape.d <= ONE_TOKEN_MAX_D:
+        # the step is one launch (moe_one_token_kernel) plus an 8-byte memset;
+        # the per-stage times above come from the three-launch form
+        gu_ms = ms_per_step
+        dom = {"kernel": "moe_one_token_kernel (router, top-k, both GEMMs and the combine, one launch)",
+               "bytes": alg["B"], "flops": alg["F"],
+               "rule": "the layer's bytes: W_router fp32 + touched experts x 6*d*f + x and out (per step, "
+                       "which also holds the 8-byte memset of its barrier counts)"}
+    elif T <= FUSED_FFN_MAX_TOKENS:
         dom = {"kernel": "grouped_ffn_fused_kernel (gate/up + SwiGLU + down, one launch)",
                "bytes": alg["ffn_bytes"], "flops": alg["ffn_flops"],
                "rule": "touched experts x 6*d*f (gate, up and down weights, bf16)"}
