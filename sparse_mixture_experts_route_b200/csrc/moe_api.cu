@@ -1314,8 +1314,15 @@ moe_status_t moe_forward_mx(const moe_bf16_t* x, const float* W_router, const fl
                                                    ticket_words);
     }
   }
-  mx_quantize_dispatch_kernel<<<static_cast<unsigned>(T), 256, 0, stream>>>(
-      reinterpret_cast<const uint4*>(x), idx, inv_perm, offsets, pre0, d, k, E, xq, sfx);
+  {
+    // few tokens: one warp per CTA and several CTAs per token (a block per thread)
+    const int nblk = d / kMxBlock;
+    const bool spread = T < 64;
+    const unsigned threads = spread ? 32u : 256u;
+    const dim3 grid(static_cast<unsigned>(T), spread ? static_cast<unsigned>(ceil_div(nblk, 32)) : 1u);
+    mx_quantize_dispatch_kernel<<<grid, threads, 0, stream>>>(reinterpret_cast<const uint4*>(x), idx, inv_perm,
+                                                             offsets, pre0, d, k, E, xq, sfx);
+  }
 
   MxGemmParams p0;
   p0.expert_offsets = offsets;

@@ -85,7 +85,9 @@ __global__ void __launch_bounds__(256)
 }
 
 // x [T][d] bf16 -> MXFP8 rows in dispatch order plus per-tile scale atoms, in
-// one pass: CTA per token, thread per 32-element block; each block's codes
+// one pass: CTA (t, s) for token t takes the blocks s * blockDim.x + i,
+// (s + gridDim.y) * blockDim.x + i, ... (one thread per 32-element block; a
+// step of few tokens spreads each token over several CTAs); each block's codes
 // and scale go to all k of the token's dispatched rows. Pair (t, j) has expert
 // e = idx[t * k + j] and row r = inv_perm[t * k + j]; its tile is
 // prefix[e] + (r - offsets[e]) / kMxTileRows and its row in the tile
@@ -110,7 +112,8 @@ __global__ void __launch_bounds__(256)
     if (!ok) record_device_error(5u /* MOE_DEVERR_BAD_ROUTE */);
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+  for (int b = static_cast<int>(blockIdx.y * blockDim.x + threadIdx.x); b < nblk;
+       b += static_cast<int>(gridDim.y * blockDim.x)) {
     uint4 q[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) q[i] = __ldg(x + (static_cast<int64_t>(t) * nblk + b) * 4 + i);
