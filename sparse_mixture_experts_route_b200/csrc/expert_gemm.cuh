@@ -888,8 +888,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // rows (h) only once h_ready[e] reaches kGemmEpiWarps * (gate/up feature
 // tiles); its weight boxes do not depend on h, so the producer issues them at
 // once and keeps up to a ring of stages whose token rows are still pending.
-// The producer lane claims the chunks and passes each id to the MMA lane and
-// the epilogue warps through a small shared-memory queue (kFusedQueue entries,
+// The producer lane claims the chunks (its CTA's index first, then from an
+// atomic counter) and passes each id to the MMA lane and the epilogue warps
+// through a small shared-memory queue (kFusedQueue entries,
 // one mbarrier pair each). The launch is cooperative (every CTA resident), so
 // a wait on another CTA always ends; it is bounded anyway, recording
 // MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY. The claim counter, the tickets and
@@ -1140,8 +1141,12 @@ __device__ __forceinline__ void fused_cta_run(const FusedCta& fc, const CUtensor
           --q_n;
         }
       };
+      // a CTA's first chunk is its own index (no atomic round trip before the
+      // first loads); later ones come from the counter, from gridDim.x on
+      bool first_claim = true;
       while (ok) {
-        const unsigned int id = atomicAdd(claim, 1u);
+        const unsigned int id = first_claim ? blockIdx.x : gridDim.x + atomicAdd(claim, 1u);
+        first_claim = false;
         const int c = id < static_cast<unsigned int>(total) ? static_cast<int>(id) : -1;
         // hand the id to the MMA lane and the epilogue warps
         if (!mbar_wait_bounded(&q_empty[qi], qph ^ 1u, kWaitLimitNs, abort_flag)) {
