@@ -869,8 +869,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // For steps in which no expert has more than 32 rows (T <= 32), the gate/up
 // GEMM (mode 2) and the down GEMM (mode 1) run in one persistent cooperative
 // launch whose CTAs take their work from a shared queue: chunk ids are handed
-// out one at a time by an atomic counter, gate/up chunks first, then down
-// chunks, both in expert-major tile order. A chunk is one tile's K-block range
+// out one at a time (a CTA's own index first, then by an atomic counter), the
+// gate/up chunks before the down chunks of the same expert, both in
+// expert-major tile order (with 64 or more experts with rows the down chunks
+// of expert i - L follow the gate/up chunks of expert i; see the claim order
+// in fused_cta_run). A chunk is one tile's K-block range
 // [j * ck, (j + 1) * ck); a GEMM with few tiles cuts each of them into up to
 // kFusedTargetChunks / tiles chunks (about four per SM) so that every SM stays busy, one with many
 // tiles hands out whole tiles. Because the queue is shared, a CTA that streams
@@ -888,10 +891,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // rows (h) only once h_ready[e] reaches kGemmEpiWarps * (gate/up feature
 // tiles); its weight boxes do not depend on h, so the producer issues them at
 // once and keeps up to a ring of stages whose token rows are still pending.
-// The producer lane claims the chunks (its CTA's index first, then from an
-// atomic counter) and passes each id to the MMA lane and the epilogue warps
-// through a small shared-memory queue (kFusedQueue entries,
-// one mbarrier pair each). The launch is cooperative (every CTA resident), so
+// The producer lane claims the chunks and passes each id to the MMA lane and
+// the epilogue warps through a small shared-memory queue (kFusedQueue
+// entries, one mbarrier pair each). The launch is cooperative (every CTA resident), so
 // a wait on another CTA always ends; it is bounded anyway, recording
 // MOE_DEVERR_WAIT_TIMEOUT_DEPENDENCY. The claim counter, the tickets and
 // h_ready start at zero (the dispatch step clears them).
